@@ -1,0 +1,228 @@
+"""CPU oracle for the INT8 ConvRot linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or calls it, and it shares no code
+with that path.
+
+The arithmetic lives in ``convrot_oracle.c`` (plain C, compiled with gcc, no
+fast-math, no FMA contraction); this module only compiles it and marshals
+numpy arrays through ctypes.  What each function computes, and the passage of
+the source pages it follows, is stated in the C file:
+
+* grouped Hadamard rotation, group 256, Sylvester order, 1/16 normalisation,
+  exact FP64 sum rounded once to FP32  (0539edu.com "minimax-h3-nvfp4-convrot",
+  section 4 "INT8 ConvRot"; zskr.cn "Qwen3-VL-32B ... INT8-ConvRot",
+  "INT8 ConvRot quantisation details")
+* row-wise symmetric INT8 round-to-nearest-even quantisation
+  (zskr.cn conversion command ``--int8 --scaling_mode row``; 0539edu.com
+  section 5, ``--simple`` = RTN)
+* exact INT8 x INT8 -> INT32 GEMM and FP32 dequantisation to BF16
+  (0539edu.com section 4 and summary item 3)
+
+Every function here is pinned by the ``-m "not gpu"`` tests against
+something other than itself (scipy's Hadamard, closed forms, brute force,
+numpy integer matmul, hand-worked tie cases).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "convrot_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c99", "-Wall",
+           "-shared", "-fPIC"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``convrot_oracle.c`` into ``liboracle.so`` next to it."""
+    if force or not os.path.exists(_LIB) or (
+            os.path.getmtime(_LIB) < os.path.getmtime(_SRC)):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        lib.oracle_sylvester_hadamard.argtypes = [ctypes.c_int, P]
+        lib.oracle_sylvester_hadamard.restype = ctypes.c_int
+        lib.oracle_rotate_rows.argtypes = [P, I64, I64, ctypes.c_int, P, P]
+        lib.oracle_rotate_rows.restype = ctypes.c_int
+        lib.oracle_rotate_rows_f64.argtypes = [P, I64, I64, ctypes.c_int, P]
+        lib.oracle_rotate_rows_f64.restype = ctypes.c_int
+        lib.oracle_quantize_rows.argtypes = [P, I64, I64, P, P]
+        lib.oracle_quantize_rows.restype = I64
+        lib.oracle_gemm_i32.argtypes = [P, P, I64, I64, I64, P]
+        lib.oracle_gemm_i32.restype = I64
+        lib.oracle_dequant_bf16.argtypes = [P, P, P, I64, I64, P]
+        lib.oracle_dequant_bf16.restype = None
+        lib.oracle_rotate_quantize.argtypes = [P, I64, I64, ctypes.c_int, P, P]
+        lib.oracle_rotate_quantize.restype = I64
+        lib.oracle_linear_int8.argtypes = [P, I64, I64, ctypes.c_int, P, P, I64,
+                                           P, P, P, P]
+        lib.oracle_linear_int8.restype = ctypes.c_int
+        lib.oracle_matmul_nt_f64.argtypes = [P, P, I64, I64, I64, P]
+        lib.oracle_matmul_nt_f64.restype = None
+        lib.oracle_float_to_bf16.argtypes = [ctypes.c_float]
+        lib.oracle_float_to_bf16.restype = ctypes.c_uint16
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bf16_bits(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("BF16 inputs are passed as their uint16 bit patterns")
+    return a
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def sylvester_hadamard(n: int) -> np.ndarray:
+    """H_n by Sylvester's recursion, int32 [n, n]."""
+    H = np.empty((n, n), dtype=np.int32)
+    if _load().oracle_sylvester_hadamard(n, _ptr(H)) != 0:
+        raise OracleError("n must be a power of two")
+    return H
+
+
+def rotate_rows(a_bf16: np.ndarray, group: int = 256):
+    """Grouped Hadamard rotation of BF16 rows, exact then rounded to FP32.
+
+    Returns ``(y_fp32, inexact_groups)``.
+    """
+    a = _bf16_bits(a_bf16)
+    rows, k = a.shape
+    y = np.empty((rows, k), dtype=np.float32)
+    bad = ctypes.c_int64(0)
+    if _load().oracle_rotate_rows(_ptr(a), rows, k, group, _ptr(y),
+                                  ctypes.byref(bad)) != 0:
+        raise OracleError("group must be a power of four dividing k")
+    return y, int(bad.value)
+
+
+def rotate_rows_f64(a: np.ndarray, group: int = 256) -> np.ndarray:
+    """The same rotation on FP64 rows, kept in FP64."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    rows, k = a.shape
+    y = np.empty((rows, k), dtype=np.float64)
+    if _load().oracle_rotate_rows_f64(_ptr(a), rows, k, group, _ptr(y)) != 0:
+        raise OracleError("group must be a power of four dividing k")
+    return y
+
+
+def quantize_rows(y: np.ndarray):
+    """Row-wise absmax INT8 RTN of FP32 rows.  Returns ``(q, s, ties)``."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    rows, k = y.shape
+    q = np.empty((rows, k), dtype=np.int8)
+    s = np.empty((rows,), dtype=np.float32)
+    ties = _load().oracle_quantize_rows(_ptr(y), rows, k, _ptr(q), _ptr(s))
+    return q, s, int(ties)
+
+
+def rotate_quantize(a_bf16: np.ndarray, group: int = 256):
+    """Rotate then quantise BF16 rows (weights offline, activations online).
+
+    Returns ``(q int8 [rows,k], s fp32 [rows])``; raises if a group's
+    rotation could not be evaluated exactly.
+    """
+    a = _bf16_bits(a_bf16)
+    rows, k = a.shape
+    q = np.empty((rows, k), dtype=np.int8)
+    s = np.empty((rows,), dtype=np.float32)
+    bad = _load().oracle_rotate_quantize(_ptr(a), rows, k, group, _ptr(q), _ptr(s))
+    if bad < 0:
+        raise OracleError("group must be a power of four dividing k")
+    if bad > 0:
+        raise OracleError("%d rotation groups span more than 37 binades" % bad)
+    return q, s
+
+
+def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:
+    """acc = xq @ wq.T, exact, int32 (raises on overflow)."""
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    wq = np.ascontiguousarray(wq, dtype=np.int8)
+    m, k = xq.shape
+    n, k2 = wq.shape
+    assert k == k2
+    acc = np.empty((m, n), dtype=np.int32)
+    if _load().oracle_gemm_i32(_ptr(xq), _ptr(wq), m, n, k, _ptr(acc)) != 0:
+        raise OracleError("INT32 overflow in the INT8 GEMM")
+    return acc
+
+
+def dequant_bf16(acc: np.ndarray, sx: np.ndarray, sw: np.ndarray) -> np.ndarray:
+    """Y = bf16(((float)acc * sx[m]) * sw[n]) as uint16 bit patterns."""
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    m, n = acc.shape
+    y = np.empty((m, n), dtype=np.uint16)
+    _load().oracle_dequant_bf16(_ptr(acc), _ptr(sx), _ptr(sw), m, n, _ptr(y))
+    return y
+
+
+def linear_int8(x_bf16: np.ndarray, wq: np.ndarray, sw: np.ndarray,
+                group: int = 256):
+    """Forward of the layer on pre-quantised weights.
+
+    Returns a dict with ``y`` (BF16 bits [m,n]), ``xq``, ``sx`` and ``acc``.
+    """
+    x = _bf16_bits(x_bf16)
+    wq = np.ascontiguousarray(wq, dtype=np.int8)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    m, k = x.shape
+    n = wq.shape[0]
+    y = np.empty((m, n), dtype=np.uint16)
+    xq = np.empty((m, k), dtype=np.int8)
+    sx = np.empty((m,), dtype=np.float32)
+    acc = np.empty((m, n), dtype=np.int32)
+    rc = _load().oracle_linear_int8(_ptr(x), m, k, group, _ptr(wq), _ptr(sw), n,
+                                    _ptr(y), _ptr(xq), _ptr(sx), _ptr(acc))
+    if rc != 0:
+        raise OracleError({-1: "bad arguments", -2: "inexact rotation group",
+                           -3: "INT32 overflow"}[rc])
+    return {"y": y, "xq": xq, "sx": sx, "acc": acc}
+
+
+def matmul_nt_f64(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """c = a @ b.T in FP64, plain triple loop."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    b = np.ascontiguousarray(b, dtype=np.float64)
+    m, k = a.shape
+    n, _ = b.shape
+    c = np.empty((m, n), dtype=np.float64)
+    _load().oracle_matmul_nt_f64(_ptr(a), _ptr(b), m, n, k, _ptr(c))
+    return c
+
+
+def float_to_bf16(f: float) -> int:
+    """Nearest-even BF16 bit pattern of one binary32 value."""
+    return int(_load().oracle_float_to_bf16(ctypes.c_float(f)))
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Widen BF16 bit patterns to FP64 (exact)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

@@ -1,0 +1,374 @@
+/*
+ * convrot_oracle.c -- CPU oracle for the INT8 ConvRot linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the package's smoke check and the CPU
+ * baseline leg of the benchmark do.  It shares no code, header, table or
+ * helper with the CUDA library.
+ *
+ * What it computes, written out plainly and slowly (no blocking, no fusion):
+ *
+ *   Grouped Hadamard pre-rotation ("ConvRot"):  the input dimension K is cut
+ *   into groups of G = 256 consecutive channels and every group of every row
+ *   is multiplied by the Sylvester Hadamard matrix H_G, normalised by
+ *   1/sqrt(G) so that the rotation is orthogonal.
+ *     [0539edu.com "minimax-h3-nvfp4-convrot", section 4 "INT8 ConvRot":
+ *      Hadamard pre-rotation in fixed groups before quantisation, group 256;
+ *      zskr.cn "Qwen3-VL-32B ... INT8-ConvRot", "INT8 ConvRot quantisation
+ *      details": row-wise, group size 256; section 5 "INT4 W4A4 ConvRot":
+ *      activations and weights are both rotated per group]
+ *   Row-wise symmetric INT8 quantisation by round-to-nearest ("--simple"):
+ *      s = max|y| / 127,  q = clamp(rne(y / s), -127, 127)
+ *     [zskr.cn, conversion command: --int8 --scaling_mode row;
+ *      0539edu.com section 4: "INT8 row-scale"; section 5: --simple = RTN]
+ *   INT8 x INT8 -> INT32 GEMM and FP32 dequantisation to BF16:
+ *      acc[m,n] = sum_k Xq[m,k] Wq[n,k];  Y[m,n] = bf16(acc * sx[m] * sw[n])
+ *     [0539edu.com section 4: INT8 tensor-core throughput; summary item 3]
+ *
+ * Readings taken where the pages are silent (each one is listed in the
+ * design notes):
+ *   - H is the natural-order Sylvester matrix, H[i][j] = (-1)^popcount(i&j),
+ *     built here by the recursion H_1 = [1], H_2n = [[H, H], [H, -H]].
+ *   - The rotated value is the exact sum of products, evaluated in FP64
+ *     (exact as long as the exponents in a group span at most 37 binades;
+ *     the routine counts the groups that break this), divided by sqrt(G)
+ *     (16 for G = 256, exact), then rounded once to FP32 (nearest-even).
+ *   - The scale is one FP32 per row; s = a / 127 in FP32; q uses an FP32
+ *     division y / s and round-half-to-even; an all-zero row has s = 0, q = 0.
+ *   - INT8 range is symmetric [-127, 127].
+ *   - Dequantisation is ((float)acc * sx[m]) * sw[n] in FP32, then rounded
+ *     to BF16 nearest-even.  No bias.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC -lm
+ * (IEEE single and double arithmetic with round-to-nearest-even, no
+ * contraction into fused multiply-adds).
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+
+/* ------------------------------------------------------------------ */
+/* BF16 and FP32 helpers                                               */
+/* ------------------------------------------------------------------ */
+
+/* A BF16 value is the upper 16 bits of an IEEE binary32; widening is exact. */
+static float bf16_bits_to_float(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static uint32_t float_bits(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return u;
+}
+
+static float float_from_bits(uint32_t u)
+{
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/*
+ * Round a finite binary32 to the nearest BF16, ties to even, by comparing
+ * the two neighbouring BF16 values: the one obtained by dropping the low 16
+ * bits (toward zero) and the next one away from zero.  Distances are exact
+ * in double.  Overflow past the largest BF16 gives infinity.
+ */
+uint16_t oracle_float_to_bf16(float f)
+{
+    uint32_t u = float_bits(f);
+    uint32_t toward_zero = u & 0xFFFF0000u;
+    float lo = float_from_bits(toward_zero);
+    if ((u & 0xFFFFu) == 0)
+        return (uint16_t)(toward_zero >> 16);
+    /* next BF16 away from zero: add one unit in the last BF16 place */
+    uint32_t away = toward_zero + 0x00010000u;
+    float hi = float_from_bits(away);
+    double d_lo = fabs((double)f - (double)lo);
+    double d_hi = fabs((double)hi - (double)f);
+    if ((away & 0x7F800000u) == 0x7F800000u) {
+        /* the candidate away from zero is infinity: compare with the
+           midpoint between the largest finite BF16 and 2^128 */
+        double big = ldexp(1.0, 128);
+        d_hi = big - fabs((double)f);
+    }
+    if (d_lo < d_hi) return (uint16_t)(toward_zero >> 16);
+    if (d_hi < d_lo) return (uint16_t)(away >> 16);
+    /* exact tie: keep the candidate whose last BF16 bit is zero */
+    return (uint16_t)(((toward_zero >> 16) & 1u) ? (away >> 16) : (toward_zero >> 16));
+}
+
+/* Round a binary32 to the nearest integer, ties to even.  Work in FP64,
+   where t - floor(t) is exact for every binary32 t. */
+static float round_half_even(float t)
+{
+    double td = (double)t;
+    double f = floor(td);
+    double d = td - f;
+    if (d > 0.5) return (float)(f + 1.0);
+    if (d < 0.5) return (float)f;
+    return (fmod(f, 2.0) == 0.0) ? (float)f : (float)(f + 1.0);
+}
+
+static int is_exact_half(float t)
+{
+    double td = (double)t;
+    return td - floor(td) == 0.5;
+}
+
+/* ------------------------------------------------------------------ */
+/* Hadamard matrix                                                     */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Sylvester's construction: H_1 = [1]; H_2n = [[H_n, H_n], [H_n, -H_n]].
+ * n must be a power of two; H is n*n, row-major.  Returns 0 on success.
+ */
+int oracle_sylvester_hadamard(int n, int32_t *H)
+{
+    if (n < 1 || (n & (n - 1)) != 0) return -1;
+    H[0] = 1;
+    for (int size = 1; size < n; size *= 2) {
+        for (int i = 0; i < size; ++i) {
+            for (int j = 0; j < size; ++j) {
+                int32_t h = H[i * n + j];
+                H[i * n + (j + size)] = h;
+                H[(i + size) * n + j] = h;
+                H[(i + size) * n + (j + size)] = -h;
+            }
+        }
+    }
+    return 0;
+}
+
+static int is_power_of_four(int g)
+{
+    if (g < 1 || (g & (g - 1)) != 0) return 0;
+    int lg = 0;
+    while ((1 << lg) < g) ++lg;
+    return (lg % 2) == 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Grouped Hadamard rotation                                           */
+/* ------------------------------------------------------------------ */
+
+/*
+ * y[r, g*G + j] = fp32( ( sum_i a[r, g*G + i] * H[i][j] ) / sqrt(G) )
+ *
+ * a is BF16 bits [rows, k], row-major; y is FP32 [rows, k].  G must be a
+ * power of four (so 1/sqrt(G) is a power of two and the division is exact)
+ * and divide k.  The sum is accumulated in FP64.  *inexact counts the groups
+ * whose nonzero magnitudes span more than 37 binades, where an FP64 sum of
+ * 256 BF16 terms might not be exact.  Returns 0, or -1 on bad arguments.
+ */
+int oracle_rotate_rows(const uint16_t *a, int64_t rows, int64_t k, int group,
+                       float *y, int64_t *inexact)
+{
+    if (!is_power_of_four(group) || k % group != 0) return -1;
+    int32_t *H = (int32_t *)malloc(sizeof(int32_t) * group * group);
+    double *x = (double *)malloc(sizeof(double) * group);
+    if (!H || !x) { free(H); free(x); return -1; }
+    oracle_sylvester_hadamard(group, H);
+    double root = sqrt((double)group);
+    int64_t bad = 0;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g0 = 0; g0 < k; g0 += group) {
+            int emin = 1000, emax = -1000;
+            for (int i = 0; i < group; ++i) {
+                x[i] = (double)bf16_bits_to_float(a[r * k + g0 + i]);
+                if (x[i] != 0.0) {
+                    int e;
+                    frexp(x[i], &e);
+                    if (e < emin) emin = e;
+                    if (e > emax) emax = e;
+                }
+            }
+            if (emax >= emin && emax - emin > 37) ++bad;
+            for (int j = 0; j < group; ++j) {
+                double s = 0.0;
+                for (int i = 0; i < group; ++i)
+                    s += x[i] * (double)H[i * group + j];
+                y[r * k + g0 + j] = (float)(s / root);
+            }
+        }
+    }
+    if (inexact) *inexact = bad;
+    free(H);
+    free(x);
+    return 0;
+}
+
+/*
+ * The same rotation kept in FP64 (no rounding to FP32), for checking the
+ * orthogonality identities of the rotation itself.  a is FP64 [rows, k].
+ */
+int oracle_rotate_rows_f64(const double *a, int64_t rows, int64_t k, int group,
+                           double *y)
+{
+    if (!is_power_of_four(group) || k % group != 0) return -1;
+    int32_t *H = (int32_t *)malloc(sizeof(int32_t) * group * group);
+    if (!H) return -1;
+    oracle_sylvester_hadamard(group, H);
+    double root = sqrt((double)group);
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g0 = 0; g0 < k; g0 += group)
+            for (int j = 0; j < group; ++j) {
+                double s = 0.0;
+                for (int i = 0; i < group; ++i)
+                    s += a[r * k + g0 + i] * (double)H[i * group + j];
+                y[r * k + g0 + j] = s / root;
+            }
+    free(H);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Row-wise symmetric INT8 quantisation (round to nearest, ties even)  */
+/* ------------------------------------------------------------------ */
+
+/*
+ * For every row r of y [rows, k] (FP32):
+ *   a = max_k |y[r,k]|            (exact in FP32)
+ *   s[r] = a / 127                (FP32 division, nearest-even)
+ *   q[r,k] = 0 if a == 0, else clamp(rne(y[r,k] / s[r]), -127, 127)
+ * Returns the number of exact .5 ties met (an FP64 check on y/s).
+ */
+int64_t oracle_quantize_rows(const float *y, int64_t rows, int64_t k,
+                             int8_t *q, float *s)
+{
+    int64_t ties = 0;
+    for (int64_t r = 0; r < rows; ++r) {
+        float a = 0.0f;
+        for (int64_t c = 0; c < k; ++c) {
+            float v = fabsf(y[r * k + c]);
+            if (v > a) a = v;
+        }
+        float scale = a / 127.0f;
+        s[r] = scale;
+        for (int64_t c = 0; c < k; ++c) {
+            if (a == 0.0f) { q[r * k + c] = 0; continue; }
+            float t = y[r * k + c] / scale;
+            if (is_exact_half(t)) ++ties;
+            float v = round_half_even(t);
+            if (v > 127.0f) v = 127.0f;
+            if (v < -127.0f) v = -127.0f;
+            q[r * k + c] = (int8_t)v;
+        }
+    }
+    return ties;
+}
+
+/* ------------------------------------------------------------------ */
+/* INT8 GEMM with INT32 result                                         */
+/* ------------------------------------------------------------------ */
+
+/*
+ * acc[m,n] = sum_k xq[m,k] * wq[n,k], summed exactly in int64.
+ * xq [m,k] and wq [n,k] are row-major; acc [m,n] row-major.
+ * Returns the number of sums that do not fit in int32 (those are stored
+ * wrapped; the caller treats a nonzero return as an error).
+ */
+int64_t oracle_gemm_i32(const int8_t *xq, const int8_t *wq, int64_t m,
+                        int64_t n, int64_t k, int32_t *acc)
+{
+    int64_t overflow = 0;
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t j = 0; j < n; ++j) {
+            int64_t sum = 0;
+            for (int64_t c = 0; c < k; ++c)
+                sum += (int64_t)xq[i * k + c] * (int64_t)wq[j * k + c];
+            if (sum > INT32_MAX || sum < INT32_MIN) ++overflow;
+            acc[i * n + j] = (int32_t)sum;
+        }
+    return overflow;
+}
+
+/* ------------------------------------------------------------------ */
+/* Dequantisation to BF16                                              */
+/* ------------------------------------------------------------------ */
+
+/* y[m,n] = bf16_rne( ((float)acc[m,n] * sx[m]) * sw[n] ), FP32 products. */
+void oracle_dequant_bf16(const int32_t *acc, const float *sx, const float *sw,
+                         int64_t m, int64_t n, uint16_t *y)
+{
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t j = 0; j < n; ++j) {
+            float v = (float)acc[i * n + j];
+            v = v * sx[i];
+            v = v * sw[j];
+            y[i * n + j] = oracle_float_to_bf16(v);
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Composites                                                          */
+/* ------------------------------------------------------------------ */
+
+/* Rotate and quantise the rows of a BF16 matrix (weights offline, or
+   activations at call time).  Returns the count of inexact groups, or -1. */
+int64_t oracle_rotate_quantize(const uint16_t *a, int64_t rows, int64_t k,
+                               int group, int8_t *q, float *s)
+{
+    float *y = (float *)malloc(sizeof(float) * (size_t)(rows * k > 0 ? rows * k : 1));
+    if (!y) return -1;
+    int64_t bad = 0;
+    if (oracle_rotate_rows(a, rows, k, group, y, &bad) != 0) { free(y); return -1; }
+    oracle_quantize_rows(y, rows, k, q, s);
+    free(y);
+    return bad;
+}
+
+/*
+ * Full forward of the layer on pre-quantised weights:
+ *   x (BF16 [m,k]) -> rotate -> quantise (xq, sx) -> GEMM with wq -> dequant.
+ * Intermediate outputs are written when their pointers are non-NULL.
+ * Returns 0 on success, -1 on bad arguments, -2 on an inexact rotation group,
+ * -3 on an INT32 overflow.
+ */
+int oracle_linear_int8(const uint16_t *x, int64_t m, int64_t k, int group,
+                       const int8_t *wq, const float *sw, int64_t n,
+                       uint16_t *y, int8_t *xq_out, float *sx_out,
+                       int32_t *acc_out)
+{
+    int8_t *xq = xq_out ? xq_out : (int8_t *)malloc((size_t)(m * k > 0 ? m * k : 1));
+    float *sx = sx_out ? sx_out : (float *)malloc(sizeof(float) * (size_t)(m > 0 ? m : 1));
+    int32_t *acc = acc_out ? acc_out
+                           : (int32_t *)malloc(sizeof(int32_t) * (size_t)(m * n > 0 ? m * n : 1));
+    int rc = 0;
+    if (!xq || !sx || !acc) { rc = -1; goto done; }
+    int64_t bad = oracle_rotate_quantize(x, m, k, group, xq, sx);
+    if (bad < 0) { rc = -1; goto done; }
+    if (bad > 0) { rc = -2; goto done; }
+    if (oracle_gemm_i32(xq, wq, m, n, k, acc) != 0) { rc = -3; goto done; }
+    oracle_dequant_bf16(acc, sx, sw, m, n, y);
+done:
+    if (!xq_out) free(xq);
+    if (!sx_out) free(sx);
+    if (!acc_out) free(acc);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* FP64 references for error reporting                                 */
+/* ------------------------------------------------------------------ */
+
+/* c[m,n] = sum_k a[m,k] * b[n,k] in FP64 (both operands row-major). */
+void oracle_matmul_nt_f64(const double *a, const double *b, int64_t m,
+                          int64_t n, int64_t k, double *c)
+{
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (int64_t t = 0; t < k; ++t)
+                s += a[i * k + t] * b[j * k + t];
+            c[i * n + j] = s;
+        }
+}

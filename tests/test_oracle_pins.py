@@ -1,0 +1,329 @@
+"""Pins for the CPU oracle, each against something other than the oracle.
+
+The oracle (``oracle/``) is the parity reference for the CUDA path, so every
+function in it is checked here against a library routine, a closed form,
+hand-worked values under ``tests/golden/``, an invariant of the mathematics,
+or brute force on tiny inputs.  These run without a GPU.
+"""
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            rows.append(line)
+    return rows
+
+
+def _f32_to_bf16_torch(f):
+    """Nearest-even BF16 via torch's own conversion (a library routine)."""
+    t = torch.from_numpy(np.ascontiguousarray(f, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_from_f32_exact(v):
+    """BF16 bits of values that are exactly representable in BF16."""
+    b = _f32_to_bf16_torch(np.asarray(v, dtype=np.float32))
+    assert np.array_equal(synth.bf16_bits_to_f32(b), np.asarray(v, dtype=np.float32))
+    return b
+
+
+# ---------------------------------------------------------------------------
+# Hadamard matrix
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 32, 64, 128, 256])
+def test_hadamard_matches_scipy(n):
+    assert np.array_equal(oracle.sylvester_hadamard(n), scipy.linalg.hadamard(n))
+
+
+def test_hadamard_8_golden():
+    H8 = np.array([[int(v) for v in r.split()] for r in _golden_rows("hadamard_8.txt")])
+    assert np.array_equal(oracle.sylvester_hadamard(8), H8)
+
+
+def test_hadamard_256_orthogonal_and_closed_form():
+    H = oracle.sylvester_hadamard(256).astype(np.int64)
+    assert np.array_equal(H @ H.T, 256 * np.eye(256, dtype=np.int64))
+    assert np.array_equal(H, H.T)
+    i = np.arange(256)
+    pc = np.vectorize(lambda v: bin(v).count("1"))(i[:, None] & i[None, :])
+    assert np.array_equal(H, np.where(pc % 2 == 0, 1, -1))
+
+
+def test_hadamard_rejects_non_power_of_two():
+    with pytest.raises(oracle.OracleError):
+        oracle.sylvester_hadamard(12)
+
+
+# ---------------------------------------------------------------------------
+# rotation
+# ---------------------------------------------------------------------------
+def _block_rotation_np(x64, group):
+    """Block-diagonal H/sqrt(G) applied with numpy's matmul and scipy's H."""
+    H = scipy.linalg.hadamard(group).astype(np.float64) / np.sqrt(group)
+    rows, k = x64.shape
+    return (x64.reshape(rows, k // group, group) @ H).reshape(rows, k)
+
+
+def test_rotation_matches_library_matmul_exactly():
+    # products with +-1 are exact and the group sums are exact (within 37
+    # binades), so numpy's FP64 matmul gives the exact value whatever its
+    # summation order; rounding it once to FP32 must equal the oracle.
+    lin = synth.tiny()[0]
+    x = lin.x_np()
+    y, bad = oracle.rotate_rows(x)
+    assert bad == 0
+    ref = _block_rotation_np(oracle.bf16_bits_to_f64(x), 256).astype(np.float32)
+    assert np.array_equal(y, ref)
+    w = lin.w_np()
+    yw, bad = oracle.rotate_rows(w)
+    assert bad == 0
+    assert np.array_equal(yw, _block_rotation_np(oracle.bf16_bits_to_f64(w), 256).astype(np.float32))
+
+
+def test_rotation_one_hot_golden():
+    for line in _golden_rows("one_hot_rotation.txt"):
+        i, c, ys, qs = [p.strip() for p in line.split("|")]
+        i, c = int(i), float(c)
+        yv = [float(v) for v in ys.split()]
+        qv = [int(v) for v in qs.split()]
+        row = np.zeros((1, 256), dtype=np.float32)
+        row[0, i] = c
+        y, bad = oracle.rotate_rows(_bf16_from_f32_exact(row))
+        assert bad == 0
+        assert list(y[0, :4]) == yv
+        q, s = oracle.rotate_quantize(_bf16_from_f32_exact(row))
+        assert list(q[0, :4]) == qv
+        assert s[0] == np.float32(np.float32(abs(c) / 16.0) / np.float32(127.0))
+
+
+def test_rotation_closed_forms_in_second_group():
+    rng = np.random.default_rng(5)
+    H = scipy.linalg.hadamard(256)
+    for _ in range(20):
+        i = int(rng.integers(256))
+        c = np.float32(rng.choice([1.0, -2.0, 0.375, 96.0]))
+        row = np.zeros((1, 512), dtype=np.float32)
+        row[0, 256 + i] = c
+        y, _ = oracle.rotate_rows(_bf16_from_f32_exact(row))
+        assert np.all(y[0, :256] == 0)
+        assert np.array_equal(y[0, 256:], (c * H[i] / 16.0).astype(np.float32))
+    # constant group -> (16c, 0, ..., 0)
+    row = np.full((1, 256), 0.75, dtype=np.float32)
+    y, _ = oracle.rotate_rows(_bf16_from_f32_exact(row))
+    assert y[0, 0] == np.float32(12.0) and np.all(y[0, 1:] == 0)
+
+
+def test_rotation_involution_and_parseval():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((3, 768))
+    y = oracle.rotate_rows_f64(x)
+    assert np.allclose(oracle.rotate_rows_f64(y), x, rtol=0, atol=1e-12)
+    for g in range(3):
+        sl = slice(256 * g, 256 * (g + 1))
+        assert np.allclose(np.linalg.norm(y[:, sl], axis=1),
+                           np.linalg.norm(x[:, sl], axis=1), rtol=1e-13)
+
+
+def test_rotation_preserves_the_layer():
+    # (X R)(W R)^T = X W^T, FP64, to 1e-5 relative
+    lin = synth.tiny()[0]
+    x = oracle.bf16_bits_to_f64(lin.x_np())
+    w = oracle.bf16_bits_to_f64(lin.w_np())
+    lhs = oracle.rotate_rows_f64(x) @ oracle.rotate_rows_f64(w).T
+    rhs = x @ w.T
+    assert np.max(np.abs(lhs - rhs)) <= 1e-5 * np.max(np.abs(rhs))
+
+
+def test_rotation_counts_inexact_groups():
+    row = np.zeros((1, 512), dtype=np.float32)
+    row[0, 0] = 2.0 ** 10
+    row[0, 1] = 2.0 ** -30      # 41 binades apart inside group 0
+    row[0, 256] = 1.0
+    row[0, 257] = 2.0 ** -20    # 21 binades apart inside group 1: fine
+    _, bad = oracle.rotate_rows(_bf16_from_f32_exact(row))
+    assert bad == 1
+    with pytest.raises(oracle.OracleError):
+        oracle.rotate_quantize(_bf16_from_f32_exact(row))
+
+
+def test_rotation_rejects_bad_group():
+    x = np.zeros((1, 384), dtype=np.uint16)
+    with pytest.raises(oracle.OracleError):
+        oracle.rotate_rows(x, 256)       # 384 is not a multiple of 256
+    with pytest.raises(oracle.OracleError):
+        oracle.rotate_rows(np.zeros((1, 256), np.uint16), 128)   # not a power of 4
+
+
+# ---------------------------------------------------------------------------
+# quantisation
+# ---------------------------------------------------------------------------
+def test_quantize_golden_ties():
+    for line in _golden_rows("quant_ties.txt"):
+        p, ys, qs, away = [v.strip() for v in line.split("|")]
+        p = int(p)
+        y = (np.array([float(v) for v in ys.split()]) * 2.0 ** p).astype(np.float32)[None, :]
+        q, s, ties = oracle.quantize_rows(y)
+        assert s[0] == np.float32(2.0 ** p)
+        assert list(q[0]) == [int(v) for v in qs.split()]
+        assert list(q[0]) != [int(v) for v in away.split()]
+        assert ties == sum(1 for v in ys.split() if float(v) % 1 == 0.5)
+
+
+def test_quantize_matches_numpy_definition():
+    rng = np.random.default_rng(2)
+    y = (rng.standard_normal((16, 1024)) * rng.uniform(0.01, 100, (16, 1))).astype(np.float32)
+    y[3] *= 0  # an all-zero row
+    q, s, _ = oracle.quantize_rows(y)
+    a = np.max(np.abs(y), axis=1)
+    s_ref = (a / np.float32(127.0)).astype(np.float32)
+    assert np.array_equal(s, s_ref)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (y / s_ref[:, None]).astype(np.float32)
+    q_ref = np.where(a[:, None] == 0, 0, np.clip(np.rint(t), -127, 127)).astype(np.int8)
+    assert np.array_equal(q, q_ref)
+    assert np.all(q[3] == 0) and s[3] == 0
+    # error bound |y - s q| <= s / 2 (plus the rounding of y / s)
+    err = np.abs(y.astype(np.float64) - s[:, None].astype(np.float64) * q)
+    assert np.all(err <= s[:, None] * (0.5 + 1e-6))
+    # the row maximum maps to +-127
+    amax = np.argmax(np.abs(y), axis=1)
+    for r in range(16):
+        if r != 3:
+            assert abs(int(q[r, amax[r]])) == 127
+
+
+def test_exhaustive_bf16_one_hot():
+    # every finite BF16 c whose scale stays a normal FP32, one-hot at a
+    # position that cycles over the group: q = 127 sign(c) H[i, :]
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = synth.bf16_bits_to_f32(bits)
+    keep = np.isfinite(vals) & (np.abs(vals) >= 2.0 ** -120)
+    bits, vals = bits[keep], vals[keep]
+    pos = np.arange(len(bits)) % 256
+    rows = np.zeros((len(bits), 256), dtype=np.uint16)
+    rows[np.arange(len(bits)), pos] = bits
+    q, s = oracle.rotate_quantize(rows)
+    H = scipy.linalg.hadamard(256)
+    expect = (127 * np.sign(vals)[:, None] * H[pos]).astype(np.int8)
+    assert np.array_equal(q, expect)
+    s_ref = ((np.abs(vals) / np.float32(16.0)).astype(np.float32) / np.float32(127.0)).astype(np.float32)
+    assert np.array_equal(s, s_ref)
+
+
+# ---------------------------------------------------------------------------
+# INT8 GEMM
+# ---------------------------------------------------------------------------
+def test_gemm_brute_force_tiny():
+    rng = np.random.default_rng(3)
+    xq = rng.integers(-127, 128, (3, 64), dtype=np.int8)
+    wq = rng.integers(-127, 128, (5, 64), dtype=np.int8)
+    acc = oracle.gemm_i32(xq, wq)
+    for i in range(3):
+        for j in range(5):
+            assert acc[i, j] == sum(int(xq[i, t]) * int(wq[j, t]) for t in range(64))
+
+
+def test_gemm_matches_numpy_int64():
+    rng = np.random.default_rng(4)
+    xq = rng.integers(-127, 128, (7, 1024), dtype=np.int8)
+    wq = rng.integers(-127, 128, (33, 1024), dtype=np.int8)
+    ref = xq.astype(np.int64) @ wq.astype(np.int64).T
+    assert np.array_equal(oracle.gemm_i32(xq, wq), ref.astype(np.int32))
+    # asymmetric operands catch a transposed index
+    assert not np.array_equal(oracle.gemm_i32(xq, wq)[:, :7], ref[:7, :7].T)
+
+
+def test_gemm_extremes_and_overflow():
+    k = 25600
+    ones = np.full((1, k), 127, dtype=np.int8)
+    assert oracle.gemm_i32(ones, -ones)[0, 0] == -k * 127 * 127
+    k_over = 140000   # 140000 * 127^2 > 2^31 - 1
+    with pytest.raises(oracle.OracleError):
+        oracle.gemm_i32(np.full((1, k_over), 127, np.int8), np.full((1, k_over), 127, np.int8))
+
+
+# ---------------------------------------------------------------------------
+# dequantisation
+# ---------------------------------------------------------------------------
+def test_float_to_bf16_matches_torch():
+    rng = np.random.default_rng(6)
+    u = rng.integers(0, 2 ** 32, 200000, dtype=np.uint64).astype(np.uint32)
+    f = u.view(np.float32)
+    f = f[np.isfinite(f) & (np.abs(f) < 3.0e38)]
+    # add exact ties and values right next to them
+    base = synth.bf16_bits_to_f32(rng.integers(0, 0x7F00, 2000).astype(np.uint16))
+    ties = (base.view(np.uint32) + np.uint32(0x8000)).view(np.float32)
+    f = np.concatenate([f, ties, -ties, np.nextafter(ties, np.float32(np.inf))])
+    mine = np.array([oracle.float_to_bf16(float(v)) for v in f[:40000]], dtype=np.uint16)
+    assert np.array_equal(mine, _f32_to_bf16_torch(f[:40000]))
+    mine_t = np.array([oracle.float_to_bf16(float(v)) for v in f[-6000:]], dtype=np.uint16)
+    assert np.array_equal(mine_t, _f32_to_bf16_torch(f[-6000:]))
+
+
+def test_dequant_matches_definition():
+    rng = np.random.default_rng(7)
+    acc = rng.integers(-400_000_000, 400_000_000, (6, 50)).astype(np.int32)
+    sx = rng.uniform(1e-3, 1, 6).astype(np.float32)
+    sw = rng.uniform(1e-5, 1e-3, 50).astype(np.float32)
+    y = oracle.dequant_bf16(acc, sx, sw)
+    v = (acc.astype(np.float32) * sx[:, None]).astype(np.float32) * sw[None, :]
+    assert np.array_equal(y, _f32_to_bf16_torch(v.astype(np.float32)))
+    # a scale applied along the wrong axis is caught
+    y_bad = oracle.dequant_bf16(acc[:, :6].copy(), sw[:6].copy(), sx)
+    assert not np.array_equal(y[:, :6], y_bad)
+
+
+# ---------------------------------------------------------------------------
+# whole layer
+# ---------------------------------------------------------------------------
+def test_linear_composes_steps_and_approximates_fp64():
+    lin = synth.tiny()[0]
+    x, w = lin.x_np(), lin.w_np()
+    wq, sw = oracle.rotate_quantize(w)
+    out = oracle.linear_int8(x, wq, sw)
+    xq, sx = oracle.rotate_quantize(x)
+    assert np.array_equal(out["xq"], xq) and np.array_equal(out["sx"], sx)
+    acc = xq.astype(np.int64) @ wq.astype(np.int64).T
+    assert np.array_equal(out["acc"], acc)
+    assert np.array_equal(out["y"], oracle.dequant_bf16(acc.astype(np.int32), sx, sw))
+    # the quantised layer approximates the FP64 layer X W^T
+    ref = oracle.bf16_bits_to_f64(x) @ oracle.bf16_bits_to_f64(w).T
+    y = oracle.bf16_bits_to_f64(out["y"])
+    assert np.max(np.abs(y - ref)) / np.max(np.abs(ref)) < 0.05
+
+
+def test_rotation_spreads_outliers():
+    # the method's purpose: with outlier channels, rotating before row INT8
+    # quantisation lowers the quantisation error of the activations
+    lin = synth.tiny()[0]
+    x = lin.x_np()
+    x64 = oracle.bf16_bits_to_f64(x)
+    q_rot, s_rot = oracle.rotate_quantize(x)
+    deq_rot = oracle.rotate_rows_f64(q_rot.astype(np.float64) * s_rot[:, None].astype(np.float64))
+    q_plain, s_plain, _ = oracle.quantize_rows(x64.astype(np.float32))
+    deq_plain = q_plain.astype(np.float64) * s_plain[:, None]
+    err_rot = np.linalg.norm(deq_rot - x64)
+    err_plain = np.linalg.norm(deq_plain - x64)
+    assert err_rot < 0.5 * err_plain
+
+
+def test_matmul_f64_matches_numpy():
+    rng = np.random.default_rng(8)
+    a = rng.standard_normal((4, 37))
+    b = rng.standard_normal((6, 37))
+    assert np.allclose(oracle.matmul_nt_f64(a, b), a @ b.T, rtol=1e-13, atol=1e-13)
