@@ -1,0 +1,171 @@
+/*
+ * convrot.h -- C ABI of libconvrot, the INT8 ConvRot linear layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (from the source pages):
+ *   - "ConvRot" is a grouped Hadamard pre-rotation: the input dimension K is
+ *     cut into fixed groups of 256 and each group is Hadamard-rotated before
+ *     quantisation, which spreads outlier energy so INT8 can hold it
+ *     [0539edu.com "minimax-h3-nvfp4-convrot", section 4 "INT8 ConvRot";
+ *      zskr.cn "Qwen3-VL-32B ... INT8-ConvRot", "INT8 ConvRot quantisation
+ *      details": row-wise, group size 256].
+ *   - Weights are rotated offline and quantised to INT8 with one FP32 scale
+ *     per output row, by round-to-nearest [zskr.cn conversion command:
+ *     "--int8 --scaling_mode row --convrot --convrot-group-size 256";
+ *     0539edu.com section 4 "INT8 row-scale", section 5 "--simple" = RTN].
+ *   - Activations are rotated the same way and quantised per token row at
+ *     call time, so the product runs on INT8 tensor cores [0539edu.com
+ *     section 4 (INT8 tensor-core throughput), section 5 (activations and
+ *     weights both rotated), section 7 (INT8 activation path on Blackwell)].
+ *
+ * Arithmetic contract (identical to the CPU oracle bit for bit):
+ *   y_j  = fp32( (sum_i a_i * H[i][j]) / 16 )   per 256-group, H Sylvester,
+ *          the sum exact (FP64; exact while the nonzero magnitudes inside a
+ *          group span at most 37 binades -- finite BF16 inputs outside that
+ *          range give unspecified low bits)
+ *   s    = fp32(max_k |y_k| / 127);  q = clamp(rne(y / s), -127, 127), q = 0
+ *          and s = 0 for an all-zero row
+ *   acc  = sum_k xq[m,k] * wq[n,k]   (INT32, exact for K <= 133144)
+ *   Y    = bf16_rne( ((float)acc * sx[m]) * sw[n] )
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, row-major,
+ *     16-byte aligned.  BF16 tensors are passed as `const void *`/`void *`
+ *     (IEEE bfloat16 bit patterns, 2 bytes each).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously; the call returns once it is launched.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and returned as a status; nothing is written then.  A launch failure
+ *     returns CONVROT_ERR_CUDA.
+ *   - Kernels never trap.  Every wait inside a kernel is bounded; a wait that
+ *     runs out records CONVROT_ERR_DEVICE_TIMEOUT in a device-side status
+ *     word that convrot_device_status() reads.
+ *   - The library allocates no device memory.  Scratch space is the
+ *     caller-provided workspace.
+ *   - Calls on different streams are independent provided they do not share
+ *     a workspace.
+ */
+#ifndef CONVROT_H
+#define CONVROT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CONVROT_OK = 0,
+    CONVROT_ERR_INVALID_ARG = 1,       /* null pointer, non-positive size */
+    CONVROT_ERR_ALIGNMENT = 2,         /* a pointer is not 16-byte aligned */
+    CONVROT_ERR_UNSUPPORTED_SHAPE = 3, /* group != 256, k % group != 0, k too large */
+    CONVROT_ERR_UNSUPPORTED_ARCH = 4,  /* current device is not compute capability 10.0 */
+    CONVROT_ERR_WORKSPACE = 5,         /* workspace missing or smaller than required */
+    CONVROT_ERR_CUDA = 6,              /* a CUDA runtime/driver call failed */
+    CONVROT_ERR_DEVICE_TIMEOUT = 7     /* a bounded in-kernel wait ran out */
+} convrot_status_t;
+
+/*
+ * Quantised-weight handle: a VIEW of caller-owned device memory.
+ *   q     : int8  [n, k] row-major -- the rotated, row-quantised weight Wq
+ *   scale : fp32  [n]              -- sw, one scale per output row
+ *   n     : out_features, k : in_features (the rotation runs along k)
+ *   group : rotation group size; must be 256
+ * The offline converter's record is an INT8 tensor, an FP32 row scale and the
+ * ConvRot group size [zskr.cn "Qwen3-VL-32B ... INT8-ConvRot": 350 INT8
+ * ConvRot matrices with FP32 scales; 0539edu.com section 4: "INT8 row-scale
+ * + ConvRot metadata"].
+ */
+typedef struct {
+    int8_t *q;
+    float *scale;
+    int64_t n;
+    int64_t k;
+    int32_t group;
+} convrot_weight_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *convrot_status_string(convrot_status_t status);
+
+/* Library version as 10000 * major + 100 * minor + patch. */
+int convrot_version(void);
+
+/*
+ * Fill a handle.  Checks: w, q, scale non-NULL; n, k >= 1; group == 256;
+ * k % 256 == 0; k <= 133120 (INT32 accumulation bound); q and scale
+ * 16-byte aligned.  Host only; touches no device.
+ */
+convrot_status_t convrot_weight_init(convrot_weight_t *w, int8_t *q, float *scale,
+                                     int64_t n, int64_t k, int32_t group);
+
+/*
+ * Offline weight conversion: rotate every row of the BF16 weight w [n, k]
+ * (PyTorch Linear layout, out x in) per 256-group and quantise it row-wise
+ * by round-to-nearest into out->q and out->scale.  The pages quantise from
+ * the BF16 source, never from an already quantised tensor [0539edu.com
+ * section 4, engineering detail 1] and use RTN in "--simple" mode
+ * [0539edu.com section 5].
+ */
+convrot_status_t convrot_quantize_weight(const void *w_bf16, const convrot_weight_t *out,
+                                         void *stream);
+
+/*
+ * Activation prologue: rotate each row of x [m, k] (BF16) per 256-group and
+ * quantise it per row into xq (int8 [m, k]) and sx (fp32 [m]).  Same
+ * arithmetic as the weight conversion.
+ */
+convrot_status_t convrot_quantize_act(const void *x_bf16, int64_t m, int64_t k, int32_t group,
+                                      int8_t *xq, float *sx, void *stream);
+
+/*
+ * Scratch bytes convrot_gemm_i8 needs for an [m x k] x [n x k]^T product on
+ * the current device (0 when no device is present is never returned: the
+ * B200's 148 SMs are assumed then).  The workspace must be zero-filled
+ * (convrot_workspace_init) before its first use; every successful call
+ * leaves it zero-filled again.
+ */
+size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/* Scratch bytes convrot_linear_int8 needs: the GEMM scratch followed by the
+   quantised activations xq [m, k] and their scales sx [m]. */
+size_t convrot_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/* Zero-fill a workspace on `stream` (an asynchronous memset). */
+convrot_status_t convrot_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * INT8 GEMM with INT32 accumulation on the tcgen05 tensor cores, with the
+ * dequantisation fused into the epilogue:
+ *   acc[m, n] = sum_k xq[m, k] * w->q[n, k]
+ *   y[m, n]   = bf16_rne(((float)acc * sx[m]) * w->scale[n])
+ * y (BF16 [m, n]) and acc (int32 [m, n]) are optional outputs; at least one
+ * must be non-NULL (acc exists for bit-exact checking).  ws/ws_bytes: see
+ * convrot_gemm_workspace_bytes.
+ */
+convrot_status_t convrot_gemm_i8(const int8_t *xq, const float *sx, int64_t m,
+                                 const convrot_weight_t *w, void *y_bf16, int32_t *acc,
+                                 void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The whole layer: y = ConvRotLinearINT8(x) for BF16 x [m, k] against the
+ * quantised weight w, BF16 y [m, n].  Runs the activation prologue into the
+ * workspace, then the GEMM; the GEMM is launched as a programmatic
+ * dependent of the prologue so its weight prefetch overlaps the prologue.
+ */
+convrot_status_t convrot_linear_int8(const void *x_bf16, int64_t m, const convrot_weight_t *w,
+                                     void *y_bf16, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device-side status word of
+ * the current device.  Returns CONVROT_OK, CONVROT_ERR_DEVICE_TIMEOUT if a
+ * bounded wait ran out in some kernel since the last call (the workspace
+ * must then be re-initialised), or CONVROT_ERR_CUDA.
+ */
+convrot_status_t convrot_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVROT_H */

@@ -1,0 +1,204 @@
+"""INT8 ConvRot linear layer on NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over ``libconvrot.so`` (C ABI in ``include/convrot.h``).
+Every function here only marshals torch tensors into device pointers and
+sizes and calls the C entry point of the same name; all arithmetic runs in
+the library's CUDA kernels.  There is no CPU fallback: if the library is
+missing or the device is not a B200, calls raise.
+
+Typical use::
+
+    w = quantize_weight(w_bf16)                 # offline, QuantizedWeight
+    ws = make_workspace(m, w)                   # zero-filled scratch
+    y = linear_int8(x_bf16, w, ws)              # BF16 [m, n]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libconvrot.so")
+GROUP = 256
+
+_STATUS = {
+    0: "CONVROT_OK", 1: "CONVROT_ERR_INVALID_ARG", 2: "CONVROT_ERR_ALIGNMENT",
+    3: "CONVROT_ERR_UNSUPPORTED_SHAPE", 4: "CONVROT_ERR_UNSUPPORTED_ARCH",
+    5: "CONVROT_ERR_WORKSPACE", 6: "CONVROT_ERR_CUDA", 7: "CONVROT_ERR_DEVICE_TIMEOUT",
+}
+
+
+class ConvrotError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed: %s" % (where, _STATUS.get(status, "status %d" % status)))
+
+
+class convrot_weight_t(ctypes.Structure):
+    """Mirror of the C struct: a view of (q int8 [n,k], scale fp32 [n])."""
+    _fields_ = [("q", ctypes.c_void_p), ("scale", ctypes.c_void_p),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("group", ctypes.c_int32)]
+
+
+# exported symbol -> (argtypes, restype); every name declared in convrot.h
+_P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+_WP = ctypes.POINTER(convrot_weight_t)
+SIGNATURES = {
+    "convrot_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "convrot_version": ([], ctypes.c_int),
+    "convrot_weight_init": ([_WP, _P, _P, _I64, _I64, _I32], ctypes.c_int),
+    "convrot_quantize_weight": ([_P, _WP, _P], ctypes.c_int),
+    "convrot_quantize_act": ([_P, _I64, _I64, _I32, _P, _P, _P], ctypes.c_int),
+    "convrot_gemm_workspace_bytes": ([_I64, _I64, _I64], _SZ),
+    "convrot_linear_workspace_bytes": ([_I64, _I64, _I64], _SZ),
+    "convrot_workspace_init": ([_P, _SZ, _P], ctypes.c_int),
+    "convrot_gemm_i8": ([_P, _P, _I64, _WP, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "convrot_linear_int8": ([_P, _I64, _WP, _P, _P, _SZ, _P], ctypes.c_int),
+    "convrot_device_status": ([_P], ctypes.c_int),
+}
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libconvrot.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError("libconvrot.so is not built (run rotated_int8_quantized_b200/build.py); "
+                              "there is no fallback path")
+        lib = ctypes.CDLL(path)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise ConvrotError(status, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+@dataclass
+class QuantizedWeight:
+    """Rotated INT8 weight q [n, k] with FP32 row scales [n] (caller-owned
+    device memory) and the C handle viewing them."""
+    q: torch.Tensor
+    scale: torch.Tensor
+    handle: convrot_weight_t
+
+    @property
+    def n(self) -> int:
+        return self.handle.n
+
+    @property
+    def k(self) -> int:
+        return self.handle.k
+
+
+def convrot_status_string(status: int) -> str:
+    return load_library().convrot_status_string(status).decode()
+
+
+def convrot_version() -> int:
+    return load_library().convrot_version()
+
+
+def convrot_weight_init(q: torch.Tensor, scale: torch.Tensor, group: int = GROUP) -> QuantizedWeight:
+    n, k = q.shape
+    h = convrot_weight_t()
+    _check(load_library().convrot_weight_init(ctypes.byref(h), _ptr(q), _ptr(scale), n, k, group),
+           "convrot_weight_init")
+    return QuantizedWeight(q, scale, h)
+
+
+def convrot_quantize_weight(w_bf16: torch.Tensor, out: QuantizedWeight, stream=None) -> QuantizedWeight:
+    assert w_bf16.dtype == torch.bfloat16 and tuple(w_bf16.shape) == (out.n, out.k)
+    _check(load_library().convrot_quantize_weight(_ptr(w_bf16), ctypes.byref(out.handle), _stream(stream)),
+           "convrot_quantize_weight")
+    return out
+
+
+def convrot_quantize_act(x_bf16: torch.Tensor, xq: torch.Tensor, sx: torch.Tensor,
+                         group: int = GROUP, stream=None) -> None:
+    assert x_bf16.dtype == torch.bfloat16 and xq.dtype == torch.int8 and sx.dtype == torch.float32
+    m, k = x_bf16.shape
+    _check(load_library().convrot_quantize_act(_ptr(x_bf16), m, k, group, _ptr(xq), _ptr(sx),
+                                               _stream(stream)), "convrot_quantize_act")
+
+
+def convrot_gemm_workspace_bytes(m: int, n: int, k: int) -> int:
+    return int(load_library().convrot_gemm_workspace_bytes(m, n, k))
+
+
+def convrot_linear_workspace_bytes(m: int, n: int, k: int) -> int:
+    return int(load_library().convrot_linear_workspace_bytes(m, n, k))
+
+
+def convrot_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check(load_library().convrot_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "convrot_workspace_init")
+
+
+def convrot_gemm_i8(xq: torch.Tensor, sx: torch.Tensor, w: QuantizedWeight, y: Optional[torch.Tensor],
+                    acc: Optional[torch.Tensor], ws: Optional[torch.Tensor], stream=None) -> None:
+    m = xq.shape[0]
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(load_library().convrot_gemm_i8(_ptr(xq), _ptr(sx), m, ctypes.byref(w.handle), _ptr(y), _ptr(acc),
+                                          _ptr(ws), ws_bytes, _stream(stream)), "convrot_gemm_i8")
+
+
+def convrot_linear_int8(x_bf16: torch.Tensor, w: QuantizedWeight, y: torch.Tensor, ws: torch.Tensor,
+                        stream=None) -> None:
+    m = x_bf16.shape[0]
+    _check(load_library().convrot_linear_int8(_ptr(x_bf16), m, ctypes.byref(w.handle), _ptr(y), _ptr(ws),
+                                              ws.numel() * ws.element_size(), _stream(stream)),
+           "convrot_linear_int8")
+
+
+def convrot_device_status(stream=None) -> None:
+    _check(load_library().convrot_device_status(_stream(stream)), "convrot_device_status")
+
+
+# ---------------------------------------------------------------- helpers
+def quantize_weight(w_bf16: torch.Tensor, stream=None) -> QuantizedWeight:
+    """Allocate q/scale and run the offline rotate+quantise kernel."""
+    n, k = w_bf16.shape
+    q = torch.empty((n, k), dtype=torch.int8, device=w_bf16.device)
+    scale = torch.empty((n,), dtype=torch.float32, device=w_bf16.device)
+    return convrot_quantize_weight(w_bf16, convrot_weight_init(q, scale), stream)
+
+
+def make_workspace(m: int, w: QuantizedWeight, device=None, linear: bool = True) -> torch.Tensor:
+    """A zero-filled workspace big enough for convrot_linear_int8 (or, with
+    linear=False, convrot_gemm_i8) at m rows against w."""
+    nbytes = (convrot_linear_workspace_bytes if linear else convrot_gemm_workspace_bytes)(m, w.n, w.k)
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device or w.q.device)
+
+
+def linear_int8(x_bf16: torch.Tensor, w: QuantizedWeight, ws: torch.Tensor, y: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    if y is None:
+        y = torch.empty((x_bf16.shape[0], w.n), dtype=torch.bfloat16, device=x_bf16.device)
+    convrot_linear_int8(x_bf16, w, y, ws, stream)
+    return y

@@ -1,0 +1,90 @@
+"""The C ABI without a GPU: the library loads, exports every entry point
+that include/convrot.h declares, and rejects bad arguments on the host
+before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "convrot.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rotated_int8_quantized_b200 import build
+    build.build()
+    import rotated_int8_quantized_b200 as cr
+    return cr.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(convrot_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("convrot_quantize_weight", "convrot_quantize_act", "convrot_gemm_i8",
+                     "convrot_linear_int8", "convrot_weight_init"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    import rotated_int8_quantized_b200 as cr
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert name in cr.SIGNATURES, name
+
+
+def test_status_strings(lib):
+    import rotated_int8_quantized_b200 as cr
+    for code, name in cr._STATUS.items():
+        assert cr.convrot_status_string(code) == name
+    assert cr.convrot_version() >= 100
+
+
+def _init(lib, q, s, n, k, g):
+    import rotated_int8_quantized_b200 as cr
+    h = cr.convrot_weight_t()
+    return lib.convrot_weight_init(ctypes.byref(h), ctypes.c_void_p(q), ctypes.c_void_p(s), n, k, g), h
+
+
+def test_weight_init_validation(lib):
+    ok, h = _init(lib, 0x10000, 0x20000, 256, 512, 256)
+    assert ok == 0 and h.n == 256 and h.k == 512 and h.group == 256
+    assert _init(lib, 0, 0x20000, 256, 512, 256)[0] == 1          # null q
+    assert _init(lib, 0x10000, 0x20000, 0, 512, 256)[0] == 1      # n = 0
+    assert _init(lib, 0x10000, 0x20000, 8, 300, 256)[0] == 3      # k % 256
+    assert _init(lib, 0x10000, 0x20000, 8, 512, 128)[0] == 3      # group
+    assert _init(lib, 0x10000, 0x20000, 8, 133376, 256)[0] == 3   # INT32 accumulation bound
+    assert _init(lib, 0x10001, 0x20000, 8, 512, 256)[0] == 2      # misaligned q
+    assert _init(lib, 0x10000, 0x20004, 8, 512, 256)[0] == 2      # misaligned scale
+
+
+def test_calls_reject_bad_arguments_before_any_device_work(lib):
+    P = ctypes.c_void_p
+    assert lib.convrot_quantize_act(P(0), 4, 512, 256, P(0x100), P(0x200), P(0)) == 1
+    assert lib.convrot_quantize_act(P(0x100), 4, 500, 256, P(0x100), P(0x200), P(0)) == 3
+    assert lib.convrot_quantize_act(P(0x101), 4, 512, 256, P(0x100), P(0x200), P(0)) == 2
+    _, h = _init(lib, 0x10000, 0x20000, 256, 512, 256)
+    assert lib.convrot_gemm_i8(P(0x100), P(0x200), 4, ctypes.byref(h), P(0), P(0), P(0), 0, P(0)) == 1
+    assert lib.convrot_linear_int8(P(0x100), 4, ctypes.byref(h), P(0x300), P(0), 0, P(0)) == 1
+    assert lib.convrot_linear_int8(P(0x100), 0, ctypes.byref(h), P(0x300), P(0x400), 1 << 20, P(0)) == 1
+
+
+def test_workspace_sizes_follow_the_tiling(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("sizes below assume the 148-SM default used without a device")
+    # decode: weight is the 128-row operand, 12 tokens pad to one 16-row
+    # tile; 64 weight tiles < 148 SMs, so every tile is split along K and
+    # needs an INT32 partial tile (16 x 128 x 4 B) and a counter.
+    assert lib.convrot_gemm_workspace_bytes(12, 8192, 5120) == 256 + 64 * 16 * 128 * 4
+    # prefill: 32 x 100 tiles of 128 x 256; 21 whole waves over 148 SMs
+    # leave 92 tiles for the stream-K tail.
+    assert lib.convrot_gemm_workspace_bytes(4096, 25600, 5120) == 512 + 92 * 256 * 128 * 4
+    lw = lib.convrot_linear_workspace_bytes(12, 8192, 5120)
+    assert lw == lib.convrot_gemm_workspace_bytes(12, 8192, 5120) + 61440 + 256

@@ -1,0 +1,227 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bit-exact: the rotated INT8 codes and FP32 scales of weights and
+activations, and the INT32 accumulators.  The BF16 output must be within
+max|Y - Y_oracle| / max|Y_oracle| <= 1e-2; since both sides evaluate
+((float)acc * sx) * sw and round once to BF16, it is in fact compared
+bit for bit as well.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def cr():
+    from rotated_int8_quantized_b200 import build
+    build.build()
+    import rotated_int8_quantized_b200 as m
+    m.load_library()
+    return m
+
+
+def to_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def from_bits(a: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def rel_err(y_bits, ref_bits):
+    y = oracle.bf16_bits_to_f64(y_bits)
+    r = oracle.bf16_bits_to_f64(ref_bits)
+    return float(np.max(np.abs(y - r)) / max(np.max(np.abs(r)), 1e-30))
+
+
+def gpu_quantize(cr, a_bits):
+    """Rotate+quantise rows on the GPU with the weight entry point."""
+    w = cr.quantize_weight(from_bits(a_bits))
+    torch.cuda.synchronize()
+    return w, w.q.cpu().numpy(), w.scale.cpu().numpy()
+
+
+# ---------------------------------------------------------------- K3 / K1
+def test_weight_quant_tiny_bit_exact(cr):
+    lin = synth.tiny()[0]
+    w_bits = lin.w_np()
+    _, q, s = gpu_quantize(cr, w_bits)
+    q_ref, s_ref = oracle.rotate_quantize(w_bits)
+    assert np.array_equal(q, q_ref)
+    assert np.array_equal(s.view(np.uint32), s_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("m,k", [(1, 256), (4, 512), (3, 768), (17, 5120), (5, 25600), (2, 65536)])
+def test_act_quant_bit_exact(cr, m, k):
+    cs = synth.outlier_scale_fraction(synth.stream_key(m * 7 + k, 2), k, 0.01, 30.0)
+    x_bits = synth.draw_np(synth.stream_key(m * 7 + k, 0), m, k, 1.0, cs)
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+    cr.convrot_quantize_act(from_bits(x_bits), xq, sx)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.rotate_quantize(x_bits)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def test_act_quant_zero_row_and_one_hot(cr):
+    x = np.zeros((3, 512), dtype=np.float32)
+    x[1, 7] = -3.0
+    x[2, :] = 0.25
+    bits = synth.f32_to_bf16_bits(x)
+    xq = torch.empty((3, 512), dtype=torch.int8, device="cuda")
+    sx = torch.empty((3,), dtype=torch.float32, device="cuda")
+    cr.convrot_quantize_act(from_bits(bits), xq, sx)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.rotate_quantize(bits)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy(), s_ref)
+    assert sx[0].item() == 0 and int(xq[0].abs().max()) == 0
+
+
+# ---------------------------------------------------------------- K2
+def _gemm_case(cr, m, n, k, seed):
+    cs = synth.outlier_scale_fraction(synth.stream_key(seed, 2), k, 0.01, 30.0)
+    x_bits = synth.draw_np(synth.stream_key(seed, 0), m, k, 1.0, cs)
+    w_bits = synth.draw_np(synth.stream_key(seed, 1), n, k, synth.W_SIGMA)
+    wq_ref, sw_ref = oracle.rotate_quantize(w_bits)
+    ref = oracle.linear_int8(x_bits, wq_ref, sw_ref)
+    w, wq, sw = gpu_quantize(cr, w_bits)
+    assert np.array_equal(wq, wq_ref) and np.array_equal(sw, sw_ref)
+    return x_bits, w, ref
+
+
+GEMM_SHAPES = [
+    (4, 256, 512),      # tiny: swap path, one 16-row activation tile, 2 weight tiles
+    (1, 384, 256),      # single token, one K block pair
+    (12, 1024, 5120),   # decode shape, stream-K across many CTAs
+    (17, 1000, 1280),   # ragged weight tile, activation tile of 32
+    (100, 640, 2560),   # swap with bn = 112
+    (256, 512, 768),    # largest swap case, bn = 256
+    (257, 512, 512),    # smallest non-swap case, ragged activation tile
+    (640, 1000, 1536),  # non-swap, ragged weight tile (1000 % 256), stream-K tail
+]
+
+
+@pytest.mark.parametrize("m,n,k", GEMM_SHAPES)
+def test_gemm_acc_and_y_bit_exact(cr, m, n, k):
+    x_bits, w, ref = _gemm_case(cr, m, n, k, seed=m * 131 + n * 7 + k)
+    xq = torch.from_numpy(ref["xq"]).cuda()
+    sx = torch.from_numpy(ref["sx"]).cuda()
+    acc = torch.empty((m, n), dtype=torch.int32, device="cuda")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    ws = cr.make_workspace(m, w, linear=False)
+    cr.convrot_gemm_i8(xq, sx, w, y, acc, ws)
+    cr.convrot_device_status()
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    yb = to_bits(y)
+    assert rel_err(yb, ref["y"]) <= TOL
+    assert np.array_equal(yb, ref["y"])
+    assert int(ws.count_nonzero()) == 0      # workspace returned to zero
+
+
+@pytest.mark.parametrize("m,n,k", [(4, 256, 512), (12, 1024, 5120), (300, 768, 1024)])
+def test_linear_end_to_end(cr, m, n, k):
+    x_bits, w, ref = _gemm_case(cr, m, n, k, seed=m + n + k)
+    ws = cr.make_workspace(m, w)
+    x = from_bits(x_bits)
+    y1 = cr.linear_int8(x, w, ws)
+    y2 = cr.linear_int8(x, w, ws)     # second call reuses the self-cleaned workspace
+    cr.convrot_device_status()
+    assert rel_err(to_bits(y1), ref["y"]) <= TOL
+    assert np.array_equal(to_bits(y1), ref["y"])
+    assert np.array_equal(to_bits(y2), ref["y"])
+
+
+def test_tiny_config_layer(cr):
+    lin = synth.tiny()[0]
+    x_bits, w_bits = lin.x_np(), lin.w_np()
+    wq_ref, sw_ref = oracle.rotate_quantize(w_bits)
+    ref = oracle.linear_int8(x_bits, wq_ref, sw_ref)
+    w = cr.quantize_weight(from_bits(w_bits))
+    y = cr.linear_int8(from_bits(x_bits), w, cr.make_workspace(lin.m, w))
+    cr.convrot_device_status()
+    assert np.array_equal(to_bits(y), ref["y"])
+
+
+def test_errors_are_statuses(cr):
+    w = cr.quantize_weight(torch.zeros((256, 512), dtype=torch.bfloat16, device="cuda"))
+    x = torch.zeros((4, 512), dtype=torch.bfloat16, device="cuda")
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(cr.ConvrotError) as e:
+        cr.linear_int8(x, w, small)
+    assert e.value.status == 5
+    with pytest.raises(cr.ConvrotError) as e:
+        cr.convrot_quantize_act(torch.zeros((4, 300), dtype=torch.bfloat16, device="cuda"),
+                                torch.empty((4, 300), dtype=torch.int8, device="cuda"),
+                                torch.empty(4, dtype=torch.float32, device="cuda"))
+    assert e.value.status == 3
+    cr.convrot_device_status()
+
+
+# ---------------------------------------------------------------- full sizes, sampled
+def _sampled_layer_check(cr, lin, rows_w, rows_x=None):
+    """Whole-size weights drawn on the GPU, quantised there; the oracle
+    recomputes the sampled weight rows (and activation rows) from the
+    counter-based generator and checks codes, scales and outputs."""
+    dev = "cuda"
+    w_bf = lin.w_torch(dev)
+    w = cr.quantize_weight(w_bf)
+    x = lin.x_torch(dev)
+    ws = cr.make_workspace(lin.m, w)
+    y = cr.linear_int8(x, w, ws)
+    acc = torch.empty((lin.m, lin.n), dtype=torch.int32, device=dev)
+    xq = torch.empty((lin.m, lin.k), dtype=torch.int8, device=dev)
+    sx = torch.empty((lin.m,), dtype=torch.float32, device=dev)
+    cr.convrot_quantize_act(x, xq, sx)
+    cr.convrot_gemm_i8(xq, sx, w, None, acc, cr.make_workspace(lin.m, w, linear=False))
+    cr.convrot_device_status()
+    del w_bf
+    w_rows = lin.w_rows_np(rows_w)
+    assert np.array_equal(to_bits(lin.w_torch(dev)[torch.as_tensor(rows_w, device=dev)]), w_rows)
+    wq_ref, sw_ref = oracle.rotate_quantize(w_rows)
+    assert np.array_equal(w.q[torch.as_tensor(rows_w, device=dev)].cpu().numpy(), wq_ref)
+    assert np.array_equal(w.scale[torch.as_tensor(rows_w, device=dev)].cpu().numpy(), sw_ref)
+    rows_x = np.arange(lin.m) if rows_x is None else np.asarray(rows_x)
+    x_rows = lin.x_rows_np(rows_x)
+    ref = oracle.linear_int8(x_rows, wq_ref, sw_ref)
+    rx = torch.as_tensor(rows_x, device=dev)
+    assert np.array_equal(xq[rx].cpu().numpy(), ref["xq"])
+    assert np.array_equal(sx[rx].cpu().numpy(), ref["sx"])
+    rw = torch.as_tensor(rows_w, device=dev)
+    assert np.array_equal(acc[rx][:, rw].cpu().numpy(), ref["acc"])
+    yb = to_bits(y[rx][:, rw])
+    assert rel_err(yb, ref["y"]) <= TOL
+    assert np.array_equal(yb, ref["y"])
+
+
+@pytest.mark.parametrize("idx", range(7))
+def test_qwen_decode_full_size_sampled(cr, idx):
+    lin = synth.qwen_layer(12)[idx]
+    rng = np.random.default_rng(idx)
+    rows = np.unique(np.concatenate([[0, lin.n - 1], rng.integers(0, lin.n, 30)]))
+    _sampled_layer_check(cr, lin, rows)
+
+
+@pytest.mark.parametrize("idx", [0, 6])
+def test_qwen_prefill_full_size_sampled(cr, idx):
+    lin = synth.qwen_layer(4096)[idx]
+    rng = np.random.default_rng(100 + idx)
+    rows_w = np.unique(np.concatenate([[0, lin.n - 1], rng.integers(0, lin.n, 14)]))
+    rows_x = np.unique(np.concatenate([[0, lin.m - 1], rng.integers(0, lin.m, 14)]))
+    _sampled_layer_check(cr, lin, rows_w, rows_x)
+
+
+def test_minimax_qkv_sampled(cr):
+    lin = synth.minimax_qkv(8192)[0]
+    rng = np.random.default_rng(4)
+    rows_w = np.unique(np.concatenate([[0, lin.n - 1], rng.integers(0, lin.n, 14)]))
+    rows_x = np.unique(np.concatenate([[0, lin.m - 1], rng.integers(0, lin.m, 14)]))
+    _sampled_layer_check(cr, lin, rows_w, rows_x)
