@@ -1,0 +1,500 @@
+"""Benchmark of the INT8 ConvRot linear layer on B200.
+
+One step = the seven Qwen3-VL-32B-shaped linears of one decoder layer at
+M = 12 conditioning tokens (q, k, v, o, gate, up, down), each a full
+ConvRot INT8 linear (activation rotation + row quantisation kernel, then the
+tcgen05 INT8 GEMM with fused dequantisation) through the C ABI, with
+weights already rotated, quantised and resident in HBM.  The metric is the
+weight-stream bandwidth in GB/s of algorithmic bytes; the roofline object
+reports the GEMM kernel against the measured HBM copy bandwidth.  A second
+measurement runs the same seven linears at prefill size M = 4096 and
+reports INT8 tensor TOPS against the dense INT8 peak.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+For N > 1 it is launched under torch.distributed.run; every rank runs an
+independent replica (the layer needs no exchange between GPUs), and the
+whole-job value is the bytes all ranks moved over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "ConvRot INT8 linear TOPS & weight-stream GB/s on 1 B200, % of INT8/HBM roofline"
+UNIT = "GB/s"
+WORKLOAD = "qwen3vl32b_layer_7linears_decode_m12"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0     # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+CPU_SAMPLE_ROWS_DIV = 64  # oracle sample: the first N/64 weight rows of every linear
+
+
+# --------------------------------------------------------------------------- helpers
+def linear_bytes(m: int, n: int, k: int) -> int:
+    """Algorithmic HBM bytes of one ConvRot INT8 linear: weight codes and
+    scales, the BF16 activations, the INT8 activations written and read
+    back, their scales, and the BF16 output."""
+    return n * k + 4 * n + 2 * m * k + m * k + m * k + 4 * m + 2 * m * n
+
+
+def gemm_bytes(m: int, n: int, k: int) -> int:
+    """Algorithmic bytes of the GEMM kernel alone."""
+    return n * k + 4 * n + m * k + 4 * m + 2 * m * n
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    csrc = os.path.join(ROOT, "rotated_int8_quantized_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.tsv")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            parts = line.rstrip("\n").split("\t")
+            if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[2] == want:
+                return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms."""
+    FIELDS = ("timestamp,index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, pci_bus_id: str | None):
+        self.pci = (pci_bus_id or "").lower()
+        self.rows = []
+        self.proc = None
+        self.windows = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.6)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons, n_all = [], None, set(), 0
+        for t, line in self.rows:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.pci and self.pci[-12:] not in parts[2].lower():
+                continue
+            n_all += 1
+            if not any(a - 0.05 <= t <= b + 0.05 for a, b in self.windows):
+                continue
+            try:
+                sm.append(float(parts[3]))
+                smax = float(parts[4])
+            except ValueError:
+                continue
+            names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+            for name, v in zip(names, parts[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm), "samples_all": n_all}
+
+
+# --------------------------------------------------------------------------- GPU arm
+class Layer:
+    """The seven quantised linears of one layer, resident on the device."""
+
+    def __init__(self, cr, lins, device):
+        self.cr = cr
+        self.lins = lins
+        self.w = []
+        for lin in lins:
+            w_bf = lin.w_torch(device)
+            self.w.append(cr.quantize_weight(w_bf))
+            del w_bf
+        torch.cuda.synchronize()
+
+
+def make_io(cr, layer, lins, device):
+    xs = [lin.x_torch(device) for lin in lins]
+    ys = [torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device) for lin in lins]
+    wss = [cr.make_workspace(lin.m, w) for lin, w in zip(lins, layer.w)]
+    return xs, ys, wss
+
+
+def run_step(cr, layer, xs, ys, wss, stream):
+    for x, w, y, ws in zip(xs, layer.w, ys, wss):
+        cr.convrot_linear_int8(x, w, y, ws, stream)
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def time_region(fn, steps, stream):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3
+
+
+def gemm_kernel_times(cr, layer, lins, xs, reps, stream, device):
+    """Per-launch GEMM kernel time per linear with CUDA events on the
+    launching stream (activation prologue launched before each, untimed)."""
+    out = []
+    for lin, w, x in zip(lins, layer.w, xs):
+        xq = torch.empty((lin.m, lin.k), dtype=torch.int8, device=device)
+        sx = torch.empty((lin.m,), dtype=torch.float32, device=device)
+        y = torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device)
+        ws = cr.make_workspace(lin.m, w, linear=False)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i in range(reps + 2):
+            cr.convrot_quantize_act(x, xq, sx, stream=stream)
+            if i >= 2:
+                evs[i - 2][0].record(stream)
+            cr.convrot_gemm_i8(xq, sx, w, y, None, ws, stream)
+            if i >= 2:
+                evs[i - 2][1].record(stream)
+        torch.cuda.synchronize()
+        t = sum(a.elapsed_time(b) for a, b in evs) / reps / 1e3
+        out.append((lin, t))
+    return out
+
+
+def all_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def cpu_baseline(lins, seconds: float = 10.0):
+    """The oracle, as it stands (single-threaded C), on a bounded sample:
+    every linear of the step with its first N/64 weight rows and all M
+    token rows; whole passes repeated for >= `seconds`."""
+    import oracle
+    prepared = []
+    for lin in lins:
+        ns = max(1, math.ceil(lin.n / CPU_SAMPLE_ROWS_DIV))
+        wq, sw = oracle.rotate_quantize(lin.w_rows_np(np.arange(ns)))
+        prepared.append((lin, ns, lin.x_np(), wq, sw))
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        for lin, ns, x, wq, sw in prepared:
+            oracle.linear_int8(x, wq, sw)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    nbytes = passes * sum(linear_bytes(lin.m, ns, lin.k) for lin, ns, *_ in prepared)
+    return {"value": nbytes / el / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d passes over the 7 linears at M=%d with the first N/%d weight rows each "
+                      "(%.2f MB INT8 weights per pass), %.1f s" % (
+                          passes, lins[0].m, CPU_SAMPLE_ROWS_DIV,
+                          sum(ns * lin.k for lin, ns, *_ in prepared) / 1e6, el)}
+
+
+def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
+    """The same seven linears at M = 4096 (same weights): TOPS vs the dense
+    INT8 peak (the bf16 peak measured on this machine x the nominal 2x)."""
+    lins = synth.qwen_layer(4096)
+    xs = [lin.x_torch(device) for lin in lins]
+    ys = [torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device) for lin in lins]
+    wss = [cr.make_workspace(lin.m, w) for lin, w in zip(lins, layer.w)]
+    fn = lambda: run_step(cr, layer, xs, ys, wss, stream)  # noqa: E731
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    t = time_region(fn, steps, stream) / steps
+    ops = sum(2 * lin.m * lin.n * lin.k for lin in lins)
+    g = gemm_kernel_times(cr, layer, lins, xs, 3, stream, device)
+    gops = sum(2 * lin.m * lin.n * lin.k for lin, _ in g)
+    gt = sum(tt for _, tt in g)
+    peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    del xs, ys, wss
+    torch.cuda.empty_cache()
+    return {"workload": "qwen3vl32b_layer_7linears_prefill_m4096", "metric": "INT8 TOPS (2MNK)",
+            "layer_tops": ops / t / 1e12, "ms_per_step": t * 1e3,
+            "gemm_tops": gops / gt / 1e12,
+            "roofline": {"bound": "tensor", "achieved": gops / gt / 1e12, "peak": peak, "unit": "TOP/s",
+                         "frac": gops / gt / 1e12 / peak,
+                         "peak_note": "measured bf16 burst x 2 (nominal int8/bf16 ratio)"},
+            "per_linear_gemm_tops": {lin.name: 2 * lin.m * lin.n * lin.k / tt / 1e12 for lin, tt in g}}
+
+
+def run_profile(args):
+    """A few plain (eager) steps of one workload for an ncu capture: no
+    timing, no JSON.  Weight generation and quantisation run first."""
+    import rotated_int8_quantized_b200 as cr
+    cr.load_library()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    m = {"decode": 12, "prefill": 4096}[args.profile]
+    lins = synth.qwen_layer(m)
+    layer = Layer(cr, lins, device)
+    xs, ys, wss = make_io(cr, layer, lins, device)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.steps):
+        run_step(cr, layer, xs, ys, wss, stream)
+    torch.cuda.synchronize()
+    cr.convrot_device_status(stream)
+    print("profile run ok: %s, %d steps" % (args.profile, args.steps))
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    import rotated_int8_quantized_b200 as cr
+    cr.load_library()
+    peaks, peak_kind = load_peaks()
+
+    lins = synth.qwen_layer(12)
+    layer = Layer(cr, lins, device)
+    xs, ys, wss = make_io(cr, layer, lins, device)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+
+    fn_eager = lambda: run_step(cr, layer, xs, ys, wss, stream)  # noqa: E731
+    with torch.cuda.stream(stream):
+        fn_eager()                      # first call configures kernels (outside capture)
+    torch.cuda.synchronize()
+    graph = capture(fn_eager, stream) if not args.no_graph else None
+    step = (lambda: graph.replay()) if graph is not None else fn_eager
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    cr.convrot_device_status(stream)
+
+    try:
+        pci = torch.cuda.get_device_properties(device).pci_bus_id
+    except Exception:
+        pci = None
+    clocks = ClockSampler(pci)
+    clocks.start()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    w0 = time.time()
+    with torch.cuda.stream(stream):
+        elapsed = time_region(step, args.steps, stream)
+    torch.cuda.synchronize()
+    clocks.mark(w0, time.time())
+    barrier(world)
+    elapsed = all_max(elapsed, world)
+    cr.convrot_device_status(stream)
+
+    bytes_step = sum(linear_bytes(lin.m, lin.n, lin.k) for lin in lins)
+    value = bytes_step * args.steps * world / elapsed / 1e9
+
+    # dominant kernel: the GEMM, per-launch CUDA-event timing
+    g = gemm_kernel_times(cr, layer, lins, xs, 20, stream, device)
+    gb = sum(gemm_bytes(lin.m, lin.n, lin.k) for lin, _ in g)
+    gt = sum(t for _, t in g)
+    achieved = gb / gt / 1e9
+    traffic = profiled_traffic("gemm_i8_tc_kernel", WORKLOAD)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "kernel": "gemm_i8_tc_kernel", "peak_source": peak_kind,
+                "per_launch_bytes_avg": gb / len(g), "per_launch_us_avg": gt / len(g) * 1e6,
+                "per_linear_gbs": {lin.name: gemm_bytes(lin.m, lin.n, lin.k) / t / 1e9 for lin, t in g}}
+
+    # end to end through the C ABI from pinned host buffers
+    hx = [x.cpu().pin_memory() for x in xs]
+    hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
+
+    def e2e_step():
+        for h, x in zip(hx, xs):
+            x.copy_(h, non_blocking=True)
+        run_step(cr, layer, xs, ys, wss, stream)
+        for h, y in zip(hy, ys):
+            h.copy_(y, non_blocking=True)
+
+    e2e_steps = max(10, min(args.steps, 500))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        w1 = time.time()
+        e2e_t = time_region(e2e_step, e2e_steps, stream)
+        clocks.mark(w1, time.time())
+    e2e_t = all_max(e2e_t, world)
+    clk = clocks.stop()
+    h2d = sum(2 * lin.m * lin.k for lin in lins)
+    d2h = sum(2 * lin.m * lin.n for lin in lins)
+    e2e = {"value": bytes_step * e2e_steps * world / e2e_t / 1e9, "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    secondary = None
+    if not args.no_prefill:
+        secondary = prefill_secondary(cr, layer, device, stream, peaks)
+    cr.convrot_device_status(stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(lins)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "m": 12,
+                       "linears": [[lin.name, lin.k, lin.n] for lin in lins],
+                       "weight_bytes_per_step": sum(lin.n * lin.k for lin in lins),
+                       "algorithmic_bytes_per_step": bytes_step,
+                       "l2": "inputs larger than L2: %.1f MB of INT8 weights streamed per step vs 126 MB L2"
+                             % (sum(lin.n * lin.k for lin in lins) / 1e6),
+                       "cuda_graph": graph is not None, "parallelism": "replicas" if world > 1 else "single"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 2 * len(lins) * args.steps, "clocks": clk,
+            "secondary": secondary, "kernel_sources": kernel_source_hash(),
+        }
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The oracle (plain single-threaded C on the host) on the same workload:
+    each step is one linear of the layer (cycling q, k, v, o, gate, up, down)
+    at M = 12 with its first N/64 weight rows."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+    lins = synth.qwen_layer(12)
+    prepared = []
+    for lin in lins:
+        ns = max(1, math.ceil(lin.n / CPU_SAMPLE_ROWS_DIV))
+        wq, sw = oracle.rotate_quantize(lin.w_rows_np(np.arange(ns)))
+        prepared.append((lin, ns, lin.x_np(), wq, sw))
+    for s in range(args.warmup):
+        lin, ns, x, wq, sw = prepared[s % 7]
+        oracle.linear_int8(x, wq, sw)
+    nbytes = 0
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        lin, ns, x, wq, sw = prepared[s % 7]
+        oracle.linear_int8(x, wq, sw)
+        nbytes += linear_bytes(lin.m, ns, lin.k)
+    el = time.perf_counter() - t0
+    value = nbytes / el / 1e9
+    sample = ("each step one linear of the layer in turn at M=12 with its first N/%d weight rows; "
+              "%d steps, %.1f s" % (CPU_SAMPLE_ROWS_DIV, args.steps, el))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / max(args.steps, 1) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "m": 12}, "gpu_launches": 0,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
+                    help="run a few eager steps of one workload for ncu (no timing)")
+    args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
