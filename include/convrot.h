@@ -91,6 +91,10 @@ const char *convrot_status_string(convrot_status_t status);
 /* Library version as 10000 * major + 100 * minor + patch. */
 int convrot_version(void);
 
+/* Text of the last CUDA error this thread's calls turned into
+   CONVROT_ERR_CUDA ("no error" if none).  Static string, never NULL. */
+const char *convrot_last_error_string(void);
+
 /*
  * Fill a handle.  Checks: w, q, scale non-NULL; n, k >= 1; group == 256;
  * k % 256 == 0; k <= 133120 (INT32 accumulation bound); q and scale
@@ -155,6 +159,65 @@ convrot_status_t convrot_gemm_i8(const int8_t *xq, const float *sx, int64_t m,
  */
 convrot_status_t convrot_linear_int8(const void *x_bf16, int64_t m, const convrot_weight_t *w,
                                      void *y_bf16, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * One product of a batched GEMM call (see convrot_gemm_i8 for the maths).
+ *   xq : int8 [m, w->k] quantised activations;  sx : fp32 [m] their scales
+ *   y_bf16 : BF16 [m, w->n] output or NULL;  acc : int32 [m, w->n] or NULL
+ */
+typedef struct {
+    const int8_t *xq;
+    const float *sx;
+    const convrot_weight_t *w;
+    void *y_bf16;
+    int32_t *acc;
+} convrot_gemm_job_t;
+
+/*
+ * Several INT8 GEMMs with the same m (1 <= m <= 256) in ONE launch: every
+ * 128-byte K block of every weight is dealt out evenly to the SMs
+ * (stream-K), so the whole set streams its weights as one long read.
+ * count <= 8.  Workspace: convrot_gemm_batch_workspace_bytes, zero-filled
+ * before first use, left zero-filled.
+ */
+convrot_status_t convrot_gemm_i8_batch(int64_t m, int count, const convrot_gemm_job_t *jobs,
+                                       void *ws, size_t ws_bytes, void *stream);
+
+size_t convrot_gemm_batch_workspace_bytes(int64_t m, int count, const convrot_gemm_job_t *jobs);
+
+/*
+ * One linear of a batched call: y = ConvRotLinearINT8(x) against w.
+ *   x_bf16 : BF16 [m, w->k] input (device)
+ *   w      : quantised weight handle
+ *   y_bf16 : BF16 [m, w->n] output (device)
+ */
+typedef struct {
+    const void *x_bf16;
+    const convrot_weight_t *w;
+    void *y_bf16;
+} convrot_linear_job_t;
+
+/*
+ * Several independent ConvRot INT8 linears with the same token count m, in
+ * two launches: one activation prologue over every job's rows, then one
+ * GEMM whose K blocks of all weights are dealt out evenly to every SM
+ * (m <= 256; larger m runs the GEMMs one after another).  This is how the
+ * linears of one decoder layer that share an input (q/k/v, gate/up) or that
+ * are otherwise ready together run at decode size, where a per-linear launch
+ * would spend more time starting and draining than streaming its weight.
+ * The pages quantise exactly these projections of every layer [zskr.cn
+ * "Qwen3-VL-32B ... INT8-ConvRot": 350 = 50 layers x 7 row-wise INT8 ConvRot
+ * matrices; 0539edu.com section 4: the attention QKV projections].
+ * count <= 8.  No job's output may overlap any job's input or another
+ * job's output (CONVROT_ERR_INVALID_ARG).  Results equal count calls of
+ * convrot_linear_int8.
+ */
+convrot_status_t convrot_linear_int8_batch(int64_t m, int count, const convrot_linear_job_t *jobs,
+                                           void *ws, size_t ws_bytes, void *stream);
+
+/* Workspace bytes convrot_linear_int8_batch needs for these jobs (0 if the
+   jobs are invalid).  Zero-fill before first use, as for the others. */
+size_t convrot_linear_batch_workspace_bytes(int64_t m, int count, const convrot_linear_job_t *jobs);
 
 /*
  * Synchronise `stream`, then read and clear the device-side status word of

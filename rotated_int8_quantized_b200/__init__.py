@@ -44,12 +44,25 @@ class convrot_weight_t(ctypes.Structure):
                 ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("group", ctypes.c_int32)]
 
 
+class convrot_linear_job_t(ctypes.Structure):
+    """Mirror of the C struct: one linear of a batched call."""
+    _fields_ = [("x_bf16", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight_t)),
+                ("y_bf16", ctypes.c_void_p)]
+
+
+class convrot_gemm_job_t(ctypes.Structure):
+    """Mirror of the C struct: one product of a batched GEMM call."""
+    _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight_t)),
+                ("y_bf16", ctypes.c_void_p), ("acc", ctypes.c_void_p)]
+
+
 # exported symbol -> (argtypes, restype); every name declared in convrot.h
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
 _WP = ctypes.POINTER(convrot_weight_t)
 SIGNATURES = {
     "convrot_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "convrot_version": ([], ctypes.c_int),
+    "convrot_last_error_string": ([], ctypes.c_char_p),
     "convrot_weight_init": ([_WP, _P, _P, _I64, _I64, _I32], ctypes.c_int),
     "convrot_quantize_weight": ([_P, _WP, _P], ctypes.c_int),
     "convrot_quantize_act": ([_P, _I64, _I64, _I32, _P, _P, _P], ctypes.c_int),
@@ -59,6 +72,11 @@ SIGNATURES = {
     "convrot_gemm_i8": ([_P, _P, _I64, _WP, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "convrot_linear_int8": ([_P, _I64, _WP, _P, _P, _SZ, _P], ctypes.c_int),
     "convrot_device_status": ([_P], ctypes.c_int),
+    "convrot_linear_int8_batch": ([_I64, ctypes.c_int, ctypes.POINTER(convrot_linear_job_t), _P, _SZ, _P],
+                                  ctypes.c_int),
+    "convrot_linear_batch_workspace_bytes": ([_I64, ctypes.c_int, ctypes.POINTER(convrot_linear_job_t)], _SZ),
+    "convrot_gemm_i8_batch": ([_I64, ctypes.c_int, ctypes.POINTER(convrot_gemm_job_t), _P, _SZ, _P], ctypes.c_int),
+    "convrot_gemm_batch_workspace_bytes": ([_I64, ctypes.c_int, ctypes.POINTER(convrot_gemm_job_t)], _SZ),
 }
 
 _lib = None
@@ -82,7 +100,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 def _check(status: int, where: str) -> None:
     if status != 0:
-        raise ConvrotError(status, where)
+        err = ConvrotError(status, where)
+        if status == 6:
+            err.args = (err.args[0] + " (" + load_library().convrot_last_error_string().decode() + ")",)
+        raise err
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -174,6 +195,73 @@ def convrot_linear_int8(x_bf16: torch.Tensor, w: QuantizedWeight, y: torch.Tenso
     _check(load_library().convrot_linear_int8(_ptr(x_bf16), m, ctypes.byref(w.handle), _ptr(y), _ptr(ws),
                                               ws.numel() * ws.element_size(), _stream(stream)),
            "convrot_linear_int8")
+
+
+def _jobs(xs, ws_, ys):
+    arr = (convrot_linear_job_t * len(xs))()
+    for i, (x, w, y) in enumerate(zip(xs, ws_, ys)):
+        arr[i].x_bf16 = _ptr(x)
+        arr[i].w = ctypes.pointer(w.handle)
+        arr[i].y_bf16 = _ptr(y)
+    return arr
+
+
+class LinearBatch:
+    """A prepared batched call: the C job array is built once and reused,
+    so a step costs one C call (argument marshalling only)."""
+
+    def __init__(self, xs, weights, ys, ws: Optional[torch.Tensor] = None):
+        self.xs, self.weights, self.ys = list(xs), list(weights), list(ys)
+        self.m = self.xs[0].shape[0]
+        self.jobs = _jobs(self.xs, self.weights, self.ys)
+        need = int(load_library().convrot_linear_batch_workspace_bytes(self.m, len(self.xs), self.jobs))
+        if need == 0:
+            raise ConvrotError(1, "convrot_linear_batch_workspace_bytes")
+        if ws is None:
+            ws = torch.zeros(need, dtype=torch.uint8, device=self.xs[0].device)
+        self.ws = ws
+
+    def __call__(self, stream=None) -> None:
+        _check(load_library().convrot_linear_int8_batch(self.m, len(self.xs), self.jobs, _ptr(self.ws),
+                                                        self.ws.numel(), _stream(stream)),
+               "convrot_linear_int8_batch")
+
+
+def convrot_linear_int8_batch(xs, weights, ys, ws: torch.Tensor, stream=None) -> None:
+    """Run len(xs) independent linears with the same token count together."""
+    m = xs[0].shape[0]
+    jobs = _jobs(xs, weights, ys)
+    _check(load_library().convrot_linear_int8_batch(m, len(xs), jobs, _ptr(ws), ws.numel() * ws.element_size(),
+                                                    _stream(stream)), "convrot_linear_int8_batch")
+
+
+def convrot_linear_batch_workspace_bytes(xs, weights, ys) -> int:
+    return int(load_library().convrot_linear_batch_workspace_bytes(xs[0].shape[0], len(xs), _jobs(xs, weights, ys)))
+
+
+class GemmBatch:
+    """A prepared batched GEMM call (job array built once)."""
+
+    def __init__(self, xqs, sxs, weights, ys, accs=None, ws: Optional[torch.Tensor] = None):
+        n = len(xqs)
+        accs = accs or [None] * n
+        self.keep = (list(xqs), list(sxs), list(weights), list(ys), list(accs))
+        self.m = xqs[0].shape[0]
+        self.jobs = (convrot_gemm_job_t * n)()
+        for i in range(n):
+            self.jobs[i].xq = _ptr(xqs[i])
+            self.jobs[i].sx = _ptr(sxs[i])
+            self.jobs[i].w = ctypes.pointer(weights[i].handle)
+            self.jobs[i].y_bf16 = _ptr(ys[i])
+            self.jobs[i].acc = _ptr(accs[i])
+        need = int(load_library().convrot_gemm_batch_workspace_bytes(self.m, n, self.jobs))
+        if need == 0:
+            raise ConvrotError(1, "convrot_gemm_batch_workspace_bytes")
+        self.ws = ws if ws is not None else torch.zeros(need, dtype=torch.uint8, device=xqs[0].device)
+
+    def __call__(self, stream=None) -> None:
+        _check(load_library().convrot_gemm_i8_batch(self.m, len(self.jobs), self.jobs, _ptr(self.ws),
+                                                    self.ws.numel(), _stream(stream)), "convrot_gemm_i8_batch")
 
 
 def convrot_device_status(stream=None) -> None:

@@ -17,6 +17,7 @@ constexpr int64_t kGroup = 256;
 constexpr int64_t kMaxK = 133120;
 constexpr int64_t kMaxRows = 0x7FFFFFFF;
 constexpr int kDefaultSms = 148;
+constexpr int kMaxBatch = convrot::kMaxJobs;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -79,8 +80,11 @@ convrot_status_t check_weight(const convrot_weight_t *w) {
     return CONVROT_OK;
 }
 
+thread_local const char *t_last_error = "no error";
+
 convrot_status_t from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return CONVROT_OK;
+    t_last_error = cudaGetErrorString(e);
     cudaGetLastError();
     return CONVROT_ERR_CUDA;
 }
@@ -106,6 +110,8 @@ const char *convrot_status_string(convrot_status_t s) {
 
 int convrot_version(void) { return 100; }
 
+const char *convrot_last_error_string(void) { return t_last_error; }
+
 convrot_status_t convrot_weight_init(convrot_weight_t *w, int8_t *q, float *scale, int64_t n, int64_t k,
                                      int32_t group) {
     if (!w) return CONVROT_ERR_INVALID_ARG;
@@ -128,8 +134,8 @@ convrot_status_t convrot_quantize_weight(const void *w_bf16, const convrot_weigh
     if (!aligned16(w_bf16)) return CONVROT_ERR_ALIGNMENT;
     DeviceInfo dev;
     if ((s = current_device(&dev)) != CONVROT_OK) return s;
-    return from_cuda(convrot::launch_rotate_quant(w_bf16, out->n, out->k, out->q, out->scale,
-                                                  static_cast<cudaStream_t>(stream), false));
+    convrot::RQProblem prob = {w_bf16, out->k, out->q, out->scale};
+    return from_cuda(convrot::launch_rotate_quant(1, out->n, &prob, static_cast<cudaStream_t>(stream), false));
 }
 
 convrot_status_t convrot_quantize_act(const void *x_bf16, int64_t m, int64_t k, int32_t group, int8_t *xq,
@@ -140,7 +146,8 @@ convrot_status_t convrot_quantize_act(const void *x_bf16, int64_t m, int64_t k, 
     if (!aligned16(x_bf16) || !aligned16(xq) || !aligned16(sx)) return CONVROT_ERR_ALIGNMENT;
     DeviceInfo dev;
     if ((s = current_device(&dev)) != CONVROT_OK) return s;
-    return from_cuda(convrot::launch_rotate_quant(x_bf16, m, k, xq, sx, static_cast<cudaStream_t>(stream), false));
+    convrot::RQProblem prob = {x_bf16, k, xq, sx};
+    return from_cuda(convrot::launch_rotate_quant(1, m, &prob, static_cast<cudaStream_t>(stream), false));
 }
 
 size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
@@ -150,28 +157,11 @@ size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     return round256(p.ws_bytes);
 }
 
-size_t convrot_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
-    if (m < 1 || n < 1 || k < kGroup) return 0;
-    return convrot_gemm_workspace_bytes(m, n, k) + round256((size_t)m * (size_t)k) + round256((size_t)m * 4);
-}
 
 convrot_status_t convrot_workspace_init(void *ws, size_t ws_bytes, void *stream) {
     if (!ws && ws_bytes) return CONVROT_ERR_INVALID_ARG;
     if (!ws_bytes) return CONVROT_OK;
     return from_cuda(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
-}
-
-static convrot_status_t gemm_impl(const int8_t *xq, const float *sx, int64_t m, const convrot_weight_t *w,
-                                  void *y, int32_t *acc, void *ws, size_t ws_bytes, cudaStream_t stream,
-                                  bool pdl, bool w_prefetch) {
-    DeviceInfo dev;
-    convrot_status_t s = current_device(&dev);
-    if (s != CONVROT_OK) return s;
-    convrot::GemmPlan p;
-    convrot::plan_gemm(m, w->n, w->k, dev.num_sms, &p);
-    if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes)) return CONVROT_ERR_WORKSPACE;
-    return from_cuda(convrot::launch_gemm_i8(p, xq, sx, m, w->q, w->scale, w->n, w->k,
-                                             static_cast<__nv_bfloat16 *>(y), acc, ws, stream, pdl, w_prefetch));
 }
 
 convrot_status_t convrot_gemm_i8(const int8_t *xq, const float *sx, int64_t m, const convrot_weight_t *w,
@@ -183,32 +173,199 @@ convrot_status_t convrot_gemm_i8(const int8_t *xq, const float *sx, int64_t m, c
     if (!aligned16(xq) || !aligned16(sx) || (y_bf16 && !aligned16(y_bf16)) || (acc && !aligned16(acc)) ||
         (ws && !aligned16(ws)))
         return CONVROT_ERR_ALIGNMENT;
-    return gemm_impl(xq, sx, m, w, y_bf16, acc, ws, ws_bytes, static_cast<cudaStream_t>(stream), false, false);
-}
-
-convrot_status_t convrot_linear_int8(const void *x_bf16, int64_t m, const convrot_weight_t *w, void *y_bf16,
-                                     void *ws, size_t ws_bytes, void *stream) {
-    if (!x_bf16 || !y_bf16 || !ws) return CONVROT_ERR_INVALID_ARG;
-    convrot_status_t s = check_weight(w);
-    if (s != CONVROT_OK) return s;
-    if ((s = check_shape(m, w->k, w->group)) != CONVROT_OK) return s;
-    if (!aligned16(x_bf16) || !aligned16(y_bf16) || !aligned16(ws)) return CONVROT_ERR_ALIGNMENT;
-    const size_t need = convrot_linear_workspace_bytes(m, w->n, w->k);
     DeviceInfo dev;
     if ((s = current_device(&dev)) != CONVROT_OK) return s;
     convrot::GemmPlan p;
     convrot::plan_gemm(m, w->n, w->k, dev.num_sms, &p);
-    const size_t gemm_ws = round256(p.ws_bytes);
-    const size_t need_here = gemm_ws + round256((size_t)m * (size_t)w->k) + round256((size_t)m * 4);
-    if (ws_bytes < need_here || ws_bytes < need) return CONVROT_ERR_WORKSPACE;
+    if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes)) return CONVROT_ERR_WORKSPACE;
+    convrot::GemmProblem prob = {m, w->n, w->k, xq, sx, w->q, w->scale, static_cast<__nv_bfloat16 *>(y_bf16), acc};
+    return from_cuda(convrot::launch_gemm_i8(p, &prob, ws, static_cast<cudaStream_t>(stream), false, false));
+}
+
+namespace {
+
+bool ranges_overlap(const void *a, size_t an, const void *b, size_t bn) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bn && b0 < a0 + an;
+}
+
+// Checks common to the single and batched layer entry points.
+convrot_status_t check_jobs(int64_t m, int count, const convrot_linear_job_t *jobs) {
+    if (!jobs || count < 1 || count > kMaxBatch) return CONVROT_ERR_INVALID_ARG;
+    for (int j = 0; j < count; ++j) {
+        const convrot_linear_job_t &J = jobs[j];
+        if (!J.x_bf16 || !J.y_bf16) return CONVROT_ERR_INVALID_ARG;
+        convrot_status_t s = check_weight(J.w);
+        if (s != CONVROT_OK) return s;
+        if ((s = check_shape(m, J.w->k, J.w->group)) != CONVROT_OK) return s;
+        if (!aligned16(J.x_bf16) || !aligned16(J.y_bf16)) return CONVROT_ERR_ALIGNMENT;
+    }
+    // no output may overlap any input or another output: the jobs run as
+    // one launch pair, so an output cannot feed a later job
+    for (int j = 0; j < count; ++j) {
+        const size_t ybytes = (size_t)m * (size_t)jobs[j].w->n * 2;
+        for (int i = 0; i < count; ++i) {
+            if (ranges_overlap(jobs[j].y_bf16, ybytes, jobs[i].x_bf16, (size_t)m * (size_t)jobs[i].w->k * 2))
+                return CONVROT_ERR_INVALID_ARG;
+            if (i != j && ranges_overlap(jobs[j].y_bf16, ybytes, jobs[i].y_bf16, (size_t)m * (size_t)jobs[i].w->n * 2))
+                return CONVROT_ERR_INVALID_ARG;
+        }
+    }
+    return CONVROT_OK;
+}
+
+// Workspace layout of the layer entry points: [GEMM scratch][xq_0][sx_0][xq_1][sx_1]...
+struct LinearLayout {
+    bool batched_gemm;
+    convrot::GemmPlan batch;       // when batched_gemm
+    size_t gemm_bytes;
+    size_t total;
+};
+
+void linear_layout(int64_t m, int count, const convrot_linear_job_t *jobs, int sms, LinearLayout *L) {
+    L->batched_gemm = (m <= 256);
+    size_t g = 0;
+    if (L->batched_gemm) {
+        int64_t n[kMaxBatch], k[kMaxBatch];
+        for (int j = 0; j < count; ++j) {
+            n[j] = jobs[j].w->n;
+            k[j] = jobs[j].w->k;
+        }
+        convrot::plan_gemm_batch(m, count, n, k, sms, &L->batch);
+        g = L->batch.ws_bytes;
+    } else {
+        for (int j = 0; j < count; ++j) {
+            convrot::GemmPlan p;
+            convrot::plan_gemm(m, jobs[j].w->n, jobs[j].w->k, sms, &p);
+            g = p.ws_bytes > g ? p.ws_bytes : g;
+        }
+    }
+    L->gemm_bytes = round256(g);
+    size_t t = L->gemm_bytes;
+    for (int j = 0; j < count; ++j) t += round256((size_t)m * (size_t)jobs[j].w->k) + round256((size_t)m * 4);
+    L->total = t;
+}
+
+convrot_status_t run_linear(int64_t m, int count, const convrot_linear_job_t *jobs, void *ws, size_t ws_bytes,
+                            cudaStream_t st) {
+    if (!ws) return CONVROT_ERR_WORKSPACE;
+    if (!aligned16(ws)) return CONVROT_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    convrot_status_t s = current_device(&dev);
+    if (s != CONVROT_OK) return s;
+    LinearLayout L;
+    linear_layout(m, count, jobs, dev.num_sms, &L);
+    if (ws_bytes < L.total) return CONVROT_ERR_WORKSPACE;
     uint8_t *base = static_cast<uint8_t *>(ws);
-    int8_t *xq = reinterpret_cast<int8_t *>(base + gemm_ws);
-    float *sx = reinterpret_cast<float *>(base + gemm_ws + round256((size_t)m * (size_t)w->k));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = convrot::launch_rotate_quant(x_bf16, m, w->k, xq, sx, st, true);
+    convrot::RQProblem rq[kMaxBatch];
+    convrot::GemmProblem gp[kMaxBatch];
+    size_t off = L.gemm_bytes;
+    for (int j = 0; j < count; ++j) {
+        int8_t *xq = reinterpret_cast<int8_t *>(base + off);
+        off += round256((size_t)m * (size_t)jobs[j].w->k);
+        float *sx = reinterpret_cast<float *>(base + off);
+        off += round256((size_t)m * 4);
+        rq[j] = {jobs[j].x_bf16, jobs[j].w->k, xq, sx};
+        gp[j] = {m, jobs[j].w->n, jobs[j].w->k, xq, sx, jobs[j].w->q, jobs[j].w->scale,
+                 static_cast<__nv_bfloat16 *>(jobs[j].y_bf16), nullptr};
+    }
+    cudaError_t e = convrot::launch_rotate_quant(count, m, rq, st, true);
     if (e != cudaSuccess) return from_cuda(e);
-    return from_cuda(convrot::launch_gemm_i8(p, xq, sx, m, w->q, w->scale, w->n, w->k,
-                                             static_cast<__nv_bfloat16 *>(y_bf16), nullptr, base, st, true, true));
+    if (L.batched_gemm) return from_cuda(convrot::launch_gemm_i8(L.batch, gp, base, st, true, true));
+    for (int j = 0; j < count; ++j) {
+        convrot::GemmPlan p;
+        convrot::plan_gemm(m, jobs[j].w->n, jobs[j].w->k, dev.num_sms, &p);
+        // the first product may prefetch weights under the prologue; later
+        // ones follow another GEMM that could still be reading the scratch
+        e = convrot::launch_gemm_i8(p, &gp[j], base, st, true, j == 0);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
+    return CONVROT_OK;
+}
+
+}  // namespace
+
+namespace {
+
+convrot_status_t check_gemm_jobs(int64_t m, int count, const convrot_gemm_job_t *jobs) {
+    if (!jobs || count < 1 || count > kMaxBatch || m < 1 || m > 256) return CONVROT_ERR_INVALID_ARG;
+    for (int j = 0; j < count; ++j) {
+        const convrot_gemm_job_t &J = jobs[j];
+        if (!J.xq || !J.sx || (!J.y_bf16 && !J.acc)) return CONVROT_ERR_INVALID_ARG;
+        convrot_status_t s = check_weight(J.w);
+        if (s != CONVROT_OK) return s;
+        if ((s = check_shape(m, J.w->k, J.w->group)) != CONVROT_OK) return s;
+        if (!aligned16(J.xq) || !aligned16(J.sx) || (J.y_bf16 && !aligned16(J.y_bf16)) ||
+            (J.acc && !aligned16(J.acc)))
+            return CONVROT_ERR_ALIGNMENT;
+    }
+    return CONVROT_OK;
+}
+
+void gemm_batch_plan(int64_t m, int count, const convrot_gemm_job_t *jobs, int sms, convrot::GemmPlan *p) {
+    int64_t n[kMaxBatch], k[kMaxBatch];
+    for (int j = 0; j < count; ++j) {
+        n[j] = jobs[j].w->n;
+        k[j] = jobs[j].w->k;
+    }
+    convrot::plan_gemm_batch(m, count, n, k, sms, p);
+}
+
+}  // namespace
+
+size_t convrot_gemm_batch_workspace_bytes(int64_t m, int count, const convrot_gemm_job_t *jobs) {
+    if (check_gemm_jobs(m, count, jobs) != CONVROT_OK) return 0;
+    convrot::GemmPlan p;
+    gemm_batch_plan(m, count, jobs, sms_for_sizing(), &p);
+    return round256(p.ws_bytes);
+}
+
+convrot_status_t convrot_gemm_i8_batch(int64_t m, int count, const convrot_gemm_job_t *jobs, void *ws,
+                                       size_t ws_bytes, void *stream) {
+    convrot_status_t s = check_gemm_jobs(m, count, jobs);
+    if (s != CONVROT_OK) return s;
+    if (ws && !aligned16(ws)) return CONVROT_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    if ((s = current_device(&dev)) != CONVROT_OK) return s;
+    convrot::GemmPlan p;
+    gemm_batch_plan(m, count, jobs, dev.num_sms, &p);
+    if (!ws || ws_bytes < p.ws_bytes) return CONVROT_ERR_WORKSPACE;
+    convrot::GemmProblem gp[kMaxBatch];
+    for (int j = 0; j < count; ++j)
+        gp[j] = {m, jobs[j].w->n, jobs[j].w->k, jobs[j].xq, jobs[j].sx, jobs[j].w->q, jobs[j].w->scale,
+                 static_cast<__nv_bfloat16 *>(jobs[j].y_bf16), jobs[j].acc};
+    return from_cuda(convrot::launch_gemm_i8(p, gp, ws, static_cast<cudaStream_t>(stream), false, false));
+}
+
+size_t convrot_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+    if (m < 1 || n < 1 || k < kGroup) return 0;
+    convrot_weight_t w = {nullptr, nullptr, n, k, (int32_t)kGroup};
+    convrot_linear_job_t job = {nullptr, &w, nullptr};
+    LinearLayout L;
+    linear_layout(m, 1, &job, sms_for_sizing(), &L);
+    return L.total;
+}
+
+convrot_status_t convrot_linear_int8(const void *x_bf16, int64_t m, const convrot_weight_t *w, void *y_bf16,
+                                     void *ws, size_t ws_bytes, void *stream) {
+    convrot_linear_job_t job = {x_bf16, w, y_bf16};
+    convrot_status_t s = check_jobs(m, 1, &job);
+    if (s != CONVROT_OK) return s;
+    return run_linear(m, 1, &job, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t convrot_linear_batch_workspace_bytes(int64_t m, int count, const convrot_linear_job_t *jobs) {
+    if (check_jobs(m, count, jobs) != CONVROT_OK) return 0;
+    LinearLayout L;
+    linear_layout(m, count, jobs, sms_for_sizing(), &L);
+    return L.total;
+}
+
+convrot_status_t convrot_linear_int8_batch(int64_t m, int count, const convrot_linear_job_t *jobs, void *ws,
+                                           size_t ws_bytes, void *stream) {
+    convrot_status_t s = check_jobs(m, count, jobs);
+    if (s != CONVROT_OK) return s;
+    return run_linear(m, count, jobs, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 convrot_status_t convrot_device_status(void *stream) {

@@ -31,6 +31,7 @@
 // per-tile ticket counter, no spin-waiting) reads the total, applies the
 // epilogue and returns the workspace tile and the counter to zero.
 #include <cstdint>
+#include <cstring>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -50,33 +51,46 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// Work of one CTA: a list of segments (tile, kb0, kb1), first the whole
-// tiles of the data-parallel waves, then its contiguous share of the
-// stream-K tail.
+// Work of one CTA: a list of segments (job, tile, kb0, kb1), first the
+// whole tiles of the data-parallel waves (single-job launches), then its
+// contiguous share of the stream-K units.  A stream-K segment never crosses
+// a tile or a job boundary.
+struct Segment {
+    int job, tile, kb0, kb1, slot;
+};
+
 struct SegmentIter {
-    int wave;
+    int wave, j;
     long long u, u_end;
     __device__ __forceinline__ void init(const GemmArgs &a) {
         wave = 0;
+        j = 0;
         const long long c = blockIdx.x, G = gridDim.x;
         u = a.tail_units * c / G;
         u_end = a.tail_units * (c + 1) / G;
     }
-    __device__ __forceinline__ bool next(const GemmArgs &a, int &tile, int &kb0, int &kb1) {
+    __device__ __forceinline__ bool next(const GemmArgs &a, Segment &s) {
         if (wave < a.full_waves) {
-            tile = wave * (int)gridDim.x + (int)blockIdx.x;
-            kb0 = 0;
-            kb1 = a.kbpt;
+            s.job = 0;
+            s.tile = wave * (int)gridDim.x + (int)blockIdx.x;
+            s.kb0 = 0;
+            s.kb1 = a.job[0].kbpt;
+            s.slot = -1;
             ++wave;
             return true;
         }
         if (u < u_end) {
-            const long long t = u / a.kbpt;
-            tile = a.tail_tile0 + (int)t;
-            kb0 = (int)(u - t * a.kbpt);
-            long long rem = u_end - u;
-            kb1 = (int)((long long)kb0 + rem < a.kbpt ? kb0 + rem : a.kbpt);
-            u += kb1 - kb0;
+            while (j + 1 < a.njobs && u >= a.job[j + 1].unit0) ++j;
+            const GemmJob &J = a.job[j];
+            const long long lu = u - J.unit0;
+            const long long t = lu / J.kbpt;
+            s.job = j;
+            s.tile = J.tile_base + (int)t;
+            s.slot = J.slot0 + (int)t;
+            s.kb0 = (int)(lu - t * J.kbpt);
+            const long long rem = u_end - u;
+            s.kb1 = (int)((long long)s.kb0 + rem < J.kbpt ? s.kb0 + rem : J.kbpt);
+            u += s.kb1 - s.kb0;
             return true;
         }
         return false;
@@ -84,54 +98,54 @@ struct SegmentIter {
 };
 
 // Dequantise and store 16 consecutive B-rows (j0 .. j0+15) of one A-row i.
-__device__ __forceinline__ void emit16(const GemmArgs &a, int i, int j0, const int32_t (&v)[16]) {
-    if (!a.swap) {
+__device__ __forceinline__ void emit16(const GemmJob &J, int swap, int i, int j0, const int32_t (&v)[16]) {
+    if (!swap) {
         const int m = i;
-        if (m >= a.m) return;
-        const float sxm = a.sx[m];
-        const bool full = (j0 + 16 <= a.n) && ((a.n & 7) == 0);
-        if (a.acc) {
-            int32_t *dst = a.acc + (size_t)m * a.n + j0;
-            if (full && (a.n & 3) == 0) {
+        if (m >= J.m) return;
+        const float sxm = J.sx[m];
+        const bool full = (j0 + 16 <= J.n) && ((J.n & 7) == 0);
+        if (J.acc) {
+            int32_t *dst = J.acc + (size_t)m * J.n + j0;
+            if (full) {
 #pragma unroll
                 for (int e = 0; e < 16; e += 4)
                     *reinterpret_cast<int4 *>(dst + e) = make_int4(v[e], v[e + 1], v[e + 2], v[e + 3]);
             } else {
-                for (int e = 0; e < 16 && j0 + e < a.n; ++e) dst[e] = v[e];
+                for (int e = 0; e < 16 && j0 + e < J.n; ++e) dst[e] = v[e];
             }
         }
-        if (a.y) {
-            __nv_bfloat16 *dst = a.y + (size_t)m * a.n + j0;
+        if (J.y) {
+            __nv_bfloat16 *dst = J.y + (size_t)m * J.n + j0;
             if (full) {
                 uint32_t pk[8];
 #pragma unroll
                 for (int e = 0; e < 16; e += 2) {
-                    float f0 = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), __ldg(a.sw + j0 + e));
-                    float f1 = __fmul_rn(__fmul_rn(__int2float_rn(v[e + 1]), sxm), __ldg(a.sw + j0 + e + 1));
+                    float f0 = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), __ldg(J.sw + j0 + e));
+                    float f1 = __fmul_rn(__fmul_rn(__int2float_rn(v[e + 1]), sxm), __ldg(J.sw + j0 + e + 1));
                     __nv_bfloat162 h = __halves2bfloat162(__float2bfloat16_rn(f0), __float2bfloat16_rn(f1));
                     pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
                 }
                 reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 reinterpret_cast<uint4 *>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             } else {
-                for (int e = 0; e < 16 && j0 + e < a.n; ++e) {
-                    float f = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), __ldg(a.sw + j0 + e));
+                for (int e = 0; e < 16 && j0 + e < J.n; ++e) {
+                    float f = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), __ldg(J.sw + j0 + e));
                     dst[e] = __float2bfloat16_rn(f);
                 }
             }
         }
     } else {
         const int n = i;
-        if (n >= a.n) return;
-        const float swn = a.sw[n];
+        if (n >= J.n) return;
+        const float swn = J.sw[n];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int m = j0 + e;
-            if (m < a.m) {
-                if (a.acc) a.acc[(size_t)m * a.n + n] = v[e];
-                if (a.y) {
-                    float f = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), __ldg(a.sx + m)), swn);
-                    a.y[(size_t)m * a.n + n] = __float2bfloat16_rn(f);
+            if (m < J.m) {
+                if (J.acc) J.acc[(size_t)m * J.n + n] = v[e];
+                if (J.y) {
+                    float f = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), __ldg(J.sx + m)), swn);
+                    J.y[(size_t)m * J.n + n] = __float2bfloat16_rn(f);
                 }
             }
         }
@@ -139,8 +153,7 @@ __device__ __forceinline__ void emit16(const GemmArgs &a, int i, int j0, const i
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const GemmArgs a) {
+    gemm_i8_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled operand tiles
     const uint32_t raw = smem_addr(smem_raw);
@@ -180,9 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         *ticket = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
+    if (warp == 0 && lane < a.njobs) {
+        tma_prefetch_desc(&maps.a[lane]);
+        tma_prefetch_desc(&maps.b[lane]);
     }
     if (warp == 1) {
         tmem_alloc(smem_addr((const void *)tmem_slot), (uint32_t)a.tmem_cols);
@@ -205,17 +218,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (waited) pdl_wait();
             // activation loads held back until the grid dependency resolves
             int pend_n = 0;
-            int pend_stage[kMaxStages], pend_x[kMaxStages], pend_y[kMaxStages];
+            int pend_stage[kMaxStages], pend_x[kMaxStages], pend_y[kMaxStages], pend_job[kMaxStages];
             uint32_t issued_mask = 0, issued_par = 0;
-            const CUtensorMap *tmW = a.swap ? &tmA : &tmB;
-            const CUtensorMap *tmX = a.swap ? &tmB : &tmA;
             SegmentIter it;
             it.init(a);
-            int tile, kb0, kb1;
+            Segment sg;
             bool ok = true;
-            while (ok && it.next(a, tile, kb0, kb1)) {
-                const int ta = tile % a.tiles_a, tb = tile / a.tiles_a;
-                for (int kb = kb0; kb < kb1; ++kb) {
+            while (ok && it.next(a, sg)) {
+                const GemmJob &J = a.job[sg.job];
+                const int ta = sg.tile % J.tiles_a, tb = sg.tile / J.tiles_a;
+                const CUtensorMap *tmW = a.swap ? &maps.a[sg.job] : &maps.b[sg.job];
+                const CUtensorMap *tmX = a.swap ? &maps.b[sg.job] : &maps.a[sg.job];
+                const int rowW = a.swap ? ta * kTileA : tb * a.bn;
+                const int rowX = a.swap ? tb * a.bn : ta * kTileA;
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!mbar_wait_bounded(empty_bar + 8u * stage, phase ^ 1u, abort_flag)) {
                         ok = false;
                         break;
@@ -226,8 +242,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sb = base + b_off + (uint32_t)stage * b_bytes;
                     const int kx = kb * kBlockK;
                     const uint32_t sW = a.swap ? sa : sb, sX = a.swap ? sb : sa;
-                    const int rowW = a.swap ? ta * kTileA : tb * a.bn;
-                    const int rowX = a.swap ? tb * a.bn : ta * kTileA;
                     tma_load_2d(sW, tmW, fb, kx, rowW);
                     if (waited) {
                         tma_load_2d(sX, tmX, fb, kx, rowX);
@@ -235,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pend_stage[pend_n] = stage;
                         pend_x[pend_n] = kx;
                         pend_y[pend_n] = rowX;
+                        pend_job[pend_n] = sg.job;
                         if (++pend_n == S) {
                             pdl_wait();
                             waited = true;
@@ -242,7 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const int st = pend_stage[p];
                                 const uint32_t sxa = a.swap ? base + b_off + (uint32_t)st * b_bytes
                                                             : base + a_off + (uint32_t)st * kATileBytes;
-                                tma_load_2d(sxa, tmX, full_bar + 8u * st, pend_x[p], pend_y[p]);
+                                const CUtensorMap *tp = a.swap ? &maps.b[pend_job[p]] : &maps.a[pend_job[p]];
+                                tma_load_2d(sxa, tp, full_bar + 8u * st, pend_x[p], pend_y[p]);
                             }
                             pend_n = 0;
                         }
@@ -261,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int st = pend_stage[p];
                     const uint32_t sxa = a.swap ? base + b_off + (uint32_t)st * b_bytes
                                                 : base + a_off + (uint32_t)st * kATileBytes;
-                    tma_load_2d(sxa, tmX, full_bar + 8u * st, pend_x[p], pend_y[p]);
+                    const CUtensorMap *tp = a.swap ? &maps.b[pend_job[p]] : &maps.a[pend_job[p]];
+                    tma_load_2d(sxa, tp, full_bar + 8u * st, pend_x[p], pend_y[p]);
                 }
             }
             if (!ok) {
@@ -282,9 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             int seg = 0;
             SegmentIter it;
             it.init(a);
-            int tile, kb0, kb1;
+            Segment sg;
             bool ok = true;
-            while (ok && it.next(a, tile, kb0, kb1)) {
+            while (ok && it.next(a, sg)) {
                 const int buf = seg & 1;
                 const uint32_t use = (uint32_t)(seg >> 1);
                 if (!mbar_wait_bounded(tempty_bar + 8u * buf, (use & 1u) ^ 1u, abort_flag)) {
@@ -293,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(buf * a.acc_cols);
-                for (int kb = kb0; kb < kb1; ++kb) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!mbar_wait_bounded(full_bar + 8u * stage, phase, abort_flag)) {
                         ok = false;
                         break;
@@ -304,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / kUmmaK; ++kk) {
                         // advance the start address by 32 bytes (2 x 16 B) along K
-                        umma_i8(d, da + 2u * kk, db + 2u * kk, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                        umma_i8(d, da + 2u * kk, db + 2u * kk, idesc, (kb > sg.kb0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(empty_bar + 8u * stage);
                     if (++stage == S) {
@@ -331,16 +348,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         int seg = 0;
         SegmentIter it;
         it.init(a);
-        int tile, kb0, kb1;
-        while (it.next(a, tile, kb0, kb1)) {
-            const int ta = tile % a.tiles_a, tb = tile / a.tiles_a;
+        Segment sg;
+        while (it.next(a, sg)) {
+            const GemmJob &J = a.job[sg.job];
+            const int ta = sg.tile % J.tiles_a, tb = sg.tile / J.tiles_a;
             const int buf = seg & 1;
             const uint32_t use = (uint32_t)(seg >> 1);
             if (!mbar_wait_bounded(tfull_bar + 8u * buf, use & 1u, abort_flag)) break;
             tc_fence_after();
             const int i = ta * kTileA + row;
-            const bool whole = (kb0 == 0 && kb1 == a.kbpt);
-            const int slot = tile - a.tail_tile0;
+            const bool whole = (sg.kb0 == 0 && sg.kb1 == J.kbpt);
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * a.acc_cols);
             for (int c = 0; c < a.bn / 16; ++c) {
                 uint32_t r[16];
@@ -351,9 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
                 if (whole) {
-                    emit16(a, i, tb * a.bn + c * 16, v);
+                    emit16(J, a.swap, i, tb * a.bn + c * 16, v);
                 } else {
-                    int32_t *p = a.partial + ((size_t)slot * a.bn + c * 16) * kTileA + row;
+                    int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         if (v[e] != 0) atomicAdd(p + (size_t)e * kTileA, v[e]);
@@ -366,24 +383,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __threadfence();
                 named_bar_sync(1, 128);
                 if (ew == 0 && lane == 0) {
-                    const int mine = kb1 - kb0;
-                    const int old = atomicAdd(a.counters + slot, mine);
-                    *ticket = (old + mine == a.kbpt) ? 1 : 0;
+                    const int mine = sg.kb1 - sg.kb0;
+                    const int old = atomicAdd(a.counters + sg.slot, mine);
+                    *ticket = (old + mine == J.kbpt) ? 1 : 0;
                 }
                 named_bar_sync(1, 128);
                 const bool last = (*ticket != 0);
                 if (last) {
                     __threadfence();
                     for (int c = 0; c < a.bn / 16; ++c) {
-                        int32_t *p = a.partial + ((size_t)slot * a.bn + c * 16) * kTileA + row;
+                        int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
                         int32_t v[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = __ldcg(p + (size_t)e * kTileA);
 #pragma unroll
                         for (int e = 0; e < 16; ++e) __stcg(p + (size_t)e * kTileA, 0);
-                        emit16(a, i, tb * a.bn + c * 16, v);
+                        emit16(J, a.swap, i, tb * a.bn + c * 16, v);
                     }
-                    if (ew == 0 && lane == 0) a.counters[slot] = 0;
+                    if (ew == 0 && lane == 0) a.counters[sg.slot] = 0;
                 }
                 named_bar_sync(1, 128);
             }
@@ -401,21 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
-    p->swap = (m <= 256) ? 1 : 0;
-    p->bn = p->swap ? (int)((m + 15) / 16 * 16) : 256;
-    p->rows_a = p->swap ? n : m;
-    p->rows_b = p->swap ? m : n;
-    p->tiles_a = (int)((p->rows_a + kTileA - 1) / kTileA);
-    p->tiles_b = (int)((p->rows_b + p->bn - 1) / p->bn);
-    p->kbpt = (int)(k / kBlockK);
-    p->num_tiles = p->tiles_a * p->tiles_b;
-    const long long units = (long long)p->num_tiles * p->kbpt;
-    p->grid = (int)(units < num_sms ? units : num_sms);
-    p->full_waves = p->num_tiles / p->grid;
-    p->tail_tile0 = p->full_waves * p->grid;
-    p->tail_tiles = p->num_tiles - p->tail_tile0;
-    p->tail_units = (long long)p->tail_tiles * p->kbpt;
+static void plan_common(GemmPlan *p) {
     const int stage_bytes = kATileBytes + p->bn * kBlockK;
     int stages = (200 * 1024) / stage_bytes;
     if (stages > kMaxStages) stages = kMaxStages;
@@ -426,11 +429,61 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
     while (cols < 2 * p->bn) cols <<= 1;
     p->tmem_cols = cols;
     p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + 5) + 16;
-    // workspace: counters, then INT32 partial tiles [tail_tiles][bn][128]
-    const size_t cnt = ((size_t)p->tail_tiles * 4 + 255) / 256 * 256;
+    // workspace: counters, then INT32 partial tiles [slots][bn][128]
+    const size_t cnt = ((size_t)p->slots * 4 + 255) / 256 * 256;
     p->ws_counters_off = 0;
     p->ws_partial_off = cnt;
-    p->ws_bytes = cnt + (size_t)p->tail_tiles * p->bn * kTileA * 4;
+    p->ws_bytes = cnt + (size_t)p->slots * p->bn * kTileA * 4;
+}
+
+void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
+    *p = GemmPlan{};
+    p->njobs = 1;
+    p->swap = (m <= 256) ? 1 : 0;
+    p->bn = p->swap ? (int)((m + 15) / 16 * 16) : 256;
+    p->rows_a[0] = p->swap ? n : m;
+    p->rows_b[0] = p->swap ? m : n;
+    const int tiles_a = (int)((p->rows_a[0] + kTileA - 1) / kTileA);
+    const int tiles_b = (int)((p->rows_b[0] + p->bn - 1) / p->bn);
+    const int kbpt = (int)(k / kBlockK);
+    const int num_tiles = tiles_a * tiles_b;
+    const long long units = (long long)num_tiles * kbpt;
+    p->grid = (int)(units < num_sms ? units : num_sms);
+    p->full_waves = num_tiles / p->grid;
+    const int tail_tile0 = p->full_waves * p->grid;
+    p->slots = num_tiles - tail_tile0;
+    p->tail_units = (long long)p->slots * kbpt;
+    p->tiles_a[0] = tiles_a;
+    p->kbpt[0] = kbpt;
+    p->tile_base[0] = tail_tile0;
+    p->slot0[0] = 0;
+    p->unit0[0] = 0;
+    plan_common(p);
+}
+
+void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p) {
+    *p = GemmPlan{};
+    p->njobs = njobs;
+    p->swap = 1;
+    p->bn = (int)((m + 15) / 16 * 16);
+    long long units = 0;
+    int slots = 0;
+    for (int j = 0; j < njobs; ++j) {
+        p->rows_a[j] = n[j];
+        p->rows_b[j] = m;
+        p->tiles_a[j] = (int)((n[j] + kTileA - 1) / kTileA);
+        p->kbpt[j] = (int)(k[j] / kBlockK);
+        p->tile_base[j] = 0;
+        p->slot0[j] = slots;
+        p->unit0[j] = units;
+        slots += p->tiles_a[j];
+        units += (long long)p->tiles_a[j] * p->kbpt[j];
+    }
+    p->grid = (int)(units < num_sms ? units : num_sms);
+    p->full_waves = 0;
+    p->slots = slots;
+    p->tail_units = units;
+    plan_common(p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -465,36 +518,43 @@ static bool make_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int64_t k
     return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gemm_i8(const GemmPlan &p, const int8_t *xq, const float *sx, int64_t m,
-                           const int8_t *wq, const float *sw, int64_t n, int64_t k, __nv_bfloat16 *y,
-                           int32_t *acc, void *ws, cudaStream_t stream, bool pdl, bool w_prefetch) {
-    CUtensorMap tmA, tmB;
-    const int8_t *A = p.swap ? wq : xq;
-    const int8_t *B = p.swap ? xq : wq;
-    if (!make_tmap(&tmA, A, p.rows_a, k, kTileA)) return cudaErrorInvalidValue;
-    if (!make_tmap(&tmB, B, p.rows_b, k, p.bn)) return cudaErrorInvalidValue;
-
-    GemmArgs a = {};
-    a.m = (int)m;
-    a.n = (int)n;
-    a.k = (int)k;
+cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws, cudaStream_t stream,
+                           bool pdl, bool w_prefetch) {
+    GemmMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.njobs = p.njobs;
     a.bn = p.bn;
     a.swap = p.swap;
-    a.tiles_a = p.tiles_a;
-    a.kbpt = p.kbpt;
     a.full_waves = p.full_waves;
-    a.tail_tile0 = p.tail_tile0;
     a.tail_units = p.tail_units;
     a.stages = p.stages;
     a.acc_cols = p.acc_cols;
     a.tmem_cols = p.tmem_cols;
     a.w_prefetch = w_prefetch ? 1 : 0;
-    a.sx = sx;
-    a.sw = sw;
-    a.y = y;
-    a.acc = acc;
     a.counters = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + p.ws_counters_off);
     a.partial = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + p.ws_partial_off);
+    for (int j = 0; j < p.njobs; ++j) {
+        const GemmProblem &q = probs[j];
+        const int8_t *A = p.swap ? q.wq : q.xq;
+        const int8_t *B = p.swap ? q.xq : q.wq;
+        if (!make_tmap(&maps.a[j], A, p.rows_a[j], q.k, kTileA)) return cudaErrorInvalidValue;
+        if (!make_tmap(&maps.b[j], B, p.rows_b[j], q.k, p.bn)) return cudaErrorInvalidValue;
+        GemmJob &J = a.job[j];
+        J.m = (int)q.m;
+        J.n = (int)q.n;
+        J.k = (int)q.k;
+        J.tiles_a = p.tiles_a[j];
+        J.kbpt = p.kbpt[j];
+        J.tile_base = p.tile_base[j];
+        J.slot0 = p.slot0[j];
+        J.unit0 = p.unit0[j];
+        J.sx = q.sx;
+        J.sw = q.sw;
+        J.y = q.y;
+        J.acc = q.acc;
+    }
 
     static bool configured[64] = {};
     int dev = 0;
@@ -516,7 +576,7 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const int8_t *xq, const float *sx,
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel, tmA, tmB, a);
+    return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel, maps, a);
 }
 
 }  // namespace convrot

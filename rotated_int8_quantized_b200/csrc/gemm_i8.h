@@ -1,56 +1,98 @@
-// gemm_i8.h -- internal interface of the tcgen05 INT8 GEMM (not part of the
+// gemm_i8.h -- internal interface of the libconvrot kernels (not part of the
 // public C ABI).
 #pragma once
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace convrot {
 
 constexpr int kMaxStages = 8;
+constexpr int kMaxJobs = 8;      // linears in one batched launch
 
-// Kernel arguments (passed by value).
-struct GemmArgs {
+// ------------------------------------------------------------------ GEMM
+// One product of a (batched) launch, as the kernel sees it.
+struct GemmJob {
     int m, n, k;
-    int bn;            // UMMA N: rows of a B tile
-    int swap;          // 1: A = weights, B = activations; 0: A = activations, B = weights
-    int tiles_a;       // 128-row tiles of A
-    int kbpt;          // 128-byte K blocks per tile
-    int full_waves;    // data-parallel waves of whole tiles
-    int tail_tile0;    // first tile of the stream-K tail
-    long long tail_units;  // K blocks in the tail
-    int stages;
-    int acc_cols;      // TMEM columns per accumulator buffer
-    int tmem_cols;     // TMEM columns allocated (power of two >= 32)
-    int w_prefetch;    // load weight tiles before the grid-dependency wait
+    int tiles_a;        // 128-row tiles of the A operand
+    int kbpt;           // 128-byte K blocks per tile
+    int tile_base;      // first tile of this job handled by stream-K
+    int slot0;          // first workspace slot of this job
+    long long unit0;    // first stream-K unit (K block) of this job
     const float *sx;
     const float *sw;
     __nv_bfloat16 *y;
     int32_t *acc;
-    int32_t *partial;  // [tail tiles][bn][128] INT32, zero on entry and exit
-    int32_t *counters; // [tail tiles], zero on entry and exit
 };
 
-// Host-side tiling of one problem.
+struct GemmArgs {
+    int njobs;
+    int bn;             // UMMA N: rows of a B tile (same for every job)
+    int swap;           // 1: A = weights, B = activations; 0: A = activations, B = weights
+    int full_waves;     // data-parallel waves of whole tiles (single job only)
+    long long tail_units;   // K blocks dealt out by stream-K
+    int stages;
+    int acc_cols;       // TMEM columns per accumulator buffer
+    int tmem_cols;      // TMEM columns allocated (power of two >= 32)
+    int w_prefetch;     // load weight tiles before the grid-dependency wait
+    int32_t *partial;   // [slots][bn][128] INT32, zero on entry and exit
+    int32_t *counters;  // [slots], zero on entry and exit
+    GemmJob job[kMaxJobs];
+};
+
+struct GemmMaps {
+    CUtensorMap a[kMaxJobs];
+    CUtensorMap b[kMaxJobs];
+};
+
+// One problem as the host describes it.
+struct GemmProblem {
+    int64_t m, n, k;
+    const int8_t *xq;
+    const float *sx;
+    const int8_t *wq;
+    const float *sw;
+    __nv_bfloat16 *y;
+    int32_t *acc;
+};
+
+// Host-side tiling of a launch.
 struct GemmPlan {
-    int swap, bn;
-    int64_t rows_a, rows_b;
-    int tiles_a, tiles_b, kbpt, num_tiles;
-    int grid, full_waves, tail_tile0, tail_tiles;
+    int njobs, swap, bn;
+    int grid, full_waves, stages, acc_cols, tmem_cols, smem_bytes;
     long long tail_units;
-    int stages, acc_cols, tmem_cols, smem_bytes;
+    int tiles_a[kMaxJobs], kbpt[kMaxJobs], tile_base[kMaxJobs], slot0[kMaxJobs];
+    long long unit0[kMaxJobs];
+    int64_t rows_a[kMaxJobs], rows_b[kMaxJobs];
+    int slots;
     size_t ws_counters_off, ws_partial_off, ws_bytes;
 };
 
+// Single product: whole tiles dealt round-robin in full waves, the last
+// partial wave split along K (stream-K).
 void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p);
+// Several products with the same m <= 256 in one launch: every K block of
+// every weight dealt out evenly by stream-K.
+void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p);
 
-cudaError_t launch_gemm_i8(const GemmPlan &p, const int8_t *xq, const float *sx, int64_t m,
-                           const int8_t *wq, const float *sw, int64_t n, int64_t k, __nv_bfloat16 *y,
-                           int32_t *acc, void *ws, cudaStream_t stream, bool pdl, bool w_prefetch);
+cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws, cudaStream_t stream,
+                           bool pdl, bool w_prefetch);
 
-cudaError_t launch_rotate_quant(const void *a, int64_t rows, int64_t k, int8_t *q, float *s,
-                                cudaStream_t stream, bool pdl);
+// ------------------------------------------------------------------ rotation + quantisation
+struct RQProblem {
+    const void *a;      // BF16 [rows, k]
+    int64_t k;
+    int8_t *q;          // int8 [rows, k]
+    float *s;           // fp32 [rows]
+};
+
+// Rotate and quantise `rows` rows of each of `njobs` matrices (same row
+// count) in one launch.
+cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl);
+// True when one launch can take all these row lengths together.
+bool rotate_quant_batchable(int njobs, const RQProblem *probs);
 
 }  // namespace convrot

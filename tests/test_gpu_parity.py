@@ -58,7 +58,10 @@ def test_weight_quant_tiny_bit_exact(cr):
     assert np.array_equal(s.view(np.uint32), s_ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("m,k", [(1, 256), (4, 512), (3, 768), (17, 5120), (5, 25600), (2, 65536)])
+# k spans every launch shape of the kernel: one slot, several groups per
+# slot (2, 3, 4, 6 and a ragged last slot), and rows too long to stage
+@pytest.mark.parametrize("m,k", [(1, 256), (4, 512), (3, 768), (17, 5120), (2, 8448), (3, 16384),
+                                 (2, 24576), (5, 25600), (2, 38912), (2, 40960), (2, 65536)])
 def test_act_quant_bit_exact(cr, m, k):
     cs = synth.outlier_scale_fraction(synth.stream_key(m * 7 + k, 2), k, 0.01, 30.0)
     x_bits = synth.draw_np(synth.stream_key(m * 7 + k, 0), m, k, 1.0, cs)
@@ -225,3 +228,86 @@ def test_minimax_qkv_sampled(cr):
     rows_w = np.unique(np.concatenate([[0, lin.n - 1], rng.integers(0, lin.n, 14)]))
     rows_x = np.unique(np.concatenate([[0, lin.m - 1], rng.integers(0, lin.m, 14)]))
     _sampled_layer_check(cr, lin, rows_w, rows_x)
+
+
+# ---------------------------------------------------------------- batched layer entry point
+BATCH_CASES = [
+    (1, [(512, 256), (768, 384), (256, 1000)]),
+    (5, [(1280, 640), (512, 128), (2560, 1024), (768, 130)]),
+    (17, [(1024, 384), (1024, 384)]),
+    (100, [(512, 512), (1536, 256), (256, 640)]),
+    (300, [(768, 512), (512, 1000)]),      # m > 256: GEMMs run one after another
+]
+
+
+@pytest.mark.parametrize("m,shapes", BATCH_CASES)
+def test_batch_matches_oracle_and_single_calls(cr, m, shapes):
+    xs, ws_, ys, refs, singles = [], [], [], [], []
+    for idx, (k, n) in enumerate(shapes):
+        x_bits, w, ref = _gemm_case(cr, m, n, k, seed=1000 + 37 * idx + m)
+        x = from_bits(x_bits)
+        xs.append(x)
+        ws_.append(w)
+        ys.append(torch.empty((m, n), dtype=torch.bfloat16, device="cuda"))
+        refs.append(ref)
+        singles.append(cr.linear_int8(x, w, cr.make_workspace(m, w)))
+    batch = cr.LinearBatch(xs, ws_, ys)
+    batch()
+    cr.convrot_device_status()
+    for y, ref, single in zip(ys, refs, singles):
+        assert np.array_equal(to_bits(y), ref["y"])
+        assert np.array_equal(to_bits(y), to_bits(single))
+    for y in ys:
+        y.zero_()
+    batch()                            # the workspace returned to zero: same result again
+    cr.convrot_device_status()
+    for y, ref in zip(ys, refs):
+        assert np.array_equal(to_bits(y), ref["y"])
+    if m <= 256:
+        # the batched GEMM alone, INT32 accumulators out
+        xqs = [torch.from_numpy(r["xq"]).cuda() for r in refs]
+        sxs = [torch.from_numpy(r["sx"]).cuda() for r in refs]
+        accs = [torch.empty((m, w.n), dtype=torch.int32, device="cuda") for w in ws_]
+        yg = [torch.empty((m, w.n), dtype=torch.bfloat16, device="cuda") for w in ws_]
+        gb = cr.GemmBatch(xqs, sxs, ws_, yg, accs)
+        gb()
+        cr.convrot_device_status()
+        for acc, y, ref in zip(accs, yg, refs):
+            assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+            assert np.array_equal(to_bits(y), ref["y"])
+        assert int(gb.ws.count_nonzero()) == 0
+
+
+def test_batch_rejects_output_overlapping_an_input(cr):
+    w = cr.quantize_weight(torch.zeros((256, 512), dtype=torch.bfloat16, device="cuda"))
+    buf = torch.zeros((4, 512), dtype=torch.bfloat16, device="cuda")
+    y_alias = buf.view(-1)[: 4 * 256].view(4, 256)      # output inside the input's memory
+    ws = torch.zeros(1 << 22, dtype=torch.uint8, device="cuda")
+    with pytest.raises(cr.ConvrotError) as e:
+        cr.convrot_linear_int8_batch([buf], [w], [y_alias], ws)
+    assert e.value.status == 1
+
+
+def test_batch_qwen_decode_layer_full_size(cr):
+    lins = synth.qwen_layer(12)
+    dev = "cuda"
+    weights, xs, ys, singles = [], [], [], []
+    for lin in lins:
+        w_bf = lin.w_torch(dev)
+        w = cr.quantize_weight(w_bf)
+        del w_bf
+        x = lin.x_torch(dev)
+        weights.append(w)
+        xs.append(x)
+        ys.append(torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=dev))
+        singles.append(cr.linear_int8(x, w, cr.make_workspace(lin.m, w)))
+    batch = cr.LinearBatch(xs, weights, ys)
+    batch()
+    batch()
+    cr.convrot_device_status()
+    for lin, w, y, single in zip(lins, weights, ys, singles):
+        assert torch.equal(y.view(torch.int16), single.view(torch.int16))
+        rows = np.array([0, 1, lin.n // 2, lin.n - 1])
+        wq_ref, sw_ref = oracle.rotate_quantize(lin.w_rows_np(rows))
+        ref = oracle.linear_int8(lin.x_np(), wq_ref, sw_ref)
+        assert np.array_equal(to_bits(y[:, torch.as_tensor(rows, device=dev)]), ref["y"])
