@@ -46,6 +46,7 @@ constexpr int kTileA = 128;            // UMMA M
 constexpr int kBlockK = 128;           // bytes of K per stage (one 128-byte swizzle row)
 constexpr int kUmmaK = 32;             // K per tcgen05.mma kind::i8
 constexpr int kATileBytes = kTileA * kBlockK;
+constexpr int kL2PrefetchBlocks = 16;  // weight K blocks pulled into L2 ahead of the grid-dependency wait
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -251,6 +252,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pend_y[pend_n] = rowX;
                         pend_job[pend_n] = sg.job;
                         if (++pend_n == S) {
+                            // while the prologue is still running, pull the
+                            // next weight tiles of this CTA into L2 as well
+                            SegmentIter it2 = it;
+                            Segment s2 = sg;
+                            int kb2 = kb + 1;
+                            for (int pf = 0; pf < kL2PrefetchBlocks;) {
+                                if (kb2 >= s2.kb1) {
+                                    if (!it2.next(a, s2)) break;
+                                    kb2 = s2.kb0;
+                                    continue;
+                                }
+                                const GemmJob &J2 = a.job[s2.job];
+                                const int ta2 = s2.tile % J2.tiles_a, tb2 = s2.tile / J2.tiles_a;
+                                const CUtensorMap *tw2 = a.swap ? &maps.a[s2.job] : &maps.b[s2.job];
+                                tma_prefetch_l2_2d(tw2, kb2 * kBlockK, a.swap ? ta2 * kTileA : tb2 * a.bn);
+                                ++kb2;
+                                ++pf;
+                            }
                             pdl_wait();
                             waited = true;
                             for (int p = 0; p < pend_n; ++p) {

@@ -92,11 +92,48 @@ __device__ __forceinline__ float block_max(float v, float *red) {
     return r;
 }
 
-__device__ __forceinline__ int8_t quant1(float y, float s, bool zero_row) {
-    if (zero_row) return 0;
-    int q = __float2int_rn(__fdiv_rn(y, s));
-    q = q > 127 ? 127 : (q < -127 ? -127 : q);
-    return (int8_t)q;
+// Row quantisation helper: everything quant1 needs about a row's scale s.
+struct RowScale {
+    float s;        // s = fl(amax / 127)
+    float r;        // fl(1 / s), correctly rounded
+    bool zero;      // all-zero row: every code is 0
+    bool fast;      // r is finite, so the rounding test below applies
+};
+
+__device__ __forceinline__ RowScale make_row_scale(float amax) {
+    RowScale rs;
+    rs.s = __fdiv_rn(amax, 127.0f);
+    rs.zero = (amax == 0.0f);
+    rs.r = rs.zero ? 0.0f : __frcp_rn(rs.s);
+    rs.fast = !rs.zero && isfinite(rs.r);
+    return rs;
+}
+
+// q = clamp(rne(fl(y / s)), -127, 127): the integer nearest to the
+// correctly rounded FP32 quotient, ties to even.
+//
+// Evaluated with Ziv's rounding test (A. Ziv, "Fast evaluation of elementary
+// mathematical functions with correctly rounded last bit", ACM TOMS 17(3),
+// 1991): a cheap approximation with a proven error bound decides the
+// rounding whenever it lies far enough from a rounding boundary, and the
+// exact evaluation runs only otherwise.  Here t = fl(y * r) with
+// r = fl(1/s) satisfies |t - y/s| <= |y/s| (2^-23 + 2^-48) and
+// |fl(y/s) - y/s| <= |y/s| 2^-24; since |y/s| <= 127 (1 + 2^-23),
+// |t - fl(y/s)| < 2.3e-5.  When t is more than 3e-5 away from every
+// half-integer, fl(y/s) rounds to the same integer as t; otherwise (about
+// 6e-5 of the elements) the IEEE division is evaluated.
+__device__ __forceinline__ int8_t quant1(float y, const RowScale &rs) {
+    if (rs.zero) return 0;
+    float f;
+    const float t = __fmul_rn(y, rs.r);
+    const float ft = rintf(t);
+    if (rs.fast && fabsf(t - ft) < 0.49997f) {
+        f = ft;
+    } else {
+        f = rintf(__fdiv_rn(y, rs.s));
+    }
+    f = fminf(fmaxf(f, -127.0f), 127.0f);
+    return (int8_t)(int)f;
 }
 
 // One CTA per row, no staging: pass 1 finds the row maximum, pass 2
@@ -118,20 +155,19 @@ __global__ void __launch_bounds__(kRQThreads) rotate_quant_rows_twopass(
         for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(y[e]));
     }
     amax = block_max(amax, red);
-    const float sc = __fdiv_rn(amax, 127.0f);
-    const bool zero_row = (amax == 0.0f);
+    const RowScale rs = make_row_scale(amax);
     int8_t *qrow = q + (size_t)row * k;
     for (int g = warp; g < groups; g += kRQWarps) {
         float y[8];
         rotate_group(arow + g * 256, lane, y);
         uint32_t lo = 0, hi = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) lo |= (uint32_t)(uint8_t)quant1(y[e], sc, zero_row) << (8 * e);
+        for (int e = 0; e < 4; ++e) lo |= (uint32_t)(uint8_t)quant1(y[e], rs) << (8 * e);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) hi |= (uint32_t)(uint8_t)quant1(y[4 + e], sc, zero_row) << (8 * e);
+        for (int e = 0; e < 4; ++e) hi |= (uint32_t)(uint8_t)quant1(y[4 + e], rs) << (8 * e);
         *reinterpret_cast<uint2 *>(qrow + g * 256 + lane * 8) = make_uint2(lo, hi);
     }
-    if (threadIdx.x == 0) s[row] = sc;
+    if (threadIdx.x == 0) s[row] = rs.s;
 }
 
 // ---------------------------------------------------------------------------
@@ -146,6 +182,7 @@ __global__ void __launch_bounds__(kRQThreads) rotate_quant_rows_twopass(
 // ---------------------------------------------------------------------------
 constexpr int kMaxSlots = 32;          // 512 threads
 constexpr int kXchStride = 16 * 17;    // doubles per slot exchange buffer
+constexpr int kMaxParts = 8;           // CTAs per row (portable cluster size)
 constexpr int kSlotsSmemMax = 226 * 1024;   // dynamic shared memory per CTA (227 KB minus the static part)
 
 __device__ __forceinline__ void fwht16_regs(double (&v)[16]) {
@@ -171,39 +208,67 @@ struct RQJobDev {
     const __nv_bfloat16 *a;
     int8_t *q;
     float *s;
-    int k, gps, slots;
+    int k, gps, slots;      // gps / slots for the groups of ONE part of a row
 };
 struct RQArgs {
     int njobs, rows;
+    int parts;              // CTAs (a thread-block cluster) per row
     RQJobDev job[kMaxJobs];
 };
 
-// Groups per slot and slots for a row of k elements.
-static void rq_shape(int64_t k, int *gps, int *slots) {
-    const int groups = (int)(k >> 8);
+// Groups per slot and slots for `groups` groups.
+static void rq_shape(int groups, int *gps, int *slots) {
     int g = (groups + kMaxSlots - 1) / kMaxSlots;
     if (g == 5) g = 6;
+    if (g < 1) g = 1;
     *gps = g;
     *slots = (groups + g - 1) / g;
 }
 
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t caddr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// One row per CTA (parts == 1) or per cluster of `parts` CTAs: CTA p of the
+// cluster rotates groups [p*G/parts, (p+1)*G/parts) of the row, the row
+// maximum is combined through distributed shared memory, then each CTA
+// quantises its own groups.  Decode-sized matrices (a few rows) are spread
+// over many SMs this way.
 template <int GPS>
 __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
     extern __shared__ __align__(16) uint8_t rq_smem[];
     __shared__ float red[kMaxSlots / 2];
+    __shared__ float part_max;
     pdl_wait();
     pdl_launch_dependents();
 
-    const int jb = blockIdx.x / args.rows;
-    const int row = blockIdx.x - jb * args.rows;
+    const int C = args.parts;
+    const int part = (int)(blockIdx.x % (unsigned)C);
+    const int rowid = (int)(blockIdx.x / (unsigned)C);
+    const int jb = rowid / args.rows;
+    const int row = rowid - jb * args.rows;
     const RQJobDev &J = args.job[jb];
     const int k = J.k, gps = J.gps, slots = J.slots;
+    const int groups = k >> 8;
+    const int g0 = part * groups / C, g1 = (part + 1) * groups / C;
     double *xch = reinterpret_cast<double *>(rq_smem);                    // slots * 272 doubles
-    float *ybuf = reinterpret_cast<float *>(rq_smem + (size_t)(blockDim.x >> 4) * kXchStride * 8);  // k floats
+    float *ybuf = reinterpret_cast<float *>(rq_smem + (size_t)(blockDim.x >> 4) * kXchStride * 8);
 
     const int tid = threadIdx.x;
     const int slot = tid >> 4, t = tid & 15;
-    const int groups = k >> 8;
     const unsigned half_mask = 0xFFFFu << (16 * (slot & 1));
     const __nv_bfloat16 *arow = J.a + (size_t)row * k;
 
@@ -211,8 +276,8 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
     uint4 raw[GPS][2];
 #pragma unroll
     for (int gi = 0; gi < GPS; ++gi) {
-        const int g = slot + gi * slots;
-        if (gi < gps && slot < slots && g < groups) {
+        const int g = g0 + slot + gi * slots;
+        if (gi < gps && slot < slots && g < g1) {
             const uint4 *src = reinterpret_cast<const uint4 *>(arow + (size_t)g * 256 + t * 16);
             raw[gi][0] = __ldg(src);
             raw[gi][1] = __ldg(src + 1);
@@ -223,8 +288,8 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
     float amax = 0.f;
 #pragma unroll
     for (int gi = 0; gi < GPS; ++gi) {
-        const int g = slot + gi * slots;
-        if (gi < gps && slot < slots && g < groups) {
+        const int g = g0 + slot + gi * slots;
+        if (gi < gps && slot < slots && g < g1) {
             double v[16];
             const uint32_t w[8] = {raw[gi][0].x, raw[gi][0].y, raw[gi][0].z, raw[gi][0].w,
                                    raw[gi][1].x, raw[gi][1].y, raw[gi][1].z, raw[gi][1].w};
@@ -238,7 +303,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
             for (int i = 0; i < 16; ++i) v[i] = xb[t + 17 * i];
             __syncwarp(half_mask);
             fwht16_regs(v);                                  // index bits 4-7
-            float *yg = ybuf + (size_t)g * 256 + t;
+            float *yg = ybuf + (size_t)(g - g0) * 256 + t;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float y = __double2float_rn(v[i] * 0.0625);   // / sqrt(256), exact
@@ -248,7 +313,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
         }
     }
 
-    // row maximum
+    // maximum over this CTA's part of the row
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const int warp = tid >> 5, lane = tid & 31, nwarps = (blockDim.x + 31) >> 5;
@@ -256,32 +321,51 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
     __syncthreads();
     float rmax = red[0];
     for (int w = 1; w < nwarps; ++w) rmax = fmaxf(rmax, red[w]);
-    const float sc = __fdiv_rn(rmax, 127.0f);
-    const bool zero_row = (rmax == 0.0f);
+    if (C > 1) {
+        // combine the parts of the row across the cluster
+        if (tid == 0) part_max = rmax;
+        cluster_arrive();
+        cluster_wait();
+        if (tid == 0) {
+            const uint32_t local = smem_addr(&part_max);
+            float m = 0.f;
+            for (int r = 0; r < C; ++r) m = fmaxf(m, ld_cluster_f32(cluster_map(local, (uint32_t)r)));
+            red[0] = m;
+        }
+        __syncthreads();
+        rmax = red[0];
+        cluster_arrive();   // this CTA no longer reads its peers; matched by the wait before exit
+    }
+    const RowScale rs = make_row_scale(rmax);
 
     // quantise 16 consecutive outputs per thread, one 16-byte store
-    int8_t *qrow = J.q + (size_t)row * k;
-    for (int c = tid; c < (k >> 4); c += blockDim.x) {
+    int8_t *qrow = J.q + (size_t)row * k + (size_t)g0 * 256;
+    const int chunks = (g1 - g0) * 16;
+    for (int c = tid; c < chunks; c += blockDim.x) {
         const float4 *src = reinterpret_cast<const float4 *>(ybuf + c * 16);
         uint32_t packed[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float4 f = src[i];
-            uint32_t b0 = (uint8_t)quant1(f.x, sc, zero_row);
-            uint32_t b1 = (uint8_t)quant1(f.y, sc, zero_row);
-            uint32_t b2 = (uint8_t)quant1(f.z, sc, zero_row);
-            uint32_t b3 = (uint8_t)quant1(f.w, sc, zero_row);
+            uint32_t b0 = (uint8_t)quant1(f.x, rs);
+            uint32_t b1 = (uint8_t)quant1(f.y, rs);
+            uint32_t b2 = (uint8_t)quant1(f.z, rs);
+            uint32_t b3 = (uint8_t)quant1(f.w, rs);
             packed[i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
         }
         *reinterpret_cast<uint4 *>(qrow + c * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
-    if (tid == 0) J.s[row] = sc;
+    if (tid == 0 && part == 0) J.s[row] = rs.s;
+    if (C > 1) {
+        __syncwarp();
+        cluster_wait();   // peers may still read part_max until they arrive
+    }
 }
 
 template <int GPS>
-static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int max_slots, int64_t max_k) {
+static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int max_slots, int max_local_groups) {
     cfg.blockDim = dim3(max_slots * 16);
-    cfg.dynamicSmemBytes = (size_t)max_slots * kXchStride * 8 + (size_t)max_k * 4;
+    cfg.dynamicSmemBytes = (size_t)max_slots * kXchStride * 8 + (size_t)max_local_groups * 256 * 4;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -295,63 +379,95 @@ static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int
     return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS>, args);
 }
 
-// Shared-memory bytes one CTA of a batched launch needs.
-static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int *max_slots, int *max_gps, int64_t *max_k) {
-    int ms = 0, mg = 0;
-    int64_t mk = 0;
+// CTAs per row: when the rows alone do not fill the GPU, split each row over
+// a cluster of CTAs so that every SM gets work, but keep the whole grid
+// within one wave (about two CTAs per SM), so that every CTA starts at once
+// and triggers the dependent GEMM's launch early.
+static int rq_parts(int njobs, int64_t rows, int num_sms) {
+    const int64_t total_rows = rows * njobs;
+    if (total_rows >= num_sms) return 1;
+    int64_t parts = (2 * (int64_t)num_sms) / total_rows;
+    if (parts > kMaxParts) parts = kMaxParts;
+    if (parts < 1) parts = 1;
+    return (int)parts;
+}
+
+// Shared-memory bytes and shape of one CTA of a launch with `parts` CTAs per row.
+static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, int *max_slots, int *max_gps,
+                            int *max_local) {
+    int ms = 0, mg = 0, ml = 0;
     for (int j = 0; j < njobs; ++j) {
+        const int groups = (int)(probs[j].k >> 8);
+        const int local = (groups + parts - 1) / parts;
         int g, sl;
-        rq_shape(probs[j].k, &g, &sl);
+        rq_shape(local, &g, &sl);
         ms = sl > ms ? sl : ms;
         mg = g > mg ? g : mg;
-        mk = probs[j].k > mk ? probs[j].k : mk;
+        ml = local > ml ? local : ml;
     }
     *max_slots = ms;
     *max_gps = mg;
-    *max_k = mk;
-    return (size_t)ms * kXchStride * 8 + (size_t)mk * 4;
+    *max_local = ml;
+    return (size_t)ms * kXchStride * 8 + (size_t)ml * 256 * 4;
 }
 
 bool rotate_quant_batchable(int njobs, const RQProblem *probs) {
-    int ms, mg;
-    int64_t mk;
-    return njobs <= kMaxJobs && rq_smem_bytes(njobs, probs, &ms, &mg, &mk) <= (size_t)kSlotsSmemMax;
+    int ms, mg, ml;
+    return njobs <= kMaxJobs && rq_smem_bytes(njobs, probs, 1, &ms, &mg, &ml) <= (size_t)kSlotsSmemMax;
 }
 
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl) {
+    int dev = 0, num_sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    const int parts = rq_parts(njobs, rows, num_sms);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3((unsigned)(rows * njobs));
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (parts > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)parts;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.gridDim = dim3((unsigned)(rows * njobs * parts));
     cfg.blockDim = dim3(kRQThreads);
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    int max_slots, max_gps;
-    int64_t max_k;
-    if (njobs <= kMaxJobs && rq_smem_bytes(njobs, probs, &max_slots, &max_gps, &max_k) <= (size_t)kSlotsSmemMax) {
+    cfg.numAttrs = na;
+    int max_slots, max_gps, max_local;
+    if (njobs <= kMaxJobs &&
+        rq_smem_bytes(njobs, probs, parts, &max_slots, &max_gps, &max_local) <= (size_t)kSlotsSmemMax) {
         RQArgs args;
         memset(&args, 0, sizeof(args));
         args.njobs = njobs;
         args.rows = (int)rows;
+        args.parts = parts;
         for (int j = 0; j < njobs; ++j) {
             RQJobDev &J = args.job[j];
             J.a = static_cast<const __nv_bfloat16 *>(probs[j].a);
             J.q = probs[j].q;
             J.s = probs[j].s;
             J.k = (int)probs[j].k;
-            rq_shape(probs[j].k, &J.gps, &J.slots);
+            const int groups = J.k >> 8;
+            rq_shape((groups + parts - 1) / parts, &J.gps, &J.slots);
         }
         switch (max_gps) {
-            case 1: return launch_slots<1>(cfg, args, max_slots, max_k);
-            case 2: return launch_slots<2>(cfg, args, max_slots, max_k);
-            case 3: return launch_slots<3>(cfg, args, max_slots, max_k);
-            case 4: return launch_slots<4>(cfg, args, max_slots, max_k);
-            default: return launch_slots<6>(cfg, args, max_slots, max_k);
+            case 1: return launch_slots<1>(cfg, args, max_slots, max_local);
+            case 2: return launch_slots<2>(cfg, args, max_slots, max_local);
+            case 3: return launch_slots<3>(cfg, args, max_slots, max_local);
+            case 4: return launch_slots<4>(cfg, args, max_slots, max_local);
+            default: return launch_slots<6>(cfg, args, max_slots, max_local);
         }
     }
-    // rows too long to stage: one launch per matrix, rotation recomputed in a second pass
+    // rows too long to stage: one plain launch per matrix, rotation recomputed in a second pass
+    cfg.numAttrs = pdl ? 1 : 0;
     cfg.dynamicSmemBytes = 0;
     cfg.gridDim = dim3((unsigned)rows);
     for (int j = 0; j < njobs; ++j) {

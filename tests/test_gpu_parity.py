@@ -58,10 +58,13 @@ def test_weight_quant_tiny_bit_exact(cr):
     assert np.array_equal(s.view(np.uint32), s_ref.view(np.uint32))
 
 
-# k spans every launch shape of the kernel: one slot, several groups per
-# slot (2, 3, 4, 6 and a ragged last slot), and rows too long to stage
+# m and k span every launch shape of the kernel: rows split over a cluster of
+# up to 8 CTAs (few rows), one CTA per row (>= 148 rows) with one slot or
+# several groups per slot (2, 3, 4, 6 and a ragged last slot), and rows too
+# long to stage (two-pass variant)
 @pytest.mark.parametrize("m,k", [(1, 256), (4, 512), (3, 768), (17, 5120), (2, 8448), (3, 16384),
-                                 (2, 24576), (5, 25600), (2, 38912), (2, 40960), (2, 65536)])
+                                 (2, 24576), (5, 25600), (2, 38912), (2, 40960), (2, 65536),
+                                 (150, 512), (160, 8448), (148, 25600), (149, 40960), (200, 65536)])
 def test_act_quant_bit_exact(cr, m, k):
     cs = synth.outlier_scale_fraction(synth.stream_key(m * 7 + k, 2), k, 0.01, 30.0)
     x_bits = synth.draw_np(synth.stream_key(m * 7 + k, 0), m, k, 1.0, cs)
@@ -87,6 +90,34 @@ def test_act_quant_zero_row_and_one_hot(cr):
     assert np.array_equal(xq.cpu().numpy(), q_ref)
     assert np.array_equal(sx.cpu().numpy(), s_ref)
     assert sx[0].item() == 0 and int(xq[0].abs().max()) == 0
+
+
+def test_act_quant_exact_ties(cr):
+    # rows whose rotated values fall exactly on half-integers of y / s: group 0
+    # is the constant 127 * 2^(p-4) (rotates to (127 * 2^p, 0, ...), so
+    # s = 2^p exactly), groups 1.. are constants c * 2^(p-4) (rotating to
+    # (c * 2^p, 0, ...)), so y / s = c exactly; ties must go to even
+    ties = [2.5, 3.5, -4.5, 0.5, -126.5, 1.5, -0.5, 6.5]
+    rows = []
+    for p in (0, -3, 5, -10):
+        row = np.zeros(256 * (1 + len(ties)), dtype=np.float32)
+        row[:256] = 127.0 * 2.0 ** (p - 4)
+        for g, c in enumerate(ties):
+            row[256 * (g + 1): 256 * (g + 2)] = c * 2.0 ** (p - 4)
+        rows.append(row)
+    x = np.stack(rows)
+    bits = synth.f32_to_bf16_bits(x)
+    assert np.array_equal(synth.bf16_bits_to_f32(bits), x)
+    m, k = x.shape
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+    cr.convrot_quantize_act(from_bits(bits), xq, sx)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.rotate_quantize(bits)
+    got = xq.cpu().numpy()
+    assert np.array_equal(got, q_ref)
+    assert np.array_equal(sx.cpu().numpy(), s_ref)
+    assert list(got[0, 256::256]) == [2, 4, -4, 0, -126, 2, 0, 6]
 
 
 # ---------------------------------------------------------------- K2
