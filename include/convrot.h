@@ -220,6 +220,33 @@ convrot_status_t convrot_linear_int8_batch(int64_t m, int count, const convrot_l
 size_t convrot_linear_batch_workspace_bytes(int64_t m, int count, const convrot_linear_job_t *jobs);
 
 /*
+ * convrot_gemm_i8 for callers that cannot allocate device memory: the same
+ * product and outputs (xq, sx, w, y_bf16, acc as for convrot_gemm_i8), but
+ * with no workspace argument.  Its scratch is an array of 8 MiB built into
+ * the library (held on every GPU that loads the library until the process
+ * exits).  It is meant for code that must not call cudaMalloc where it runs
+ * the layer -- for example a plugin inside an engine that owns all device
+ * memory through its own pool -- and cannot be handed a workspace either.
+ * (The source pages have no counterpart of this entry point; it is an
+ * integration convenience.)
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before
+ *     any stream capture.
+ *   - Problems whose scratch needs more than 8 MiB are rejected with
+ *     CONVROT_ERR_WORKSPACE before anything is launched
+ *     (convrot_last_error_string says so).  convrot_gemm_workspace_bytes
+ *     gives the need.
+ *   - Each call clears the part of the array it uses (an asynchronous memset
+ *     on `stream`) and then launches the GEMM; it allocates nothing.
+ *   - Every call on a device shares the one array: calls whose GPU work can
+ *     overlap (other streams, other host threads) race and corrupt each
+ *     other's results.  Serialise them.
+ */
+convrot_status_t convrot_gemm_i8_noalloc(const int8_t *xq, const float *sx, int64_t m,
+                                         const convrot_weight_t *w, void *y_bf16, int32_t *acc,
+                                         void *stream);
+
+/*
  * Synchronise `stream`, then read and clear the device-side status word of
  * the current device.  Returns CONVROT_OK, CONVROT_ERR_DEVICE_TIMEOUT if a
  * bounded wait ran out in some kernel since the last call (the workspace

@@ -77,6 +77,7 @@ SIGNATURES = {
     "convrot_linear_batch_workspace_bytes": ([_I64, ctypes.c_int, ctypes.POINTER(convrot_linear_job_t)], _SZ),
     "convrot_gemm_i8_batch": ([_I64, ctypes.c_int, ctypes.POINTER(convrot_gemm_job_t), _P, _SZ, _P], ctypes.c_int),
     "convrot_gemm_batch_workspace_bytes": ([_I64, ctypes.c_int, ctypes.POINTER(convrot_gemm_job_t)], _SZ),
+    "convrot_gemm_i8_noalloc": ([_P, _P, _I64, _WP, _P, _P, _P], ctypes.c_int),
 }
 
 _lib = None

@@ -3,3 +3,4 @@
 #include "rotate_quant.cu"
 #include "gemm_i8.cu"
 #include "api.cu"
+#include "noalloc.cu"
