@@ -10,17 +10,16 @@
 //  section 5: activations and weights both rotated, "--simple" RTN;
 //  zskr.cn "Qwen3-VL-32B ... INT8-ConvRot": "--int8 --scaling_mode row"]
 //
-// Design (B200): one warp rotates one 256-wide group.  Each lane loads 8
-// consecutive BF16 values with one 16-byte load (the warp reads the group's
-// 512 bytes fully coalesced), widens them to FP64 and runs the fast
-// Walsh-Hadamard transform: three butterfly stages inside the lane (index
-// bits 0-2) and five across lanes with xor-shuffles (index bits 3-7).  Every
-// partial sum of +-BF16 values is exact in FP64, so the butterfly order
-// gives the same exact sum as the explicit matrix product, and one rounding
-// to FP32 follows.  The row's rotated FP32 values wait in shared memory
-// while the CTA reduces the row maximum; then each thread packs 16 INT8
-// codes into one 16-byte store.  Rows too long for shared memory take a
-// two-pass variant that recomputes the (cheap, L2-resident) rotation.
+// Design (B200): the main kernel (rotate_quant_rows_slots, below) gives 16
+// threads to each 256-wide group and splits H_256 = H_16 (x) H_16; rows are
+// split over a thread-block cluster when there are too few to fill the GPU.
+// Every partial sum of +-BF16 values is exact in FP64, so any butterfly order
+// gives the exact sum of the explicit matrix product, and one rounding to
+// FP32 follows.  The row's rotated FP32 values wait in shared memory while
+// the row maximum is reduced; then each thread packs 16 INT8 codes into one
+// 16-byte store.  Rows too long for shared memory take a two-pass variant
+// (one warp per group, the 8-stage butterfly across lanes with shuffles)
+// that recomputes the L2-resident rotation instead of staging it.
 #include <cstdint>
 #include <cstring>
 #include <cuda_bf16.h>
@@ -136,6 +135,37 @@ __device__ __forceinline__ int8_t quant1(float y, const RowScale &rs) {
     return (int8_t)(int)f;
 }
 
+// The same for 16 consecutive values packed into one 16-byte word, with the
+// fast path as straight-line code (independent lanes of work for the
+// scheduler) and the exact division only where some thread of the warp
+// needs it.  Every thread of the warp must call it together (`mask` = the
+// active threads).
+__device__ __forceinline__ uint4 quant16(const float (&y)[16], const RowScale &rs, unsigned mask) {
+    float f[16];
+    bool slow = false;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float t = __fmul_rn(y[e], rs.r);
+        f[e] = rintf(t);
+        slow |= !(fabsf(t - f[e]) < 0.49997f);
+    }
+    slow = slow || !rs.fast;
+    if (__any_sync(mask, slow) && slow) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float t = __fmul_rn(y[e], rs.r);
+            if (!rs.fast || !(fabsf(t - rintf(t)) < 0.49997f)) f[e] = rintf(__fdiv_rn(y[e], rs.s));
+        }
+    }
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float c = rs.zero ? 0.0f : fminf(fmaxf(f[e], -127.0f), 127.0f);
+        w[e >> 2] |= (uint32_t)(uint8_t)(int8_t)(int)c << (8 * (e & 3));
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // One CTA per row, no staging: pass 1 finds the row maximum, pass 2
 // recomputes the rotation (the row is L2-resident) and quantises.
 __global__ void __launch_bounds__(kRQThreads) rotate_quant_rows_twopass(
@@ -174,14 +204,15 @@ __global__ void __launch_bounds__(kRQThreads) rotate_quant_rows_twopass(
 // Main variant: 16 threads ("a slot") per 256-group, H_256 = H_16 (x) H_16.
 // Thread t of a slot loads elements 16t .. 16t+15 (32 contiguous bytes; the
 // slot reads the group's 512 bytes coalesced), transforms index bits 0-3 in
-// registers, exchanges through a padded shared-memory transpose (stride 17
-// doubles: conflict-free both ways), transforms index bits 4-7 in registers
+// registers, exchanges through a padded shared-memory transpose (in two
+// halves through a 16 x 9 buffer: conflict-free both ways), transforms index
+// bits 4-7 in registers
 // and so ends up holding outputs t, t+16, ..., t+240.  Every group of a row
 // is in flight at once (up to 32 slots per CTA, several groups per slot for
 // long rows), so a decode-sized matrix of a few rows costs one load latency.
 // ---------------------------------------------------------------------------
 constexpr int kMaxSlots = 32;          // 512 threads
-constexpr int kXchStride = 16 * 17;    // doubles per slot exchange buffer
+constexpr int kXchStride = 16 * 9;     // doubles per slot exchange buffer (half a 16 x 16 transpose + padding)
 constexpr int kMaxParts = 8;           // CTAs per row (portable cluster size)
 constexpr int kSlotsSmemMax = 226 * 1024;   // dynamic shared memory per CTA (227 KB minus the static part)
 
@@ -296,17 +327,26 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
 #pragma unroll
             for (int i = 0; i < 8; ++i) bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
             fwht16_regs(v);                                  // index bits 0-3
+            // transpose across the slot's 16 threads in two halves (a 16 x 9
+            // buffer: conflict-free): thread u needs element 16*j + u of every
+            // thread j, i.e. v[u] of thread j
+            double x[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) xb[17 * t + i] = v[i];
-            __syncwarp(half_mask);
+            for (int h = 0; h < 2; ++h) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = xb[t + 17 * i];
-            __syncwarp(half_mask);
-            fwht16_regs(v);                                  // index bits 4-7
+                for (int i = 0; i < 8; ++i) xb[9 * t + i] = v[8 * h + i];
+                __syncwarp(half_mask);
+                if ((t >> 3) == h) {
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) x[jj] = xb[9 * jj + (t & 7)];
+                }
+                __syncwarp(half_mask);
+            }
+            fwht16_regs(x);                                  // index bits 4-7
             float *yg = ybuf + (size_t)(g - g0) * 256 + t;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float y = __double2float_rn(v[i] * 0.0625);   // / sqrt(256), exact
+                const float y = __double2float_rn(x[i] * 0.0625);   // / sqrt(256), exact
                 yg[16 * i] = y;
                 amax = fmaxf(amax, fabsf(y));
             }
@@ -341,19 +381,22 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
     // quantise 16 consecutive outputs per thread, one 16-byte store
     int8_t *qrow = J.q + (size_t)row * k + (size_t)g0 * 256;
     const int chunks = (g1 - g0) * 16;
-    for (int c = tid; c < chunks; c += blockDim.x) {
-        const float4 *src = reinterpret_cast<const float4 *>(ybuf + c * 16);
-        uint32_t packed[4];
+    for (int c0 = 0; c0 < chunks; c0 += blockDim.x) {
+        const int c = c0 + tid;
+        const unsigned mask = __ballot_sync(__activemask(), c < chunks);
+        if (c < chunks) {
+            const float4 *src = reinterpret_cast<const float4 *>(ybuf + c * 16);
+            float y[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float4 f = src[i];
-            uint32_t b0 = (uint8_t)quant1(f.x, rs);
-            uint32_t b1 = (uint8_t)quant1(f.y, rs);
-            uint32_t b2 = (uint8_t)quant1(f.z, rs);
-            uint32_t b3 = (uint8_t)quant1(f.w, rs);
-            packed[i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            for (int i = 0; i < 4; ++i) {
+                const float4 f = src[i];
+                y[4 * i] = f.x;
+                y[4 * i + 1] = f.y;
+                y[4 * i + 2] = f.z;
+                y[4 * i + 3] = f.w;
+            }
+            *reinterpret_cast<uint4 *>(qrow + c * 16) = quant16(y, rs, mask);
         }
-        *reinterpret_cast<uint4 *>(qrow + c * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
     if (tid == 0 && part == 0) J.s[row] = rs.s;
     if (C > 1) {

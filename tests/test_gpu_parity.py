@@ -262,12 +262,20 @@ def test_minimax_qkv_sampled(cr):
 
 
 # ---------------------------------------------------------------- batched layer entry point
+# (m, [(k, n), ...]): fewer K blocks than SMs (grid < 148), ragged N, many
+# jobs, long rows split over a cluster of up to 8 CTAs in the prologue, many
+# K blocks per SM, and m > 256, where the GEMMs run one after another
 BATCH_CASES = [
     (1, [(512, 256), (768, 384), (256, 1000)]),
     (5, [(1280, 640), (512, 128), (2560, 1024), (768, 130)]),
+    (3, [(5120, 2048), (2560, 1024)]),
+    (5, [(5120, 8192), (2560, 512)]),       # many K blocks per SM
     (17, [(1024, 384), (1024, 384)]),
+    (32, [(1024, 2048), (3072, 512), (256, 1280)]),
+    (24, [(25600, 1024)]),
     (100, [(512, 512), (1536, 256), (256, 640)]),
-    (300, [(768, 512), (512, 1000)]),      # m > 256: GEMMs run one after another
+    (64, [(25600, 640)]),
+    (300, [(768, 512), (512, 1000)]),
 ]
 
 
