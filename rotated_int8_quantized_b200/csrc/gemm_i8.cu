@@ -71,7 +71,7 @@ struct SegmentIter {
         u_end = a.tail_units * (c + 1) / G;
     }
     __device__ __forceinline__ bool next(const GemmArgs &a, Segment &s) {
-        if (wave < a.full_waves) {
+        if (wave < a.full_waves && wave * (int)gridDim.x + (int)blockIdx.x < a.full_tiles) {
             s.job = 0;
             s.tile = wave * (int)gridDim.x + (int)blockIdx.x;
             s.kb0 = 0;
@@ -467,9 +467,23 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
     const int kbpt = (int)(k / kBlockK);
     const int num_tiles = tiles_a * tiles_b;
     const long long units = (long long)num_tiles * kbpt;
-    p->grid = (int)(units < num_sms ? units : num_sms);
-    p->full_waves = num_tiles / p->grid;
-    const int tail_tile0 = p->full_waves * p->grid;
+    int tail_tile0;
+    if (p->swap) {
+        // few weight tiles: whole tiles in full waves, the rest split along K
+        // (the INT32 partial tiles are small: bn <= 256 columns x 128 rows)
+        p->grid = (int)(units < num_sms ? units : num_sms);
+        p->full_waves = num_tiles / p->grid;
+        tail_tile0 = p->full_waves * p->grid;
+        p->full_tiles = tail_tile0;
+    } else {
+        // large M: whole 128 x 256 tiles only, the last wave partly idle;
+        // splitting the last wave along K would cost a 128 KB INT32 partial
+        // flush per split tile, more than the idle SMs lose
+        p->grid = num_tiles < num_sms ? num_tiles : num_sms;
+        p->full_waves = (num_tiles + p->grid - 1) / p->grid;
+        tail_tile0 = num_tiles;
+        p->full_tiles = num_tiles;
+    }
     p->slots = num_tiles - tail_tile0;
     p->tail_units = (long long)p->slots * kbpt;
     p->tiles_a[0] = tiles_a;
@@ -547,6 +561,7 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
     a.bn = p.bn;
     a.swap = p.swap;
     a.full_waves = p.full_waves;
+    a.full_tiles = p.full_tiles;
     a.tail_units = p.tail_units;
     a.stages = p.stages;
     a.acc_cols = p.acc_cols;

@@ -33,6 +33,7 @@ struct GemmArgs {
     int bn;             // UMMA N: rows of a B tile (same for every job)
     int swap;           // 1: A = weights, B = activations; 0: A = activations, B = weights
     int full_waves;     // data-parallel waves of whole tiles (single job only)
+    int full_tiles;     // tiles those waves cover (the last wave may be partial)
     long long tail_units;   // K blocks dealt out by stream-K
     int stages;
     int acc_cols;       // TMEM columns per accumulator buffer
@@ -62,7 +63,7 @@ struct GemmProblem {
 // Host-side tiling of a launch.
 struct GemmPlan {
     int njobs, swap, bn;
-    int grid, full_waves, stages, acc_cols, tmem_cols, smem_bytes;
+    int grid, full_waves, full_tiles, stages, acc_cols, tmem_cols, smem_bytes;
     long long tail_units;
     int tiles_a[kMaxJobs], kbpt[kMaxJobs], tile_base[kMaxJobs], slot0[kMaxJobs];
     long long unit0[kMaxJobs];

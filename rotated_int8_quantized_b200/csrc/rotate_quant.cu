@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(kRQThreads) rotate_quant_rows_twopass(
 // long rows), so a decode-sized matrix of a few rows costs one load latency.
 // ---------------------------------------------------------------------------
 constexpr int kMaxSlots = 32;          // 512 threads
-constexpr int kXchStride = 16 * 9;     // doubles per slot exchange buffer (half a 16 x 16 transpose + padding)
+constexpr int kXchFull = 16 * 17;     // doubles per slot: whole 16 x 16 transpose, padded
+constexpr int kXchHalf = 16 * 9;      // doubles per slot: half of it at a time, padded
 constexpr int kMaxParts = 8;           // CTAs per row (portable cluster size)
 constexpr int kSlotsSmemMax = 226 * 1024;   // dynamic shared memory per CTA (227 KB minus the static part)
 
@@ -278,8 +279,14 @@ __device__ __forceinline__ void cluster_wait() {
 // maximum is combined through distributed shared memory, then each CTA
 // quantises its own groups.  Decode-sized matrices (a few rows) are spread
 // over many SMs this way.
-template <int GPS>
-__global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
+// HALF: transpose in two halves through a 16 x 9 buffer (half the shared
+// memory, used for decode-sized launches whose CTAs should fit beside a
+// GEMM CTA); otherwise in one pass through a 16 x 17 buffer and in place
+// (fewer registers, for launches with a row per CTA).
+template <int GPS, bool HALF>
+__global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
+    rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
+    constexpr int kXchStride = HALF ? kXchHalf : kXchFull;
     extern __shared__ __align__(16) uint8_t rq_smem[];
     __shared__ float red[kMaxSlots / 2];
     __shared__ float part_max;
@@ -327,19 +334,28 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
 #pragma unroll
             for (int i = 0; i < 8; ++i) bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
             fwht16_regs(v);                                  // index bits 0-3
-            // transpose across the slot's 16 threads in two halves (a 16 x 9
-            // buffer: conflict-free): thread u needs element 16*j + u of every
-            // thread j, i.e. v[u] of thread j
+            // transpose across the slot's 16 threads: thread u needs element
+            // 16*j + u of every thread j, i.e. v[u] of thread j (padded rows:
+            // conflict-free both ways)
             double x[16];
+            if (HALF) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < 2; ++h) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) xb[9 * t + i] = v[8 * h + i];
-                __syncwarp(half_mask);
-                if ((t >> 3) == h) {
+                    for (int i = 0; i < 8; ++i) xb[9 * t + i] = v[8 * h + i];
+                    __syncwarp(half_mask);
+                    if ((t >> 3) == h) {
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) x[jj] = xb[9 * jj + (t & 7)];
+                        for (int jj = 0; jj < 16; ++jj) x[jj] = xb[9 * jj + (t & 7)];
+                    }
+                    __syncwarp(half_mask);
                 }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) xb[17 * t + i] = v[i];
+                __syncwarp(half_mask);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = xb[t + 17 * i];
                 __syncwarp(half_mask);
             }
             fwht16_regs(x);                                  // index bits 4-7
@@ -405,21 +421,21 @@ __global__ void __launch_bounds__(kMaxSlots * 16, 1) rotate_quant_rows_slots(con
     }
 }
 
-template <int GPS>
+template <int GPS, bool HALF>
 static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int max_slots, int max_local_groups) {
     cfg.blockDim = dim3(max_slots * 16);
-    cfg.dynamicSmemBytes = (size_t)max_slots * kXchStride * 8 + (size_t)max_local_groups * 256 * 4;
+    cfg.dynamicSmemBytes = (size_t)max_slots * (HALF ? kXchHalf : kXchFull) * 8 + (size_t)max_local_groups * 256 * 4;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(rotate_quant_rows_slots<GPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(rotate_quant_rows_slots<GPS, HALF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSlotsSmemMax);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev] = true;
     }
-    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS>, args);
+    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS, HALF>, args);
 }
 
 // CTAs per row: when the rows alone do not fill the GPU, split each row over
@@ -451,7 +467,7 @@ static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, int *m
     *max_slots = ms;
     *max_gps = mg;
     *max_local = ml;
-    return (size_t)ms * kXchStride * 8 + (size_t)ml * 256 * 4;
+    return (size_t)ms * (parts > 1 ? kXchHalf : kXchFull) * 8 + (size_t)ml * 256 * 4;
 }
 
 bool rotate_quant_batchable(int njobs, const RQProblem *probs) {
@@ -464,6 +480,16 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     const int parts = rq_parts(njobs, rows, num_sms);
+    if (parts == 1 && njobs > 1) {
+        // rows fill the GPU: one launch per matrix, each with the CTA shape of
+        // its own row length (a shared shape would size every CTA for the
+        // longest rows)
+        for (int jj = 0; jj < njobs; ++jj) {
+            cudaError_t e = launch_rotate_quant(1, rows, probs + jj, stream, pdl);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     int na = 0;
@@ -501,12 +527,21 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
             const int groups = J.k >> 8;
             rq_shape((groups + parts - 1) / parts, &J.gps, &J.slots);
         }
+        if (parts > 1) {
+            switch (max_gps) {
+                case 1: return launch_slots<1, true>(cfg, args, max_slots, max_local);
+                case 2: return launch_slots<2, true>(cfg, args, max_slots, max_local);
+                case 3: return launch_slots<3, true>(cfg, args, max_slots, max_local);
+                case 4: return launch_slots<4, true>(cfg, args, max_slots, max_local);
+                default: return launch_slots<6, true>(cfg, args, max_slots, max_local);
+            }
+        }
         switch (max_gps) {
-            case 1: return launch_slots<1>(cfg, args, max_slots, max_local);
-            case 2: return launch_slots<2>(cfg, args, max_slots, max_local);
-            case 3: return launch_slots<3>(cfg, args, max_slots, max_local);
-            case 4: return launch_slots<4>(cfg, args, max_slots, max_local);
-            default: return launch_slots<6>(cfg, args, max_slots, max_local);
+            case 1: return launch_slots<1, false>(cfg, args, max_slots, max_local);
+            case 2: return launch_slots<2, false>(cfg, args, max_slots, max_local);
+            case 3: return launch_slots<3, false>(cfg, args, max_slots, max_local);
+            case 4: return launch_slots<4, false>(cfg, args, max_slots, max_local);
+            default: return launch_slots<6, false>(cfg, args, max_slots, max_local);
         }
     }
     // rows too long to stage: one plain launch per matrix, rotation recomputed in a second pass

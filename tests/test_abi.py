@@ -83,8 +83,8 @@ def test_workspace_sizes_follow_the_tiling(lib):
     # tile; 64 weight tiles < 148 SMs, so every tile is split along K and
     # needs an INT32 partial tile (16 x 128 x 4 B) and a counter.
     assert lib.convrot_gemm_workspace_bytes(12, 8192, 5120) == 256 + 64 * 16 * 128 * 4
-    # prefill: 32 x 100 tiles of 128 x 256; 21 whole waves over 148 SMs
-    # leave 92 tiles for the stream-K tail.
-    assert lib.convrot_gemm_workspace_bytes(4096, 25600, 5120) == 512 + 92 * 256 * 128 * 4
+    # prefill: 32 x 100 tiles of 128 x 256, whole tiles only (22 waves over
+    # 148 SMs, the last one partial): no scratch at all
+    assert lib.convrot_gemm_workspace_bytes(4096, 25600, 5120) == 0
     lw = lib.convrot_linear_workspace_bytes(12, 8192, 5120)
     assert lw == lib.convrot_gemm_workspace_bytes(12, 8192, 5120) + 61440 + 256
