@@ -47,6 +47,7 @@ constexpr int kBlockK = 128;           // bytes of K per stage (one 128-byte swi
 constexpr int kUmmaK = 32;             // K per tcgen05.mma kind::i8
 constexpr int kATileBytes = kTileA * kBlockK;
 constexpr int kL2PrefetchBlocks = 16;  // weight K blocks pulled into L2 ahead of the grid-dependency wait
+constexpr int kMaxSplitWays = 8;       // K ranges per split tail tile (large M)
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -58,14 +59,17 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 // a tile or a job boundary.
 struct Segment {
     int job, tile, kb0, kb1, slot;
+    int split;          // >= 0: a piece of a split tail tile (private partial)
 };
 
 struct SegmentIter {
     int wave, j;
+    bool piece_done;
     long long u, u_end;
     __device__ __forceinline__ void init(const GemmArgs &a) {
         wave = 0;
         j = 0;
+        piece_done = false;
         const long long c = blockIdx.x, G = gridDim.x;
         u = a.tail_units * c / G;
         u_end = a.tail_units * (c + 1) / G;
@@ -77,8 +81,23 @@ struct SegmentIter {
             s.kb0 = 0;
             s.kb1 = a.job[0].kbpt;
             s.slot = -1;
+            s.split = -1;
             ++wave;
             return true;
+        }
+        if (a.split_ways > 1 && !piece_done) {
+            piece_done = true;
+            const int c = (int)blockIdx.x;
+            if (c < a.split_pieces) {
+                const int kbpt = a.job[0].kbpt;
+                s.job = 0;
+                s.slot = c / a.split_ways;
+                s.split = c - s.slot * a.split_ways;
+                s.tile = a.full_tiles + s.slot;
+                s.kb0 = s.split * kbpt / a.split_ways;
+                s.kb1 = (s.split + 1) * kbpt / a.split_ways;
+                return true;
+            }
         }
         if (u < u_end) {
             while (j + 1 < a.njobs && u >= a.job[j + 1].unit0) ++j;
@@ -91,6 +110,7 @@ struct SegmentIter {
             s.kb0 = (int)(lu - t * J.kbpt);
             const long long rem = u_end - u;
             s.kb1 = (int)((long long)s.kb0 + rem < J.kbpt ? s.kb0 + rem : J.kbpt);
+            s.split = -1;
             u += s.kb1 - s.kb0;
             return true;
         }
@@ -388,6 +408,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
                 if (whole) {
                     emit16(J, a.swap, i, tb * a.bn + c * 16, v);
+                } else if (sg.split >= 0) {
+                    // private partial: plain coalesced stores, no atomics
+                    int32_t *p = a.partial +
+                                 (((size_t)sg.slot * a.split_ways + sg.split) * a.bn + c * 16) * kTileA + row;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) __stcg(p + (size_t)e * kTileA, v[e]);
                 } else {
                     int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
 #pragma unroll
@@ -395,10 +421,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (v[e] != 0) atomicAdd(p + (size_t)e * kTileA, v[e]);
                 }
             }
+            if (sg.split >= 0) {
+                // the last piece of the tile adds the others' partials to its
+                // own accumulator (still in TMEM) and writes the tile
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (ew == 0 && lane == 0) {
+                    const int old = atomicAdd(a.counters + sg.slot, 1);
+                    *ticket = (old == a.split_ways - 1) ? 1 : 0;
+                }
+                named_bar_sync(1, 128);
+                if (*ticket != 0) {
+                    __threadfence();
+                    for (int c = 0; c < a.bn / 16; ++c) {
+                        uint32_t r[16];
+                        __syncwarp();
+                        tmem_ld_32x32b_x16(tbase + (uint32_t)(c * 16), r);
+                        tmem_ld_wait();
+                        int32_t v[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
+                        // add the other pieces' partials; leave every piece's
+                        // region zero again (the scratch is zero between calls)
+                        for (int sp = 0; sp < a.split_ways; ++sp) {
+                            int32_t *p = a.partial + (((size_t)sg.slot * a.split_ways + sp) * a.bn + c * 16) * kTileA + row;
+                            if (sp != sg.split) {
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) v[e] += __ldcg(p + (size_t)e * kTileA);
+                            }
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) __stcg(p + (size_t)e * kTileA, 0);
+                        }
+                        emit16(J, a.swap, i, tb * a.bn + c * 16, v);
+                    }
+                    if (ew == 0 && lane == 0) a.counters[sg.slot] = 0;
+                }
+                named_bar_sync(1, 128);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar + 8u * buf);
-            if (!whole) {
+            if (!whole && sg.split < 0) {
                 __threadfence();
                 named_bar_sync(1, 128);
                 if (ew == 0 && lane == 0) {
@@ -452,7 +515,8 @@ static void plan_common(GemmPlan *p) {
     const size_t cnt = ((size_t)p->slots * 4 + 255) / 256 * 256;
     p->ws_counters_off = 0;
     p->ws_partial_off = cnt;
-    p->ws_bytes = cnt + (size_t)p->slots * p->bn * kTileA * 4;
+    const int per_slot = p->split_ways > 1 ? p->split_ways : 1;
+    p->ws_bytes = cnt + (size_t)p->slots * per_slot * p->bn * kTileA * 4;
 }
 
 void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
@@ -476,16 +540,30 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
         tail_tile0 = p->full_waves * p->grid;
         p->full_tiles = tail_tile0;
     } else {
-        // large M: whole 128 x 256 tiles only, the last wave partly idle;
-        // splitting the last wave along K would cost a 128 KB INT32 partial
-        // flush per split tile, more than the idle SMs lose
+        // large M: whole 128 x 256 tiles in full waves.  A last, partial wave
+        // that would leave most SMs idle is split instead: each of its tiles
+        // into `ways` K ranges, one CTA each, with private INT32 partial tiles
+        // (plain stores) summed by the tile's last piece.  Atomic stream-K
+        // partials would cost more than the idle SMs lose at 128 x 256.
         p->grid = num_tiles < num_sms ? num_tiles : num_sms;
-        p->full_waves = (num_tiles + p->grid - 1) / p->grid;
+        p->full_waves = num_tiles / p->grid;
+        const int tail = num_tiles - p->full_waves * p->grid;
+        int ways = tail > 0 ? p->grid / tail : 0;
+        if (ways > kMaxSplitWays) ways = kMaxSplitWays;
+        if (ways > kbpt / 4) ways = kbpt / 4;
+        if (ways >= 2) {
+            p->full_tiles = p->full_waves * p->grid;
+            p->split_ways = ways;
+            p->split_pieces = tail * ways;
+            p->slots = tail;
+        } else {
+            p->full_waves += tail > 0 ? 1 : 0;
+            p->full_tiles = num_tiles;
+        }
         tail_tile0 = num_tiles;
-        p->full_tiles = num_tiles;
     }
-    p->slots = num_tiles - tail_tile0;
-    p->tail_units = (long long)p->slots * kbpt;
+    if (p->swap) p->slots = num_tiles - tail_tile0;
+    p->tail_units = p->swap ? (long long)p->slots * kbpt : 0;
     p->tiles_a[0] = tiles_a;
     p->kbpt[0] = kbpt;
     p->tile_base[0] = tail_tile0;
@@ -562,6 +640,8 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
     a.swap = p.swap;
     a.full_waves = p.full_waves;
     a.full_tiles = p.full_tiles;
+    a.split_ways = p.split_ways;
+    a.split_pieces = p.split_pieces;
     a.tail_units = p.tail_units;
     a.stages = p.stages;
     a.acc_cols = p.acc_cols;

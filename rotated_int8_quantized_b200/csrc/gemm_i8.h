@@ -34,6 +34,11 @@ struct GemmArgs {
     int swap;           // 1: A = weights, B = activations; 0: A = activations, B = weights
     int full_waves;     // data-parallel waves of whole tiles (single job only)
     int full_tiles;     // tiles those waves cover (the last wave may be partial)
+    // split tail (large M): the tiles after the full waves are each split into
+    // split_ways K ranges, one per CTA; every piece stores its INT32 partial
+    // tile privately and the last piece of a tile (ticket counter) sums them
+    int split_ways;     // 0: no split tail
+    int split_pieces;   // tail tiles x split_ways (CTAs 0 .. pieces-1 take one each)
     long long tail_units;   // K blocks dealt out by stream-K
     int stages;
     int acc_cols;       // TMEM columns per accumulator buffer
@@ -63,7 +68,7 @@ struct GemmProblem {
 // Host-side tiling of a launch.
 struct GemmPlan {
     int njobs, swap, bn;
-    int grid, full_waves, full_tiles, stages, acc_cols, tmem_cols, smem_bytes;
+    int grid, full_waves, full_tiles, split_ways, split_pieces, stages, acc_cols, tmem_cols, smem_bytes;
     long long tail_units;
     int tiles_a[kMaxJobs], kbpt[kMaxJobs], tile_base[kMaxJobs], slot0[kMaxJobs];
     long long unit0[kMaxJobs];
@@ -93,7 +98,5 @@ struct RQProblem {
 // Rotate and quantise `rows` rows of each of `njobs` matrices (same row
 // count) in one launch.
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl);
-// True when one launch can take all these row lengths together.
-bool rotate_quant_batchable(int njobs, const RQProblem *probs);
 
 }  // namespace convrot

@@ -17,9 +17,9 @@
 // gives the exact sum of the explicit matrix product, and one rounding to
 // FP32 follows.  The row's rotated FP32 values wait in shared memory while
 // the row maximum is reduced; then each thread packs 16 INT8 codes into one
-// 16-byte store.  Rows too long for shared memory take a two-pass variant
-// (one warp per group, the 8-stage butterfly across lanes with shuffles)
-// that recomputes the L2-resident rotation instead of staging it.
+// 16-byte store.  Long rows are split over a cluster too (at most one group
+// per slot), so every row the API accepts (k <= 133120) stages in shared
+// memory.
 #include <cstdint>
 #include <cstring>
 #include <cuda_bf16.h>
@@ -30,68 +30,7 @@
 
 namespace convrot {
 
-constexpr int kRQThreads = 256;
-constexpr int kRQWarps = kRQThreads / 32;
-
-// In-place unnormalised Walsh-Hadamard transform of one 256-group held as
-// 8 values per lane (lane L holds elements 8L .. 8L+7).  Natural (Sylvester)
-// order: y_j = sum_i x_i * (-1)^popcount(i & j).
-__device__ __forceinline__ void fwht256_warp(double (&v)[8], int lane) {
-#pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            if ((e & h) == 0) {
-                double a = v[e], b = v[e + h];
-                v[e] = a + b;
-                v[e + h] = a - b;
-            }
-        }
-    }
-#pragma unroll
-    for (int lm = 1; lm < 32; lm <<= 1) {
-        const bool upper = (lane & lm) != 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            double p = __shfl_xor_sync(0xffffffffu, v[e], lm);
-            v[e] = upper ? (p - v[e]) : (v[e] + p);
-        }
-    }
-}
-
-// Load 8 BF16 (one 16-byte vector) and widen to FP64 (exact).
-__device__ __forceinline__ void load8_bf16_as_f64(const __nv_bfloat16 *p, double (&v)[8]) {
-    uint4 raw = __ldg(reinterpret_cast<const uint4 *>(p));
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = (double)__uint_as_float(w[i] << 16);
-        v[2 * i + 1] = (double)__uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-
-// Rotate one group: returns the 8 FP32 outputs of this lane.
-__device__ __forceinline__ void rotate_group(const __nv_bfloat16 *grp, int lane, float (&y)[8]) {
-    double v[8];
-    load8_bf16_as_f64(grp + lane * 8, v);
-    fwht256_warp(v, lane);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] = __double2float_rn(v[e] * 0.0625);   // / sqrt(256), exact
-}
-
-__device__ __forceinline__ float block_max(float v, float *red) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float r = red[0];
-#pragma unroll
-    for (int w = 1; w < kRQWarps; ++w) r = fmaxf(r, red[w]);
-    return r;
-}
-
-// Row quantisation helper: everything quant1 needs about a row's scale s.
+// Row quantisation helper: everything quant16 needs about a row's scale s.
 struct RowScale {
     float s;        // s = fl(amax / 127)
     float r;        // fl(1 / s), correctly rounded
@@ -108,8 +47,9 @@ __device__ __forceinline__ RowScale make_row_scale(float amax) {
     return rs;
 }
 
-// q = clamp(rne(fl(y / s)), -127, 127): the integer nearest to the
-// correctly rounded FP32 quotient, ties to even.
+// q = clamp(rne(fl(y / s)), -127, 127) for 16 consecutive values y: the
+// integer nearest to the correctly rounded FP32 quotient, ties to even,
+// packed into one 16-byte word.
 //
 // Evaluated with Ziv's rounding test (A. Ziv, "Fast evaluation of elementary
 // mathematical functions with correctly rounded last bit", ACM TOMS 17(3),
@@ -121,25 +61,9 @@ __device__ __forceinline__ RowScale make_row_scale(float amax) {
 // |t - fl(y/s)| < 2.3e-5.  When t is more than 3e-5 away from every
 // half-integer, fl(y/s) rounds to the same integer as t; otherwise (about
 // 6e-5 of the elements) the IEEE division is evaluated.
-__device__ __forceinline__ int8_t quant1(float y, const RowScale &rs) {
-    if (rs.zero) return 0;
-    float f;
-    const float t = __fmul_rn(y, rs.r);
-    const float ft = rintf(t);
-    if (rs.fast && fabsf(t - ft) < 0.49997f) {
-        f = ft;
-    } else {
-        f = rintf(__fdiv_rn(y, rs.s));
-    }
-    f = fminf(fmaxf(f, -127.0f), 127.0f);
-    return (int8_t)(int)f;
-}
-
-// The same for 16 consecutive values packed into one 16-byte word, with the
-// fast path as straight-line code (independent lanes of work for the
-// scheduler) and the exact division only where some thread of the warp
-// needs it.  Every thread of the warp must call it together (`mask` = the
-// active threads).
+// The fast path is straight-line code over the 16 values (independent work
+// for the scheduler); the division runs only where some thread of the warp
+// needs it.  Every thread of `mask` (the active threads) must call it.
 __device__ __forceinline__ uint4 quant16(const float (&y)[16], const RowScale &rs, unsigned mask) {
     float f[16];
     bool slow = false;
@@ -166,50 +90,15 @@ __device__ __forceinline__ uint4 quant16(const float (&y)[16], const RowScale &r
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// One CTA per row, no staging: pass 1 finds the row maximum, pass 2
-// recomputes the rotation (the row is L2-resident) and quantises.
-__global__ void __launch_bounds__(kRQThreads) rotate_quant_rows_twopass(
-    const __nv_bfloat16 *__restrict__ a, int k, int8_t *__restrict__ q, float *__restrict__ s) {
-    __shared__ float red[kRQWarps];
-    pdl_wait();
-    pdl_launch_dependents();
-    const int row = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const __nv_bfloat16 *arow = a + (size_t)row * k;
-    const int groups = k >> 8;
-    float amax = 0.f;
-    for (int g = warp; g < groups; g += kRQWarps) {
-        float y[8];
-        rotate_group(arow + g * 256, lane, y);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(y[e]));
-    }
-    amax = block_max(amax, red);
-    const RowScale rs = make_row_scale(amax);
-    int8_t *qrow = q + (size_t)row * k;
-    for (int g = warp; g < groups; g += kRQWarps) {
-        float y[8];
-        rotate_group(arow + g * 256, lane, y);
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) lo |= (uint32_t)(uint8_t)quant1(y[e], rs) << (8 * e);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) hi |= (uint32_t)(uint8_t)quant1(y[4 + e], rs) << (8 * e);
-        *reinterpret_cast<uint2 *>(qrow + g * 256 + lane * 8) = make_uint2(lo, hi);
-    }
-    if (threadIdx.x == 0) s[row] = rs.s;
-}
-
 // ---------------------------------------------------------------------------
 // Main variant: 16 threads ("a slot") per 256-group, H_256 = H_16 (x) H_16.
 // Thread t of a slot loads elements 16t .. 16t+15 (32 contiguous bytes; the
 // slot reads the group's 512 bytes coalesced), transforms index bits 0-3 in
-// registers, exchanges through a padded shared-memory transpose (in two
-// halves through a 16 x 9 buffer: conflict-free both ways), transforms index
-// bits 4-7 in registers
-// and so ends up holding outputs t, t+16, ..., t+240.  Every group of a row
-// is in flight at once (up to 32 slots per CTA, several groups per slot for
-// long rows), so a decode-sized matrix of a few rows costs one load latency.
+// registers, exchanges through a padded shared-memory transpose, transforms
+// index bits 4-7 in registers and so ends up holding outputs t, t+16, ...,
+// t+240.  Every group of a row is in flight at once (up to 32 slots per CTA,
+// several groups per slot for long rows), so a decode-sized matrix of a few
+// rows costs one load latency.
 // ---------------------------------------------------------------------------
 constexpr int kMaxSlots = 32;          // 512 threads
 constexpr int kXchFull = 16 * 17;     // doubles per slot: whole 16 x 16 transpose, padded
@@ -438,22 +327,32 @@ static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int
     return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS, HALF>, args);
 }
 
-// CTAs per row: when the rows alone do not fill the GPU, split each row over
-// a cluster of CTAs so that every SM gets work, but keep the whole grid
-// within one wave (about two CTAs per SM), so that every CTA starts at once
-// and triggers the dependent GEMM's launch early.
-static int rq_parts(int njobs, int64_t rows, int num_sms) {
+// CTAs per row (a thread-block cluster).  When the rows alone do not fill
+// the GPU, enough to spread the work over the SMs while the whole grid stays
+// within one wave (about two CTAs per SM), so every CTA starts at once and
+// triggers the dependent GEMM's launch early.  Otherwise one, unless a row is
+// too long to stage in one CTA's shared memory.
+static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, bool half, int *max_slots,
+                            int *max_gps, int *max_local);
+
+static int rq_parts(int njobs, int64_t rows, const RQProblem *probs, int num_sms, bool half) {
+    int parts = 1;
+    int ms, mg, ml;
+    while (parts < kMaxParts &&
+           (rq_smem_bytes(njobs, probs, parts, half, &ms, &mg, &ml) > (size_t)kSlotsSmemMax || mg > 6))
+        ++parts;
     const int64_t total_rows = rows * njobs;
-    if (total_rows >= num_sms) return 1;
-    int64_t parts = (2 * (int64_t)num_sms) / total_rows;
-    if (parts > kMaxParts) parts = kMaxParts;
-    if (parts < 1) parts = 1;
-    return (int)parts;
+    if (total_rows < num_sms) {
+        int64_t spread = (2 * (int64_t)num_sms) / total_rows;
+        if (spread > kMaxParts) spread = kMaxParts;
+        if (spread > parts) parts = (int)spread;
+    }
+    return parts;
 }
 
 // Shared-memory bytes and shape of one CTA of a launch with `parts` CTAs per row.
-static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, int *max_slots, int *max_gps,
-                            int *max_local) {
+static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, bool half, int *max_slots,
+                            int *max_gps, int *max_local) {
     int ms = 0, mg = 0, ml = 0;
     for (int j = 0; j < njobs; ++j) {
         const int groups = (int)(probs[j].k >> 8);
@@ -467,20 +366,15 @@ static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, int *m
     *max_slots = ms;
     *max_gps = mg;
     *max_local = ml;
-    return (size_t)ms * (parts > 1 ? kXchHalf : kXchFull) * 8 + (size_t)ml * 256 * 4;
-}
-
-bool rotate_quant_batchable(int njobs, const RQProblem *probs) {
-    int ms, mg, ml;
-    return njobs <= kMaxJobs && rq_smem_bytes(njobs, probs, 1, &ms, &mg, &ml) <= (size_t)kSlotsSmemMax;
+    return (size_t)ms * (half ? kXchHalf : kXchFull) * 8 + (size_t)ml * 256 * 4;
 }
 
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl) {
     int dev = 0, num_sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    const int parts = rq_parts(njobs, rows, num_sms);
-    if (parts == 1 && njobs > 1) {
+    const bool few_rows = rows * njobs < num_sms;
+    if (!few_rows && njobs > 1) {
         // rows fill the GPU: one launch per matrix, each with the CTA shape of
         // its own row length (a shared shape would size every CTA for the
         // longest rows)
@@ -490,6 +384,10 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         }
         return cudaSuccess;
     }
+    // decode-sized launches use the half-size transpose buffer, so that their
+    // CTAs fit beside the GEMM's
+    const bool half = few_rows;
+    const int parts = rq_parts(njobs, rows, probs, num_sms, half);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     int na = 0;
@@ -506,13 +404,12 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         ++na;
     }
     cfg.gridDim = dim3((unsigned)(rows * njobs * parts));
-    cfg.blockDim = dim3(kRQThreads);
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = na;
     int max_slots, max_gps, max_local;
     if (njobs <= kMaxJobs &&
-        rq_smem_bytes(njobs, probs, parts, &max_slots, &max_gps, &max_local) <= (size_t)kSlotsSmemMax) {
+        rq_smem_bytes(njobs, probs, parts, half, &max_slots, &max_gps, &max_local) <= (size_t)kSlotsSmemMax) {
         RQArgs args;
         memset(&args, 0, sizeof(args));
         args.njobs = njobs;
@@ -527,7 +424,7 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
             const int groups = J.k >> 8;
             rq_shape((groups + parts - 1) / parts, &J.gps, &J.slots);
         }
-        if (parts > 1) {
+        if (half) {
             switch (max_gps) {
                 case 1: return launch_slots<1, true>(cfg, args, max_slots, max_local);
                 case 2: return launch_slots<2, true>(cfg, args, max_slots, max_local);
@@ -544,17 +441,10 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
             default: return launch_slots<6, false>(cfg, args, max_slots, max_local);
         }
     }
-    // rows too long to stage: one plain launch per matrix, rotation recomputed in a second pass
-    cfg.numAttrs = pdl ? 1 : 0;
-    cfg.dynamicSmemBytes = 0;
-    cfg.gridDim = dim3((unsigned)rows);
-    for (int j = 0; j < njobs; ++j) {
-        cudaError_t e = cudaLaunchKernelEx(&cfg, rotate_quant_rows_twopass,
-                                           static_cast<const __nv_bfloat16 *>(probs[j].a), (int)probs[j].k,
-                                           probs[j].q, probs[j].s);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+    // unreachable within the shapes the API accepts (k <= 133120 stages in
+    // at most 114 KB per CTA with 8 parts)
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace convrot
+

@@ -86,5 +86,9 @@ def test_workspace_sizes_follow_the_tiling(lib):
     # prefill: 32 x 100 tiles of 128 x 256, whole tiles only (22 waves over
     # 148 SMs, the last one partial): no scratch at all
     assert lib.convrot_gemm_workspace_bytes(4096, 25600, 5120) == 0
+    # prefill down projection: 32 x 20 = 640 tiles, 4 full waves; the 48 tail
+    # tiles are split into 148 // 48 = 3 K ranges with private 128 KB INT32
+    # partial tiles
+    assert lib.convrot_gemm_workspace_bytes(4096, 5120, 25600) == 256 + 48 * 3 * 256 * 128 * 4
     lw = lib.convrot_linear_workspace_bytes(12, 8192, 5120)
     assert lw == lib.convrot_gemm_workspace_bytes(12, 8192, 5120) + 61440 + 256

@@ -59,12 +59,13 @@ def test_weight_quant_tiny_bit_exact(cr):
 
 
 # m and k span every launch shape of the kernel: rows split over a cluster of
-# up to 8 CTAs (few rows), one CTA per row (>= 148 rows) with one slot or
-# several groups per slot (2, 3, 4, 6 and a ragged last slot), and rows too
-# long to stage (two-pass variant)
+# up to 8 CTAs (few rows, or rows of more than 32 groups), one CTA per row
+# (>= 148 rows), one or several groups per slot and a ragged last slot, and
+# the longest rows the API accepts
 @pytest.mark.parametrize("m,k", [(1, 256), (4, 512), (3, 768), (17, 5120), (2, 8448), (3, 16384),
                                  (2, 24576), (5, 25600), (2, 38912), (2, 40960), (2, 65536),
-                                 (150, 512), (160, 8448), (148, 25600), (149, 40960), (200, 65536)])
+                                 (150, 512), (160, 8448), (148, 25600), (149, 40960), (200, 65536),
+                                 (3, 133120), (150, 133120)])
 def test_act_quant_bit_exact(cr, m, k):
     cs = synth.outlier_scale_fraction(synth.stream_key(m * 7 + k, 2), k, 0.01, 30.0)
     x_bits = synth.draw_np(synth.stream_key(m * 7 + k, 0), m, k, 1.0, cs)
@@ -140,7 +141,9 @@ GEMM_SHAPES = [
     (100, 640, 2560),   # swap with bn = 112
     (256, 512, 768),    # largest swap case, bn = 256
     (257, 512, 512),    # smallest non-swap case, ragged activation tile
-    (640, 1000, 1536),  # non-swap, ragged weight tile (1000 % 256), stream-K tail
+    (640, 1000, 1536),  # non-swap, ragged weight tile (1000 % 256), one partial wave
+    (9500, 500, 1024),  # 150 tiles: one full wave, 2 tail tiles split in 2 K ranges
+    (5083, 1000, 4096), # 160 tiles: 12 tail tiles split in 8 K ranges, ragged both ways
 ]
 
 
