@@ -47,10 +47,31 @@ constexpr int kBlockK = 128;           // bytes of K per stage (one 128-byte swi
 constexpr int kUmmaK = 32;             // K per tcgen05.mma kind::i8
 constexpr int kATileBytes = kTileA * kBlockK;
 constexpr int kL2PrefetchBlocks = 16;  // weight K blocks pulled into L2 ahead of the grid-dependency wait
-constexpr int kMaxSplitWays = 8;       // K ranges per split tail tile (large M)
+constexpr int kMaxSplitWays = 6;       // K ranges per split tail tile (large M)
+constexpr int kExtraBars = 7;          // tfull[2], tempty[2], drain, red[2]
+// The split-tail reduction double-buffers at least 32 columns of every other
+// piece's partial in the operand ring of a bn = 256 launch.
+static_assert(2 * (kMaxSplitWays - 1) * 32 * kTileA * 4 <=
+                  (200 * 1024 / (kATileBytes + 256 * kBlockK)) * (kATileBytes + 256 * kBlockK),
+              "split-tail reduction buffers exceed the operand ring");
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Barrier over `n` threads that also returns the AND of their predicates, so
+// that all of them take the same branch after a bounded wait.
+__device__ __forceinline__ bool named_bar_and(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
 }
 
 // Work of one CTA: a list of segments (job, tile, kb0, kb1), first the
@@ -173,6 +194,56 @@ __device__ __forceinline__ void emit16(const GemmJob &J, int swap, int i, int j0
     }
 }
 
+// Large-M orientation: dequantise and store columns j0 .. j0+15 of output
+// row m, with the row scale sxm in a register and the tile's weight scales
+// staged in shared memory (sws[e] = sw[j0 + e]).
+__device__ __forceinline__ void emit_row16(const GemmJob &J, int m, int j0, const int32_t (&v)[16], float sxm,
+                                           const float *sws) {
+    if (m >= J.m) return;
+    const bool full = (j0 + 16 <= J.n) && ((J.n & 7) == 0);
+    if (J.acc) {
+        int32_t *dst = J.acc + (size_t)m * J.n + j0;
+        if (full) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                *reinterpret_cast<int4 *>(dst + e) = make_int4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        } else {
+            for (int e = 0; e < 16 && j0 + e < J.n; ++e) dst[e] = v[e];
+        }
+    }
+    if (J.y) {
+        __nv_bfloat16 *dst = J.y + (size_t)m * J.n + j0;
+        if (full) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+                const float f0 = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), sws[e]);
+                const float f1 = __fmul_rn(__fmul_rn(__int2float_rn(v[e + 1]), sxm), sws[e + 1]);
+                __nv_bfloat162 h = __halves2bfloat162(__float2bfloat16_rn(f0), __float2bfloat16_rn(f1));
+                pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
+            }
+            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+            for (int e = 0; e < 16 && j0 + e < J.n; ++e)
+                dst[e] = __float2bfloat16_rn(__fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), sws[e]));
+        }
+    }
+}
+
+// Two TMEM loads of 16 columns each, one wait.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, int32_t (&v0)[16], int32_t (&v1)[16]) {
+    uint32_t r0[16], r1[16];
+    tmem_ld_32x32b_x16(taddr, r0);
+    tmem_ld_32x32b_x16(taddr + 16u, r1);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        v0[e] = (int32_t)r0[e];
+        v1[e] = (int32_t)r1[e];
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -186,16 +257,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t a_off = 0;
     const uint32_t b_off = (uint32_t)S * kATileBytes;
     const uint32_t bar_off = b_off + (uint32_t)S * b_bytes;
-    // barriers: full[S], empty[S], tfull[2], tempty[2], drain
+    // barriers: full[S], empty[S], tfull[2], tempty[2], drain, red[2]
     const uint32_t full_bar = base + bar_off;
     const uint32_t empty_bar = full_bar + 8u * S;
     const uint32_t tfull_bar = empty_bar + 8u * S;
     const uint32_t tempty_bar = tfull_bar + 16u;
     const uint32_t drain_bar = tempty_bar + 16u;
-    uint8_t *misc = smem + bar_off + 8u * (2 * S + 5);
+    const uint32_t red_bar = drain_bar + 8u;
+    uint8_t *misc = smem + bar_off + 8u * (2 * S + kExtraBars);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(misc);
     volatile int *ticket = reinterpret_cast<volatile int *>(misc + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 8);
+    volatile int *red_ok = reinterpret_cast<volatile int *>(misc + 12);
+    float *sw_stage = reinterpret_cast<float *>(misc + 16);     // [2][256] weight scales of a tile
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -210,6 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(tempty_bar + 8u * b, 4);
         }
         mbar_init(drain_bar, 1);
+        mbar_init(red_bar, 1);
+        mbar_init(red_bar + 8u, 1);
         *abort_flag = 0;
         *ticket = 0;
         fence_mbar_init();
@@ -393,68 +469,185 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ta = sg.tile % J.tiles_a, tb = sg.tile / J.tiles_a;
             const int buf = seg & 1;
             const uint32_t use = (uint32_t)(seg >> 1);
-            if (!mbar_wait_bounded(tfull_bar + 8u * buf, use & 1u, abort_flag)) break;
-            tc_fence_after();
             const int i = ta * kTileA + row;
+            // large M: the tile's weight scales go to shared memory and the
+            // row scale to a register while the accumulator is still being
+            // computed (double-buffered by segment parity; the barrier
+            // below publishes them)
+            float *sws = sw_stage + (seg & 1) * 256;
+            float sxm = 0.f;
+            if (!a.swap) {
+                const int tid = ew * 32 + lane;
+                for (int cidx = tid; cidx < a.bn; cidx += 128) {
+                    const int col = tb * a.bn + cidx;
+                    sws[cidx] = col < J.n ? __ldg(J.sw + col) : 0.f;
+                }
+                if (i < J.m) sxm = __ldg(J.sx + i);
+            }
+            const bool full = mbar_wait_bounded(tfull_bar + 8u * buf, use & 1u, abort_flag);
+            if (!named_bar_and(1, 128, full)) break;
+            tc_fence_after();
             const bool whole = (sg.kb0 == 0 && sg.kb1 == J.kbpt);
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * a.acc_cols);
-            for (int c = 0; c < a.bn / 16; ++c) {
-                uint32_t r[16];
-                __syncwarp();
-                tmem_ld_32x32b_x16(tbase + (uint32_t)(c * 16), r);
-                tmem_ld_wait();
-                int32_t v[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
-                if (whole) {
-                    emit16(J, a.swap, i, tb * a.bn + c * 16, v);
-                } else if (sg.split >= 0) {
-                    // private partial: plain coalesced stores, no atomics
-                    int32_t *p = a.partial +
-                                 (((size_t)sg.slot * a.split_ways + sg.split) * a.bn + c * 16) * kTileA + row;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) __stcg(p + (size_t)e * kTileA, v[e]);
-                } else {
-                    int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (v[e] != 0) atomicAdd(p + (size_t)e * kTileA, v[e]);
+            if (sg.split < 0 && whole && !a.swap) {
+                for (int c = 0; c < a.bn; c += 32) {
+                    int32_t v0[16], v1[16];
+                    __syncwarp();
+                    tmem_ld32(tbase + (uint32_t)c, v0, v1);
+                    const int j0 = tb * a.bn + c;
+                    emit_row16(J, i, j0, v0, sxm, sws + c);
+                    emit_row16(J, i, j0 + 16, v1, sxm, sws + c + 16);
                 }
-            }
-            if (sg.split >= 0) {
-                // the last piece of the tile adds the others' partials to its
-                // own accumulator (still in TMEM) and writes the tile
-                __threadfence();
+            } else if (sg.split < 0) {
+                for (int c = 0; c < a.bn / 16; ++c) {
+                    uint32_t r[16];
+                    __syncwarp();
+                    tmem_ld_32x32b_x16(tbase + (uint32_t)(c * 16), r);
+                    tmem_ld_wait();
+                    int32_t v[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
+                    if (whole) {
+                        emit16(J, a.swap, i, tb * a.bn + c * 16, v);
+                    } else {
+                        int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (v[e] != 0) atomicAdd(p + (size_t)e * kTileA, v[e]);
+                    }
+                }
+            } else {
+                // A piece of a split tail tile.  The tile's counter holds the
+                // pieces that finished their K range (low 16 bits) and the
+                // pieces whose partial is stored (high bits).  Every piece
+                // but the last to finish stores its INT32 partial in its own
+                // region; the last one waits for those stores (the pieces it
+                // waits on are already running), pulls the partials into
+                // shared memory with bulk copies (the operand ring is idle:
+                // this is the CTA's last segment and its MMAs are complete),
+                // adds them to its accumulator in TMEM and writes the tile.
+                const int ways = a.split_ways;
                 named_bar_sync(1, 128);
                 if (ew == 0 && lane == 0) {
                     const int old = atomicAdd(a.counters + sg.slot, 1);
-                    *ticket = (old == a.split_ways - 1) ? 1 : 0;
+                    *ticket = ((old & 0xFFFF) == ways - 1) ? 1 : 0;
                 }
                 named_bar_sync(1, 128);
-                if (*ticket != 0) {
-                    __threadfence();
-                    for (int c = 0; c < a.bn / 16; ++c) {
-                        uint32_t r[16];
+                if (*ticket == 0) {
+                    int32_t *pbase = a.partial + ((size_t)sg.slot * ways + sg.split) * a.bn * kTileA + row;
+                    for (int c = 0; c < a.bn; c += 32) {
+                        int32_t v0[16], v1[16];
                         __syncwarp();
-                        tmem_ld_32x32b_x16(tbase + (uint32_t)(c * 16), r);
-                        tmem_ld_wait();
-                        int32_t v[16];
+                        tmem_ld32(tbase + (uint32_t)c, v0, v1);
+                        int32_t *p = pbase + (size_t)c * kTileA;
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
-                        // add the other pieces' partials; leave every piece's
-                        // region zero again (the scratch is zero between calls)
-                        for (int sp = 0; sp < a.split_ways; ++sp) {
-                            int32_t *p = a.partial + (((size_t)sg.slot * a.split_ways + sp) * a.bn + c * 16) * kTileA + row;
-                            if (sp != sg.split) {
-#pragma unroll
-                                for (int e = 0; e < 16; ++e) v[e] += __ldcg(p + (size_t)e * kTileA);
-                            }
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) __stcg(p + (size_t)e * kTileA, 0);
+                        for (int e = 0; e < 16; ++e) {
+                            __stcg(p + (size_t)e * kTileA, v0[e]);
+                            __stcg(p + (size_t)(e + 16) * kTileA, v1[e]);
                         }
-                        emit16(J, a.swap, i, tb * a.bn + c * 16, v);
                     }
-                    if (ew == 0 && lane == 0) a.counters[sg.slot] = 0;
+                    __threadfence();
+                    named_bar_sync(1, 128);
+                    if (ew == 0 && lane == 0) atomicAdd(a.counters + sg.slot, 1 << 16);
+                } else {
+                    const int others = ways - 1;
+                    // column rounds, double-buffered in the operand ring
+                    const uint32_t ring = (uint32_t)S * ((uint32_t)kATileBytes + b_bytes);
+                    int cols = (int)(ring / (2u * (uint32_t)others * kTileA * 4u)) / 32 * 32;
+                    if (cols > a.bn) cols = a.bn;
+                    const int rounds = (a.bn + cols - 1) / cols;
+                    const uint32_t buf_bytes = (uint32_t)others * (uint32_t)cols * kTileA * 4u;
+                    const int32_t *tile_parts = a.partial + (size_t)sg.slot * ways * a.bn * kTileA;
+                    auto issue = [&](int r) {
+                        const int col0 = r * cols;
+                        const int nc = (a.bn - col0 < cols) ? a.bn - col0 : cols;
+                        const uint32_t bytes = (uint32_t)nc * kTileA * 4u;
+                        const uint32_t bar = red_bar + 8u * (uint32_t)(r & 1);
+                        const uint32_t dst = base + (uint32_t)(r & 1) * buf_bytes;
+                        mbar_arrive_expect_tx(bar, bytes * (uint32_t)others);
+                        int o = 0;
+                        for (int sp = 0; sp < ways; ++sp) {
+                            if (sp == sg.split) continue;
+                            bulk_load_1d(dst + (uint32_t)o * bytes,
+                                         tile_parts + ((size_t)sp * a.bn + col0) * kTileA, bytes, bar);
+                            ++o;
+                        }
+                    };
+                    if (ew == 0 && lane == 0) {
+                        int ok_wait = 1;
+                        if ((ld_acquire_gpu(a.counters + sg.slot) >> 16) < others) {
+                            const unsigned long long t0 = global_timer_ns();
+                            for (uint32_t it_w = 1;; ++it_w) {
+                                if ((ld_acquire_gpu(a.counters + sg.slot) >> 16) >= others) break;
+                                if ((it_w & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+                                    atomicExch(&g_device_status, 7 /* CONVROT_ERR_DEVICE_TIMEOUT */);
+                                    ok_wait = 0;
+                                    break;
+                                }
+                            }
+                        }
+                        if (ok_wait) {
+                            fence_proxy_async();
+                            issue(0);
+                            if (rounds > 1) issue(1);
+                        }
+                        *red_ok = ok_wait;
+                    }
+                    named_bar_sync(1, 128);
+                    bool ok_red = *red_ok != 0;
+                    int r = 0;
+                    for (; r < rounds && ok_red; ++r) {
+                        const int col0 = r * cols;
+                        const int nc = (a.bn - col0 < cols) ? a.bn - col0 : cols;
+                        const bool landed =
+                            mbar_wait_bounded(red_bar + 8u * (uint32_t)(r & 1), (uint32_t)((r >> 1) & 1), abort_flag);
+                        ok_red = named_bar_and(1, 128, landed);
+                        if (!ok_red) break;
+                        const int32_t *sbuf =
+                            reinterpret_cast<const int32_t *>(smem + (size_t)(r & 1) * buf_bytes) + row;
+                        for (int cc = 0; cc < nc; cc += 32) {
+                            int32_t v0[16], v1[16];
+                            __syncwarp();
+                            tmem_ld32(tbase + (uint32_t)(col0 + cc), v0, v1);
+                            for (int o = 0; o < others; ++o) {
+                                const int32_t *q = sbuf + ((size_t)o * nc + cc) * kTileA;
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) {
+                                    v0[e] += q[(size_t)e * kTileA];
+                                    v1[e] += q[(size_t)(e + 16) * kTileA];
+                                }
+                            }
+                            const int j0 = tb * a.bn + col0 + cc;
+                            emit_row16(J, i, j0, v0, sxm, sws + col0 + cc);
+                            emit_row16(J, i, j0 + 16, v1, sxm, sws + col0 + cc + 16);
+                        }
+                        named_bar_sync(1, 128);     // buffer (r & 1) is read by everyone
+                        if (r + 2 < rounds && ew == 0 && lane == 0) {
+                            fence_proxy_async();
+                            issue(r + 2);
+                        }
+                    }
+                    if (ok_red) {
+                        // leave the other pieces' regions zero again (the
+                        // workspace is zero between calls), then the counter
+                        const int4 z = make_int4(0, 0, 0, 0);
+                        const int tid = ew * 32 + lane;
+                        const size_t n4 = (size_t)a.bn * kTileA / 4;
+                        for (int sp = 0; sp < ways; ++sp) {
+                            if (sp == sg.split) continue;
+                            int4 *dst = reinterpret_cast<int4 *>(const_cast<int32_t *>(tile_parts) +
+                                                                 (size_t)sp * a.bn * kTileA);
+                            for (size_t x = (size_t)tid; x < n4; x += 128) __stcg(dst + x, z);
+                        }
+                        if (ew == 0 && lane == 0) a.counters[sg.slot] = 0;
+                    } else if (ew == 0 && lane == 0 && *red_ok) {
+                        // a wait gave up at round r: let the copies already
+                        // started (rounds r and r + 1 at most) land first
+                        volatile int no_abort = 0;
+                        const int issued = rounds < r + 2 ? rounds : r + 2;
+                        for (int q = r; q < issued; ++q)
+                            mbar_wait_bounded(red_bar + 8u * (uint32_t)(q & 1), (uint32_t)((q >> 1) & 1), &no_abort);
+                    }
                 }
                 named_bar_sync(1, 128);
             }
@@ -510,7 +703,7 @@ static void plan_common(GemmPlan *p) {
     int cols = 32;
     while (cols < 2 * p->bn) cols <<= 1;
     p->tmem_cols = cols;
-    p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + 5) + 16;
+    p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + kExtraBars) + 16 + 2 * 256 * 4;
     // workspace: counters, then INT32 partial tiles [slots][bn][128]
     const size_t cnt = ((size_t)p->slots * 4 + 255) / 256 * 256;
     p->ws_counters_off = 0;
