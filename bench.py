@@ -229,6 +229,13 @@ def time_region(fn, steps, stream):
     return start.elapsed_time(end) / 1e3
 
 
+def keep_busy(stream, us: float = 60.0):
+    """Queue a short device-side spin ahead of a timed launch so that the
+    host's launch overhead is not inside the CUDA-event interval."""
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(us * 2000))
+
+
 def gemm_batch_kernel_time(cr, layer, lins, xs, reps, stream, device):
     """Per-launch time of the batched GEMM kernel (all linears of the step in
     one launch) with CUDA events on the launching stream; the activation
@@ -240,6 +247,7 @@ def gemm_batch_kernel_time(cr, layer, lins, xs, reps, stream, device):
     torch.cuda.synchronize()        # the zeroed workspace is ready before `stream` uses it
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
     for i in range(reps + 2):
+        keep_busy(stream)
         for x, xq, sx in zip(xs, xqs, sxs):
             cr.convrot_quantize_act(x, xq, sx, stream=stream)
         if i >= 2:
@@ -263,6 +271,7 @@ def gemm_kernel_times(cr, layer, lins, xs, reps, stream, device):
         torch.cuda.synchronize()    # the zeroed workspace is ready before `stream` uses it
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
         for i in range(reps + 2):
+            keep_busy(stream)
             cr.convrot_quantize_act(x, xq, sx, stream=stream)
             if i >= 2:
                 evs[i - 2][0].record(stream)
@@ -334,6 +343,7 @@ def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
+    keep_busy(stream)
     t = time_region(fn, steps, stream) / steps
     ops = sum(2 * lin.m * lin.n * lin.k for lin in lins)
     g = gemm_kernel_times(cr, layer, lins, xs, 3, stream, device)
@@ -349,6 +359,90 @@ def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
                          "frac": gops / gt / 1e12 / peak,
                          "peak_note": "measured bf16 burst x 2 (nominal int8/bf16 ratio)"},
             "per_linear_gemm_tops": {lin.name: 2 * lin.m * lin.n * lin.k / tt / 1e12 for lin, tt in g}}
+
+
+def minimax_secondary(cr, device, stream, peaks, steps=5, warmup=2):
+    """MiniMax-H3-shaped qkv projection (K = 5376, N = 16128) at M = 8192 and
+    32768 video tokens through the single-linear entry point: INT8 TOPS."""
+    out = {"workload": "minimax_h3_qkv_k5376_n16128", "metric": "INT8 TOPS (2MNK)"}
+    w = None
+    peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    for m in (8192, 32768):
+        lin = synth.minimax_qkv(m)[0]
+        if w is None:
+            w_bf = lin.w_torch(device)
+            w = cr.quantize_weight(w_bf)
+            del w_bf
+        x = lin.x_torch(device)
+        y = torch.empty((m, lin.n), dtype=torch.bfloat16, device=device)
+        ws = cr.make_workspace(m, w)
+        torch.cuda.synchronize()
+        fn = lambda: cr.convrot_linear_int8(x, w, y, ws, stream)  # noqa: E731
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        keep_busy(stream)
+        t = time_region(fn, steps, stream) / steps
+        g = gemm_kernel_times(cr, _OneWeight(w), [lin], [x], 3, stream, device)[0][1]
+        ops = 2 * m * lin.n * lin.k
+        out["m%d" % m] = {"linear_tops": ops / t / 1e12, "ms": t * 1e3, "gemm_tops": ops / g / 1e12,
+                          "gemm_frac": ops / g / 1e12 / peak, "gemm_ms": g * 1e3}
+        del x, y, ws
+        torch.cuda.empty_cache()
+    out["peak"] = peak
+    return out
+
+
+class _OneWeight:
+    def __init__(self, w):
+        self.w = [w]
+
+
+def stack_secondary(cr, device, stream, peaks, layers=50, steps=5, warmup=2):
+    """The 50-layer stack of the seven Qwen linears (350 INT8 weights,
+    24.4 GB resident) run back to back, one batched call per layer, at
+    M = 12 and M = 512 (one CUDA graph per pass): weight-stream GB/s."""
+    lins12 = synth.qwen_stack(12, layers)
+    t0 = time.time()
+    ws = []
+    for lin in lins12:
+        w_bf = lin.w_torch(device)
+        ws.append(cr.quantize_weight(w_bf))
+        del w_bf
+    torch.cuda.synchronize()
+    out = {"workload": "qwen3vl32b_stack_%dlayers" % layers, "weights": len(ws),
+           "weight_gb": sum(lin.n * lin.k for lin in lins12) / 1e9, "setup_s": time.time() - t0}
+    for m in (12, 512):
+        lins = synth.qwen_stack(m, layers)
+        xs = [lin.x_torch(device) for lin in lins]
+        ys = [torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device) for lin in lins]
+        batches = [cr.LinearBatch(xs[7 * i:7 * i + 7], ws[7 * i:7 * i + 7], ys[7 * i:7 * i + 7])
+                   for i in range(layers)]
+        torch.cuda.synchronize()
+
+        def one_pass():
+            for b in batches:
+                b(stream)
+        with torch.cuda.stream(stream):
+            one_pass()
+        torch.cuda.synchronize()
+        g = capture(one_pass, stream)
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                g.replay()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):     # replay() launches on the current stream
+            t = time_region(g.replay, steps, stream) / steps
+        nbytes = sum(linear_bytes(lin.m, lin.n, lin.k) for lin in lins)
+        ops = sum(2 * lin.m * lin.n * lin.k for lin in lins)
+        out["m%d" % m] = {"gb_s": nbytes / t / 1e9, "ms_per_pass": t * 1e3, "tops": ops / t / 1e12,
+                          "frac_of_measured_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"],
+                          "launches_per_pass": 2 * layers if m <= 256 else None}
+        del g, batches, xs, ys
+        torch.cuda.empty_cache()
+    del ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_profile(args):
@@ -493,6 +587,15 @@ def run_ours(args):
     if not args.no_prefill:
         secondary = prefill_secondary(cr, layer, device, stream, peaks)
     cr.convrot_device_status(stream)
+    others = {}
+    if not args.no_minimax:
+        others["minimax_qkv"] = minimax_secondary(cr, device, stream, peaks)
+        cr.convrot_device_status(stream)
+    if not args.no_stack:
+        del layer, xs, ys, wss, batch, batch_e, dx, dy
+        torch.cuda.empty_cache()
+        others["stack"] = stack_secondary(cr, device, stream, peaks)
+        cr.convrot_device_status(stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -516,7 +619,7 @@ def run_ours(args):
             "per_linear_entry_point": {"ms_per_step": per_linear_t * 1e3,
                                        "value": bytes_step / per_linear_t / 1e9,
                                        "launches_per_step": 2 * len(lins)},
-            "secondary": secondary, "kernel_sources": kernel_source_hash(),
+            "secondary": secondary, "more": others or None, "kernel_sources": kernel_source_hash(),
         }
         print(json.dumps(line), flush=True)
     del graph
@@ -571,6 +674,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-minimax", action="store_true", help="skip the MiniMax qkv TOPS measurement")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 50-layer stack measurement")
     ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
                     help="run a few eager steps of one workload for ncu (no timing)")
     args = ap.parse_args()

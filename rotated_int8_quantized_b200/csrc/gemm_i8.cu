@@ -48,6 +48,7 @@ constexpr int kUmmaK = 32;             // K per tcgen05.mma kind::i8
 constexpr int kATileBytes = kTileA * kBlockK;
 constexpr int kL2PrefetchBlocks = 16;  // weight K blocks pulled into L2 ahead of the grid-dependency wait
 constexpr int kMaxSplitWays = 6;       // K ranges per split tail tile (large M)
+constexpr long long kGroupABytes = 48ll << 20;   // INT8 A operand above this is taken in tile groups
 constexpr int kExtraBars = 7;          // tfull[2], tempty[2], drain, red[2]
 // The split-tail reduction double-buffers at least 32 columns of every other
 // piece's partial in the operand ring of a bn = 256 launch.
@@ -138,6 +139,19 @@ struct SegmentIter {
         return false;
     }
 };
+
+// Tile index -> (A tile, B tile).  Tiles run in groups of group_a A tiles;
+// inside a group the A tile varies fastest, so the CTAs of one wave share a
+// few B tiles and a group's A rows stay in L2 while the group sweeps B.
+__device__ __forceinline__ void tile_coords(const GemmJob &J, int tile, int &ta, int &tb) {
+    const int per_group = J.group_a * (J.n_tiles_b);
+    const int g = tile / per_group;
+    const int w = tile - g * per_group;
+    const int a0 = g * J.group_a;
+    const int ga = (J.tiles_a - a0 < J.group_a) ? J.tiles_a - a0 : J.group_a;
+    tb = w / ga;
+    ta = a0 + (w - tb * ga);
+}
 
 // Dequantise and store 16 consecutive B-rows (j0 .. j0+15) of one A-row i.
 __device__ __forceinline__ void emit16(const GemmJob &J, int swap, int i, int j0, const int32_t (&v)[16]) {
@@ -323,7 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             while (ok && it.next(a, sg)) {
                 const GemmJob &J = a.job[sg.job];
-                const int ta = sg.tile % J.tiles_a, tb = sg.tile / J.tiles_a;
+                int ta, tb;
+                tile_coords(J, sg.tile, ta, tb);
                 const CUtensorMap *tmW = a.swap ? &maps.a[sg.job] : &maps.b[sg.job];
                 const CUtensorMap *tmX = a.swap ? &maps.b[sg.job] : &maps.a[sg.job];
                 const int rowW = a.swap ? ta * kTileA : tb * a.bn;
@@ -360,7 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     continue;
                                 }
                                 const GemmJob &J2 = a.job[s2.job];
-                                const int ta2 = s2.tile % J2.tiles_a, tb2 = s2.tile / J2.tiles_a;
+                                int ta2, tb2;
+                                tile_coords(J2, s2.tile, ta2, tb2);
                                 const CUtensorMap *tw2 = a.swap ? &maps.a[s2.job] : &maps.b[s2.job];
                                 tma_prefetch_l2_2d(tw2, kb2 * kBlockK, a.swap ? ta2 * kTileA : tb2 * a.bn);
                                 ++kb2;
@@ -466,7 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         Segment sg;
         while (it.next(a, sg)) {
             const GemmJob &J = a.job[sg.job];
-            const int ta = sg.tile % J.tiles_a, tb = sg.tile / J.tiles_a;
+            int ta, tb;
+            tile_coords(J, sg.tile, ta, tb);
             const int buf = seg & 1;
             const uint32_t use = (uint32_t)(seg >> 1);
             const int i = ta * kTileA + row;
@@ -758,6 +775,10 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
     if (p->swap) p->slots = num_tiles - tail_tile0;
     p->tail_units = p->swap ? (long long)p->slots * kbpt : 0;
     p->tiles_a[0] = tiles_a;
+    p->tiles_b[0] = tiles_b;
+    // an A operand that would not stay in L2 while a wave sweeps it is
+    // taken in groups of 16 tiles (2048 rows)
+    p->group_a[0] = (!p->swap && (long long)p->rows_a[0] * k > kGroupABytes && tiles_a > 16) ? 16 : tiles_a;
     p->kbpt[0] = kbpt;
     p->tile_base[0] = tail_tile0;
     p->slot0[0] = 0;
@@ -776,6 +797,8 @@ void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, i
         p->rows_a[j] = n[j];
         p->rows_b[j] = m;
         p->tiles_a[j] = (int)((n[j] + kTileA - 1) / kTileA);
+        p->tiles_b[j] = 1;
+        p->group_a[j] = p->tiles_a[j];
         p->kbpt[j] = (int)(k[j] / kBlockK);
         p->tile_base[j] = 0;
         p->slot0[j] = slots;
@@ -853,6 +876,8 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
         J.n = (int)q.n;
         J.k = (int)q.k;
         J.tiles_a = p.tiles_a[j];
+        J.n_tiles_b = p.tiles_b[j];
+        J.group_a = p.group_a[j];
         J.kbpt = p.kbpt[j];
         J.tile_base = p.tile_base[j];
         J.slot0 = p.slot0[j];

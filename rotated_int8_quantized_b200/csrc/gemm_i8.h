@@ -18,6 +18,8 @@ constexpr int kMaxJobs = 8;      // linears in one batched launch
 struct GemmJob {
     int m, n, k;
     int tiles_a;        // 128-row tiles of the A operand
+    int n_tiles_b;      // tiles of the B operand
+    int group_a;        // tile order: groups of group_a A tiles, B tiles outer within a group
     int kbpt;           // 128-byte K blocks per tile
     int tile_base;      // first tile of this job handled by stream-K
     int slot0;          // first workspace slot of this job
@@ -70,7 +72,7 @@ struct GemmPlan {
     int njobs, swap, bn;
     int grid, full_waves, full_tiles, split_ways, split_pieces, stages, acc_cols, tmem_cols, smem_bytes;
     long long tail_units;
-    int tiles_a[kMaxJobs], kbpt[kMaxJobs], tile_base[kMaxJobs], slot0[kMaxJobs];
+    int tiles_a[kMaxJobs], tiles_b[kMaxJobs], group_a[kMaxJobs], kbpt[kMaxJobs], tile_base[kMaxJobs], slot0[kMaxJobs];
     long long unit0[kMaxJobs];
     int64_t rows_a[kMaxJobs], rows_b[kMaxJobs];
     int slots;

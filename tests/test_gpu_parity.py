@@ -143,7 +143,7 @@ GEMM_SHAPES = [
     (257, 512, 512),    # smallest non-swap case, ragged activation tile
     (640, 1000, 1536),  # non-swap, ragged weight tile (1000 % 256), one partial wave
     (9500, 500, 1024),  # 150 tiles: one full wave, 2 tail tiles split in 2 K ranges
-    (5083, 1000, 4096), # 160 tiles: 12 tail tiles split in 8 K ranges, ragged both ways
+    (5083, 1000, 4096), # 160 tiles: 12 tail tiles split in 6 K ranges, ragged both ways
 ]
 
 
@@ -261,6 +261,27 @@ def test_minimax_qkv_sampled(cr):
     rng = np.random.default_rng(4)
     rows_w = np.unique(np.concatenate([[0, lin.n - 1], rng.integers(0, lin.n, 14)]))
     rows_x = np.unique(np.concatenate([[0, lin.m - 1], rng.integers(0, lin.m, 14)]))
+    _sampled_layer_check(cr, lin, rows_w, rows_x)
+
+
+def test_minimax_qkv_m32768_sampled(cr):
+    # 176 MB of INT8 activations: tiles are taken in groups of 16 A tiles
+    lin = synth.minimax_qkv(32768)[0]
+    rng = np.random.default_rng(5)
+    rows_w = np.unique(np.concatenate([[0, lin.n - 1], rng.integers(0, lin.n, 10)]))
+    rows_x = np.unique(np.concatenate([[0, 2047, 2048, lin.m - 1], rng.integers(0, lin.m, 10)]))
+    _sampled_layer_check(cr, lin, rows_w, rows_x)
+
+
+def test_grouped_tile_order_ragged_sampled(cr):
+    # 79 A tiles = 4 groups of 16 + a ragged group of 15, 4 B tiles (the last
+    # ragged), 316 tiles = 2 full waves + 20 tail tiles split along K
+    k = 5376
+    lin = synth.Linear("grouped", 10000, k, 1000, 77, synth.student_t3_scale(synth.stream_key(77, 2), k))
+    rng = np.random.default_rng(77)
+    rows_w = np.unique(np.concatenate([[0, 255, 256, 767, 768, lin.n - 1], rng.integers(0, lin.n, 8)]))
+    rows_x = np.unique(np.concatenate([[0, 2047, 2048, 8191, 8192, 9983, 9984, lin.m - 1],
+                                       rng.integers(0, lin.m, 8)]))
     _sampled_layer_check(cr, lin, rows_w, rows_x)
 
 
