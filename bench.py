@@ -284,6 +284,26 @@ def gemm_kernel_times(cr, layer, lins, xs, reps, stream, device):
     return out
 
 
+def prologue_kernel_times(cr, lins, xs, reps, stream, device):
+    """Per-launch time of the activation prologue (rotation + row
+    quantisation) per linear, CUDA events on the launching stream."""
+    out = []
+    for lin, x in zip(lins, xs):
+        xq = torch.empty((lin.m, lin.k), dtype=torch.int8, device=device)
+        sx = torch.empty((lin.m,), dtype=torch.float32, device=device)
+        torch.cuda.synchronize()
+        cr.convrot_quantize_act(x, xq, sx, stream=stream)
+        keep_busy(stream, 200.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            cr.convrot_quantize_act(x, xq, sx, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out.append((lin, e0.elapsed_time(e1) / reps / 1e3))
+    return out
+
+
 def all_max(v: float, world: int, device="cuda") -> float:
     """The maximum of `v` over the ranks (the slowest rank's time)."""
     if world == 1:
@@ -350,6 +370,7 @@ def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
     gops = sum(2 * lin.m * lin.n * lin.k for lin, _ in g)
     gt = sum(tt for _, tt in g)
     peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    pro = prologue_kernel_times(cr, lins, xs, 5, stream, device)
     del xs, ys, batch
     torch.cuda.empty_cache()
     return {"workload": "qwen3vl32b_layer_7linears_prefill_m4096", "metric": "INT8 TOPS (2MNK)",
@@ -358,7 +379,11 @@ def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
             "roofline": {"bound": "tensor", "achieved": gops / gt / 1e12, "peak": peak, "unit": "TOP/s",
                          "frac": gops / gt / 1e12 / peak,
                          "peak_note": "measured bf16 burst x 2 (nominal int8/bf16 ratio)"},
-            "per_linear_gemm_tops": {lin.name: 2 * lin.m * lin.n * lin.k / tt / 1e12 for lin, tt in g}}
+            "per_linear_gemm_tops": {lin.name: 2 * lin.m * lin.n * lin.k / tt / 1e12 for lin, tt in g},
+            "prologue": {"bytes": "2MK read + MK + 4M written",
+                         "per_linear_us": {lin.name: tt * 1e6 for lin, tt in pro},
+                         "per_linear_gbs": {lin.name: (3 * lin.m * lin.k + 4 * lin.m) / tt / 1e9 for lin, tt in pro},
+                         "layer_us": sum(tt for _, tt in pro) * 1e6}}
 
 
 def minimax_secondary(cr, device, stream, peaks, steps=5, warmup=2):
@@ -437,7 +462,7 @@ def stack_secondary(cr, device, stream, peaks, layers=50, steps=5, warmup=2):
         ops = sum(2 * lin.m * lin.n * lin.k for lin in lins)
         out["m%d" % m] = {"gb_s": nbytes / t / 1e9, "ms_per_pass": t * 1e3, "tops": ops / t / 1e12,
                           "frac_of_measured_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"],
-                          "launches_per_pass": 2 * layers if m <= 256 else None}
+                          "launches_per_pass": 2 * layers if m <= 512 else None}
         del g, batches, xs, ys
         torch.cuda.empty_cache()
     del ws

@@ -174,9 +174,10 @@ typedef struct {
 } convrot_gemm_job_t;
 
 /*
- * Several INT8 GEMMs with the same m (1 <= m <= 256) in ONE launch: every
- * 128-byte K block of every weight is dealt out evenly to the SMs
- * (stream-K), so the whole set streams its weights as one long read.
+ * Several INT8 GEMMs with the same m (1 <= m <= 512) in ONE launch: every
+ * 128-byte K block of every output tile of every product is dealt out
+ * evenly to the SMs (stream-K), so the whole set streams its weights as one
+ * long read.  m > 512: CONVROT_ERR_INVALID_ARG.
  * count <= 8.  Workspace: convrot_gemm_batch_workspace_bytes, zero-filled
  * before first use, left zero-filled.
  */
@@ -201,7 +202,7 @@ typedef struct {
  * Several independent ConvRot INT8 linears with the same token count m, in
  * two launches: one activation prologue over every job's rows, then one
  * GEMM whose K blocks of all weights are dealt out evenly to every SM
- * (m <= 256; larger m runs the GEMMs one after another).  This is how the
+ * (m <= 512; larger m runs the GEMMs one after another).  This is how the
  * linears of one decoder layer that share an input (q/k/v, gate/up) or that
  * are otherwise ready together run at decode size, where a per-linear launch
  * would spend more time starting and draining than streaming its weight.

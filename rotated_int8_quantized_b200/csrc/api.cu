@@ -223,7 +223,7 @@ struct LinearLayout {
 };
 
 void linear_layout(int64_t m, int count, const convrot_linear_job_t *jobs, int sms, LinearLayout *L) {
-    L->batched_gemm = (m <= 256);
+    L->batched_gemm = (m <= convrot::kMaxSwapM);
     size_t g = 0;
     if (L->batched_gemm) {
         int64_t n[kMaxBatch], k[kMaxBatch];
@@ -288,7 +288,7 @@ convrot_status_t run_linear(int64_t m, int count, const convrot_linear_job_t *jo
 namespace {
 
 convrot_status_t check_gemm_jobs(int64_t m, int count, const convrot_gemm_job_t *jobs) {
-    if (!jobs || count < 1 || count > kMaxBatch || m < 1 || m > 256) return CONVROT_ERR_INVALID_ARG;
+    if (!jobs || count < 1 || count > kMaxBatch || m < 1 || m > convrot::kMaxSwapM) return CONVROT_ERR_INVALID_ARG;
     for (int j = 0; j < count; ++j) {
         const convrot_gemm_job_t &J = jobs[j];
         if (!J.xq || !J.sx || (!J.y_bf16 && !J.acc)) return CONVROT_ERR_INVALID_ARG;

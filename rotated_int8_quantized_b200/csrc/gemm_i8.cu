@@ -84,17 +84,32 @@ struct Segment {
     int split;          // >= 0: a piece of a split tail tile (private partial)
 };
 
+// The stream-K CTA whose unit range [total*c/G, total*(c+1)/G) holds unit u.
+__device__ __forceinline__ int stream_k_cta(long long u, long long total, int G) {
+    int c = (int)((u * G) / total);
+    while (c + 1 < G && (total * (c + 1)) / G <= u) ++c;
+    while (c > 0 && (total * c) / G > u) --c;
+    return c;
+}
+
+// Stream-K with replication R = a.rep: the grid is Q = G / R groups of R
+// consecutive CTAs; group q takes a contiguous share of the units (K blocks
+// of B tiles when R > 1, of whole tiles when R = 1) and CTA r of the group
+// computes A tile r for them, so the R CTAs of a group read the same weight
+// blocks at about the same time and share them in L2.
 struct SegmentIter {
-    int wave, j;
+    int wave, j, r;
     bool piece_done;
     long long u, u_end;
     __device__ __forceinline__ void init(const GemmArgs &a) {
         wave = 0;
         j = 0;
         piece_done = false;
-        const long long c = blockIdx.x, G = gridDim.x;
-        u = a.tail_units * c / G;
-        u_end = a.tail_units * (c + 1) / G;
+        const int R = a.rep;
+        const long long q = blockIdx.x / R, Q = gridDim.x / R;
+        r = (int)blockIdx.x - (int)q * R;
+        u = a.tail_units * q / Q;
+        u_end = a.tail_units * (q + 1) / Q;
     }
     __device__ __forceinline__ bool next(const GemmArgs &a, Segment &s) {
         if (wave < a.full_waves && wave * (int)gridDim.x + (int)blockIdx.x < a.full_tiles) {
@@ -127,8 +142,11 @@ struct SegmentIter {
             const long long lu = u - J.unit0;
             const long long t = lu / J.kbpt;
             s.job = j;
-            s.tile = J.tile_base + (int)t;
-            s.slot = J.slot0 + (int)t;
+            s.tile = J.tile_base + (int)t * a.rep + r;
+            // a tile shared by several CTAs sums in the workspace slot of the
+            // last of them (its range starts inside this tile, so no other
+            // shared tile maps to the same slot)
+            s.slot = stream_k_cta(J.unit0 + (t + 1) * J.kbpt - 1, a.tail_units, (int)gridDim.x / a.rep) * a.rep + r;
             s.kb0 = (int)(lu - t * J.kbpt);
             const long long rem = u_end - u;
             s.kb1 = (int)((long long)s.kb0 + rem < J.kbpt ? s.kb0 + rem : J.kbpt);
@@ -151,61 +169,6 @@ __device__ __forceinline__ void tile_coords(const GemmJob &J, int tile, int &ta,
     const int ga = (J.tiles_a - a0 < J.group_a) ? J.tiles_a - a0 : J.group_a;
     tb = w / ga;
     ta = a0 + (w - tb * ga);
-}
-
-// Dequantise and store 16 consecutive B-rows (j0 .. j0+15) of one A-row i.
-__device__ __forceinline__ void emit16(const GemmJob &J, int swap, int i, int j0, const int32_t (&v)[16]) {
-    if (!swap) {
-        const int m = i;
-        if (m >= J.m) return;
-        const float sxm = J.sx[m];
-        const bool full = (j0 + 16 <= J.n) && ((J.n & 7) == 0);
-        if (J.acc) {
-            int32_t *dst = J.acc + (size_t)m * J.n + j0;
-            if (full) {
-#pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<int4 *>(dst + e) = make_int4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-            } else {
-                for (int e = 0; e < 16 && j0 + e < J.n; ++e) dst[e] = v[e];
-            }
-        }
-        if (J.y) {
-            __nv_bfloat16 *dst = J.y + (size_t)m * J.n + j0;
-            if (full) {
-                uint32_t pk[8];
-#pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    float f0 = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), __ldg(J.sw + j0 + e));
-                    float f1 = __fmul_rn(__fmul_rn(__int2float_rn(v[e + 1]), sxm), __ldg(J.sw + j0 + e + 1));
-                    __nv_bfloat162 h = __halves2bfloat162(__float2bfloat16_rn(f0), __float2bfloat16_rn(f1));
-                    pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
-                }
-                reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                reinterpret_cast<uint4 *>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            } else {
-                for (int e = 0; e < 16 && j0 + e < J.n; ++e) {
-                    float f = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), __ldg(J.sw + j0 + e));
-                    dst[e] = __float2bfloat16_rn(f);
-                }
-            }
-        }
-    } else {
-        const int n = i;
-        if (n >= J.n) return;
-        const float swn = J.sw[n];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int m = j0 + e;
-            if (m < J.m) {
-                if (J.acc) J.acc[(size_t)m * J.n + n] = v[e];
-                if (J.y) {
-                    float f = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), __ldg(J.sx + m)), swn);
-                    J.y[(size_t)m * J.n + n] = __float2bfloat16_rn(f);
-                }
-            }
-        }
-    }
 }
 
 // Large-M orientation: dequantise and store columns j0 .. j0+15 of output
@@ -245,6 +208,60 @@ __device__ __forceinline__ void emit_row16(const GemmJob &J, int m, int j0, cons
     }
 }
 
+// Swapped orientation (A = weight rows n, B = activation rows m): the 16
+// accumulators of weight row n = a0 + row for activation rows j0 .. j0+15.
+// The BF16 results are transposed through `stg` ([16][128], this chunk's
+// buffer) so that each output row leaves as 16-byte segments instead of
+// 2-byte scatters.  Called by all 128 epilogue threads (it holds a barrier).
+__device__ __forceinline__ void emit_swap16(const GemmJob &J, int a0, int row, int tid, int j0,
+                                            const int32_t (&v)[16], float srow, const float *scol,
+                                            __nv_bfloat16 *stg) {
+    const int n = a0 + row;
+    if (J.acc && n < J.n) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (j0 + e < J.m) J.acc[(size_t)(j0 + e) * J.n + n] = v[e];
+    }
+    if (!J.y) return;
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+        stg[e * kTileA + row] = __float2bfloat16_rn(__fmul_rn(__fmul_rn(__int2float_rn(v[e]), scol[e]), srow));
+    named_bar_sync(1, 128);
+    const bool vec = (J.n & 7) == 0;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int idx = tid + q * 128;          // 16 rows x 16 segments of 8 columns
+        const int ml = idx >> 4, seg8 = idx & 15;
+        const int m = j0 + ml, nb = a0 + seg8 * 8;
+        if (m >= J.m || nb >= J.n) continue;
+        const __nv_bfloat16 *src = stg + ml * kTileA + seg8 * 8;
+        __nv_bfloat16 *dst = J.y + (size_t)m * J.n + nb;
+        if (vec && nb + 8 <= J.n) {
+            *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
+        } else {
+            for (int e = 0; e < 8 && nb + e < J.n; ++e) dst[e] = src[e];
+        }
+    }
+}
+
+// Dequantise and store the 16 accumulators of A-row a0 + row and B-rows
+// j0 .. j0+15 in either orientation.  srow is the scale of the A row and
+// scol[e] the scale of B-row j0 + e (both staged by the caller): sx[m] and
+// sw[n] for large M, sw[n] and sx[m] for the swapped (weights = A)
+// orientation.  Both compute bf16(((float)acc * sx[m]) * sw[n]).  Called by
+// all 128 epilogue threads; `chunk` counts the calls (it picks the transpose
+// buffer of the swapped orientation).
+__device__ __forceinline__ void emit16s(const GemmJob &J, int swap, int a0, int row, int tid, int j0,
+                                        const int32_t (&v)[16], float srow, const float *scol,
+                                        __nv_bfloat16 *y_stage, int &chunk) {
+    if (!swap) {
+        emit_row16(J, a0 + row, j0, v, srow, scol);
+        return;
+    }
+    emit_swap16(J, a0, row, tid, j0, v, srow, scol, y_stage + (chunk & 1) * 16 * kTileA);
+    ++chunk;
+}
+
 // Two TMEM loads of 16 columns each, one wait.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, int32_t (&v0)[16], int32_t (&v1)[16]) {
     uint32_t r0[16], r1[16];
@@ -278,12 +295,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tempty_bar = tfull_bar + 16u;
     const uint32_t drain_bar = tempty_bar + 16u;
     const uint32_t red_bar = drain_bar + 8u;
-    uint8_t *misc = smem + bar_off + 8u * (2 * S + kExtraBars);
+    uint8_t *misc = smem + ((bar_off + 8u * (2 * S + kExtraBars) + 15u) & ~15u);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(misc);
     volatile int *ticket = reinterpret_cast<volatile int *>(misc + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 8);
     volatile int *red_ok = reinterpret_cast<volatile int *>(misc + 12);
-    float *sw_stage = reinterpret_cast<float *>(misc + 16);     // [2][256] weight scales of a tile
+    float *sw_stage = reinterpret_cast<float *>(misc + 16);     // [2][256] B-row scales of a tile
+    // [2][16][128] BF16: swapped-orientation output chunks, transposed so
+    // that they leave as 16-byte row segments
+    __nv_bfloat16 *y_stage = reinterpret_cast<__nv_bfloat16 *>(misc + 16 + 2 * 256 * 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -476,6 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;       // row of the A tile
         const int ew = warp - 2;
+        const int tid = ew * 32 + lane;
+        int ychunk = 0;
         int seg = 0;
         SegmentIter it;
         it.init(a);
@@ -487,19 +509,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int buf = seg & 1;
             const uint32_t use = (uint32_t)(seg >> 1);
             const int i = ta * kTileA + row;
-            // large M: the tile's weight scales go to shared memory and the
-            // row scale to a register while the accumulator is still being
-            // computed (double-buffered by segment parity; the barrier
-            // below publishes them)
-            float *sws = sw_stage + (seg & 1) * 256;
-            float sxm = 0.f;
-            if (!a.swap) {
-                const int tid = ew * 32 + lane;
+            // the scales of the tile's B rows go to shared memory and the
+            // scale of this thread's A row to a register while the
+            // accumulator is still being computed (double-buffered by
+            // segment parity; the barrier below publishes them)
+            float *scol = sw_stage + (seg & 1) * 256;
+            float srow = 0.f;
+            {
+                const float *cs = a.swap ? J.sx : J.sw;
+                const int clim = a.swap ? J.m : J.n;
                 for (int cidx = tid; cidx < a.bn; cidx += 128) {
                     const int col = tb * a.bn + cidx;
-                    sws[cidx] = col < J.n ? __ldg(J.sw + col) : 0.f;
+                    scol[cidx] = col < clim ? __ldg(cs + col) : 0.f;
                 }
-                if (i < J.m) sxm = __ldg(J.sx + i);
+                const float *rs = a.swap ? J.sw : J.sx;
+                if (i < (a.swap ? J.n : J.m)) srow = __ldg(rs + i);
             }
             const bool full = mbar_wait_bounded(tfull_bar + 8u * buf, use & 1u, abort_flag);
             if (!named_bar_and(1, 128, full)) break;
@@ -512,8 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     tmem_ld32(tbase + (uint32_t)c, v0, v1);
                     const int j0 = tb * a.bn + c;
-                    emit_row16(J, i, j0, v0, sxm, sws + c);
-                    emit_row16(J, i, j0 + 16, v1, sxm, sws + c + 16);
+                    emit_row16(J, i, j0, v0, srow, scol + c);
+                    emit_row16(J, i, j0 + 16, v1, srow, scol + c + 16);
                 }
             } else if (sg.split < 0) {
                 for (int c = 0; c < a.bn / 16; ++c) {
@@ -525,7 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
                     if (whole) {
-                        emit16(J, a.swap, i, tb * a.bn + c * 16, v);
+                        emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + c * 16, v, srow, scol + c * 16,
+                                y_stage, ychunk);
                     } else {
                         int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
 #pragma unroll
@@ -635,8 +660,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
                             }
                             const int j0 = tb * a.bn + col0 + cc;
-                            emit_row16(J, i, j0, v0, sxm, sws + col0 + cc);
-                            emit_row16(J, i, j0 + 16, v1, sxm, sws + col0 + cc + 16);
+                            emit_row16(J, i, j0, v0, srow, scol + col0 + cc);
+                            emit_row16(J, i, j0 + 16, v1, srow, scol + col0 + cc + 16);
                         }
                         named_bar_sync(1, 128);     // buffer (r & 1) is read by everyone
                         if (r + 2 < rounds && ew == 0 && lane == 0) {
@@ -648,7 +673,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // leave the other pieces' regions zero again (the
                         // workspace is zero between calls), then the counter
                         const int4 z = make_int4(0, 0, 0, 0);
-                        const int tid = ew * 32 + lane;
                         const size_t n4 = (size_t)a.bn * kTileA / 4;
                         for (int sp = 0; sp < ways; ++sp) {
                             if (sp == sg.split) continue;
@@ -683,14 +707,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool last = (*ticket != 0);
                 if (last) {
                     __threadfence();
-                    for (int c = 0; c < a.bn / 16; ++c) {
+                    const int chunks = a.bn / 16;
+                    int c = 0;
+                    // four 16-column chunks in flight at a time (wide tiles)
+                    for (; c + 4 <= chunks; c += 4) {
+                        int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
+                        int32_t v[4][16];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h)
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) v[h][e] = __ldcg(p + (size_t)(h * 16 + e) * kTileA);
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) __stcg(p + (size_t)e * kTileA, 0);
+#pragma unroll
+                        for (int h = 0; h < 4; ++h)
+                            emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + (c + h) * 16, v[h], srow,
+                                    scol + (c + h) * 16, y_stage, ychunk);
+                    }
+                    for (; c < chunks; ++c) {
                         int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
                         int32_t v[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = __ldcg(p + (size_t)e * kTileA);
 #pragma unroll
                         for (int e = 0; e < 16; ++e) __stcg(p + (size_t)e * kTileA, 0);
-                        emit16(J, a.swap, i, tb * a.bn + c * 16, v);
+                        emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + c * 16, v, srow, scol + c * 16,
+                                y_stage, ychunk);
                     }
                     if (ew == 0 && lane == 0) a.counters[sg.slot] = 0;
                 }
@@ -720,7 +762,8 @@ static void plan_common(GemmPlan *p) {
     int cols = 32;
     while (cols < 2 * p->bn) cols <<= 1;
     p->tmem_cols = cols;
-    p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + kExtraBars) + 16 + 2 * 256 * 4;
+    p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + kExtraBars) + 16 + 16 + 2 * 256 * 4 +
+                    2 * 16 * kTileA * 2;
     // workspace: counters, then INT32 partial tiles [slots][bn][128]
     const size_t cnt = ((size_t)p->slots * 4 + 255) / 256 * 256;
     p->ws_counters_off = 0;
@@ -730,6 +773,12 @@ static void plan_common(GemmPlan *p) {
 }
 
 void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
+    if (m > 256 && m <= kMaxSwapM) {
+        // a few hundred rows: too few 128 x 256 tiles for 148 SMs; stream-K
+        // over all of them, as in a batched launch
+        plan_gemm_batch(m, 1, &n, &k, num_sms, p);
+        return;
+    }
     *p = GemmPlan{};
     p->njobs = 1;
     p->swap = (m <= 256) ? 1 : 0;
@@ -772,8 +821,12 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
         }
         tail_tile0 = num_tiles;
     }
-    if (p->swap) p->slots = num_tiles - tail_tile0;
-    p->tail_units = p->swap ? (long long)p->slots * kbpt : 0;
+    if (p->swap) {
+        // stream-K over the tiles after the full waves; a tile shared by
+        // several CTAs sums in the slot of one of them (one slot per CTA)
+        p->tail_units = (long long)(num_tiles - tail_tile0) * kbpt;
+        p->slots = p->tail_units > 0 ? p->grid : 0;
+    }
     p->tiles_a[0] = tiles_a;
     p->tiles_b[0] = tiles_b;
     // an A operand that would not stay in L2 while a wave sweeps it is
@@ -781,7 +834,6 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
     p->group_a[0] = (!p->swap && (long long)p->rows_a[0] * k > kGroupABytes && tiles_a > 16) ? 16 : tiles_a;
     p->kbpt[0] = kbpt;
     p->tile_base[0] = tail_tile0;
-    p->slot0[0] = 0;
     p->unit0[0] = 0;
     plan_common(p);
 }
@@ -789,26 +841,32 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
 void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p) {
     *p = GemmPlan{};
     p->njobs = njobs;
-    p->swap = 1;
-    p->bn = (int)((m + 15) / 16 * 16);
+    // m <= 256: the weights are the 128-row A operand and the activations
+    // one B tile of roundup16(m) rows.  256 < m <= 512: activations are A
+    // (up to four 128-row tiles), weights B (256-row tiles), and the A tiles
+    // vary fastest, so a CTA reuses a weight tile from L2 for every
+    // activation tile
+    p->swap = m <= 256 ? 1 : 0;
+    p->bn = p->swap ? (int)((m + 15) / 16 * 16) : 256;
+    // large-M orientation: the A tiles (<= 4) are replicated over groups of
+    // CTAs, the units are the K blocks of the weight (B) tiles
+    p->rep = p->swap ? 1 : (int)((m + kTileA - 1) / kTileA);
     long long units = 0;
-    int slots = 0;
     for (int j = 0; j < njobs; ++j) {
-        p->rows_a[j] = n[j];
-        p->rows_b[j] = m;
-        p->tiles_a[j] = (int)((n[j] + kTileA - 1) / kTileA);
-        p->tiles_b[j] = 1;
+        p->rows_a[j] = p->swap ? n[j] : m;
+        p->rows_b[j] = p->swap ? m : n[j];
+        p->tiles_a[j] = (int)((p->rows_a[j] + kTileA - 1) / kTileA);
+        p->tiles_b[j] = (int)((p->rows_b[j] + p->bn - 1) / p->bn);
         p->group_a[j] = p->tiles_a[j];
         p->kbpt[j] = (int)(k[j] / kBlockK);
         p->tile_base[j] = 0;
-        p->slot0[j] = slots;
         p->unit0[j] = units;
-        slots += p->tiles_a[j];
-        units += (long long)p->tiles_a[j] * p->kbpt[j];
+        units += (long long)(p->swap ? p->tiles_a[j] : p->tiles_b[j]) * p->kbpt[j];
     }
-    p->grid = (int)(units < num_sms ? units : num_sms);
+    const long long groups = num_sms / p->rep;
+    p->grid = (int)(units < groups ? units : groups) * p->rep;
     p->full_waves = 0;
-    p->slots = slots;
+    p->slots = p->grid;
     p->tail_units = units;
     plan_common(p);
 }
@@ -858,6 +916,7 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
     a.full_tiles = p.full_tiles;
     a.split_ways = p.split_ways;
     a.split_pieces = p.split_pieces;
+    a.rep = p.rep > 0 ? p.rep : 1;
     a.tail_units = p.tail_units;
     a.stages = p.stages;
     a.acc_cols = p.acc_cols;
@@ -880,7 +939,6 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
         J.group_a = p.group_a[j];
         J.kbpt = p.kbpt[j];
         J.tile_base = p.tile_base[j];
-        J.slot0 = p.slot0[j];
         J.unit0 = p.unit0[j];
         J.sx = q.sx;
         J.sw = q.sw;

@@ -12,6 +12,7 @@ namespace convrot {
 
 constexpr int kMaxStages = 8;
 constexpr int kMaxJobs = 8;      // linears in one batched launch
+constexpr int kMaxSwapM = 512;   // rows up to which the weights are the A operand (stream-K)
 
 // ------------------------------------------------------------------ GEMM
 // One product of a (batched) launch, as the kernel sees it.
@@ -22,7 +23,6 @@ struct GemmJob {
     int group_a;        // tile order: groups of group_a A tiles, B tiles outer within a group
     int kbpt;           // 128-byte K blocks per tile
     int tile_base;      // first tile of this job handled by stream-K
-    int slot0;          // first workspace slot of this job
     long long unit0;    // first stream-K unit (K block) of this job
     const float *sx;
     const float *sw;
@@ -42,6 +42,7 @@ struct GemmArgs {
     int split_ways;     // 0: no split tail
     int split_pieces;   // tail tiles x split_ways (CTAs 0 .. pieces-1 take one each)
     long long tail_units;   // K blocks dealt out by stream-K
+    int rep;            // stream-K CTAs per group sharing a weight tile (one per A tile), 1: none
     int stages;
     int acc_cols;       // TMEM columns per accumulator buffer
     int tmem_cols;      // TMEM columns allocated (power of two >= 32)
@@ -70,9 +71,9 @@ struct GemmProblem {
 // Host-side tiling of a launch.
 struct GemmPlan {
     int njobs, swap, bn;
-    int grid, full_waves, full_tiles, split_ways, split_pieces, stages, acc_cols, tmem_cols, smem_bytes;
+    int grid, full_waves, full_tiles, split_ways, split_pieces, stages, acc_cols, tmem_cols, smem_bytes, rep;
     long long tail_units;
-    int tiles_a[kMaxJobs], tiles_b[kMaxJobs], group_a[kMaxJobs], kbpt[kMaxJobs], tile_base[kMaxJobs], slot0[kMaxJobs];
+    int tiles_a[kMaxJobs], tiles_b[kMaxJobs], group_a[kMaxJobs], kbpt[kMaxJobs], tile_base[kMaxJobs];
     long long unit0[kMaxJobs];
     int64_t rows_a[kMaxJobs], rows_b[kMaxJobs];
     int slots;
@@ -82,8 +83,9 @@ struct GemmPlan {
 // Single product: whole tiles dealt round-robin in full waves, the last
 // partial wave split along K (stream-K).
 void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p);
-// Several products with the same m <= 256 in one launch: every K block of
-// every weight dealt out evenly by stream-K.
+// Several products with the same m <= kMaxSwapM in one launch: every K
+// block of every (weight tile, activation tile) pair dealt out evenly by
+// stream-K.
 void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p);
 
 cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws, cudaStream_t stream,

@@ -64,28 +64,38 @@ __device__ __forceinline__ RowScale make_row_scale(float amax) {
 // The fast path is straight-line code over the 16 values (independent work
 // for the scheduler); the division runs only where some thread of the warp
 // needs it.  Every thread of `mask` (the active threads) must call it.
+// Rounding to the nearest integer, ties to even, on the FP32 pipe instead of
+// the conversion unit: for |t| < 2^22 the sum fl(t + 1.5 * 2^23) has an ulp
+// of 1, so the addition itself rounds t to an integer (round-to-nearest-even
+// is the FP32 mode) and that integer sits in the low mantissa bits of the sum.
+constexpr float kRoundMagic = 12582912.0f;          // 1.5 * 2^23
+constexpr int kRoundMagicBits = 0x4B400000;         // its bit pattern
+
 __device__ __forceinline__ uint4 quant16(const float (&y)[16], const RowScale &rs, unsigned mask) {
-    float f[16];
+    int code[16];
     bool slow = false;
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const float t = __fmul_rn(y[e], rs.r);
-        f[e] = rintf(t);
-        slow |= !(fabsf(t - f[e]) < 0.49997f);
+        const float big = __fadd_rn(t, kRoundMagic);
+        code[e] = __float_as_int(big) - kRoundMagicBits;            // rne(t)
+        slow |= !(fabsf(__fsub_rn(t, __fsub_rn(big, kRoundMagic))) < 0.49997f);
     }
     slow = slow || !rs.fast;
     if (__any_sync(mask, slow) && slow) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const float t = __fmul_rn(y[e], rs.r);
-            if (!rs.fast || !(fabsf(t - rintf(t)) < 0.49997f)) f[e] = rintf(__fdiv_rn(y[e], rs.s));
+            const float f = __fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic);
+            if (!rs.fast || !(fabsf(__fsub_rn(t, f)) < 0.49997f))
+                code[e] = __float_as_int(__fadd_rn(__fdiv_rn(y[e], rs.s), kRoundMagic)) - kRoundMagicBits;
         }
     }
     uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-        const float c = rs.zero ? 0.0f : fminf(fmaxf(f[e], -127.0f), 127.0f);
-        w[e >> 2] |= (uint32_t)(uint8_t)(int8_t)(int)c << (8 * (e & 3));
+        const int c = rs.zero ? 0 : min(max(code[e], -127), 127);
+        w[e >> 2] |= (uint32_t)(c & 0xFF) << (8 * (e & 3));
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
@@ -104,6 +114,11 @@ constexpr int kMaxSlots = 32;          // 512 threads
 constexpr int kXchFull = 16 * 17;     // doubles per slot: whole 16 x 16 transpose, padded
 constexpr int kXchHalf = 16 * 9;      // doubles per slot: half of it at a time, padded
 constexpr int kMaxParts = 8;           // CTAs per row (portable cluster size)
+// FP32 staging of a rotated group: 256 values padded to 272 so that the two
+// slots of a warp write different banks; inside, 16-value chunks whose four
+// float4 parts are XOR-swizzled so that the quantiser's 16-byte reads of
+// consecutive chunks are conflict-free.
+constexpr int kYGroupStride = 272;
 constexpr int kSlotsSmemMax = 226 * 1024;   // dynamic shared memory per CTA (227 KB minus the static part)
 
 __device__ __forceinline__ void fwht16_regs(double (&v)[16]) {
@@ -248,11 +263,12 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                 __syncwarp(half_mask);
             }
             fwht16_regs(x);                                  // index bits 4-7
-            float *yg = ybuf + (size_t)(g - g0) * 256 + t;
+            // output 16*i + t of the group is element t of chunk i
+            float *yg = ybuf + (size_t)(g - g0) * kYGroupStride + (t & 3);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float y = __double2float_rn(x[i] * 0.0625);   // / sqrt(256), exact
-                yg[16 * i] = y;
+                yg[16 * i + 4 * ((t >> 2) ^ ((i >> 1) & 3))] = y;
                 amax = fmaxf(amax, fabsf(y));
             }
         }
@@ -290,11 +306,12 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
         const int c = c0 + tid;
         const unsigned mask = __ballot_sync(__activemask(), c < chunks);
         if (c < chunks) {
-            const float4 *src = reinterpret_cast<const float4 *>(ybuf + c * 16);
+            const int ci = c & 15;     // chunk within its group
+            const float4 *src = reinterpret_cast<const float4 *>(ybuf + (size_t)(c >> 4) * kYGroupStride + ci * 16);
             float y[16];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float4 f = src[i];
+                const float4 f = src[i ^ ((ci >> 1) & 3)];
                 y[4 * i] = f.x;
                 y[4 * i + 1] = f.y;
                 y[4 * i + 2] = f.z;
@@ -313,7 +330,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
 template <int GPS, bool HALF>
 static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int max_slots, int max_local_groups) {
     cfg.blockDim = dim3(max_slots * 16);
-    cfg.dynamicSmemBytes = (size_t)max_slots * (HALF ? kXchHalf : kXchFull) * 8 + (size_t)max_local_groups * 256 * 4;
+    cfg.dynamicSmemBytes = (size_t)max_slots * (HALF ? kXchHalf : kXchFull) * 8 + (size_t)max_local_groups * kYGroupStride * 4;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -366,7 +383,7 @@ static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, bool h
     *max_slots = ms;
     *max_gps = mg;
     *max_local = ml;
-    return (size_t)ms * (half ? kXchHalf : kXchFull) * 8 + (size_t)ml * 256 * 4;
+    return (size_t)ms * (half ? kXchHalf : kXchFull) * 8 + (size_t)ml * kYGroupStride * 4;
 }
 
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl) {

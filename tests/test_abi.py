@@ -80,9 +80,14 @@ def test_workspace_sizes_follow_the_tiling(lib):
     if torch.cuda.is_available():
         pytest.skip("sizes below assume the 148-SM default used without a device")
     # decode: weight is the 128-row operand, 12 tokens pad to one 16-row
-    # tile; 64 weight tiles < 148 SMs, so every tile is split along K and
-    # needs an INT32 partial tile (16 x 128 x 4 B) and a counter.
-    assert lib.convrot_gemm_workspace_bytes(12, 8192, 5120) == 256 + 64 * 16 * 128 * 4
+    # tile; 64 weight tiles < 148 SMs, so the K blocks are dealt out over all
+    # 148 CTAs (stream-K) and a tile shared by several CTAs sums in the slot
+    # of one of them: 148 counters (768 B) + 148 INT32 partial tiles of
+    # 16 x 128 x 4 B
+    assert lib.convrot_gemm_workspace_bytes(12, 8192, 5120) == 768 + 148 * 16 * 128 * 4
+    # 512 rows: four 128-row activation tiles x 20 weight tiles of 256 rows,
+    # stream-K again (128 x 256 INT32 partial tiles)
+    assert lib.convrot_gemm_workspace_bytes(512, 5120, 5120) == 768 + 148 * 256 * 128 * 4
     # prefill: 32 x 100 tiles of 128 x 256, whole tiles only (22 waves over
     # 148 SMs, the last one partial): no scratch at all
     assert lib.convrot_gemm_workspace_bytes(4096, 25600, 5120) == 0

@@ -140,7 +140,10 @@ GEMM_SHAPES = [
     (17, 1000, 1280),   # ragged weight tile, activation tile of 32
     (100, 640, 2560),   # swap with bn = 112
     (256, 512, 768),    # largest swap case, bn = 256
-    (257, 512, 512),    # smallest non-swap case, ragged activation tile
+    (257, 512, 512),    # stream-K with activations = A: 3 tiles, the last of 1 row
+    (400, 640, 5120),   # stream-K, 4 x 3 tiles, many K blocks per CTA
+    (512, 1000, 2560),  # stream-K, 4 full activation tiles, ragged weight tile
+    (513, 512, 512),    # smallest large-M case, ragged activation tile
     (640, 1000, 1536),  # non-swap, ragged weight tile (1000 % 256), one partial wave
     (9500, 500, 1024),  # 150 tiles: one full wave, 2 tail tiles split in 2 K ranges
     (5083, 1000, 4096), # 160 tiles: 12 tail tiles split in 6 K ranges, ragged both ways
@@ -300,6 +303,8 @@ BATCH_CASES = [
     (100, [(512, 512), (1536, 256), (256, 640)]),
     (64, [(25600, 640)]),
     (300, [(768, 512), (512, 1000)]),
+    (512, [(5120, 1024), (2560, 640), (512, 384)]),
+    (600, [(768, 512), (512, 1000)]),
 ]
 
 
