@@ -68,6 +68,7 @@ def _load():
         lib.oracle_gemm_i32.argtypes = [P, P, I64, I64, I64, P]
         lib.oracle_gemm_i32.restype = I64
         lib.oracle_dequant_bf16.argtypes = [P, P, P, I64, I64, P]
+        lib.oracle_dequant_bf16_bias.argtypes = [P, P, P, P, I64, I64, P]
         lib.oracle_dequant_bf16.restype = None
         lib.oracle_rotate_quantize.argtypes = [P, I64, I64, ctypes.c_int, P, P]
         lib.oracle_rotate_quantize.restype = I64
@@ -172,20 +173,27 @@ def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:
     return acc
 
 
-def dequant_bf16(acc: np.ndarray, sx: np.ndarray, sw: np.ndarray) -> np.ndarray:
-    """Y = bf16(((float)acc * sx[m]) * sw[n]) as uint16 bit patterns."""
+def dequant_bf16(acc: np.ndarray, sx: np.ndarray, sw: np.ndarray, bias=None) -> np.ndarray:
+    """Y = bf16(((float)acc * sx[m]) * sw[n] [+ bias[n]]) as uint16 bit
+    patterns; ``bias`` is BF16 bits [n] or None."""
     acc = np.ascontiguousarray(acc, dtype=np.int32)
     sx = np.ascontiguousarray(sx, dtype=np.float32)
     sw = np.ascontiguousarray(sw, dtype=np.float32)
     m, n = acc.shape
     y = np.empty((m, n), dtype=np.uint16)
-    _load().oracle_dequant_bf16(_ptr(acc), _ptr(sx), _ptr(sw), m, n, _ptr(y))
+    if bias is None:
+        _load().oracle_dequant_bf16(_ptr(acc), _ptr(sx), _ptr(sw), m, n, _ptr(y))
+    else:
+        b = _bf16_bits(np.asarray(bias).reshape(-1))
+        assert b.shape == (n,)
+        _load().oracle_dequant_bf16_bias(_ptr(acc), _ptr(sx), _ptr(sw), _ptr(b), m, n, _ptr(y))
     return y
 
 
 def linear_int8(x_bf16: np.ndarray, wq: np.ndarray, sw: np.ndarray,
-                group: int = 256):
-    """Forward of the layer on pre-quantised weights.
+                group: int = 256, bias=None):
+    """Forward of the layer on pre-quantised weights (optional BF16 bias
+    bits [n], added in FP32 before the rounding to BF16).
 
     Returns a dict with ``y`` (BF16 bits [m,n]), ``xq``, ``sx`` and ``acc``.
     """
@@ -203,6 +211,8 @@ def linear_int8(x_bf16: np.ndarray, wq: np.ndarray, sw: np.ndarray,
     if rc != 0:
         raise OracleError({-1: "bad arguments", -2: "inexact rotation group",
                            -3: "INT32 overflow"}[rc])
+    if bias is not None:
+        y = dequant_bf16(acc, sx, sw, bias)
     return {"y": y, "xq": xq, "sx": sx, "acc": acc}
 
 

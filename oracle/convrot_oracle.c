@@ -308,6 +308,26 @@ void oracle_dequant_bf16(const int32_t *acc, const float *sx, const float *sw,
         }
 }
 
+/*
+ * The same with an optional per-output-channel bias (BF16 bits [n], or
+ * NULL for none): y[m,n] = bf16_rne( ((float)acc * sx[m]) * sw[n] + b[n] ),
+ * the bias added to the FP32 product and the sum rounded once to BF16.  The
+ * source pages quantise bias-free projections; the bias is this library's
+ * extension for layers that carry one.
+ */
+void oracle_dequant_bf16_bias(const int32_t *acc, const float *sx, const float *sw,
+                              const uint16_t *bias, int64_t m, int64_t n, uint16_t *y)
+{
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t j = 0; j < n; ++j) {
+            float v = (float)acc[i * n + j];
+            v = v * sx[i];
+            v = v * sw[j];
+            if (bias) v = v + bf16_bits_to_float(bias[j]);
+            y[i * n + j] = oracle_float_to_bf16(v);
+        }
+}
+
 /* ------------------------------------------------------------------ */
 /* Composites                                                          */
 /* ------------------------------------------------------------------ */

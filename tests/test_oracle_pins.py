@@ -288,6 +288,33 @@ def test_dequant_matches_definition():
     assert not np.array_equal(y[:, :6], y_bad)
 
 
+def test_dequant_bias_closed_forms():
+    f2b = synth.f32_to_bf16_bits
+    # acc = 0: the output is the bias itself, bit for bit
+    bias = f2b(np.array([1.5, -3.25, 0.0, 2.0 ** -20, -65504.0], np.float32))
+    y = oracle.dequant_bf16(np.zeros((2, 5), np.int32), np.ones(2, np.float32), np.ones(5, np.float32), bias)
+    assert np.array_equal(y, np.stack([bias, bias]))
+    # a zero bias changes nothing; None means no bias
+    rng = np.random.default_rng(8)
+    acc = rng.integers(-10 ** 6, 10 ** 6, (3, 7)).astype(np.int32)
+    sx, sw = rng.uniform(0.1, 1, 3).astype(np.float32), rng.uniform(0.1, 1, 7).astype(np.float32)
+    assert np.array_equal(oracle.dequant_bf16(acc, sx, sw, np.zeros(7, np.uint16)), oracle.dequant_bf16(acc, sx, sw))
+    # 3 * 0.5 * 2 + 1.5 = 4.5 exactly
+    y = oracle.dequant_bf16(np.array([[3]], np.int32), np.array([0.5], np.float32), np.array([2.0], np.float32),
+                            f2b(np.array([1.5], np.float32)))
+    assert synth.bf16_bits_to_f32(y)[0, 0] == 4.5
+    # the bias joins the FP32 product before the one rounding to BF16:
+    # 513 * 2^-9 + 2^-8 = 1 + 3 * 2^-9 rounds up to 1 + 2^-7, while rounding
+    # the product first (to 1.0) and then adding would give a tie -> 1.0
+    y = oracle.dequant_bf16(np.array([[513]], np.int32), np.array([2.0 ** -9], np.float32),
+                            np.array([1.0], np.float32), f2b(np.array([2.0 ** -8], np.float32)))
+    assert synth.bf16_bits_to_f32(y)[0, 0] == np.float32(1 + 2.0 ** -7)
+    # the bias is indexed by the output column
+    b = f2b(np.arange(7, dtype=np.float32))
+    y = oracle.dequant_bf16(np.zeros((3, 7), np.int32), sx, sw, b)
+    assert np.array_equal(synth.bf16_bits_to_f32(y), np.tile(np.arange(7, dtype=np.float32), (3, 1)))
+
+
 # ---------------------------------------------------------------------------
 # whole layer
 # ---------------------------------------------------------------------------
