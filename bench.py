@@ -386,6 +386,37 @@ def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
                          "layer_us": sum(tt for _, tt in pro) * 1e6}}
 
 
+def shared_input_secondary(cr, layer, lins, device, stream, peaks, steps=2000, warmup=20):
+    """The decode layer as the model feeds it: q, k and v read one input,
+    gate and up another (their rotation runs once), o and down their own.
+    Algorithmic bytes count each distinct input once."""
+    groups = {"q": "attn", "k": "attn", "v": "attn", "o": "o", "gate": "mlp", "up": "mlp", "down": "down"}
+    src = {}
+    for lin in lins:
+        src.setdefault(groups[lin.name], lin)
+    xin = {g: l.x_torch(device) for g, l in src.items()}
+    xs = [xin[groups[lin.name]] for lin in lins]
+    ys = [torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device) for lin in lins]
+    batch = cr.LinearBatch(xs, layer.w, ys)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        batch(stream)
+    torch.cuda.synchronize()
+    g = capture(lambda: batch(stream), stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        t = time_region(g.replay, steps, stream) / steps
+    m = lins[0].m
+    nbytes = sum(lin.n * lin.k + 4 * lin.n + m * lin.k + 2 * m * lin.n for lin in lins)   # weights, xq reads, y
+    nbytes += sum(2 * m * l.k + m * l.k + 4 * m for l in src.values())                      # one prologue per input
+    del g, batch
+    return {"workload": "qwen3vl32b_layer_shared_inputs_decode_m12", "distinct_inputs": len(src),
+            "gb_s": nbytes / t / 1e9, "us_per_step": t * 1e6,
+            "frac_of_measured_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"]}
+
+
 def minimax_secondary(cr, device, stream, peaks, steps=5, warmup=2):
     """MiniMax-H3-shaped qkv projection (K = 5376, N = 16128) at M = 8192 and
     32768 video tokens through the single-linear entry point: INT8 TOPS."""
@@ -612,7 +643,7 @@ def run_ours(args):
     if not args.no_prefill:
         secondary = prefill_secondary(cr, layer, device, stream, peaks)
     cr.convrot_device_status(stream)
-    others = {}
+    others = {"shared_inputs": shared_input_secondary(cr, layer, lins, device, stream, peaks)}
     if not args.no_minimax:
         others["minimax_qkv"] = minimax_secondary(cr, device, stream, peaks)
         cr.convrot_device_status(stream)

@@ -164,6 +164,11 @@ convrot_status_t convrot_linear_int8(const void *x_bf16, int64_t m, const convro
  * One product of a batched GEMM call (see convrot_gemm_i8 for the maths).
  *   xq : int8 [m, w->k] quantised activations;  sx : fp32 [m] their scales
  *   y_bf16 : BF16 [m, w->n] output or NULL;  acc : int32 [m, w->n] or NULL
+ *   bias_bf16 : BF16 [w->n] per-output-channel bias or NULL (none).  With a
+ *     bias, y = bf16_rne( ((float)acc * sx[m]) * sw[n] + bias[n] ): the bias
+ *     joins the FP32 product and the sum is rounded once.  The source pages
+ *     quantise bias-free projections; the bias is this library's extension
+ *     for layers that carry one.  16-byte aligned.
  */
 typedef struct {
     const int8_t *xq;
@@ -171,6 +176,7 @@ typedef struct {
     const convrot_weight_t *w;
     void *y_bf16;
     int32_t *acc;
+    const void *bias_bf16;
 } convrot_gemm_job_t;
 
 /*
@@ -187,24 +193,28 @@ convrot_status_t convrot_gemm_i8_batch(int64_t m, int count, const convrot_gemm_
 size_t convrot_gemm_batch_workspace_bytes(int64_t m, int count, const convrot_gemm_job_t *jobs);
 
 /*
- * One linear of a batched call: y = ConvRotLinearINT8(x) against w.
- *   x_bf16 : BF16 [m, w->k] input (device)
+ * One linear of a batched call: y = ConvRotLinearINT8(x) (+ bias) against w.
+ *   x_bf16 : BF16 [m, w->k] input (device).  Jobs that pass the same x_bf16
+ *            pointer (same k) share one activation prologue.
  *   w      : quantised weight handle
  *   y_bf16 : BF16 [m, w->n] output (device)
+ *   bias_bf16 : BF16 [w->n] bias or NULL, as in convrot_gemm_job_t
  */
 typedef struct {
     const void *x_bf16;
     const convrot_weight_t *w;
     void *y_bf16;
+    const void *bias_bf16;
 } convrot_linear_job_t;
 
 /*
- * Several independent ConvRot INT8 linears with the same token count m, in
- * two launches: one activation prologue over every job's rows, then one
- * GEMM whose K blocks of all weights are dealt out evenly to every SM
- * (m <= 512; larger m runs the GEMMs one after another).  This is how the
- * linears of one decoder layer that share an input (q/k/v, gate/up) or that
- * are otherwise ready together run at decode size, where a per-linear launch
+ * Several ConvRot INT8 linears with the same token count m, in two
+ * launches: one activation prologue over the rows of every distinct input
+ * (jobs with the same x_bf16 share its rotated INT8 copy), then one GEMM
+ * whose K blocks of all weights are dealt out evenly to every SM (m <= 512;
+ * larger m runs the GEMMs one after another).  This is how the linears of
+ * one decoder layer that share an input (q/k/v, gate/up) or that are
+ * otherwise ready together run at decode size, where a per-linear launch
  * would spend more time starting and draining than streaming its weight.
  * The pages quantise exactly these projections of every layer [zskr.cn
  * "Qwen3-VL-32B ... INT8-ConvRot": 350 = 50 layers x 7 row-wise INT8 ConvRot

@@ -47,13 +47,13 @@ class convrot_weight_t(ctypes.Structure):
 class convrot_linear_job_t(ctypes.Structure):
     """Mirror of the C struct: one linear of a batched call."""
     _fields_ = [("x_bf16", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight_t)),
-                ("y_bf16", ctypes.c_void_p)]
+                ("y_bf16", ctypes.c_void_p), ("bias_bf16", ctypes.c_void_p)]
 
 
 class convrot_gemm_job_t(ctypes.Structure):
     """Mirror of the C struct: one product of a batched GEMM call."""
     _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight_t)),
-                ("y_bf16", ctypes.c_void_p), ("acc", ctypes.c_void_p)]
+                ("y_bf16", ctypes.c_void_p), ("acc", ctypes.c_void_p), ("bias_bf16", ctypes.c_void_p)]
 
 
 # exported symbol -> (argtypes, restype); every name declared in convrot.h
@@ -198,23 +198,28 @@ def convrot_linear_int8(x_bf16: torch.Tensor, w: QuantizedWeight, y: torch.Tenso
            "convrot_linear_int8")
 
 
-def _jobs(xs, ws_, ys):
+def _jobs(xs, ws_, ys, biases=None):
     arr = (convrot_linear_job_t * len(xs))()
-    for i, (x, w, y) in enumerate(zip(xs, ws_, ys)):
+    biases = biases or [None] * len(xs)
+    for i, (x, w, y, b) in enumerate(zip(xs, ws_, ys, biases)):
         arr[i].x_bf16 = _ptr(x)
         arr[i].w = ctypes.pointer(w.handle)
         arr[i].y_bf16 = _ptr(y)
+        arr[i].bias_bf16 = _ptr(b)
     return arr
 
 
 class LinearBatch:
     """A prepared batched call: the C job array is built once and reused,
-    so a step costs one C call (argument marshalling only)."""
+    so a step costs one C call (argument marshalling only).  ``biases``: an
+    optional BF16 [n] tensor (or None) per linear.  Linears given the same
+    input tensor share its rotation."""
 
-    def __init__(self, xs, weights, ys, ws: Optional[torch.Tensor] = None):
+    def __init__(self, xs, weights, ys, ws: Optional[torch.Tensor] = None, biases=None):
         self.xs, self.weights, self.ys = list(xs), list(weights), list(ys)
+        self.biases = list(biases) if biases is not None else None
         self.m = self.xs[0].shape[0]
-        self.jobs = _jobs(self.xs, self.weights, self.ys)
+        self.jobs = _jobs(self.xs, self.weights, self.ys, self.biases)
         need = int(load_library().convrot_linear_batch_workspace_bytes(self.m, len(self.xs), self.jobs))
         if need == 0:
             raise ConvrotError(1, "convrot_linear_batch_workspace_bytes")
@@ -228,25 +233,27 @@ class LinearBatch:
                "convrot_linear_int8_batch")
 
 
-def convrot_linear_int8_batch(xs, weights, ys, ws: torch.Tensor, stream=None) -> None:
-    """Run len(xs) independent linears with the same token count together."""
+def convrot_linear_int8_batch(xs, weights, ys, ws: torch.Tensor, stream=None, biases=None) -> None:
+    """Run len(xs) linears with the same token count together."""
     m = xs[0].shape[0]
-    jobs = _jobs(xs, weights, ys)
+    jobs = _jobs(xs, weights, ys, biases)
     _check(load_library().convrot_linear_int8_batch(m, len(xs), jobs, _ptr(ws), ws.numel() * ws.element_size(),
                                                     _stream(stream)), "convrot_linear_int8_batch")
 
 
-def convrot_linear_batch_workspace_bytes(xs, weights, ys) -> int:
-    return int(load_library().convrot_linear_batch_workspace_bytes(xs[0].shape[0], len(xs), _jobs(xs, weights, ys)))
+def convrot_linear_batch_workspace_bytes(xs, weights, ys, biases=None) -> int:
+    return int(load_library().convrot_linear_batch_workspace_bytes(xs[0].shape[0], len(xs),
+                                                                   _jobs(xs, weights, ys, biases)))
 
 
 class GemmBatch:
     """A prepared batched GEMM call (job array built once)."""
 
-    def __init__(self, xqs, sxs, weights, ys, accs=None, ws: Optional[torch.Tensor] = None):
+    def __init__(self, xqs, sxs, weights, ys, accs=None, ws: Optional[torch.Tensor] = None, biases=None):
         n = len(xqs)
         accs = accs or [None] * n
-        self.keep = (list(xqs), list(sxs), list(weights), list(ys), list(accs))
+        biases = biases or [None] * n
+        self.keep = (list(xqs), list(sxs), list(weights), list(ys), list(accs), list(biases))
         self.m = xqs[0].shape[0]
         self.jobs = (convrot_gemm_job_t * n)()
         for i in range(n):
@@ -255,6 +262,7 @@ class GemmBatch:
             self.jobs[i].w = ctypes.pointer(weights[i].handle)
             self.jobs[i].y_bf16 = _ptr(ys[i])
             self.jobs[i].acc = _ptr(accs[i])
+            self.jobs[i].bias_bf16 = _ptr(biases[i])
         need = int(load_library().convrot_gemm_batch_workspace_bytes(self.m, n, self.jobs))
         if need == 0:
             raise ConvrotError(1, "convrot_gemm_batch_workspace_bytes")

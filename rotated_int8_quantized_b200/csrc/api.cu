@@ -198,7 +198,8 @@ convrot_status_t check_jobs(int64_t m, int count, const convrot_linear_job_t *jo
         convrot_status_t s = check_weight(J.w);
         if (s != CONVROT_OK) return s;
         if ((s = check_shape(m, J.w->k, J.w->group)) != CONVROT_OK) return s;
-        if (!aligned16(J.x_bf16) || !aligned16(J.y_bf16)) return CONVROT_ERR_ALIGNMENT;
+        if (!aligned16(J.x_bf16) || !aligned16(J.y_bf16) || (J.bias_bf16 && !aligned16(J.bias_bf16)))
+            return CONVROT_ERR_ALIGNMENT;
     }
     // no output may overlap any input or another output: the jobs run as
     // one launch pair, so an output cannot feed a later job
@@ -206,6 +207,8 @@ convrot_status_t check_jobs(int64_t m, int count, const convrot_linear_job_t *jo
         const size_t ybytes = (size_t)m * (size_t)jobs[j].w->n * 2;
         for (int i = 0; i < count; ++i) {
             if (ranges_overlap(jobs[j].y_bf16, ybytes, jobs[i].x_bf16, (size_t)m * (size_t)jobs[i].w->k * 2))
+                return CONVROT_ERR_INVALID_ARG;
+            if (jobs[i].bias_bf16 && ranges_overlap(jobs[j].y_bf16, ybytes, jobs[i].bias_bf16, (size_t)jobs[i].w->n * 2))
                 return CONVROT_ERR_INVALID_ARG;
             if (i != j && ranges_overlap(jobs[j].y_bf16, ybytes, jobs[i].y_bf16, (size_t)m * (size_t)jobs[i].w->n * 2))
                 return CONVROT_ERR_INVALID_ARG;
@@ -260,16 +263,27 @@ convrot_status_t run_linear(int64_t m, int count, const convrot_linear_job_t *jo
     convrot::RQProblem rq[kMaxBatch];
     convrot::GemmProblem gp[kMaxBatch];
     size_t off = L.gemm_bytes;
+    int nrq = 0;
     for (int j = 0; j < count; ++j) {
         int8_t *xq = reinterpret_cast<int8_t *>(base + off);
         off += round256((size_t)m * (size_t)jobs[j].w->k);
         float *sx = reinterpret_cast<float *>(base + off);
         off += round256((size_t)m * 4);
-        rq[j] = {jobs[j].x_bf16, jobs[j].w->k, xq, sx};
+        // a job whose input an earlier job already rotates reuses its codes
+        int same = -1;
+        for (int i = 0; i < j && same < 0; ++i)
+            if (jobs[i].x_bf16 == jobs[j].x_bf16 && jobs[i].w->k == jobs[j].w->k) same = i;
+        if (same >= 0) {
+            xq = const_cast<int8_t *>(gp[same].xq);
+            sx = const_cast<float *>(gp[same].sx);
+        } else {
+            rq[nrq++] = {jobs[j].x_bf16, jobs[j].w->k, xq, sx};
+        }
         gp[j] = {m, jobs[j].w->n, jobs[j].w->k, xq, sx, jobs[j].w->q, jobs[j].w->scale,
-                 static_cast<__nv_bfloat16 *>(jobs[j].y_bf16), nullptr};
+                 static_cast<__nv_bfloat16 *>(jobs[j].y_bf16), nullptr,
+                 static_cast<const __nv_bfloat16 *>(jobs[j].bias_bf16)};
     }
-    cudaError_t e = convrot::launch_rotate_quant(count, m, rq, st, true);
+    cudaError_t e = convrot::launch_rotate_quant(nrq, m, rq, st, true);
     if (e != cudaSuccess) return from_cuda(e);
     if (L.batched_gemm) return from_cuda(convrot::launch_gemm_i8(L.batch, gp, base, st, true, true));
     for (int j = 0; j < count; ++j) {
@@ -296,7 +310,7 @@ convrot_status_t check_gemm_jobs(int64_t m, int count, const convrot_gemm_job_t 
         if (s != CONVROT_OK) return s;
         if ((s = check_shape(m, J.w->k, J.w->group)) != CONVROT_OK) return s;
         if (!aligned16(J.xq) || !aligned16(J.sx) || (J.y_bf16 && !aligned16(J.y_bf16)) ||
-            (J.acc && !aligned16(J.acc)))
+            (J.acc && !aligned16(J.acc)) || (J.bias_bf16 && !aligned16(J.bias_bf16)))
             return CONVROT_ERR_ALIGNMENT;
     }
     return CONVROT_OK;
@@ -333,14 +347,15 @@ convrot_status_t convrot_gemm_i8_batch(int64_t m, int count, const convrot_gemm_
     convrot::GemmProblem gp[kMaxBatch];
     for (int j = 0; j < count; ++j)
         gp[j] = {m, jobs[j].w->n, jobs[j].w->k, jobs[j].xq, jobs[j].sx, jobs[j].w->q, jobs[j].w->scale,
-                 static_cast<__nv_bfloat16 *>(jobs[j].y_bf16), jobs[j].acc};
+                 static_cast<__nv_bfloat16 *>(jobs[j].y_bf16), jobs[j].acc,
+                 static_cast<const __nv_bfloat16 *>(jobs[j].bias_bf16)};
     return from_cuda(convrot::launch_gemm_i8(p, gp, ws, static_cast<cudaStream_t>(stream), false, false));
 }
 
 size_t convrot_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     if (m < 1 || n < 1 || k < kGroup) return 0;
     convrot_weight_t w = {nullptr, nullptr, n, k, (int32_t)kGroup};
-    convrot_linear_job_t job = {nullptr, &w, nullptr};
+    convrot_linear_job_t job = {nullptr, &w, nullptr, nullptr};
     LinearLayout L;
     linear_layout(m, 1, &job, sms_for_sizing(), &L);
     return L.total;
@@ -348,7 +363,7 @@ size_t convrot_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
 
 convrot_status_t convrot_linear_int8(const void *x_bf16, int64_t m, const convrot_weight_t *w, void *y_bf16,
                                      void *ws, size_t ws_bytes, void *stream) {
-    convrot_linear_job_t job = {x_bf16, w, y_bf16};
+    convrot_linear_job_t job = {x_bf16, w, y_bf16, nullptr};
     convrot_status_t s = check_jobs(m, 1, &job);
     if (s != CONVROT_OK) return s;
     return run_linear(m, 1, &job, ws, ws_bytes, static_cast<cudaStream_t>(stream));

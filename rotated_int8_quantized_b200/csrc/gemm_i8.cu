@@ -49,6 +49,7 @@ constexpr int kATileBytes = kTileA * kBlockK;
 constexpr int kL2PrefetchBlocks = 16;  // weight K blocks pulled into L2 ahead of the grid-dependency wait
 constexpr int kMaxSplitWays = 6;       // K ranges per split tail tile (large M)
 constexpr long long kGroupABytes = 48ll << 20;   // INT8 A operand above this is taken in tile groups
+constexpr int kBiasStage = 256;        // offset of the staged bias after the staged scales of a tile
 constexpr int kExtraBars = 7;          // tfull[2], tempty[2], drain, red[2]
 // The split-tail reduction double-buffers at least 32 columns of every other
 // piece's partial in the operand ring of a bn = 256 launch.
@@ -111,7 +112,9 @@ struct SegmentIter {
         u = a.tail_units * q / Q;
         u_end = a.tail_units * (q + 1) / Q;
     }
-    __device__ __forceinline__ bool next(const GemmArgs &a, Segment &s) {
+    // want_slot: also find the workspace slot of a shared (partial) tile;
+    // only the epilogue needs it
+    __device__ __forceinline__ bool next(const GemmArgs &a, Segment &s, bool want_slot = false) {
         if (wave < a.full_waves && wave * (int)gridDim.x + (int)blockIdx.x < a.full_tiles) {
             s.job = 0;
             s.tile = wave * (int)gridDim.x + (int)blockIdx.x;
@@ -139,18 +142,21 @@ struct SegmentIter {
         if (u < u_end) {
             while (j + 1 < a.njobs && u >= a.job[j + 1].unit0) ++j;
             const GemmJob &J = a.job[j];
-            const long long lu = u - J.unit0;
-            const long long t = lu / J.kbpt;
+            const int lu = (int)(u - J.unit0);           // < tiles x kbpt of one job
+            const int t = lu / J.kbpt;
             s.job = j;
-            s.tile = J.tile_base + (int)t * a.rep + r;
-            // a tile shared by several CTAs sums in the workspace slot of the
-            // last of them (its range starts inside this tile, so no other
-            // shared tile maps to the same slot)
-            s.slot = stream_k_cta(J.unit0 + (t + 1) * J.kbpt - 1, a.tail_units, (int)gridDim.x / a.rep) * a.rep + r;
-            s.kb0 = (int)(lu - t * J.kbpt);
+            s.tile = J.tile_base + t * a.rep + r;
+            s.kb0 = lu - t * J.kbpt;
             const long long rem = u_end - u;
             s.kb1 = (int)((long long)s.kb0 + rem < J.kbpt ? s.kb0 + rem : J.kbpt);
             s.split = -1;
+            s.slot = -1;
+            // a tile shared by several CTAs sums in the workspace slot of the
+            // last of them (its range starts inside this tile, so no other
+            // shared tile maps to the same slot)
+            if (want_slot && (s.kb0 != 0 || s.kb1 != J.kbpt))
+                s.slot = stream_k_cta(J.unit0 + (long long)(t + 1) * J.kbpt - 1, a.tail_units,
+                                      (int)gridDim.x / a.rep) * a.rep + r;
             u += s.kb1 - s.kb0;
             return true;
         }
@@ -162,6 +168,11 @@ struct SegmentIter {
 // inside a group the A tile varies fastest, so the CTAs of one wave share a
 // few B tiles and a group's A rows stay in L2 while the group sweeps B.
 __device__ __forceinline__ void tile_coords(const GemmJob &J, int tile, int &ta, int &tb) {
+    if (J.n_tiles_b == 1) {         // one B tile (decode): no division
+        ta = tile;
+        tb = 0;
+        return;
+    }
     const int per_group = J.group_a * (J.n_tiles_b);
     const int g = tile / per_group;
     const int w = tile - g * per_group;
@@ -173,7 +184,13 @@ __device__ __forceinline__ void tile_coords(const GemmJob &J, int tile, int &ta,
 
 // Large-M orientation: dequantise and store columns j0 .. j0+15 of output
 // row m, with the row scale sxm in a register and the tile's weight scales
-// staged in shared memory (sws[e] = sw[j0 + e]).
+// staged in shared memory (sws[e] = sw[j0 + e]; with a bias, the bias
+// values follow kBiasStage floats later: sws[kBiasStage + e] = bias[j0 + e]).
+__device__ __forceinline__ float dq_row(int32_t acc, float sxm, const float *sws, int e, bool bias) {
+    const float f = __fmul_rn(__fmul_rn(__int2float_rn(acc), sxm), sws[e]);
+    return bias ? __fadd_rn(f, sws[kBiasStage + e]) : f;
+}
+
 __device__ __forceinline__ void emit_row16(const GemmJob &J, int m, int j0, const int32_t (&v)[16], float sxm,
                                            const float *sws) {
     if (m >= J.m) return;
@@ -192,18 +209,18 @@ __device__ __forceinline__ void emit_row16(const GemmJob &J, int m, int j0, cons
         __nv_bfloat16 *dst = J.y + (size_t)m * J.n + j0;
         if (full) {
             uint32_t pk[8];
+            const bool bias = J.bias != nullptr;
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
-                const float f0 = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), sws[e]);
-                const float f1 = __fmul_rn(__fmul_rn(__int2float_rn(v[e + 1]), sxm), sws[e + 1]);
+                const float f0 = dq_row(v[e], sxm, sws, e, bias);
+                const float f1 = dq_row(v[e + 1], sxm, sws, e + 1, bias);
                 __nv_bfloat162 h = __halves2bfloat162(__float2bfloat16_rn(f0), __float2bfloat16_rn(f1));
                 pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
             }
             reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             reinterpret_cast<uint4 *>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         } else {
-            for (int e = 0; e < 16 && j0 + e < J.n; ++e)
-                dst[e] = __float2bfloat16_rn(__fmul_rn(__fmul_rn(__int2float_rn(v[e]), sxm), sws[e]));
+            for (int e = 0; e < 16 && j0 + e < J.n; ++e) dst[e] = __float2bfloat16_rn(dq_row(v[e], sxm, sws, e, J.bias));
         }
     }
 }
@@ -214,7 +231,7 @@ __device__ __forceinline__ void emit_row16(const GemmJob &J, int m, int j0, cons
 // buffer) so that each output row leaves as 16-byte segments instead of
 // 2-byte scatters.  Called by all 128 epilogue threads (it holds a barrier).
 __device__ __forceinline__ void emit_swap16(const GemmJob &J, int a0, int row, int tid, int j0,
-                                            const int32_t (&v)[16], float srow, const float *scol,
+                                            const int32_t (&v)[16], float srow, float brow, const float *scol,
                                             __nv_bfloat16 *stg) {
     const int n = a0 + row;
     if (J.acc && n < J.n) {
@@ -223,9 +240,12 @@ __device__ __forceinline__ void emit_swap16(const GemmJob &J, int a0, int row, i
             if (j0 + e < J.m) J.acc[(size_t)(j0 + e) * J.n + n] = v[e];
     }
     if (!J.y) return;
+    const bool bias = J.bias != nullptr;
 #pragma unroll
-    for (int e = 0; e < 16; ++e)
-        stg[e * kTileA + row] = __float2bfloat16_rn(__fmul_rn(__fmul_rn(__int2float_rn(v[e]), scol[e]), srow));
+    for (int e = 0; e < 16; ++e) {
+        const float f = __fmul_rn(__fmul_rn(__int2float_rn(v[e]), scol[e]), srow);
+        stg[e * kTileA + row] = __float2bfloat16_rn(bias ? __fadd_rn(f, brow) : f);
+    }
     named_bar_sync(1, 128);
     const bool vec = (J.n & 7) == 0;
 #pragma unroll
@@ -252,13 +272,13 @@ __device__ __forceinline__ void emit_swap16(const GemmJob &J, int a0, int row, i
 // all 128 epilogue threads; `chunk` counts the calls (it picks the transpose
 // buffer of the swapped orientation).
 __device__ __forceinline__ void emit16s(const GemmJob &J, int swap, int a0, int row, int tid, int j0,
-                                        const int32_t (&v)[16], float srow, const float *scol,
+                                        const int32_t (&v)[16], float srow, float brow, const float *scol,
                                         __nv_bfloat16 *y_stage, int &chunk) {
     if (!swap) {
         emit_row16(J, a0 + row, j0, v, srow, scol);
         return;
     }
-    emit_swap16(J, a0, row, tid, j0, v, srow, scol, y_stage + (chunk & 1) * 16 * kTileA);
+    emit_swap16(J, a0, row, tid, j0, v, srow, brow, scol, y_stage + (chunk & 1) * 16 * kTileA);
     ++chunk;
 }
 
@@ -300,10 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *ticket = reinterpret_cast<volatile int *>(misc + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 8);
     volatile int *red_ok = reinterpret_cast<volatile int *>(misc + 12);
-    float *sw_stage = reinterpret_cast<float *>(misc + 16);     // [2][256] B-row scales of a tile
+    // [2][2 * kBiasStage]: B-row scales of a tile, then (large M, with a
+    // bias) the bias of its columns
+    float *sw_stage = reinterpret_cast<float *>(misc + 16);
     // [2][16][128] BF16: swapped-orientation output chunks, transposed so
     // that they leave as 16-byte row segments
-    __nv_bfloat16 *y_stage = reinterpret_cast<__nv_bfloat16 *>(misc + 16 + 2 * 256 * 4);
+    __nv_bfloat16 *y_stage = reinterpret_cast<__nv_bfloat16 *>(misc + 16 + 2 * 2 * kBiasStage * 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -502,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         SegmentIter it;
         it.init(a);
         Segment sg;
-        while (it.next(a, sg)) {
+        while (it.next(a, sg, true)) {
             const GemmJob &J = a.job[sg.job];
             int ta, tb;
             tile_coords(J, sg.tile, ta, tb);
@@ -513,15 +535,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             // scale of this thread's A row to a register while the
             // accumulator is still being computed (double-buffered by
             // segment parity; the barrier below publishes them)
-            float *scol = sw_stage + (seg & 1) * 256;
-            float srow = 0.f;
+            float *scol = sw_stage + (seg & 1) * 2 * kBiasStage;
+            float srow = 0.f, brow = 0.f;
             {
                 const float *cs = a.swap ? J.sx : J.sw;
                 const int clim = a.swap ? J.m : J.n;
                 for (int cidx = tid; cidx < a.bn; cidx += 128) {
                     const int col = tb * a.bn + cidx;
                     scol[cidx] = col < clim ? __ldg(cs + col) : 0.f;
+                    if (!a.swap && J.bias) scol[kBiasStage + cidx] = col < clim ? __bfloat162float(J.bias[col]) : 0.f;
                 }
+                if (a.swap && J.bias && i < J.n) brow = __bfloat162float(J.bias[i]);
                 const float *rs = a.swap ? J.sw : J.sx;
                 if (i < (a.swap ? J.n : J.m)) srow = __ldg(rs + i);
             }
@@ -549,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
                     if (whole) {
-                        emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + c * 16, v, srow, scol + c * 16,
+                        emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + c * 16, v, srow, brow, scol + c * 16,
                                 y_stage, ychunk);
                     } else {
                         int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
@@ -721,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e = 0; e < 64; ++e) __stcg(p + (size_t)e * kTileA, 0);
 #pragma unroll
                         for (int h = 0; h < 4; ++h)
-                            emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + (c + h) * 16, v[h], srow,
+                            emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + (c + h) * 16, v[h], srow, brow,
                                     scol + (c + h) * 16, y_stage, ychunk);
                     }
                     for (; c < chunks; ++c) {
@@ -731,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e = 0; e < 16; ++e) v[e] = __ldcg(p + (size_t)e * kTileA);
 #pragma unroll
                         for (int e = 0; e < 16; ++e) __stcg(p + (size_t)e * kTileA, 0);
-                        emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + c * 16, v, srow, scol + c * 16,
+                        emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + c * 16, v, srow, brow, scol + c * 16,
                                 y_stage, ychunk);
                     }
                     if (ew == 0 && lane == 0) a.counters[sg.slot] = 0;
@@ -762,7 +786,7 @@ static void plan_common(GemmPlan *p) {
     int cols = 32;
     while (cols < 2 * p->bn) cols <<= 1;
     p->tmem_cols = cols;
-    p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + kExtraBars) + 16 + 16 + 2 * 256 * 4 +
+    p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + kExtraBars) + 16 + 16 + 2 * 2 * kBiasStage * 4 +
                     2 * 16 * kTileA * 2;
     // workspace: counters, then INT32 partial tiles [slots][bn][128]
     const size_t cnt = ((size_t)p->slots * 4 + 255) / 256 * 256;
@@ -944,6 +968,7 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
         J.sw = q.sw;
         J.y = q.y;
         J.acc = q.acc;
+        J.bias = q.bias;
     }
 
     static bool configured[64] = {};

@@ -28,6 +28,7 @@ struct GemmJob {
     const float *sw;
     __nv_bfloat16 *y;
     int32_t *acc;
+    const __nv_bfloat16 *bias;   // [n] or null
 };
 
 struct GemmArgs {
@@ -66,6 +67,7 @@ struct GemmProblem {
     const float *sw;
     __nv_bfloat16 *y;
     int32_t *acc;
+    const __nv_bfloat16 *bias;   // [n] or null
 };
 
 // Host-side tiling of a launch.

@@ -100,6 +100,7 @@ __device__ __forceinline__ uint4 quant16(const float (&y)[16], const RowScale &r
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+
 // ---------------------------------------------------------------------------
 // Main variant: 16 threads ("a slot") per 256-group, H_256 = H_16 (x) H_16.
 // Thread t of a slot loads elements 16t .. 16t+15 (32 contiguous bytes; the
@@ -117,8 +118,13 @@ constexpr int kMaxParts = 8;           // CTAs per row (portable cluster size)
 // FP32 staging of a rotated group: 256 values padded to 272 so that the two
 // slots of a warp write different banks; inside, 16-value chunks whose four
 // float4 parts are XOR-swizzled so that the quantiser's 16-byte reads of
-// consecutive chunks are conflict-free.
+// consecutive chunks are conflict-free.  Decode-sized launches (HALF) keep
+// the plain layout: a few rows are latency-bound, not bank-bound, and the
+// extra address arithmetic raised the decode variant above 96 registers,
+// which cost a co-resident GEMM CTA during the programmatic-launch overlap
+// (2 us per decode step).
 constexpr int kYGroupStride = 272;
+__host__ __device__ constexpr int y_group_stride(bool half) { return half ? 256 : kYGroupStride; }
 constexpr int kSlotsSmemMax = 226 * 1024;   // dynamic shared memory per CTA (227 KB minus the static part)
 
 __device__ __forceinline__ void fwht16_regs(double (&v)[16]) {
@@ -263,12 +269,13 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                 __syncwarp(half_mask);
             }
             fwht16_regs(x);                                  // index bits 4-7
-            // output 16*i + t of the group is element t of chunk i
-            float *yg = ybuf + (size_t)(g - g0) * kYGroupStride + (t & 3);
+            // output 16*i + t of the group is element t of chunk i (its
+            // float4 part XOR-swizzled in launches with a row per CTA)
+            float *yg = ybuf + (size_t)(g - g0) * y_group_stride(HALF) + (HALF ? t : (t & 3));
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float y = __double2float_rn(x[i] * 0.0625);   // / sqrt(256), exact
-                yg[16 * i + 4 * ((t >> 2) ^ ((i >> 1) & 3))] = y;
+                yg[16 * i + (HALF ? 0 : 4 * ((t >> 2) ^ ((i >> 1) & 3)))] = y;
                 amax = fmaxf(amax, fabsf(y));
             }
         }
@@ -307,11 +314,12 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
         const unsigned mask = __ballot_sync(__activemask(), c < chunks);
         if (c < chunks) {
             const int ci = c & 15;     // chunk within its group
-            const float4 *src = reinterpret_cast<const float4 *>(ybuf + (size_t)(c >> 4) * kYGroupStride + ci * 16);
+            const float4 *src = reinterpret_cast<const float4 *>(
+                HALF ? ybuf + c * 16 : ybuf + (size_t)(c >> 4) * kYGroupStride + ci * 16);
             float y[16];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float4 f = src[i ^ ((ci >> 1) & 3)];
+                const float4 f = src[HALF ? i : (i ^ ((ci >> 1) & 3))];
                 y[4 * i] = f.x;
                 y[4 * i + 1] = f.y;
                 y[4 * i + 2] = f.z;
@@ -330,7 +338,8 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
 template <int GPS, bool HALF>
 static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int max_slots, int max_local_groups) {
     cfg.blockDim = dim3(max_slots * 16);
-    cfg.dynamicSmemBytes = (size_t)max_slots * (HALF ? kXchHalf : kXchFull) * 8 + (size_t)max_local_groups * kYGroupStride * 4;
+    cfg.dynamicSmemBytes =
+        (size_t)max_slots * (HALF ? kXchHalf : kXchFull) * 8 + (size_t)max_local_groups * y_group_stride(HALF) * 4;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -383,7 +392,7 @@ static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, bool h
     *max_slots = ms;
     *max_gps = mg;
     *max_local = ml;
-    return (size_t)ms * (half ? kXchHalf : kXchFull) * 8 + (size_t)ml * kYGroupStride * 4;
+    return (size_t)ms * (half ? kXchHalf : kXchFull) * 8 + (size_t)ml * y_group_stride(half) * 4;
 }
 
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl) {

@@ -97,3 +97,38 @@ def test_workspace_sizes_follow_the_tiling(lib):
     assert lib.convrot_gemm_workspace_bytes(4096, 5120, 25600) == 256 + 48 * 3 * 256 * 128 * 4
     lw = lib.convrot_linear_workspace_bytes(12, 8192, 5120)
     assert lw == lib.convrot_gemm_workspace_bytes(12, 8192, 5120) + 61440 + 256
+
+
+def test_binding_structs_match_the_header(tmp_path):
+    """The ctypes mirrors of the job structs have the C layout: a C program
+    compiled against include/convrot.h prints sizes and offsets."""
+    import subprocess
+    import rotated_int8_quantized_b200 as cr
+    src = tmp_path / "layout.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "convrot.h"
+#define F(T, f) printf(#T "." #f " %zu\n", offsetof(T, f));
+int main(void) {
+    printf("convrot_weight_t %zu\n", sizeof(convrot_weight_t));
+    printf("convrot_gemm_job_t %zu\n", sizeof(convrot_gemm_job_t));
+    printf("convrot_linear_job_t %zu\n", sizeof(convrot_linear_job_t));
+    F(convrot_weight_t, group) F(convrot_gemm_job_t, acc) F(convrot_gemm_job_t, bias_bf16)
+    F(convrot_linear_job_t, y_bf16) F(convrot_linear_job_t, bias_bf16)
+    return 0;
+}
+''')
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = dict(line.split() for line in subprocess.check_output([str(exe)], text=True).splitlines())
+    want = {
+        "convrot_weight_t": ctypes.sizeof(cr.convrot_weight_t),
+        "convrot_gemm_job_t": ctypes.sizeof(cr.convrot_gemm_job_t),
+        "convrot_linear_job_t": ctypes.sizeof(cr.convrot_linear_job_t),
+        "convrot_weight_t.group": cr.convrot_weight_t.group.offset,
+        "convrot_gemm_job_t.acc": cr.convrot_gemm_job_t.acc.offset,
+        "convrot_gemm_job_t.bias_bf16": cr.convrot_gemm_job_t.bias_bf16.offset,
+        "convrot_linear_job_t.y_bf16": cr.convrot_linear_job_t.y_bf16.offset,
+        "convrot_linear_job_t.bias_bf16": cr.convrot_linear_job_t.bias_bf16.offset,
+    }
+    assert {k: int(v) for k, v in got.items()} == want

@@ -379,3 +379,66 @@ def test_batch_qwen_decode_layer_full_size(cr):
         wq_ref, sw_ref = oracle.rotate_quantize(lin.w_rows_np(rows))
         ref = oracle.linear_int8(lin.x_np(), wq_ref, sw_ref)
         assert np.array_equal(to_bits(y[:, torch.as_tensor(rows, device=dev)]), ref["y"])
+
+
+# ---------------------------------------------------------------- bias, shared inputs
+# (m, [(k, n), ...]): jobs with equal k read the same input tensor (one
+# prologue for them); every other job has a BF16 bias.  Decode orientation,
+# the stream-K large-M orientation (m <= 512), and per-job launches (m > 512)
+BIAS_CASES = [
+    (12, [(5120, 1024), (5120, 768), (2560, 512)]),
+    (300, [(768, 512), (768, 1000), (512, 384)]),
+    (700, [(512, 640), (512, 384), (1024, 256)]),
+]
+
+
+def _bias_bits(seed, n):
+    return synth.draw_np(synth.stream_key(seed, 5), 1, n, 1.0).reshape(n)
+
+
+@pytest.mark.parametrize("m,shapes", BIAS_CASES)
+def test_batch_bias_and_shared_inputs(cr, m, shapes):
+    x_by_k, xs, ws_, ys, biases, refs = {}, [], [], [], [], []
+    for idx, (k, n) in enumerate(shapes):
+        seed = 4000 + 17 * idx + m
+        if k not in x_by_k:
+            cs = synth.outlier_scale_fraction(synth.stream_key(seed, 2), k, 0.01, 30.0)
+            x_by_k[k] = synth.draw_np(synth.stream_key(seed, 0), m, k, 1.0, cs)
+        x_bits = x_by_k[k]
+        w_bits = synth.draw_np(synth.stream_key(seed, 1), n, k, synth.W_SIGMA)
+        wq_ref, sw_ref = oracle.rotate_quantize(w_bits)
+        b_bits = _bias_bits(seed, n) if idx % 2 == 0 else None
+        refs.append(oracle.linear_int8(x_bits, wq_ref, sw_ref, bias=b_bits))
+        ws_.append(cr.quantize_weight(from_bits(w_bits)))
+        ys.append(torch.empty((m, n), dtype=torch.bfloat16, device="cuda"))
+        biases.append(None if b_bits is None else from_bits(b_bits))
+    x_dev = {k: from_bits(v) for k, v in x_by_k.items()}
+    xs = [x_dev[k] for k, _ in shapes]
+    batch = cr.LinearBatch(xs, ws_, ys, biases=biases)
+    batch()
+    batch()                      # the workspace is left reusable
+    cr.convrot_device_status()
+    for y, ref in zip(ys, refs):
+        yb = to_bits(y)
+        assert rel_err(yb, ref["y"]) <= TOL
+        assert np.array_equal(yb, ref["y"])
+
+
+@pytest.mark.parametrize("m", [12, 400])
+def test_gemm_batch_bias(cr, m):
+    shapes = [(1024, 640), (2048, 256)]
+    xqs, sxs, ws_, ys, biases, refs = [], [], [], [], [], []
+    for idx, (k, n) in enumerate(shapes):
+        x_bits, w, ref = _gemm_case(cr, m, n, k, seed=5000 + idx + m)
+        b_bits = _bias_bits(5000 + idx, n)
+        xqs.append(torch.from_numpy(ref["xq"]).cuda())
+        sxs.append(torch.from_numpy(ref["sx"]).cuda())
+        ws_.append(w)
+        ys.append(torch.empty((m, n), dtype=torch.bfloat16, device="cuda"))
+        biases.append(from_bits(b_bits))
+        refs.append(oracle.dequant_bf16(ref["acc"], ref["sx"], w.scale.cpu().numpy(), b_bits))
+    gb = cr.GemmBatch(xqs, sxs, ws_, ys, biases=biases)
+    gb()
+    cr.convrot_device_status()
+    for y, ref in zip(ys, refs):
+        assert np.array_equal(to_bits(y), ref)
