@@ -18,7 +18,10 @@ the source pages it follows, is stated in the C file:
   (zskr.cn conversion command ``--int8 --scaling_mode row``; 0539edu.com
   section 5, ``--simple`` = RTN)
 * exact INT8 x INT8 -> INT32 GEMM and FP32 dequantisation to BF16
-  (0539edu.com section 4 and summary item 3)
+  (0539edu.com section 4 and summary item 3), with an optional BF16 bias
+  (an extension; the pages' projections carry none)
+* the group --dynamic-convrot picks: the largest power of two <= 256 that
+  divides k, with rotations of such groups (0539edu.com section 4, item 3)
 
 Every function here is pinned by the ``-m "not gpu"`` tests against
 something other than itself (scipy's Hadamard, closed forms, brute force,
@@ -68,6 +71,8 @@ def _load():
         lib.oracle_gemm_i32.argtypes = [P, P, I64, I64, I64, P]
         lib.oracle_gemm_i32.restype = I64
         lib.oracle_dequant_bf16.argtypes = [P, P, P, I64, I64, P]
+        lib.oracle_dynamic_group.argtypes = [I64, ctypes.c_int]
+        lib.oracle_dynamic_group.restype = ctypes.c_int
         lib.oracle_dequant_bf16_bias.argtypes = [P, P, P, P, I64, I64, P]
         lib.oracle_dequant_bf16.restype = None
         lib.oracle_rotate_quantize.argtypes = [P, I64, I64, ctypes.c_int, P, P]
@@ -107,6 +112,11 @@ def sylvester_hadamard(n: int) -> np.ndarray:
     return H
 
 
+def dynamic_group(k: int, max_group: int = 256) -> int:
+    """The largest power of two <= max_group dividing k (--dynamic-convrot)."""
+    return int(_load().oracle_dynamic_group(k, max_group))
+
+
 def rotate_rows(a_bf16: np.ndarray, group: int = 256):
     """Grouped Hadamard rotation of BF16 rows, exact then rounded to FP32.
 
@@ -118,7 +128,7 @@ def rotate_rows(a_bf16: np.ndarray, group: int = 256):
     bad = ctypes.c_int64(0)
     if _load().oracle_rotate_rows(_ptr(a), rows, k, group, _ptr(y),
                                   ctypes.byref(bad)) != 0:
-        raise OracleError("group must be a power of four dividing k")
+        raise OracleError("group must be a power of two dividing k")
     return y, int(bad.value)
 
 
@@ -128,7 +138,7 @@ def rotate_rows_f64(a: np.ndarray, group: int = 256) -> np.ndarray:
     rows, k = a.shape
     y = np.empty((rows, k), dtype=np.float64)
     if _load().oracle_rotate_rows_f64(_ptr(a), rows, k, group, _ptr(y)) != 0:
-        raise OracleError("group must be a power of four dividing k")
+        raise OracleError("group must be a power of two dividing k")
     return y
 
 
@@ -154,7 +164,7 @@ def rotate_quantize(a_bf16: np.ndarray, group: int = 256):
     s = np.empty((rows,), dtype=np.float32)
     bad = _load().oracle_rotate_quantize(_ptr(a), rows, k, group, _ptr(q), _ptr(s))
     if bad < 0:
-        raise OracleError("group must be a power of four dividing k")
+        raise OracleError("group must be a power of two dividing k")
     if bad > 0:
         raise OracleError("%d rotation groups span more than 37 binades" % bad)
     return q, s

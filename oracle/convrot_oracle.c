@@ -148,12 +148,26 @@ int oracle_sylvester_hadamard(int n, int32_t *H)
     return 0;
 }
 
-static int is_power_of_four(int g)
+static int is_power_of_two(int g)
 {
-    if (g < 1 || (g & (g - 1)) != 0) return 0;
-    int lg = 0;
-    while ((1 << lg) < g) ++lg;
-    return (lg % 2) == 0;
+    return g >= 1 && (g & (g - 1)) == 0;
+}
+
+/*
+ * The rotation group --dynamic-convrot picks for a layer: the largest
+ * compatible group size, i.e. the largest power of two that divides k and
+ * does not exceed max_group (the --convrot-group-size cap, 256).
+ * [0539edu.com "minimax-h3-nvfp4-convrot", section 4, item 3: the flag
+ *  selects, per layer, the largest compatible group size.]
+ * Counts down from max_group and tests divisibility (0 if max_group < 1).
+ */
+int oracle_dynamic_group(int64_t k, int max_group)
+{
+    int g = 1;
+    while (g * 2 <= max_group) g *= 2;
+    if (max_group < 1 || k < 1) return 0;
+    while (g > 1 && k % g != 0) g /= 2;
+    return g;
 }
 
 /* ------------------------------------------------------------------ */
@@ -164,15 +178,20 @@ static int is_power_of_four(int g)
  * y[r, g*G + j] = fp32( ( sum_i a[r, g*G + i] * H[i][j] ) / sqrt(G) )
  *
  * a is BF16 bits [rows, k], row-major; y is FP32 [rows, k].  G must be a
- * power of four (so 1/sqrt(G) is a power of two and the division is exact)
- * and divide k.  The sum is accumulated in FP64.  *inexact counts the groups
- * whose nonzero magnitudes span more than 37 binades, where an FP64 sum of
- * 256 BF16 terms might not be exact.  Returns 0, or -1 on bad arguments.
+ * power of two dividing k.  The sum S is accumulated in FP64 (exact, see
+ * below).  When G is a power of four (256 and the other sizes the pages
+ * use by default), sqrt(G) is a power of two and S / sqrt(G) is exact, so y
+ * is S/sqrt(G) rounded once to FP32.  Otherwise (the smaller groups
+ * --dynamic-convrot may pick, e.g. 128) S is divided by the FP64 square
+ * root of G, both correctly rounded, and that quotient rounded to FP32.
+ * *inexact counts the groups whose nonzero magnitudes span more than 37
+ * binades, where an FP64 sum of 256 BF16 terms might not be exact.
+ * Returns 0, or -1 on bad arguments.
  */
 int oracle_rotate_rows(const uint16_t *a, int64_t rows, int64_t k, int group,
                        float *y, int64_t *inexact)
 {
-    if (!is_power_of_four(group) || k % group != 0) return -1;
+    if (!is_power_of_two(group) || k % group != 0) return -1;
     int32_t *H = (int32_t *)malloc(sizeof(int32_t) * group * group);
     double *x = (double *)malloc(sizeof(double) * group);
     if (!H || !x) { free(H); free(x); return -1; }
@@ -213,7 +232,7 @@ int oracle_rotate_rows(const uint16_t *a, int64_t rows, int64_t k, int group,
 int oracle_rotate_rows_f64(const double *a, int64_t rows, int64_t k, int group,
                            double *y)
 {
-    if (!is_power_of_four(group) || k % group != 0) return -1;
+    if (!is_power_of_two(group) || k % group != 0) return -1;
     int32_t *H = (int32_t *)malloc(sizeof(int32_t) * group * group);
     if (!H) return -1;
     oracle_sylvester_hadamard(group, H);

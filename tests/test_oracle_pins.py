@@ -166,7 +166,54 @@ def test_rotation_rejects_bad_group():
     with pytest.raises(oracle.OracleError):
         oracle.rotate_rows(x, 256)       # 384 is not a multiple of 256
     with pytest.raises(oracle.OracleError):
-        oracle.rotate_rows(np.zeros((1, 256), np.uint16), 128)   # not a power of 4
+        oracle.rotate_rows(np.zeros((1, 288), np.uint16), 96)   # not a power of 2
+
+
+# ---------------------------------------------------------------------------
+# --dynamic-convrot: smaller power-of-two groups
+# ---------------------------------------------------------------------------
+def test_dynamic_group_choice():
+    # the pages' own case: in_features 5376 = 21 x 256 keeps the full group
+    assert oracle.dynamic_group(5376) == 256
+    assert oracle.dynamic_group(640) == 128 and oracle.dynamic_group(5440) == 64
+    assert oracle.dynamic_group(48) == 16 and oracle.dynamic_group(1024, 64) == 64
+    # brute force: the largest power of two <= cap dividing k
+    for cap in (256, 128, 100):
+        for k in range(1, 3000):
+            best = max(g for g in (1, 2, 4, 8, 16, 32, 64, 128, 256) if g <= cap and k % g == 0)
+            assert oracle.dynamic_group(k, cap) == best, (k, cap)
+
+
+@pytest.mark.parametrize("group", [16, 32, 64, 128])
+def test_small_group_rotation_matches_scipy(group):
+    # S exact in FP64 (any summation order), then S / sqrt(G) correctly
+    # rounded in FP64, then rounded to FP32: numpy with scipy's Hadamard
+    # computes the same value bit for bit
+    rng = np.random.default_rng(group)
+    x = synth.f32_to_bf16_bits(rng.standard_normal((5, 4 * group)).astype(np.float32))
+    y, bad = oracle.rotate_rows(x, group)
+    assert bad == 0
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64).reshape(5, 4, group)
+    ref = (xf @ scipy.linalg.hadamard(group).astype(np.float64)) / np.sqrt(np.float64(group))
+    assert np.array_equal(y, ref.reshape(5, 4 * group).astype(np.float32))
+
+
+def test_small_group_closed_forms():
+    # one-hot c * e_i in a group of 128 -> +-c / sqrt(128) everywhere in it,
+    # zero in the other groups; orthonormal: applying it twice returns x
+    c = 3.0
+    x = np.zeros((1, 256), np.float32)
+    x[0, 128 + 5] = c
+    y, _ = oracle.rotate_rows(synth.f32_to_bf16_bits(x), 128)
+    assert np.all(y[0, :128] == 0)
+    assert np.array_equal(np.abs(y[0, 128:]), np.full(128, np.float32(c / np.sqrt(128.0))))
+    h = scipy.linalg.hadamard(128)
+    assert np.array_equal(np.sign(y[0, 128:]), h[5].astype(np.float32))
+    rng = np.random.default_rng(9)
+    xf = rng.standard_normal((3, 384))
+    twice = oracle.rotate_rows_f64(oracle.rotate_rows_f64(xf, 128), 128)
+    assert np.max(np.abs(twice - xf)) < 1e-12
+    assert np.allclose(np.sum(oracle.rotate_rows_f64(xf, 32) ** 2, axis=1), np.sum(xf ** 2, axis=1), rtol=1e-12)
 
 
 # ---------------------------------------------------------------------------
