@@ -22,7 +22,11 @@
  *   y_j  = fp32( (sum_i a_i * H[i][j]) / 16 )   per 256-group, H Sylvester,
  *          the sum exact (FP64; exact while the nonzero magnitudes inside a
  *          group span at most 37 binades -- finite BF16 inputs outside that
- *          range give unspecified low bits)
+ *          range give unspecified low bits).  Groups G of 16 .. 128 (the
+ *          sizes --dynamic-convrot falls back to, see convrot_dynamic_group):
+ *          the same with H_G and sqrt(G); for G = 32 and 128 the exact sum
+ *          is divided by fp64(sqrt(G)) in FP64 and that quotient rounded to
+ *          FP32.
  *   s    = fp32(max_k |y_k| / 127);  q = clamp(rne(y / s), -127, 127), q = 0
  *          and s = 0 for an all-zero row
  *   acc  = sum_k xq[m,k] * wq[n,k]   (INT32, exact for K <= 133144)
@@ -59,7 +63,7 @@ typedef enum {
     CONVROT_OK = 0,
     CONVROT_ERR_INVALID_ARG = 1,       /* null pointer, non-positive size */
     CONVROT_ERR_ALIGNMENT = 2,         /* a pointer is not 16-byte aligned */
-    CONVROT_ERR_UNSUPPORTED_SHAPE = 3, /* group != 256, k % group != 0, k too large */
+    CONVROT_ERR_UNSUPPORTED_SHAPE = 3, /* bad group, k % group != 0, k too large */
     CONVROT_ERR_UNSUPPORTED_ARCH = 4,  /* current device is not compute capability 10.0 */
     CONVROT_ERR_WORKSPACE = 5,         /* workspace missing or smaller than required */
     CONVROT_ERR_CUDA = 6,              /* a CUDA runtime/driver call failed */
@@ -71,7 +75,8 @@ typedef enum {
  *   q     : int8  [n, k] row-major -- the rotated, row-quantised weight Wq
  *   scale : fp32  [n]              -- sw, one scale per output row
  *   n     : out_features, k : in_features (the rotation runs along k)
- *   group : rotation group size; must be 256
+ *   group : rotation group size: 256 (the pages' setting), or a smaller power
+ *           of two >= 16 dividing k (convrot_dynamic_group)
  * The offline converter's record is an INT8 tensor, an FP32 row scale and the
  * ConvRot group size [zskr.cn "Qwen3-VL-32B ... INT8-ConvRot": 350 INT8
  * ConvRot matrices with FP32 scales; 0539edu.com section 4: "INT8 row-scale
@@ -96,16 +101,28 @@ int convrot_version(void);
 const char *convrot_last_error_string(void);
 
 /*
- * Fill a handle.  Checks: w, q, scale non-NULL; n, k >= 1; group == 256;
- * k % 256 == 0; k <= 133120 (INT32 accumulation bound); q and scale
- * 16-byte aligned.  Host only; touches no device.
+ * Fill a handle.  Checks: w, q, scale non-NULL; n, k >= 1; group a power
+ * of two in 16 .. 256 with k % group == 0; k <= 133120 (INT32 accumulation
+ * bound); q and scale 16-byte aligned.  Host only; touches no device.
  */
 convrot_status_t convrot_weight_init(convrot_weight_t *w, int8_t *q, float *scale,
                                      int64_t n, int64_t k, int32_t group);
 
 /*
+ * The rotation group --dynamic-convrot picks for a layer with k input
+ * features: the largest power of two <= max_group (the configured group
+ * size, 256) that divides k [0539edu.com "minimax-h3-nvfp4-convrot",
+ * section 4, item 3: the flag picks the largest compatible group size per
+ * layer; in_features 5376 keeps 256].  Returns 0 when that group would be
+ * below 16 (k not a multiple of 16: INT8 rows must be 16-byte multiples
+ * for the tensor-memory-access loads), which the other entry points reject.
+ * Host only.
+ */
+int32_t convrot_dynamic_group(int64_t k, int32_t max_group);
+
+/*
  * Offline weight conversion: rotate every row of the BF16 weight w [n, k]
- * (PyTorch Linear layout, out x in) per 256-group and quantise it row-wise
+ * (PyTorch Linear layout, out x in) per group and quantise it row-wise
  * by round-to-nearest into out->q and out->scale.  The pages quantise from
  * the BF16 source, never from an already quantised tensor [0539edu.com
  * section 4, engineering detail 1] and use RTN in "--simple" mode
@@ -115,9 +132,9 @@ convrot_status_t convrot_quantize_weight(const void *w_bf16, const convrot_weigh
                                          void *stream);
 
 /*
- * Activation prologue: rotate each row of x [m, k] (BF16) per 256-group and
- * quantise it per row into xq (int8 [m, k]) and sx (fp32 [m]).  Same
- * arithmetic as the weight conversion.
+ * Activation prologue: rotate each row of x [m, k] (BF16) per group (the
+ * weight's group) and quantise it per row into xq (int8 [m, k]) and sx
+ * (fp32 [m]).  Same arithmetic as the weight conversion.
  */
 convrot_status_t convrot_quantize_act(const void *x_bf16, int64_t m, int64_t k, int32_t group,
                                       int8_t *xq, float *sx, void *stream);

@@ -62,6 +62,7 @@ _WP = ctypes.POINTER(convrot_weight_t)
 SIGNATURES = {
     "convrot_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "convrot_version": ([], ctypes.c_int),
+    "convrot_dynamic_group": ([_I64, _I32], _I32),
     "convrot_last_error_string": ([], ctypes.c_char_p),
     "convrot_weight_init": ([_WP, _P, _P, _I64, _I64, _I32], ctypes.c_int),
     "convrot_quantize_weight": ([_P, _WP, _P], ctypes.c_int),
@@ -136,6 +137,10 @@ class QuantizedWeight:
     @property
     def k(self) -> int:
         return self.handle.k
+
+    @property
+    def group(self) -> int:
+        return self.handle.group
 
 
 def convrot_status_string(status: int) -> str:
@@ -278,12 +283,20 @@ def convrot_device_status(stream=None) -> None:
 
 
 # ---------------------------------------------------------------- helpers
-def quantize_weight(w_bf16: torch.Tensor, stream=None) -> QuantizedWeight:
-    """Allocate q/scale and run the offline rotate+quantise kernel."""
+def convrot_dynamic_group(k: int, max_group: int = GROUP) -> int:
+    """The group --dynamic-convrot picks for k input features (0: none)."""
+    return int(load_library().convrot_dynamic_group(k, max_group))
+
+
+def quantize_weight(w_bf16: torch.Tensor, stream=None, group: int = GROUP, dynamic: bool = False) -> QuantizedWeight:
+    """Allocate q/scale and run the offline rotate+quantise kernel; with
+    dynamic=True the group is the largest power of two <= group dividing k."""
     n, k = w_bf16.shape
+    if dynamic:
+        group = convrot_dynamic_group(k, group)
     q = torch.empty((n, k), dtype=torch.int8, device=w_bf16.device)
     scale = torch.empty((n,), dtype=torch.float32, device=w_bf16.device)
-    return convrot_quantize_weight(w_bf16, convrot_weight_init(q, scale), stream)
+    return convrot_quantize_weight(w_bf16, convrot_weight_init(q, scale, group), stream)
 
 
 def make_workspace(m: int, w: QuantizedWeight, device=None, linear: bool = True) -> torch.Tensor:

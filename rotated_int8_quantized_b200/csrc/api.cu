@@ -12,7 +12,8 @@
 
 namespace {
 
-constexpr int64_t kGroup = 256;
+constexpr int64_t kGroup = 256;         // the pages' group; also the largest
+constexpr int64_t kMinGroup = 16;       // INT8 rows must be 16-byte multiples (TMA row stride)
 // |acc| <= k * 127^2 must fit in INT32: k <= 133144; largest multiple of 256.
 constexpr int64_t kMaxK = 133120;
 constexpr int64_t kMaxRows = 0x7FFFFFFF;
@@ -65,10 +66,12 @@ int sms_for_sizing() {
     return kDefaultSms;
 }
 
+bool is_pow2(int64_t g) { return g > 0 && (g & (g - 1)) == 0; }
+
 convrot_status_t check_shape(int64_t rows, int64_t k, int64_t group) {
     if (rows < 1 || k < 1) return CONVROT_ERR_INVALID_ARG;
-    if (group != kGroup) return CONVROT_ERR_UNSUPPORTED_SHAPE;
-    if (k % kGroup != 0 || k > kMaxK || rows > kMaxRows) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    if (!is_pow2(group) || group < kMinGroup || group > kGroup) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    if (k % group != 0 || k > kMaxK || rows > kMaxRows) return CONVROT_ERR_UNSUPPORTED_SHAPE;
     return CONVROT_OK;
 }
 
@@ -110,6 +113,14 @@ const char *convrot_status_string(convrot_status_t s) {
 
 int convrot_version(void) { return 100; }
 
+int32_t convrot_dynamic_group(int64_t k, int32_t max_group) {
+    if (k < 1 || max_group < 1) return 0;
+    int64_t g = 1;
+    while (g * 2 <= max_group && g * 2 <= kGroup) g *= 2;
+    while (g > 1 && k % g != 0) g /= 2;
+    return g >= kMinGroup ? (int32_t)g : 0;
+}
+
 const char *convrot_last_error_string(void) { return t_last_error; }
 
 convrot_status_t convrot_weight_init(convrot_weight_t *w, int8_t *q, float *scale, int64_t n, int64_t k,
@@ -134,7 +145,7 @@ convrot_status_t convrot_quantize_weight(const void *w_bf16, const convrot_weigh
     if (!aligned16(w_bf16)) return CONVROT_ERR_ALIGNMENT;
     DeviceInfo dev;
     if ((s = current_device(&dev)) != CONVROT_OK) return s;
-    convrot::RQProblem prob = {w_bf16, out->k, out->q, out->scale};
+    convrot::RQProblem prob = {w_bf16, out->k, out->group, out->q, out->scale};
     return from_cuda(convrot::launch_rotate_quant(1, out->n, &prob, static_cast<cudaStream_t>(stream), false));
 }
 
@@ -146,12 +157,12 @@ convrot_status_t convrot_quantize_act(const void *x_bf16, int64_t m, int64_t k, 
     if (!aligned16(x_bf16) || !aligned16(xq) || !aligned16(sx)) return CONVROT_ERR_ALIGNMENT;
     DeviceInfo dev;
     if ((s = current_device(&dev)) != CONVROT_OK) return s;
-    convrot::RQProblem prob = {x_bf16, k, xq, sx};
+    convrot::RQProblem prob = {x_bf16, k, (int)group, xq, sx};
     return from_cuda(convrot::launch_rotate_quant(1, m, &prob, static_cast<cudaStream_t>(stream), false));
 }
 
 size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
-    if (m < 1 || n < 1 || k < kGroup) return 0;
+    if (m < 1 || n < 1 || k < kMinGroup || k % kMinGroup != 0 || k > kMaxK) return 0;
     convrot::GemmPlan p;
     convrot::plan_gemm(m, n, k, sms_for_sizing(), &p);
     return round256(p.ws_bytes);
@@ -272,12 +283,14 @@ convrot_status_t run_linear(int64_t m, int count, const convrot_linear_job_t *jo
         // a job whose input an earlier job already rotates reuses its codes
         int same = -1;
         for (int i = 0; i < j && same < 0; ++i)
-            if (jobs[i].x_bf16 == jobs[j].x_bf16 && jobs[i].w->k == jobs[j].w->k) same = i;
+            if (jobs[i].x_bf16 == jobs[j].x_bf16 && jobs[i].w->k == jobs[j].w->k &&
+                jobs[i].w->group == jobs[j].w->group)
+                same = i;
         if (same >= 0) {
             xq = const_cast<int8_t *>(gp[same].xq);
             sx = const_cast<float *>(gp[same].sx);
         } else {
-            rq[nrq++] = {jobs[j].x_bf16, jobs[j].w->k, xq, sx};
+            rq[nrq++] = {jobs[j].x_bf16, jobs[j].w->k, jobs[j].w->group, xq, sx};
         }
         gp[j] = {m, jobs[j].w->n, jobs[j].w->k, xq, sx, jobs[j].w->q, jobs[j].w->scale,
                  static_cast<__nv_bfloat16 *>(jobs[j].y_bf16), nullptr,
@@ -353,7 +366,7 @@ convrot_status_t convrot_gemm_i8_batch(int64_t m, int count, const convrot_gemm_
 }
 
 size_t convrot_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
-    if (m < 1 || n < 1 || k < kGroup) return 0;
+    if (m < 1 || n < 1 || k < kMinGroup || k % kMinGroup != 0 || k > kMaxK) return 0;
     convrot_weight_t w = {nullptr, nullptr, n, k, (int32_t)kGroup};
     convrot_linear_job_t job = {nullptr, &w, nullptr, nullptr};
     LinearLayout L;

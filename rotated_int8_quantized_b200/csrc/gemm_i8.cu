@@ -811,7 +811,7 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
     p->rows_b[0] = p->swap ? m : n;
     const int tiles_a = (int)((p->rows_a[0] + kTileA - 1) / kTileA);
     const int tiles_b = (int)((p->rows_b[0] + p->bn - 1) / p->bn);
-    const int kbpt = (int)(k / kBlockK);
+    const int kbpt = (int)((k + kBlockK - 1) / kBlockK);   // a partial last block reads zeros past k
     const int num_tiles = tiles_a * tiles_b;
     const long long units = (long long)num_tiles * kbpt;
     int tail_tile0;
@@ -882,7 +882,7 @@ void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, i
         p->tiles_a[j] = (int)((p->rows_a[j] + kTileA - 1) / kTileA);
         p->tiles_b[j] = (int)((p->rows_b[j] + p->bn - 1) / p->bn);
         p->group_a[j] = p->tiles_a[j];
-        p->kbpt[j] = (int)(k[j] / kBlockK);
+        p->kbpt[j] = (int)((k[j] + kBlockK - 1) / kBlockK);
         p->tile_base[j] = 0;
         p->unit0[j] = units;
         units += (long long)(p->swap ? p->tiles_a[j] : p->tiles_b[j]) * p->kbpt[j];

@@ -97,6 +97,7 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
 struct RQProblem {
     const void *a;      // BF16 [rows, k]
     int64_t k;
+    int group;          // rotation group (power of two, 16 .. 256)
     int8_t *q;          // int8 [rows, k]
     float *s;           // fp32 [rows]
 };

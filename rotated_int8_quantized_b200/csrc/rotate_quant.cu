@@ -20,6 +20,7 @@
 // 16-byte store.  Long rows are split over a cluster too (at most one group
 // per slot), so every row the API accepts (k <= 133120) stages in shared
 // memory.
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <cuda_bf16.h>
@@ -127,6 +128,24 @@ constexpr int kYGroupStride = 272;
 __host__ __device__ constexpr int y_group_stride(bool half) { return half ? 256 : kYGroupStride; }
 constexpr int kSlotsSmemMax = 226 * 1024;   // dynamic shared memory per CTA (227 KB minus the static part)
 
+// Butterflies of strides h < hmax only (hmax a power of two <= 16): the
+// transform of groups smaller than 16 along these index bits.
+__device__ __forceinline__ void fwht16_regs_upto(double (&v)[16], int hmax) {
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+        if (h < hmax) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                if ((e & h) == 0) {
+                    double a = v[e], b = v[e + h];
+                    v[e] = a + b;
+                    v[e + h] = a - b;
+                }
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ void fwht16_regs(double (&v)[16]) {
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1) {
@@ -150,7 +169,11 @@ struct RQJobDev {
     const __nv_bfloat16 *a;
     int8_t *q;
     float *s;
-    int k, gps, slots;      // gps / slots for the groups of ONE part of a row
+    int k, gps, slots;      // gps / slots for the 256-element chunks of ONE part of a row
+    int group;              // rotation group G (power of two, 16 .. 256; 256 unless DYN)
+    int exact_scale;        // G a power of four: 1/sqrt(G) is a power of two
+    double scale;           // 1/sqrt(G) when exact_scale
+    double root;            // fl64(sqrt(G)) otherwise (the quotient is rounded once in FP64)
 };
 struct RQArgs {
     int njobs, rows;
@@ -193,7 +216,11 @@ __device__ __forceinline__ void cluster_wait() {
 // memory, used for decode-sized launches whose CTAs should fit beside a
 // GEMM CTA); otherwise in one pass through a 16 x 17 buffer and in place
 // (fewer registers, for launches with a row per CTA).
-template <int GPS, bool HALF>
+// DYN: groups other than 256 (--dynamic-convrot): a 256-element chunk holds
+// 256/G independent groups (butterflies of strides < G only), a row's last
+// chunk may be partial (k % 256 != 0; k is a multiple of G), and the
+// normalisation divides by sqrt(G) in FP64 when G is not a power of four.
+template <int GPS, bool HALF, bool DYN>
 __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
     constexpr int kXchStride = HALF ? kXchHalf : kXchFull;
@@ -210,7 +237,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     const int row = rowid - jb * args.rows;
     const RQJobDev &J = args.job[jb];
     const int k = J.k, gps = J.gps, slots = J.slots;
-    const int groups = k >> 8;
+    const int groups = DYN ? (k + 255) >> 8 : k >> 8;     // 256-element chunks
     const int g0 = part * groups / C, g1 = (part + 1) * groups / C;
     double *xch = reinterpret_cast<double *>(rq_smem);                    // slots * 272 doubles
     float *ybuf = reinterpret_cast<float *>(rq_smem + (size_t)(blockDim.x >> 4) * kXchStride * 8);
@@ -226,9 +253,14 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     for (int gi = 0; gi < GPS; ++gi) {
         const int g = g0 + slot + gi * slots;
         if (gi < gps && slot < slots && g < g1) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(arow + (size_t)g * 256 + t * 16);
-            raw[gi][0] = __ldg(src);
-            raw[gi][1] = __ldg(src + 1);
+            if (!DYN || g * 256 + t * 16 < k) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(arow + (size_t)g * 256 + t * 16);
+                raw[gi][0] = __ldg(src);
+                raw[gi][1] = __ldg(src + 1);
+            } else {        // past the end of the row: zeros rotate to zeros
+                raw[gi][0] = make_uint4(0u, 0u, 0u, 0u);
+                raw[gi][1] = make_uint4(0u, 0u, 0u, 0u);
+            }
         }
     }
 
@@ -243,7 +275,10 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                                    raw[gi][1].x, raw[gi][1].y, raw[gi][1].z, raw[gi][1].w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
-            fwht16_regs(v);                                  // index bits 0-3
+            if (DYN)
+                fwht16_regs_upto(v, J.group < 16 ? J.group : 16);
+            else
+                fwht16_regs(v);                              // index bits 0-3
             // transpose across the slot's 16 threads: thread u needs element
             // 16*j + u of every thread j, i.e. v[u] of thread j (padded rows:
             // conflict-free both ways)
@@ -268,13 +303,17 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                 for (int i = 0; i < 16; ++i) x[i] = xb[t + 17 * i];
                 __syncwarp(half_mask);
             }
-            fwht16_regs(x);                                  // index bits 4-7
+            if (DYN)
+                fwht16_regs_upto(x, J.group >> 4);
+            else
+                fwht16_regs(x);                              // index bits 4-7
             // output 16*i + t of the group is element t of chunk i (its
             // float4 part XOR-swizzled in launches with a row per CTA)
             float *yg = ybuf + (size_t)(g - g0) * y_group_stride(HALF) + (HALF ? t : (t & 3));
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float y = __double2float_rn(x[i] * 0.0625);   // / sqrt(256), exact
+                const float y = DYN ? __double2float_rn(J.exact_scale ? x[i] * J.scale : __ddiv_rn(x[i], J.root))
+                                    : __double2float_rn(x[i] * 0.0625);   // / sqrt(256), exact
                 yg[16 * i + (HALF ? 0 : 4 * ((t >> 2) ^ ((i >> 1) & 3)))] = y;
                 amax = fmaxf(amax, fabsf(y));
             }
@@ -308,7 +347,8 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
 
     // quantise 16 consecutive outputs per thread, one 16-byte store
     int8_t *qrow = J.q + (size_t)row * k + (size_t)g0 * 256;
-    const int chunks = (g1 - g0) * 16;
+    int chunks = (g1 - g0) * 16;
+    if (DYN && g0 * 256 + chunks * 16 > k) chunks = (k - g0 * 256) / 16;     // partial last chunk
     for (int c0 = 0; c0 < chunks; c0 += blockDim.x) {
         const int c = c0 + tid;
         const unsigned mask = __ballot_sync(__activemask(), c < chunks);
@@ -335,7 +375,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     }
 }
 
-template <int GPS, bool HALF>
+template <int GPS, bool HALF, bool DYN>
 static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int max_slots, int max_local_groups) {
     cfg.blockDim = dim3(max_slots * 16);
     cfg.dynamicSmemBytes =
@@ -345,12 +385,33 @@ static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(rotate_quant_rows_slots<GPS, HALF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(rotate_quant_rows_slots<GPS, HALF, DYN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSlotsSmemMax);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev] = true;
     }
-    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS, HALF>, args);
+    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS, HALF, DYN>, args);
+}
+
+template <bool DYN>
+static cudaError_t launch_gps(cudaLaunchConfig_t &cfg, const RQArgs &args, bool half, int max_gps, int max_slots,
+                              int max_local) {
+    if (half) {
+        switch (max_gps) {
+            case 1: return launch_slots<1, true, DYN>(cfg, args, max_slots, max_local);
+            case 2: return launch_slots<2, true, DYN>(cfg, args, max_slots, max_local);
+            case 3: return launch_slots<3, true, DYN>(cfg, args, max_slots, max_local);
+            case 4: return launch_slots<4, true, DYN>(cfg, args, max_slots, max_local);
+            default: return launch_slots<6, true, DYN>(cfg, args, max_slots, max_local);
+        }
+    }
+    switch (max_gps) {
+        case 1: return launch_slots<1, false, DYN>(cfg, args, max_slots, max_local);
+        case 2: return launch_slots<2, false, DYN>(cfg, args, max_slots, max_local);
+        case 3: return launch_slots<3, false, DYN>(cfg, args, max_slots, max_local);
+        case 4: return launch_slots<4, false, DYN>(cfg, args, max_slots, max_local);
+        default: return launch_slots<6, false, DYN>(cfg, args, max_slots, max_local);
+    }
 }
 
 // CTAs per row (a thread-block cluster).  When the rows alone do not fill
@@ -381,7 +442,7 @@ static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, bool h
                             int *max_gps, int *max_local) {
     int ms = 0, mg = 0, ml = 0;
     for (int j = 0; j < njobs; ++j) {
-        const int groups = (int)(probs[j].k >> 8);
+        const int groups = (int)((probs[j].k + 255) >> 8);
         const int local = (groups + parts - 1) / parts;
         int g, sl;
         rq_shape(local, &g, &sl);
@@ -438,6 +499,7 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         rq_smem_bytes(njobs, probs, parts, half, &max_slots, &max_gps, &max_local) <= (size_t)kSlotsSmemMax) {
         RQArgs args;
         memset(&args, 0, sizeof(args));
+        bool dyn = false;
         args.njobs = njobs;
         args.rows = (int)rows;
         args.parts = parts;
@@ -447,25 +509,18 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
             J.q = probs[j].q;
             J.s = probs[j].s;
             J.k = (int)probs[j].k;
-            const int groups = J.k >> 8;
+            J.group = probs[j].group;
+            int lg = 0;
+            while ((1 << lg) < J.group) ++lg;
+            J.exact_scale = (lg % 2 == 0) ? 1 : 0;
+            J.scale = 1.0 / (double)(1 << (lg / 2));
+            J.root = sqrt((double)J.group);
+            const int groups = (J.k + 255) >> 8;
             rq_shape((groups + parts - 1) / parts, &J.gps, &J.slots);
+            dyn = dyn || J.group != 256 || (J.k & 255) != 0;
         }
-        if (half) {
-            switch (max_gps) {
-                case 1: return launch_slots<1, true>(cfg, args, max_slots, max_local);
-                case 2: return launch_slots<2, true>(cfg, args, max_slots, max_local);
-                case 3: return launch_slots<3, true>(cfg, args, max_slots, max_local);
-                case 4: return launch_slots<4, true>(cfg, args, max_slots, max_local);
-                default: return launch_slots<6, true>(cfg, args, max_slots, max_local);
-            }
-        }
-        switch (max_gps) {
-            case 1: return launch_slots<1, false>(cfg, args, max_slots, max_local);
-            case 2: return launch_slots<2, false>(cfg, args, max_slots, max_local);
-            case 3: return launch_slots<3, false>(cfg, args, max_slots, max_local);
-            case 4: return launch_slots<4, false>(cfg, args, max_slots, max_local);
-            default: return launch_slots<6, false>(cfg, args, max_slots, max_local);
-        }
+        if (dyn) return launch_gps<true>(cfg, args, half, max_gps, max_slots, max_local);
+        return launch_gps<false>(cfg, args, half, max_gps, max_slots, max_local);
     }
     // unreachable within the shapes the API accepts (k <= 133120 stages in
     // at most 114 KB per CTA with 8 parts)

@@ -58,7 +58,12 @@ def test_weight_init_validation(lib):
     assert _init(lib, 0, 0x20000, 256, 512, 256)[0] == 1          # null q
     assert _init(lib, 0x10000, 0x20000, 0, 512, 256)[0] == 1      # n = 0
     assert _init(lib, 0x10000, 0x20000, 8, 300, 256)[0] == 3      # k % 256
-    assert _init(lib, 0x10000, 0x20000, 8, 512, 128)[0] == 3      # group
+    assert _init(lib, 0x10000, 0x20000, 8, 512, 128)[0] == 0      # a smaller power-of-two group
+    assert _init(lib, 0x10000, 0x20000, 8, 640, 128)[0] == 0      # ... need not divide 256
+    assert _init(lib, 0x10000, 0x20000, 8, 512, 96)[0] == 3       # not a power of two
+    assert _init(lib, 0x10000, 0x20000, 8, 512, 8)[0] == 3        # below 16
+    assert _init(lib, 0x10000, 0x20000, 8, 512, 512)[0] == 3      # above 256
+    assert _init(lib, 0x10000, 0x20000, 8, 640, 256)[0] == 3      # k % group
     assert _init(lib, 0x10000, 0x20000, 8, 133376, 256)[0] == 3   # INT32 accumulation bound
     assert _init(lib, 0x10001, 0x20000, 8, 512, 256)[0] == 2      # misaligned q
     assert _init(lib, 0x10000, 0x20004, 8, 512, 256)[0] == 2      # misaligned scale
@@ -132,3 +137,15 @@ int main(void) {
         "convrot_linear_job_t.bias_bf16": cr.convrot_linear_job_t.bias_bf16.offset,
     }
     assert {k: int(v) for k, v in got.items()} == want
+
+
+def test_dynamic_group(lib):
+    # the largest power of two <= the cap dividing k; 0 below 16
+    assert lib.convrot_dynamic_group(5376, 256) == 256
+    assert lib.convrot_dynamic_group(640, 256) == 128
+    assert lib.convrot_dynamic_group(5440, 256) == 64
+    assert lib.convrot_dynamic_group(1024, 64) == 64
+    assert lib.convrot_dynamic_group(40, 256) == 0
+    for k in range(16, 4000, 16):
+        g = lib.convrot_dynamic_group(k, 256)
+        assert g >= 16 and g <= 256 and k % g == 0 and (g == 256 or k % (2 * g) != 0)

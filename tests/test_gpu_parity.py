@@ -442,3 +442,54 @@ def test_gemm_batch_bias(cr, m):
     cr.convrot_device_status()
     for y, ref in zip(ys, refs):
         assert np.array_equal(to_bits(y), ref)
+
+
+# ---------------------------------------------------------------- --dynamic-convrot groups
+# (m, k, group): groups below 256, rows that end in a partial 256-element
+# chunk, rows shorter than 256, decode-sized launches (rows over a cluster)
+# and one-CTA-per-row launches, the FP64 division by sqrt(G) for G = 32, 128
+DYN_ACT = [(3, 640, 128), (150, 640, 128), (4, 48, 16), (160, 48, 16), (2, 5440, 64), (150, 5440, 64),
+           (5, 1376, 32), (149, 1376, 32), (3, 1024, 128), (2, 25600, 128), (148, 8192, 32)]
+
+
+@pytest.mark.parametrize("m,k,group", DYN_ACT)
+def test_act_quant_dynamic_group_bit_exact(cr, m, k, group):
+    assert cr.convrot_dynamic_group(k) == group or k % 256 == 0
+    cs = synth.outlier_scale_fraction(synth.stream_key(m + k + group, 2), k, 0.01, 30.0)
+    x_bits = synth.draw_np(synth.stream_key(m + k + group, 0), m, k, 1.0, cs)
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+    cr.convrot_quantize_act(from_bits(x_bits), xq, sx, group=group)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.rotate_quantize(x_bits, group)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# (m, n, k): K not a multiple of the 128-byte K block (the last block reads
+# zeros past k), through both GEMM orientations and the batched layer
+DYN_LINEAR = [(12, 384, 640), (4, 256, 48), (300, 512, 640), (700, 640, 5440), (12, 1000, 1376)]
+
+
+@pytest.mark.parametrize("m,n,k", DYN_LINEAR)
+def test_linear_dynamic_group(cr, m, n, k):
+    group = cr.convrot_dynamic_group(k)
+    seed = 7000 + m + n + k
+    cs = synth.outlier_scale_fraction(synth.stream_key(seed, 2), k, 0.01, 30.0)
+    x_bits = synth.draw_np(synth.stream_key(seed, 0), m, k, 1.0, cs)
+    w_bits = synth.draw_np(synth.stream_key(seed, 1), n, k, synth.W_SIGMA)
+    wq_ref, sw_ref = oracle.rotate_quantize(w_bits, group)
+    ref = oracle.linear_int8(x_bits, wq_ref, sw_ref, group=group)
+    w = cr.quantize_weight(from_bits(w_bits), dynamic=True)
+    assert w.group == group
+    assert np.array_equal(w.q.cpu().numpy(), wq_ref) and np.array_equal(w.scale.cpu().numpy(), sw_ref)
+    y = cr.linear_int8(from_bits(x_bits), w, cr.make_workspace(m, w))
+    acc = torch.empty((m, n), dtype=torch.int32, device="cuda")
+    cr.convrot_gemm_i8(torch.from_numpy(ref["xq"]).cuda(), torch.from_numpy(ref["sx"]).cuda(), w, None, acc,
+                       cr.make_workspace(m, w, linear=False))
+    ys = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    cr.LinearBatch([from_bits(x_bits)], [w], [ys])()
+    cr.convrot_device_status()
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(to_bits(y), ref["y"])
+    assert np.array_equal(to_bits(ys), ref["y"])
