@@ -22,6 +22,8 @@ the source pages it follows, is stated in the C file:
   (an extension; the pages' projections carry none)
 * the group --dynamic-convrot picks: the largest power of two <= 256 that
   divides k, with rotations of such groups (0539edu.com section 4, item 3)
+* tensor-wise simple INT8 of the embedding table and the lookup from it
+  (zskr.cn quantisation configuration and conversion command)
 
 Every function here is pinned by the ``-m "not gpu"`` tests against
 something other than itself (scipy's Hadamard, closed forms, brute force,
@@ -71,6 +73,10 @@ def _load():
         lib.oracle_gemm_i32.argtypes = [P, P, I64, I64, I64, P]
         lib.oracle_gemm_i32.restype = I64
         lib.oracle_dequant_bf16.argtypes = [P, P, P, I64, I64, P]
+        lib.oracle_quantize_tensor.argtypes = [P, I64, P, P]
+        lib.oracle_quantize_tensor.restype = I64
+        lib.oracle_embed_lookup.argtypes = [P, I64, P, ctypes.c_float, I64, I64, P]
+        lib.oracle_embed_lookup.restype = I64
         lib.oracle_dynamic_group.argtypes = [I64, ctypes.c_int]
         lib.oracle_dynamic_group.restype = ctypes.c_int
         lib.oracle_dequant_bf16_bias.argtypes = [P, P, P, P, I64, I64, P]
@@ -168,6 +174,29 @@ def rotate_quantize(a_bf16: np.ndarray, group: int = 256):
     if bad > 0:
         raise OracleError("%d rotation groups span more than 37 binades" % bad)
     return q, s
+
+
+def quantize_tensor(a_bf16: np.ndarray):
+    """Tensor-wise simple INT8 (embedding table): ``(q int8, s fp32 scalar,
+    ties)`` with one scale for the whole tensor, no rotation."""
+    a = _bf16_bits(a_bf16)
+    q = np.empty(a.shape, dtype=np.int8)
+    s = np.empty((1,), dtype=np.float32)
+    ties = _load().oracle_quantize_tensor(_ptr(a), a.size, _ptr(q), _ptr(s))
+    if ties < 0:
+        raise OracleError("out of memory")
+    return q, s[0], int(ties)
+
+
+def embed_lookup(tokens: np.ndarray, q: np.ndarray, s) -> np.ndarray:
+    """out[i] = bf16(q[tokens[i]] * s) as BF16 bits; zero rows for tokens
+    outside the table."""
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    vocab, dim = q.shape
+    out = np.empty((tokens.size, dim), dtype=np.uint16)
+    _load().oracle_embed_lookup(_ptr(tokens), tokens.size, _ptr(q), float(np.float32(s)), vocab, dim, _ptr(out))
+    return out
 
 
 def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:

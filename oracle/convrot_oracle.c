@@ -286,6 +286,51 @@ int64_t oracle_quantize_rows(const float *y, int64_t rows, int64_t k,
 }
 
 /* ------------------------------------------------------------------ */
+/* Tensor-wise "simple" INT8 (the word-embedding table)                */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The converter treats the embedding table apart from the ConvRot matrices:
+ * simple tensor-wise INT8, i.e. no rotation, ONE FP32 scale for the whole
+ * tensor and round-to-nearest [zskr.cn "Qwen3-VL-32B ... INT8-ConvRot",
+ * quantisation configuration: word embedding "simple tensor-wise INT8";
+ * conversion command: --custom-layers embed_tokens --custom-type int8
+ * --custom-scaling-mode tensor --custom-simple].  The scale and codes follow
+ * the row rule above with the whole tensor as the row:
+ *   a = max |x| over all elements,  s = a / 127,  q = clamp(rne(x / s)).
+ * a is BF16 bits [count].  Returns the number of exact .5 ties met.
+ */
+int64_t oracle_quantize_tensor(const uint16_t *a, int64_t count, int8_t *q, float *s)
+{
+    float *x = (float *)malloc(sizeof(float) * (size_t)(count > 0 ? count : 1));
+    if (!x) return -1;
+    for (int64_t i = 0; i < count; ++i) x[i] = bf16_bits_to_float(a[i]);
+    int64_t ties = oracle_quantize_rows(x, 1, count, q, s);
+    free(x);
+    return ties;
+}
+
+/*
+ * Embedding lookup from the tensor-wise table q [vocab, dim] with scale s:
+ *   out[i, d] = bf16_rne( (float)q[tokens[i], d] * s ).
+ * A token outside [0, vocab) gives a zero row.  Returns the number of such
+ * tokens.
+ */
+int64_t oracle_embed_lookup(const int32_t *tokens, int64_t t, const int8_t *q, float s,
+                            int64_t vocab, int64_t dim, uint16_t *out)
+{
+    int64_t bad = 0;
+    for (int64_t i = 0; i < t; ++i) {
+        int64_t tok = tokens[i];
+        int ok = tok >= 0 && tok < vocab;
+        if (!ok) ++bad;
+        for (int64_t d = 0; d < dim; ++d)
+            out[i * dim + d] = ok ? oracle_float_to_bf16((float)q[tok * dim + d] * s) : 0;
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------ */
 /* INT8 GEMM with INT32 result                                         */
 /* ------------------------------------------------------------------ */
 

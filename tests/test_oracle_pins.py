@@ -170,6 +170,45 @@ def test_rotation_rejects_bad_group():
 
 
 # ---------------------------------------------------------------------------
+# tensor-wise simple INT8 (embedding table) and the lookup
+# ---------------------------------------------------------------------------
+def test_tensor_quant_closed_forms():
+    f2b = synth.f32_to_bf16_bits
+    p = -3
+    # the largest magnitude 127 * 2^p sets s = 2^p exactly; y / s are then
+    # exact, ties go to even, and one scale serves every row
+    x = np.array([[127.0, 2.5, 3.5, -0.5, 1.0], [0.25, -4.5, 6.5, 0.0, -127.0]], np.float32) * 2.0 ** p
+    q, sc, ties = oracle.quantize_tensor(f2b(x))
+    assert sc == np.float32(2.0 ** p) and ties == 5
+    assert np.array_equal(q, np.array([[127, 2, 4, 0, 1], [0, -4, 6, 0, -127]], np.int8))
+    # per-row scales would differ (row 1's own maximum is the same here, so
+    # use a table whose rows have different maxima)
+    y = np.array([[127.0, 1.0], [1.0, 0.5]], np.float32)
+    qt, st, _ = oracle.quantize_tensor(f2b(y))
+    qr, sr, _ = oracle.quantize_rows(y)
+    assert st == sr[0] and np.array_equal(qt[0], qr[0]) and not np.array_equal(qt[1], qr[1])
+    assert list(qt[1]) == [1, 0]                     # 0.5 / 1 = 0.5 -> 0 (ties to even)
+    # all-zero table
+    q0, s0, _ = oracle.quantize_tensor(np.zeros((3, 4), np.uint16))
+    assert s0 == 0 and not q0.any()
+
+
+def test_embed_lookup_closed_forms():
+    rng = np.random.default_rng(11)
+    q = rng.integers(-127, 128, (50, 32)).astype(np.int8)
+    s = np.float32(2.0 ** -5)
+    tokens = np.array([3, 49, 0, 3, -1, 50], np.int32)
+    out = oracle.embed_lookup(tokens, q, s)
+    want = q[[3, 49, 0, 3]].astype(np.float32) * np.float32(2.0 ** -5)     # exact in BF16
+    assert np.array_equal(synth.bf16_bits_to_f32(out[:4]), want)
+    assert not out[4:].any()                                                # out of range -> zero rows
+    # a scale that is not a power of two rounds each product once to BF16
+    s2 = np.float32(0.0123)
+    out2 = oracle.embed_lookup(np.array([7], np.int32), q, s2)
+    assert np.array_equal(out2[0], _f32_to_bf16_torch(q[7].astype(np.float32) * s2))
+
+
+# ---------------------------------------------------------------------------
 # --dynamic-convrot: smaller power-of-two groups
 # ---------------------------------------------------------------------------
 def test_dynamic_group_choice():
