@@ -275,10 +275,42 @@ convrot_status_t convrot_gemm_i8_noalloc(const int8_t *xq, const float *sx, int6
                                          void *stream);
 
 /*
+ * Tensor-wise "simple" INT8 of a BF16 tensor of `count` elements (the
+ * word-embedding table [vocab, dim]): no rotation, ONE scale for the whole
+ * tensor, round-to-nearest-even --
+ *   a = max |x|;  *scale = fl(a / 127);  q = clamp(rne(fl(x / s)), -127, 127)
+ * (q = 0, s = 0 for an all-zero tensor) -- the treatment the converter gives
+ * the embedding table instead of ConvRot [zskr.cn "Qwen3-VL-32B ...
+ * INT8-ConvRot": word embedding "simple tensor-wise INT8"; conversion
+ * command --custom-layers embed_tokens --custom-type int8
+ * --custom-scaling-mode tensor --custom-simple].
+ *   w_bf16 : BF16 [count] (device);  q : int8 [count] (device)
+ *   scale  : ONE fp32 (device), overwritten; it also holds the running
+ *            maximum between the launches, so it may not alias w or q.
+ * count >= 16 and a multiple of 16.  Offline: four stream-ordered steps (a
+ * memset of *scale and three kernels).
+ */
+convrot_status_t convrot_quantize_tensor(const void *w_bf16, int64_t count, int8_t *q, float *scale,
+                                         void *stream);
+
+/*
+ * Rows of the tensor-wise table: out[i, :] = bf16_rne(fl((float)q[tokens[i], :]
+ * * scale)) for i < t.
+ *   tokens : int32 [t] (device);  q : int8 [vocab, dim];  scale : one fp32
+ *   out_bf16 : BF16 [t, dim]
+ * dim a multiple of 16.  A token id outside [0, vocab) cannot be checked on
+ * the host: its row is written as zeros and CONVROT_ERR_INVALID_ARG is
+ * recorded for convrot_device_status().
+ */
+convrot_status_t convrot_embed_lookup(const int32_t *tokens, int64_t t, const int8_t *q, const float *scale,
+                                      int64_t vocab, int64_t dim, void *out_bf16, void *stream);
+
+/*
  * Synchronise `stream`, then read and clear the device-side status word of
  * the current device.  Returns CONVROT_OK, CONVROT_ERR_DEVICE_TIMEOUT if a
  * bounded wait ran out in some kernel since the last call (the workspace
- * must then be re-initialised), or CONVROT_ERR_CUDA.
+ * must then be re-initialised), CONVROT_ERR_INVALID_ARG if a lookup met a
+ * token outside its table, or CONVROT_ERR_CUDA.
  */
 convrot_status_t convrot_device_status(void *stream);
 

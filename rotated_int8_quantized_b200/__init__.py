@@ -63,6 +63,8 @@ SIGNATURES = {
     "convrot_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "convrot_version": ([], ctypes.c_int),
     "convrot_dynamic_group": ([_I64, _I32], _I32),
+    "convrot_quantize_tensor": ([_P, _I64, _P, _P, _P], ctypes.c_int),
+    "convrot_embed_lookup": ([_P, _I64, _P, _P, _I64, _I64, _P, _P], ctypes.c_int),
     "convrot_last_error_string": ([], ctypes.c_char_p),
     "convrot_weight_init": ([_WP, _P, _P, _I64, _I64, _I32], ctypes.c_int),
     "convrot_quantize_weight": ([_P, _WP, _P], ctypes.c_int),
@@ -276,6 +278,23 @@ class GemmBatch:
     def __call__(self, stream=None) -> None:
         _check(load_library().convrot_gemm_i8_batch(self.m, len(self.jobs), self.jobs, _ptr(self.ws),
                                                     self.ws.numel(), _stream(stream)), "convrot_gemm_i8_batch")
+
+
+def convrot_quantize_tensor(w_bf16: torch.Tensor, q: torch.Tensor, scale: torch.Tensor, stream=None) -> None:
+    """Tensor-wise simple INT8 (embedding table): q int8 like w, scale a
+    one-element fp32 tensor."""
+    assert w_bf16.dtype == torch.bfloat16 and q.dtype == torch.int8 and q.numel() == w_bf16.numel()
+    assert scale.dtype == torch.float32 and scale.numel() == 1
+    _check(load_library().convrot_quantize_tensor(_ptr(w_bf16), w_bf16.numel(), _ptr(q), _ptr(scale),
+                                                  _stream(stream)), "convrot_quantize_tensor")
+
+
+def convrot_embed_lookup(tokens: torch.Tensor, q: torch.Tensor, scale: torch.Tensor, out: torch.Tensor,
+                         stream=None) -> None:
+    """out[i] = bf16(q[tokens[i]] * scale) for int32 tokens [t], q [vocab, dim]."""
+    assert tokens.dtype == torch.int32 and q.dim() == 2 and out.shape == (tokens.numel(), q.shape[1])
+    _check(load_library().convrot_embed_lookup(_ptr(tokens), tokens.numel(), _ptr(q), _ptr(scale), q.shape[0],
+                                               q.shape[1], _ptr(out), _stream(stream)), "convrot_embed_lookup")
 
 
 def convrot_device_status(stream=None) -> None:

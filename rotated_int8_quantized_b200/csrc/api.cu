@@ -396,6 +396,34 @@ convrot_status_t convrot_linear_int8_batch(int64_t m, int count, const convrot_l
     return run_linear(m, count, jobs, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+convrot_status_t convrot_quantize_tensor(const void *w_bf16, int64_t count, int8_t *q, float *scale,
+                                         void *stream) {
+    if (!w_bf16 || !q || !scale || count < 16) return CONVROT_ERR_INVALID_ARG;
+    if (count % 16 != 0) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(w_bf16) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+        return CONVROT_ERR_ALIGNMENT;
+    if (ranges_overlap(scale, 4, w_bf16, (size_t)count * 2) || ranges_overlap(scale, 4, q, (size_t)count))
+        return CONVROT_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    convrot_status_t s = current_device(&dev);
+    if (s != CONVROT_OK) return s;
+    return from_cuda(convrot::launch_quantize_tensor(w_bf16, count, q, scale, static_cast<cudaStream_t>(stream)));
+}
+
+convrot_status_t convrot_embed_lookup(const int32_t *tokens, int64_t t, const int8_t *q, const float *scale,
+                                      int64_t vocab, int64_t dim, void *out_bf16, void *stream) {
+    if (!tokens || !q || !scale || !out_bf16 || t < 1 || vocab < 1 || dim < 16) return CONVROT_ERR_INVALID_ARG;
+    if (dim % 16 != 0) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(q) || !aligned16(out_bf16) || (reinterpret_cast<uintptr_t>(tokens) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+        return CONVROT_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    convrot_status_t s = current_device(&dev);
+    if (s != CONVROT_OK) return s;
+    return from_cuda(convrot::launch_embed_lookup(tokens, t, q, scale, vocab, dim, out_bf16,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
 convrot_status_t convrot_device_status(void *stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) {

@@ -106,4 +106,9 @@ struct RQProblem {
 // count) in one launch.
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl);
 
+// ------------------------------------------------------------------ tensor-wise INT8 (embedding table)
+cudaError_t launch_quantize_tensor(const void *a, int64_t count, int8_t *q, float *scale, cudaStream_t stream);
+cudaError_t launch_embed_lookup(const int32_t *tokens, int64_t t, const int8_t *q, const float *scale,
+                                int64_t vocab, int64_t dim, void *out, cudaStream_t stream);
+
 }  // namespace convrot

@@ -2,5 +2,6 @@
 // status word and all kernels in one module without relocatable device code).
 #include "rotate_quant.cu"
 #include "gemm_i8.cu"
+#include "tensor_quant.cu"
 #include "api.cu"
 #include "noalloc.cu"

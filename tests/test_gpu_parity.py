@@ -493,3 +493,57 @@ def test_linear_dynamic_group(cr, m, n, k):
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
     assert np.array_equal(to_bits(y), ref["y"])
     assert np.array_equal(to_bits(ys), ref["y"])
+
+
+# ---------------------------------------------------------------- tensor-wise INT8 (embedding table)
+@pytest.mark.parametrize("vocab,dim", [(4096, 5120), (3, 16), (1000, 48)])
+def test_tensor_quant_bit_exact(cr, vocab, dim):
+    w_bits = synth.draw_np(synth.stream_key(vocab + dim, 7), vocab, dim, 0.05, None)
+    q = torch.empty((vocab, dim), dtype=torch.int8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    cr.convrot_quantize_tensor(from_bits(w_bits), q, s)
+    torch.cuda.synchronize()
+    q_ref, s_ref, _ = oracle.quantize_tensor(w_bits)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert s.cpu().numpy().view(np.uint32)[0] == np.float32(s_ref).view(np.uint32)
+
+
+def test_tensor_quant_ties_and_zero(cr):
+    p = -6
+    row = np.array([127.0, 2.5, -3.5, 0.5, -126.5, 1.5, 6.5, -0.5] * 4, np.float32) * 2.0 ** p
+    bits = synth.f32_to_bf16_bits(np.tile(row, (3, 1)))
+    q = torch.empty((3, 32), dtype=torch.int8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    cr.convrot_quantize_tensor(from_bits(bits), q, s)
+    torch.cuda.synchronize()
+    q_ref, s_ref, ties = oracle.quantize_tensor(bits)
+    assert ties > 0 and np.array_equal(q.cpu().numpy(), q_ref) and s.item() == s_ref == 2.0 ** p
+    qz = torch.full((2, 16), 5, dtype=torch.int8, device="cuda")
+    cr.convrot_quantize_tensor(torch.zeros((2, 16), dtype=torch.bfloat16, device="cuda"), qz, s)
+    torch.cuda.synchronize()
+    assert s.item() == 0 and int(qz.abs().max()) == 0
+
+
+def test_embed_lookup_matches_oracle(cr):
+    vocab, dim = 2000, 1024
+    w_bits = synth.draw_np(synth.stream_key(99, 7), vocab, dim, 0.05, None)
+    q = torch.empty((vocab, dim), dtype=torch.int8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    cr.convrot_quantize_tensor(from_bits(w_bits), q, s)
+    rng = np.random.default_rng(3)
+    tokens = np.concatenate([[0, vocab - 1, 5, 5], rng.integers(0, vocab, 60)]).astype(np.int32)
+    out = torch.empty((tokens.size, dim), dtype=torch.bfloat16, device="cuda")
+    cr.convrot_embed_lookup(torch.from_numpy(tokens).cuda(), q, s, out)
+    cr.convrot_device_status()
+    q_ref, s_ref, _ = oracle.quantize_tensor(w_bits)
+    assert np.array_equal(to_bits(out), oracle.embed_lookup(tokens, q_ref, s_ref))
+    # an id outside the table: zero row, reported by the status word
+    bad = torch.tensor([1, vocab, -3], dtype=torch.int32, device="cuda")
+    out2 = torch.full((3, dim), 1.0, dtype=torch.bfloat16, device="cuda")
+    cr.convrot_embed_lookup(bad, q, s, out2)
+    with pytest.raises(cr.ConvrotError) as e:
+        cr.convrot_device_status()
+    assert e.value.status == 1
+    cr.convrot_device_status()           # cleared by the read
+    assert np.array_equal(to_bits(out2[:1]), oracle.embed_lookup(np.array([1], np.int32), q_ref, s_ref))
+    assert not to_bits(out2[1:]).any()
