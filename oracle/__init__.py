@@ -24,6 +24,9 @@ the source pages it follows, is stated in the C file:
   divides k, with rotations of such groups (0539edu.com section 4, item 3)
 * tensor-wise simple INT8 of the embedding table and the lookup from it
   (zskr.cn quantisation configuration and conversion command)
+* INT4 ConvRot weights (levels -7..7, row scale a/7) packed two per byte,
+  with INT8 activations: the W4A4 variant's Blackwell route (0539edu.com
+  sections 5 and 7)
 
 Every function here is pinned by the ``-m "not gpu"`` tests against
 something other than itself (scipy's Hadamard, closed forms, brute force,
@@ -77,6 +80,12 @@ def _load():
         lib.oracle_quantize_tensor.restype = I64
         lib.oracle_embed_lookup.argtypes = [P, I64, P, ctypes.c_float, I64, I64, P]
         lib.oracle_embed_lookup.restype = I64
+        lib.oracle_quantize_rows4.argtypes = [P, I64, I64, P, P]
+        lib.oracle_quantize_rows4.restype = I64
+        lib.oracle_pack_int4.argtypes = [P, I64, I64, P]
+        lib.oracle_unpack_int4.argtypes = [P, I64, I64, P]
+        lib.oracle_rotate_quantize4.argtypes = [P, I64, I64, ctypes.c_int, P, P]
+        lib.oracle_rotate_quantize4.restype = I64
         lib.oracle_dynamic_group.argtypes = [I64, ctypes.c_int]
         lib.oracle_dynamic_group.restype = ctypes.c_int
         lib.oracle_dequant_bf16_bias.argtypes = [P, P, P, P, I64, I64, P]
@@ -197,6 +206,55 @@ def embed_lookup(tokens: np.ndarray, q: np.ndarray, s) -> np.ndarray:
     out = np.empty((tokens.size, dim), dtype=np.uint16)
     _load().oracle_embed_lookup(_ptr(tokens), tokens.size, _ptr(q), float(np.float32(s)), vocab, dim, _ptr(out))
     return out
+
+
+def quantize_rows4(y: np.ndarray):
+    """Row-wise absmax INT4 RTN (levels -7..7) of FP32 rows: ``(q int8, s, ties)``."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    rows, k = y.shape
+    q = np.empty((rows, k), dtype=np.int8)
+    s = np.empty((rows,), dtype=np.float32)
+    ties = _load().oracle_quantize_rows4(_ptr(y), rows, k, _ptr(q), _ptr(s))
+    return q, s, int(ties)
+
+
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """INT4 codes [rows, k] (int8 holding -8..7) -> packed uint8 [rows, k/2]."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    rows, k = q.shape
+    assert k % 16 == 0
+    out = np.empty((rows, k // 2), dtype=np.uint8)
+    _load().oracle_pack_int4(_ptr(q), rows, k, _ptr(out))
+    return out
+
+
+def unpack_int4(packed: np.ndarray) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    rows, half = packed.shape
+    out = np.empty((rows, 2 * half), dtype=np.int8)
+    _load().oracle_unpack_int4(_ptr(packed), rows, 2 * half, _ptr(out))
+    return out
+
+
+def rotate_quantize4(a_bf16: np.ndarray, group: int = 256):
+    """Rotate, INT4-quantise and pack BF16 weight rows: ``(packed uint8 [rows, k/2], s fp32 [rows])``."""
+    a = _bf16_bits(a_bf16)
+    rows, k = a.shape
+    packed = np.empty((rows, k // 2), dtype=np.uint8)
+    s = np.empty((rows,), dtype=np.float32)
+    bad = _load().oracle_rotate_quantize4(_ptr(a), rows, k, group, _ptr(packed), _ptr(s))
+    if bad < 0:
+        raise OracleError("group must be a power of two dividing k, k % 16 == 0")
+    if bad > 0:
+        raise OracleError("%d rotation groups span more than 37 binades" % bad)
+    return packed, s
+
+
+def linear_w4a8(x_bf16: np.ndarray, packed: np.ndarray, sw: np.ndarray, group: int = 256, bias=None):
+    """W4A8 layer: the activations as in linear_int8 (INT8 rows), the weight
+    codes unpacked from INT4; exact INT32 GEMM; the same dequantisation."""
+    wq = unpack_int4(packed)
+    return linear_int8(x_bf16, wq, sw, group=group, bias=bias)
 
 
 def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:

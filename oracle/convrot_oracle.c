@@ -331,6 +331,93 @@ int64_t oracle_embed_lookup(const int32_t *tokens, int64_t t, const int8_t *q, f
 }
 
 /* ------------------------------------------------------------------ */
+/* INT4 ConvRot weights (W4A8)                                         */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The INT4 variants rotate weights (and activations) with the same grouped
+ * Hadamard before a 4-bit round-to-nearest quantisation [0539edu.com
+ * "minimax-h3-nvfp4-convrot", section 5 "INT4 W4A4 ConvRot": both operands
+ * rotated per group, then 4-bit quantised; --simple = RTN].  On Blackwell the
+ * W4A4 kernels take the INT8-activation path [same page, section 7], so the
+ * product here is INT4 weights x INT8 activations (W4A8).
+ *
+ * Weight rows, after the rotation (same rule as the INT8 rows, levels 7):
+ *   a = max_k |y[r,k]|;  s[r] = a / 7;  q = 0 if a == 0 else clamp(rne(y / s), -7, 7)
+ * Returns the number of exact .5 ties met.
+ */
+int64_t oracle_quantize_rows4(const float *y, int64_t rows, int64_t k, int8_t *q, float *s)
+{
+    int64_t ties = 0;
+    for (int64_t r = 0; r < rows; ++r) {
+        float a = 0.0f;
+        for (int64_t c = 0; c < k; ++c) {
+            float v = fabsf(y[r * k + c]);
+            if (v > a) a = v;
+        }
+        float scale = a / 7.0f;
+        s[r] = scale;
+        for (int64_t c = 0; c < k; ++c) {
+            if (a == 0.0f) { q[r * k + c] = 0; continue; }
+            float t = y[r * k + c] / scale;
+            if (is_exact_half(t)) ++ties;
+            float v = round_half_even(t);
+            if (v > 7.0f) v = 7.0f;
+            if (v < -7.0f) v = -7.0f;
+            q[r * k + c] = (int8_t)v;
+        }
+    }
+    return ties;
+}
+
+/*
+ * Storage of INT4 codes (this library's format; the pages fix none): each
+ * row of k codes (k % 16 == 0) is k/2 bytes; within every 16-code chunk c,
+ * byte 8c + j holds code 16c + j in its low nibble and code 16c + 8 + j in
+ * its high nibble (two's complement nibbles).
+ */
+void oracle_pack_int4(const int8_t *q, int64_t rows, int64_t k, uint8_t *packed)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < k / 16; ++c)
+            for (int j = 0; j < 8; ++j) {
+                uint8_t lo = (uint8_t)q[r * k + 16 * c + j] & 0x0F;
+                uint8_t hi = (uint8_t)q[r * k + 16 * c + 8 + j] & 0x0F;
+                packed[r * (k / 2) + 8 * c + j] = (uint8_t)(lo | (hi << 4));
+            }
+}
+
+void oracle_unpack_int4(const uint8_t *packed, int64_t rows, int64_t k, int8_t *q)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < k / 16; ++c)
+            for (int j = 0; j < 8; ++j) {
+                uint8_t b = packed[r * (k / 2) + 8 * c + j];
+                int lo = b & 0x0F, hi = b >> 4;
+                q[r * k + 16 * c + j] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+                q[r * k + 16 * c + 8 + j] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+            }
+}
+
+/* Rotate, quantise to INT4 and pack the rows of a BF16 weight.  Returns the
+   count of inexact rotation groups, or -1 on bad arguments. */
+int64_t oracle_rotate_quantize4(const uint16_t *a, int64_t rows, int64_t k, int group,
+                                uint8_t *packed, float *s)
+{
+    if (k % 16 != 0) return -1;
+    float *y = (float *)malloc(sizeof(float) * (size_t)(rows * k > 0 ? rows * k : 1));
+    int8_t *q = (int8_t *)malloc((size_t)(rows * k > 0 ? rows * k : 1));
+    if (!y || !q) { free(y); free(q); return -1; }
+    int64_t bad = 0;
+    if (oracle_rotate_rows(a, rows, k, group, y, &bad) != 0) { free(y); free(q); return -1; }
+    oracle_quantize_rows4(y, rows, k, q, s);
+    oracle_pack_int4(q, rows, k, packed);
+    free(y);
+    free(q);
+    return bad;
+}
+
+/* ------------------------------------------------------------------ */
 /* INT8 GEMM with INT32 result                                         */
 /* ------------------------------------------------------------------ */
 

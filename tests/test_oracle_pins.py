@@ -209,6 +209,58 @@ def test_embed_lookup_closed_forms():
 
 
 # ---------------------------------------------------------------------------
+# INT4 weights (W4A8)
+# ---------------------------------------------------------------------------
+def test_int4_quant_closed_forms():
+    p = 4
+    y = np.array([[7.0, 2.5, 3.5, -0.5, 6.5, -1.5, -7.0, 0.25]], np.float32) * 2.0 ** p
+    q, s, ties = oracle.quantize_rows4(y)
+    assert s[0] == np.float32(2.0 ** p) and ties == 5
+    assert list(q[0]) == [7, 2, 4, 0, 6, -2, -7, 0]
+    q0, s0, _ = oracle.quantize_rows4(np.zeros((1, 16), np.float32))
+    assert s0[0] == 0 and not q0.any()
+    rng = np.random.default_rng(12)
+    yr = (rng.standard_normal((4, 512)) * rng.uniform(0.1, 10, (4, 1))).astype(np.float32)
+    qr, sr, _ = oracle.quantize_rows4(yr)
+    assert np.all(np.abs(yr - sr[:, None] * qr) <= sr[:, None] / 2 * (1 + 1e-6))
+    assert np.array_equal(np.abs(qr).max(axis=1), np.full(4, 7))
+    want = np.clip(np.rint(yr / (np.abs(yr).max(axis=1) / np.float32(7))[:, None]), -7, 7)
+    assert np.array_equal(qr, want.astype(np.int8))
+
+
+def test_int4_pack_golden_and_round_trip():
+    lines = [l.split() for l in open(os.path.join(GOLDEN, "int4_pack.txt")) if l.strip() and not l.startswith("#")]
+    codes = np.array([int(v) for v in lines[0]], np.int8).reshape(1, 16)
+    want = np.array([int(v, 16) for v in lines[1]], np.uint8).reshape(1, 8)
+    assert np.array_equal(oracle.pack_int4(codes), want)
+    assert np.array_equal(oracle.unpack_int4(want), codes)
+    rng = np.random.default_rng(13)
+    q = rng.integers(-8, 8, (5, 96)).astype(np.int8)
+    assert np.array_equal(oracle.unpack_int4(oracle.pack_int4(q)), q)
+    # every code at every position of a chunk
+    allq = np.array([[(v + j) % 16 - 8 for j in range(16)] for v in range(16)], np.int8)
+    assert np.array_equal(oracle.unpack_int4(oracle.pack_int4(allq)), allq)
+
+
+def test_w4a8_linear_composes():
+    lin = synth.tiny()[0]
+    x, w = lin.x_np(), lin.w_np()
+    packed, sw = oracle.rotate_quantize4(w)
+    y_rot, _ = oracle.rotate_rows(w)
+    q4, s4, _ = oracle.quantize_rows4(y_rot)
+    assert np.array_equal(oracle.unpack_int4(packed), q4) and np.array_equal(sw, s4)
+    out = oracle.linear_w4a8(x, packed, sw)
+    xq, sx = oracle.rotate_quantize(x)
+    acc = xq.astype(np.int64) @ q4.astype(np.int64).T
+    assert np.array_equal(out["acc"], acc)
+    assert np.array_equal(out["y"], oracle.dequant_bf16(acc.astype(np.int32), sx, sw))
+    # the 4-bit layer still approximates X W^T (coarser than INT8)
+    ref = oracle.bf16_bits_to_f64(x) @ oracle.bf16_bits_to_f64(w).T
+    err = np.max(np.abs(oracle.bf16_bits_to_f64(out["y"]) - ref)) / np.max(np.abs(ref))
+    assert err < 0.3
+
+
+# ---------------------------------------------------------------------------
 # --dynamic-convrot: smaller power-of-two groups
 # ---------------------------------------------------------------------------
 def test_dynamic_group_choice():
