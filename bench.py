@@ -417,6 +417,37 @@ def shared_input_secondary(cr, layer, lins, device, stream, peaks, steps=2000, w
             "frac_of_measured_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"]}
 
 
+def w4a8_secondary(cr, lins, device, stream, peaks, steps=2000, warmup=20):
+    """The decode layer with INT4 ConvRot weights (W4A8): the same seven
+    linears at M = 12, half the weight bytes, one batched call per step."""
+    ws4, keep = [], []
+    for lin in lins:
+        w_bf = lin.w_torch(device)
+        ws4.append(cr.quantize_weight4(w_bf))
+        del w_bf
+    xs = [lin.x_torch(device) for lin in lins]
+    ys = [torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device) for lin in lins]
+    batch = cr.LinearBatchW4(xs, ws4, ys)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        batch(stream)
+    torch.cuda.synchronize()
+    g = capture(lambda: batch(stream), stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        t = time_region(g.replay, steps, stream) / steps
+    m = lins[0].m
+    nbytes = sum(lin.n * lin.k // 2 + 4 * lin.n + 2 * m * lin.k + 2 * m * lin.k + 4 * m + 2 * m * lin.n for lin in lins)
+    del g, batch, ws4
+    torch.cuda.empty_cache()
+    return {"workload": "qwen3vl32b_layer_7linears_decode_m12_w4a8", "int4_weight_bytes": sum(l.n * l.k // 2 for l in lins),
+            "gb_s": nbytes / t / 1e9, "us_per_step": t * 1e6,
+            "frac_of_measured_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"],
+            "weight_stream_gb_s_int8_equivalent": sum(l.n * l.k for l in lins) / t / 1e9}
+
+
 def minimax_secondary(cr, device, stream, peaks, steps=5, warmup=2):
     """MiniMax-H3-shaped qkv projection (K = 5376, N = 16128) at M = 8192 and
     32768 video tokens through the single-linear entry point: INT8 TOPS."""
@@ -643,7 +674,8 @@ def run_ours(args):
     if not args.no_prefill:
         secondary = prefill_secondary(cr, layer, device, stream, peaks)
     cr.convrot_device_status(stream)
-    others = {"shared_inputs": shared_input_secondary(cr, layer, lins, device, stream, peaks)}
+    others = {"shared_inputs": shared_input_secondary(cr, layer, lins, device, stream, peaks),
+              "w4a8": w4a8_secondary(cr, lins, device, stream, peaks)}
     if not args.no_minimax:
         others["minimax_qkv"] = minimax_secondary(cr, device, stream, peaks)
         cr.convrot_device_status(stream)

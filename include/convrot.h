@@ -275,6 +275,64 @@ convrot_status_t convrot_gemm_i8_noalloc(const int8_t *xq, const float *sx, int6
                                          void *stream);
 
 /*
+ * ---------------------------------------------------------------- INT4 ConvRot weights (W4A8)
+ * The INT4 variants rotate weights and activations with the same grouped
+ * Hadamard and quantise to 4 bits by round-to-nearest [0539edu.com
+ * "minimax-h3-nvfp4-convrot", section 5 "INT4 W4A4 ConvRot", --simple = RTN];
+ * on Blackwell those kernels take the INT8-activation path [same page,
+ * section 7].  Here: weights INT4 (levels -7..7, one FP32 scale per row,
+ * s = max|Wr[n,:]| / 7), activations INT8 exactly as in the INT8 layer, the
+ * product on the INT8 tensor cores after unpacking the weight tile in shared
+ * memory, so the weight stream (the decode bound) is half as many bytes.
+ *
+ * Packed INT4 weight handle (caller-owned device memory):
+ *   q     : uint8 [n, k/2] -- within each 16-code chunk c of a row, byte
+ *           8c + j holds code 16c + j in its low nibble and code 16c + 8 + j
+ *           in its high nibble (two's complement)
+ *   scale : fp32 [n];  group as in convrot_weight_t;  k % 32 == 0
+ */
+typedef struct {
+    uint8_t *q;
+    float *scale;
+    int64_t n;
+    int64_t k;
+    int32_t group;
+} convrot_weight4_t;
+
+/* Fill an INT4 handle; the checks of convrot_weight_init plus k % 32 == 0. */
+convrot_status_t convrot_weight4_init(convrot_weight4_t *w, uint8_t *q, float *scale,
+                                      int64_t n, int64_t k, int32_t group);
+
+/* Offline: rotate every row of the BF16 weight w [n, k] per group, quantise
+   it to INT4 (row scale max/7, RTN, clamp to -7..7) and pack it into out->q. */
+convrot_status_t convrot_quantize_weight4(const void *w_bf16, const convrot_weight4_t *out, void *stream);
+
+/* One W4A8 linear of a call: y [m, w->n] = the ConvRot layer of x [m, w->k]. */
+typedef struct {
+    const void *x_bf16;
+    const convrot_weight4_t *w;
+    void *y_bf16;
+    const void *bias_bf16;      /* BF16 [w->n] or NULL, as in convrot_linear_job_t */
+} convrot_linear4_job_t;
+
+/*
+ * count (<= 8) W4A8 linears with the same token count m in two launches:
+ * the activation prologue (INT8 codes, shared by jobs with the same input),
+ * then one weight-streaming GEMM whose K blocks of all weights are dealt out
+ * to every SM, the packed tiles unpacked to INT8 by four dedicated warps per
+ * CTA.  1 <= m <= 256 (larger m: CONVROT_ERR_UNSUPPORTED_SHAPE; there the
+ * layer is tensor-bound and the INT4 format saves no time).  Results:
+ * y = bf16(((float)acc * sx[m]) * sw[n] [+ bias[n]]) with acc the exact INT32
+ * product of the INT8 activation codes and the INT4 weight codes.
+ * Workspace: convrot_linear_w4a8_workspace_bytes, zero-filled before first
+ * use, left zero-filled.
+ */
+convrot_status_t convrot_linear_w4a8(int64_t m, int count, const convrot_linear4_job_t *jobs,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+size_t convrot_linear_w4a8_workspace_bytes(int64_t m, int count, const convrot_linear4_job_t *jobs);
+
+/*
  * Tensor-wise "simple" INT8 of a BF16 tensor of `count` elements (the
  * word-embedding table [vocab, dim]): no rotation, ONE scale for the whole
  * tensor, round-to-nearest-even --

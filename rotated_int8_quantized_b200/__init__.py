@@ -50,6 +50,18 @@ class convrot_linear_job_t(ctypes.Structure):
                 ("y_bf16", ctypes.c_void_p), ("bias_bf16", ctypes.c_void_p)]
 
 
+class convrot_weight4_t(ctypes.Structure):
+    """Mirror of the C struct: packed INT4 weight (q uint8 [n, k/2], scale fp32 [n])."""
+    _fields_ = [("q", ctypes.c_void_p), ("scale", ctypes.c_void_p),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("group", ctypes.c_int32)]
+
+
+class convrot_linear4_job_t(ctypes.Structure):
+    """Mirror of the C struct: one W4A8 linear of a call."""
+    _fields_ = [("x_bf16", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight4_t)),
+                ("y_bf16", ctypes.c_void_p), ("bias_bf16", ctypes.c_void_p)]
+
+
 class convrot_gemm_job_t(ctypes.Structure):
     """Mirror of the C struct: one product of a batched GEMM call."""
     _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight_t)),
@@ -64,6 +76,10 @@ SIGNATURES = {
     "convrot_version": ([], ctypes.c_int),
     "convrot_dynamic_group": ([_I64, _I32], _I32),
     "convrot_quantize_tensor": ([_P, _I64, _P, _P, _P], ctypes.c_int),
+    "convrot_weight4_init": ([ctypes.POINTER(convrot_weight4_t), _P, _P, _I64, _I64, _I32], ctypes.c_int),
+    "convrot_quantize_weight4": ([_P, ctypes.POINTER(convrot_weight4_t), _P], ctypes.c_int),
+    "convrot_linear_w4a8": ([_I64, ctypes.c_int, _P, _P, _SZ, _P], ctypes.c_int),
+    "convrot_linear_w4a8_workspace_bytes": ([_I64, ctypes.c_int, _P], _SZ),
     "convrot_embed_lookup": ([_P, _I64, _P, _P, _I64, _I64, _P, _P], ctypes.c_int),
     "convrot_last_error_string": ([], ctypes.c_char_p),
     "convrot_weight_init": ([_WP, _P, _P, _I64, _I64, _I32], ctypes.c_int),
@@ -295,6 +311,65 @@ def convrot_embed_lookup(tokens: torch.Tensor, q: torch.Tensor, scale: torch.Ten
     assert tokens.dtype == torch.int32 and q.dim() == 2 and out.shape == (tokens.numel(), q.shape[1])
     _check(load_library().convrot_embed_lookup(_ptr(tokens), tokens.numel(), _ptr(q), _ptr(scale), q.shape[0],
                                                q.shape[1], _ptr(out), _stream(stream)), "convrot_embed_lookup")
+
+
+# ---------------------------------------------------------------- INT4 weights (W4A8)
+@dataclass
+class QuantizedWeight4:
+    """Packed INT4 weight q [n, k/2] (uint8) with FP32 row scales [n] and the C handle."""
+    q: torch.Tensor
+    scale: torch.Tensor
+    handle: convrot_weight4_t
+
+    @property
+    def n(self) -> int:
+        return self.handle.n
+
+    @property
+    def k(self) -> int:
+        return self.handle.k
+
+    @property
+    def group(self) -> int:
+        return self.handle.group
+
+
+def quantize_weight4(w_bf16: torch.Tensor, stream=None, group: int = GROUP, dynamic: bool = False) -> QuantizedWeight4:
+    """Offline INT4 ConvRot conversion of a BF16 weight [n, k]."""
+    n, k = w_bf16.shape
+    if dynamic:
+        group = convrot_dynamic_group(k, group)
+    q = torch.empty((n, k // 2), dtype=torch.uint8, device=w_bf16.device)
+    scale = torch.empty((n,), dtype=torch.float32, device=w_bf16.device)
+    h = convrot_weight4_t()
+    lib = load_library()
+    _check(lib.convrot_weight4_init(ctypes.byref(h), _ptr(q), _ptr(scale), n, k, group), "convrot_weight4_init")
+    _check(lib.convrot_quantize_weight4(_ptr(w_bf16), ctypes.byref(h), _stream(stream)), "convrot_quantize_weight4")
+    return QuantizedWeight4(q, scale, h)
+
+
+class LinearBatchW4:
+    """A prepared W4A8 call over up to 8 linears with the same token count."""
+
+    def __init__(self, xs, weights, ys, ws: Optional[torch.Tensor] = None, biases=None):
+        self.keep = (list(xs), list(weights), list(ys), list(biases) if biases else None)
+        self.m = xs[0].shape[0]
+        n = len(xs)
+        biases = biases or [None] * n
+        self.jobs = (convrot_linear4_job_t * n)()
+        for i in range(n):
+            self.jobs[i].x_bf16 = _ptr(xs[i])
+            self.jobs[i].w = ctypes.pointer(weights[i].handle)
+            self.jobs[i].y_bf16 = _ptr(ys[i])
+            self.jobs[i].bias_bf16 = _ptr(biases[i])
+        need = int(load_library().convrot_linear_w4a8_workspace_bytes(self.m, n, self.jobs))
+        if need == 0:
+            raise ConvrotError(3, "convrot_linear_w4a8_workspace_bytes")
+        self.ws = ws if ws is not None else torch.zeros(need, dtype=torch.uint8, device=xs[0].device)
+
+    def __call__(self, stream=None) -> None:
+        _check(load_library().convrot_linear_w4a8(self.m, len(self.jobs), self.jobs, _ptr(self.ws),
+                                                  self.ws.numel(), _stream(stream)), "convrot_linear_w4a8")
 
 
 def convrot_device_status(stream=None) -> None:

@@ -19,6 +19,7 @@ constexpr int64_t kMaxK = 133120;
 constexpr int64_t kMaxRows = 0x7FFFFFFF;
 constexpr int kDefaultSms = 148;
 constexpr int kMaxBatch = convrot::kMaxJobs;
+constexpr int64_t kMaxW4Rows = 256;     // INT4 weights: the swapped (weight-streaming) orientation only
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -79,6 +80,16 @@ convrot_status_t check_weight(const convrot_weight_t *w) {
     if (!w || !w->q || !w->scale) return CONVROT_ERR_INVALID_ARG;
     convrot_status_t s = check_shape(w->n, w->k, w->group);
     if (s != CONVROT_OK) return s;
+    if (!aligned16(w->q) || !aligned16(w->scale)) return CONVROT_ERR_ALIGNMENT;
+    return CONVROT_OK;
+}
+
+// INT4 rows are k/2 bytes: a multiple of 16 (TMA row stride) needs k % 32 == 0.
+convrot_status_t check_weight4(const convrot_weight4_t *w) {
+    if (!w || !w->q || !w->scale) return CONVROT_ERR_INVALID_ARG;
+    convrot_status_t s = check_shape(w->n, w->k, w->group);
+    if (s != CONVROT_OK) return s;
+    if (w->k % 32 != 0) return CONVROT_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(w->q) || !aligned16(w->scale)) return CONVROT_ERR_ALIGNMENT;
     return CONVROT_OK;
 }
@@ -200,32 +211,68 @@ bool ranges_overlap(const void *a, size_t an, const void *b, size_t bn) {
     return a0 < b0 + bn && b0 < a0 + an;
 }
 
-// Checks common to the single and batched layer entry points.
-convrot_status_t check_jobs(int64_t m, int count, const convrot_linear_job_t *jobs) {
-    if (!jobs || count < 1 || count > kMaxBatch) return CONVROT_ERR_INVALID_ARG;
+// One linear as the layer entry points see it (INT8 or packed INT4 weight).
+struct LinJob {
+    const void *x;
+    const int8_t *wq;       // int8 [n, k], or INT4 codes [n, k/2] bytes
+    const float *sw;
+    int64_t n, k;
+    int32_t group;
+    void *y;
+    const void *bias;
+};
+
+LinJob lin_job(const convrot_linear_job_t &J) {
+    return {J.x_bf16, J.w->q, J.w->scale, J.w->n, J.w->k, J.w->group, J.y_bf16, J.bias_bf16};
+}
+
+// Checks common to the layer entry points, after the weights' own checks.
+convrot_status_t check_lin_jobs(int64_t m, int count, const LinJob *jobs) {
     for (int j = 0; j < count; ++j) {
-        const convrot_linear_job_t &J = jobs[j];
-        if (!J.x_bf16 || !J.y_bf16) return CONVROT_ERR_INVALID_ARG;
-        convrot_status_t s = check_weight(J.w);
+        const LinJob &J = jobs[j];
+        if (!J.x || !J.y) return CONVROT_ERR_INVALID_ARG;
+        convrot_status_t s = check_shape(m, J.k, J.group);
         if (s != CONVROT_OK) return s;
-        if ((s = check_shape(m, J.w->k, J.w->group)) != CONVROT_OK) return s;
-        if (!aligned16(J.x_bf16) || !aligned16(J.y_bf16) || (J.bias_bf16 && !aligned16(J.bias_bf16)))
-            return CONVROT_ERR_ALIGNMENT;
+        if (!aligned16(J.x) || !aligned16(J.y) || (J.bias && !aligned16(J.bias))) return CONVROT_ERR_ALIGNMENT;
     }
     // no output may overlap any input or another output: the jobs run as
     // one launch pair, so an output cannot feed a later job
     for (int j = 0; j < count; ++j) {
-        const size_t ybytes = (size_t)m * (size_t)jobs[j].w->n * 2;
+        const size_t ybytes = (size_t)m * (size_t)jobs[j].n * 2;
         for (int i = 0; i < count; ++i) {
-            if (ranges_overlap(jobs[j].y_bf16, ybytes, jobs[i].x_bf16, (size_t)m * (size_t)jobs[i].w->k * 2))
+            if (ranges_overlap(jobs[j].y, ybytes, jobs[i].x, (size_t)m * (size_t)jobs[i].k * 2))
                 return CONVROT_ERR_INVALID_ARG;
-            if (jobs[i].bias_bf16 && ranges_overlap(jobs[j].y_bf16, ybytes, jobs[i].bias_bf16, (size_t)jobs[i].w->n * 2))
+            if (jobs[i].bias && ranges_overlap(jobs[j].y, ybytes, jobs[i].bias, (size_t)jobs[i].n * 2))
                 return CONVROT_ERR_INVALID_ARG;
-            if (i != j && ranges_overlap(jobs[j].y_bf16, ybytes, jobs[i].y_bf16, (size_t)m * (size_t)jobs[i].w->n * 2))
+            if (i != j && ranges_overlap(jobs[j].y, ybytes, jobs[i].y, (size_t)m * (size_t)jobs[i].n * 2))
                 return CONVROT_ERR_INVALID_ARG;
         }
     }
     return CONVROT_OK;
+}
+
+// INT8 jobs -> LinJob array (and the weights' checks).
+convrot_status_t collect_jobs(int64_t m, int count, const convrot_linear_job_t *jobs, LinJob *out) {
+    if (!jobs || count < 1 || count > kMaxBatch) return CONVROT_ERR_INVALID_ARG;
+    for (int j = 0; j < count; ++j) {
+        convrot_status_t s = check_weight(jobs[j].w);
+        if (s != CONVROT_OK) return s;
+        out[j] = lin_job(jobs[j]);
+    }
+    return check_lin_jobs(m, count, out);
+}
+
+convrot_status_t collect_jobs4(int64_t m, int count, const convrot_linear4_job_t *jobs, LinJob *out) {
+    if (!jobs || count < 1 || count > kMaxBatch) return CONVROT_ERR_INVALID_ARG;
+    if (m < 1 || m > kMaxW4Rows) return m < 1 ? CONVROT_ERR_INVALID_ARG : CONVROT_ERR_UNSUPPORTED_SHAPE;
+    for (int j = 0; j < count; ++j) {
+        const convrot_linear4_job_t &J = jobs[j];
+        convrot_status_t s = check_weight4(J.w);
+        if (s != CONVROT_OK) return s;
+        out[j] = {J.x_bf16, reinterpret_cast<const int8_t *>(J.w->q), J.w->scale, J.w->n, J.w->k, J.w->group,
+                  J.y_bf16, J.bias_bf16};
+    }
+    return check_lin_jobs(m, count, out);
 }
 
 // Workspace layout of the layer entry points: [GEMM scratch][xq_0][sx_0][xq_1][sx_1]...
@@ -236,31 +283,31 @@ struct LinearLayout {
     size_t total;
 };
 
-void linear_layout(int64_t m, int count, const convrot_linear_job_t *jobs, int sms, LinearLayout *L) {
-    L->batched_gemm = (m <= convrot::kMaxSwapM);
+void linear_layout(int64_t m, int count, const LinJob *jobs, bool w4, int sms, LinearLayout *L) {
+    L->batched_gemm = w4 || (m <= convrot::kMaxSwapM);
     size_t g = 0;
     if (L->batched_gemm) {
         int64_t n[kMaxBatch], k[kMaxBatch];
         for (int j = 0; j < count; ++j) {
-            n[j] = jobs[j].w->n;
-            k[j] = jobs[j].w->k;
+            n[j] = jobs[j].n;
+            k[j] = jobs[j].k;
         }
-        convrot::plan_gemm_batch(m, count, n, k, sms, &L->batch);
+        convrot::plan_gemm_batch(m, count, n, k, sms, &L->batch, w4);
         g = L->batch.ws_bytes;
     } else {
         for (int j = 0; j < count; ++j) {
             convrot::GemmPlan p;
-            convrot::plan_gemm(m, jobs[j].w->n, jobs[j].w->k, sms, &p);
+            convrot::plan_gemm(m, jobs[j].n, jobs[j].k, sms, &p);
             g = p.ws_bytes > g ? p.ws_bytes : g;
         }
     }
     L->gemm_bytes = round256(g);
     size_t t = L->gemm_bytes;
-    for (int j = 0; j < count; ++j) t += round256((size_t)m * (size_t)jobs[j].w->k) + round256((size_t)m * 4);
+    for (int j = 0; j < count; ++j) t += round256((size_t)m * (size_t)jobs[j].k) + round256((size_t)m * 4);
     L->total = t;
 }
 
-convrot_status_t run_linear(int64_t m, int count, const convrot_linear_job_t *jobs, void *ws, size_t ws_bytes,
+convrot_status_t run_linear(int64_t m, int count, const LinJob *jobs, bool w4, void *ws, size_t ws_bytes,
                             cudaStream_t st) {
     if (!ws) return CONVROT_ERR_WORKSPACE;
     if (!aligned16(ws)) return CONVROT_ERR_ALIGNMENT;
@@ -268,7 +315,7 @@ convrot_status_t run_linear(int64_t m, int count, const convrot_linear_job_t *jo
     convrot_status_t s = current_device(&dev);
     if (s != CONVROT_OK) return s;
     LinearLayout L;
-    linear_layout(m, count, jobs, dev.num_sms, &L);
+    linear_layout(m, count, jobs, w4, dev.num_sms, &L);
     if (ws_bytes < L.total) return CONVROT_ERR_WORKSPACE;
     uint8_t *base = static_cast<uint8_t *>(ws);
     convrot::RQProblem rq[kMaxBatch];
@@ -277,31 +324,28 @@ convrot_status_t run_linear(int64_t m, int count, const convrot_linear_job_t *jo
     int nrq = 0;
     for (int j = 0; j < count; ++j) {
         int8_t *xq = reinterpret_cast<int8_t *>(base + off);
-        off += round256((size_t)m * (size_t)jobs[j].w->k);
+        off += round256((size_t)m * (size_t)jobs[j].k);
         float *sx = reinterpret_cast<float *>(base + off);
         off += round256((size_t)m * 4);
         // a job whose input an earlier job already rotates reuses its codes
         int same = -1;
         for (int i = 0; i < j && same < 0; ++i)
-            if (jobs[i].x_bf16 == jobs[j].x_bf16 && jobs[i].w->k == jobs[j].w->k &&
-                jobs[i].w->group == jobs[j].w->group)
-                same = i;
+            if (jobs[i].x == jobs[j].x && jobs[i].k == jobs[j].k && jobs[i].group == jobs[j].group) same = i;
         if (same >= 0) {
             xq = const_cast<int8_t *>(gp[same].xq);
             sx = const_cast<float *>(gp[same].sx);
         } else {
-            rq[nrq++] = {jobs[j].x_bf16, jobs[j].w->k, jobs[j].w->group, xq, sx};
+            rq[nrq++] = {jobs[j].x, jobs[j].k, jobs[j].group, xq, sx, 0};
         }
-        gp[j] = {m, jobs[j].w->n, jobs[j].w->k, xq, sx, jobs[j].w->q, jobs[j].w->scale,
-                 static_cast<__nv_bfloat16 *>(jobs[j].y_bf16), nullptr,
-                 static_cast<const __nv_bfloat16 *>(jobs[j].bias_bf16)};
+        gp[j] = {m, jobs[j].n, jobs[j].k, xq, sx, jobs[j].wq, jobs[j].sw, static_cast<__nv_bfloat16 *>(jobs[j].y),
+                 nullptr, static_cast<const __nv_bfloat16 *>(jobs[j].bias)};
     }
     cudaError_t e = convrot::launch_rotate_quant(nrq, m, rq, st, true);
     if (e != cudaSuccess) return from_cuda(e);
     if (L.batched_gemm) return from_cuda(convrot::launch_gemm_i8(L.batch, gp, base, st, true, true));
     for (int j = 0; j < count; ++j) {
         convrot::GemmPlan p;
-        convrot::plan_gemm(m, jobs[j].w->n, jobs[j].w->k, dev.num_sms, &p);
+        convrot::plan_gemm(m, jobs[j].n, jobs[j].k, dev.num_sms, &p);
         // the first product may prefetch weights under the prologue; later
         // ones follow another GEMM that could still be reading the scratch
         e = convrot::launch_gemm_i8(p, &gp[j], base, st, true, j == 0);
@@ -367,33 +411,74 @@ convrot_status_t convrot_gemm_i8_batch(int64_t m, int count, const convrot_gemm_
 
 size_t convrot_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     if (m < 1 || n < 1 || k < kMinGroup || k % kMinGroup != 0 || k > kMaxK) return 0;
-    convrot_weight_t w = {nullptr, nullptr, n, k, (int32_t)kGroup};
-    convrot_linear_job_t job = {nullptr, &w, nullptr, nullptr};
+    LinJob job = {nullptr, nullptr, nullptr, n, k, (int32_t)kGroup, nullptr, nullptr};
     LinearLayout L;
-    linear_layout(m, 1, &job, sms_for_sizing(), &L);
+    linear_layout(m, 1, &job, false, sms_for_sizing(), &L);
     return L.total;
 }
 
 convrot_status_t convrot_linear_int8(const void *x_bf16, int64_t m, const convrot_weight_t *w, void *y_bf16,
                                      void *ws, size_t ws_bytes, void *stream) {
     convrot_linear_job_t job = {x_bf16, w, y_bf16, nullptr};
-    convrot_status_t s = check_jobs(m, 1, &job);
+    LinJob lj[1];
+    convrot_status_t s = collect_jobs(m, 1, &job, lj);
     if (s != CONVROT_OK) return s;
-    return run_linear(m, 1, &job, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    return run_linear(m, 1, lj, false, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 size_t convrot_linear_batch_workspace_bytes(int64_t m, int count, const convrot_linear_job_t *jobs) {
-    if (check_jobs(m, count, jobs) != CONVROT_OK) return 0;
+    LinJob lj[kMaxBatch];
+    if (collect_jobs(m, count, jobs, lj) != CONVROT_OK) return 0;
     LinearLayout L;
-    linear_layout(m, count, jobs, sms_for_sizing(), &L);
+    linear_layout(m, count, lj, false, sms_for_sizing(), &L);
     return L.total;
 }
 
 convrot_status_t convrot_linear_int8_batch(int64_t m, int count, const convrot_linear_job_t *jobs, void *ws,
                                            size_t ws_bytes, void *stream) {
-    convrot_status_t s = check_jobs(m, count, jobs);
+    LinJob lj[kMaxBatch];
+    convrot_status_t s = collect_jobs(m, count, jobs, lj);
     if (s != CONVROT_OK) return s;
-    return run_linear(m, count, jobs, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    return run_linear(m, count, lj, false, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------- INT4 weights (W4A8)
+convrot_status_t convrot_weight4_init(convrot_weight4_t *w, uint8_t *q, float *scale, int64_t n, int64_t k,
+                                      int32_t group) {
+    if (!w) return CONVROT_ERR_INVALID_ARG;
+    convrot_weight4_t t = {q, scale, n, k, group};
+    convrot_status_t s = check_weight4(&t);
+    if (s != CONVROT_OK) return s;
+    *w = t;
+    return CONVROT_OK;
+}
+
+convrot_status_t convrot_quantize_weight4(const void *w_bf16, const convrot_weight4_t *out, void *stream) {
+    if (!w_bf16) return CONVROT_ERR_INVALID_ARG;
+    convrot_status_t s = check_weight4(out);
+    if (s != CONVROT_OK) return s;
+    if (!aligned16(w_bf16)) return CONVROT_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    if ((s = current_device(&dev)) != CONVROT_OK) return s;
+    convrot::RQProblem prob = {w_bf16, out->k, out->group, reinterpret_cast<int8_t *>(out->q), out->scale, 1};
+    return from_cuda(convrot::launch_rotate_quant(1, out->n, &prob, static_cast<cudaStream_t>(stream), false));
+}
+
+
+size_t convrot_linear_w4a8_workspace_bytes(int64_t m, int count, const convrot_linear4_job_t *jobs) {
+    LinJob lj[kMaxBatch];
+    if (collect_jobs4(m, count, jobs, lj) != CONVROT_OK) return 0;
+    LinearLayout L;
+    linear_layout(m, count, lj, true, sms_for_sizing(), &L);
+    return L.total;
+}
+
+convrot_status_t convrot_linear_w4a8(int64_t m, int count, const convrot_linear4_job_t *jobs, void *ws,
+                                     size_t ws_bytes, void *stream) {
+    LinJob lj[kMaxBatch];
+    convrot_status_t s = collect_jobs4(m, count, jobs, lj);
+    if (s != CONVROT_OK) return s;
+    return run_linear(m, count, lj, true, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 convrot_status_t convrot_quantize_tensor(const void *w_bf16, int64_t count, int8_t *q, float *scale,

@@ -42,10 +42,14 @@
 namespace convrot {
 
 constexpr int kThreads = 192;          // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
+constexpr int kW4Warps = 8;            // INT4 weights: warps 6.. unpack the packed weight tiles
+constexpr int kMaxRing = kMaxStages;
+constexpr int kThreadsW4 = kThreads + 32 * kW4Warps;
 constexpr int kTileA = 128;            // UMMA M
 constexpr int kBlockK = 128;           // bytes of K per stage (one 128-byte swizzle row)
 constexpr int kUmmaK = 32;             // K per tcgen05.mma kind::i8
 constexpr int kATileBytes = kTileA * kBlockK;
+constexpr uint32_t kPackedTileBytes = kTileA * kBlockK / 2;   // 128 rows x 64 bytes of INT4 codes
 constexpr int kL2PrefetchBlocks = 16;  // weight K blocks pulled into L2 ahead of the grid-dependency wait
 constexpr int kMaxSplitWays = 6;       // K ranges per split tail tile (large M)
 constexpr long long kGroupABytes = 48ll << 20;   // INT8 A operand above this is taken in tile groups
@@ -295,7 +299,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, int32_t (&v0)[16], int
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Sign-extend the low nibble of each byte of v (bytes 0..15) to int8: the
+// bit 3 of a byte times 30 is 0xF0, which lands in its empty high nibble.
+__device__ __forceinline__ uint32_t sext_nibbles(uint32_t v) {
+    return (v & 0x08080808u) * 30u + v;
+}
+
+// W4: the weight (A operand, swapped orientation) arrives as packed INT4
+// codes; warps 6-9 unpack each 128 x 64-byte tile into the 128 x 128-byte
+// 128B-swizzled INT8 tile the MMA reads.
+template <bool W4>
+__global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
     gemm_i8_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled operand tiles
@@ -307,15 +321,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t b_bytes = (uint32_t)a.bn * kBlockK;
     const uint32_t a_off = 0;
     const uint32_t b_off = (uint32_t)S * kATileBytes;
-    const uint32_t bar_off = b_off + (uint32_t)S * b_bytes;
-    // barriers: full[S], empty[S], tfull[2], tempty[2], drain, red[2]
+    // W4: a staging slot per stage where the packed weight tile lands
+    const uint32_t p_off = b_off + (uint32_t)S * b_bytes;
+    const uint32_t bar_off = p_off + (W4 ? (uint32_t)S * kPackedTileBytes : 0u);
+    // barriers: full[S], empty[S], tfull[2], tempty[2], drain, red[2], W4: pfull[S]
     const uint32_t full_bar = base + bar_off;
     const uint32_t empty_bar = full_bar + 8u * S;
     const uint32_t tfull_bar = empty_bar + 8u * S;
     const uint32_t tempty_bar = tfull_bar + 16u;
     const uint32_t drain_bar = tempty_bar + 16u;
     const uint32_t red_bar = drain_bar + 8u;
-    uint8_t *misc = smem + ((bar_off + 8u * (2 * S + kExtraBars) + 15u) & ~15u);
+    const uint32_t pfull_bar = red_bar + 16u;
+    // W4: TMA copies land on pfull; the unpacking warps then arrive on full
+    const uint32_t land_bar = W4 ? pfull_bar : full_bar;
+    uint8_t *misc = smem + ((bar_off + 8u * (2 * S + kExtraBars + (W4 ? S : 0)) + 15u) & ~15u);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(misc);
     volatile int *ticket = reinterpret_cast<volatile int *>(misc + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 8);
@@ -332,8 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar + 8u * s, 1);
+            mbar_init(full_bar + 8u * s, W4 ? kW4Warps : 1);
             mbar_init(empty_bar + 8u * s, 1);
+            if (W4) mbar_init(pfull_bar + 8u * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar + 8u * b, 1);
@@ -364,14 +384,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint32_t tx = (uint32_t)kATileBytes + b_bytes;
+            // W4: the packed weight tile lands in the stage's staging slot
+            // (unpacked into its operand slot by the unpacking warps)
+            const uint32_t tx = (W4 ? kPackedTileBytes : (uint32_t)kATileBytes) + b_bytes;
+            const int RS = S;
+            const uint32_t free_bar = empty_bar;
             int stage = 0;
             uint32_t phase = 0;
             bool waited = !a.w_prefetch;
             if (waited) pdl_wait();
             // activation loads held back until the grid dependency resolves
             int pend_n = 0;
-            int pend_stage[kMaxStages], pend_x[kMaxStages], pend_y[kMaxStages], pend_job[kMaxStages];
+            int pend_stage[kMaxRing], pend_x[kMaxRing], pend_y[kMaxRing], pend_job[kMaxRing];
             uint32_t issued_mask = 0, issued_par = 0;
             SegmentIter it;
             it.init(a);
@@ -386,25 +410,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int rowW = a.swap ? ta * kTileA : tb * a.bn;
                 const int rowX = a.swap ? tb * a.bn : ta * kTileA;
                 for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
-                    if (!mbar_wait_bounded(empty_bar + 8u * stage, phase ^ 1u, abort_flag)) {
+                    if (!mbar_wait_bounded(free_bar + 8u * stage, phase ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = full_bar + 8u * stage;
-                    mbar_arrive_expect_tx(fb, tx);
+                    const uint32_t lb = land_bar + 8u * stage;
+                    mbar_arrive_expect_tx(lb, tx);
                     const uint32_t sa = base + a_off + (uint32_t)stage * kATileBytes;
                     const uint32_t sb = base + b_off + (uint32_t)stage * b_bytes;
                     const int kx = kb * kBlockK;
-                    const uint32_t sW = a.swap ? sa : sb, sX = a.swap ? sb : sa;
-                    tma_load_2d(sW, tmW, fb, kx, rowW);
+                    const uint32_t sp = base + p_off + (uint32_t)stage * kPackedTileBytes;   // W4 staging
+                    const uint32_t sW = W4 ? sp : (a.swap ? sa : sb);
+                    const uint32_t sX = a.swap ? sb : sa;
+                    tma_load_2d(sW, tmW, lb, W4 ? kx / 2 : kx, rowW);
                     if (waited) {
-                        tma_load_2d(sX, tmX, fb, kx, rowX);
+                        tma_load_2d(sX, tmX, lb, kx, rowX);
                     } else {
                         pend_stage[pend_n] = stage;
                         pend_x[pend_n] = kx;
                         pend_y[pend_n] = rowX;
                         pend_job[pend_n] = sg.job;
-                        if (++pend_n == S) {
+                        if (++pend_n == RS) {
                             // while the prologue is still running, pull the
                             // next weight tiles of this CTA into L2 as well
                             SegmentIter it2 = it;
@@ -420,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 int ta2, tb2;
                                 tile_coords(J2, s2.tile, ta2, tb2);
                                 const CUtensorMap *tw2 = a.swap ? &maps.a[s2.job] : &maps.b[s2.job];
-                                tma_prefetch_l2_2d(tw2, kb2 * kBlockK, a.swap ? ta2 * kTileA : tb2 * a.bn);
+                                tma_prefetch_l2_2d(tw2, kb2 * (W4 ? kBlockK / 2 : kBlockK),
+                                                   a.swap ? ta2 * kTileA : tb2 * a.bn);
                                 ++kb2;
                                 ++pf;
                             }
@@ -431,14 +458,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const uint32_t sxa = a.swap ? base + b_off + (uint32_t)st * b_bytes
                                                             : base + a_off + (uint32_t)st * kATileBytes;
                                 const CUtensorMap *tp = a.swap ? &maps.b[pend_job[p]] : &maps.a[pend_job[p]];
-                                tma_load_2d(sxa, tp, full_bar + 8u * st, pend_x[p], pend_y[p]);
+                                tma_load_2d(sxa, tp, land_bar + 8u * st, pend_x[p], pend_y[p]);
                             }
                             pend_n = 0;
                         }
                     }
                     issued_mask |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-                    if (++stage == S) {
+                    if (++stage == RS) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -451,15 +478,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sxa = a.swap ? base + b_off + (uint32_t)st * b_bytes
                                                 : base + a_off + (uint32_t)st * kATileBytes;
                     const CUtensorMap *tp = a.swap ? &maps.b[pend_job[p]] : &maps.a[pend_job[p]];
-                    tma_load_2d(sxa, tp, full_bar + 8u * st, pend_x[p], pend_y[p]);
+                    tma_load_2d(sxa, tp, land_bar + 8u * st, pend_x[p], pend_y[p]);
                 }
             }
             if (!ok) {
                 // let every copy this thread started land before the CTA exits
                 volatile int no_abort = 0;
-                for (int s = 0; s < S; ++s)
+                for (int s = 0; s < RS; ++s)
                     if (issued_mask & (1u << s))
-                        mbar_wait_bounded(full_bar + 8u * s, (issued_par >> s) & 1u, &no_abort);
+                        mbar_wait_bounded(land_bar + 8u * s, (issued_par >> s) & 1u, &no_abort);
             }
         }
     } else if (warp == 1) {
@@ -510,6 +537,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                 volatile int no_abort = 0;
                 umma_commit(drain_bar);
                 mbar_wait_bounded(drain_bar, 0, &no_abort);
+            }
+        }
+    } else if (W4 && warp >= 6) {
+        // ------------------------------------------------ INT4 unpacking (kW4Warps warps)
+        // All unpacking warps walk every K block in ring order (so no wait
+        // runs ahead of a phase) and each unpacks its share of the stage:
+        // 128 rows x 8 chunks of 16 codes, 8 B of nibbles -> 16 B of INT8 at
+        // the chunk's swizzled position (chunk c of row r sits at
+        // 16 * (c ^ (r & 7)) in the row's 128 bytes); then full[stage].
+        const int ct = (int)threadIdx.x - kThreads;
+        constexpr int kCT = 32 * kW4Warps;
+        int stage = 0;
+        uint32_t phase = 0;
+        SegmentIter it;
+        it.init(a);
+        Segment sg;
+        bool ok = true;
+        while (ok && it.next(a, sg)) {
+            for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                if (!mbar_wait_bounded(pfull_bar + 8u * stage, phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *src = smem + p_off + (uint32_t)stage * kPackedTileBytes;
+                uint8_t *dst = smem + a_off + (uint32_t)stage * kATileBytes;
+#pragma unroll
+                for (int i = 0; i < 1024 / kCT; ++i) {
+                    const int item = ct + kCT * i;
+                    const int r = item >> 3, c = item & 7;
+                    const uint2 w = *reinterpret_cast<const uint2 *>(src + r * 64 + c * 8);
+                    uint4 o;
+                    o.x = sext_nibbles(w.x & 0x0F0F0F0Fu);            // codes 0-3 of the chunk
+                    o.y = sext_nibbles(w.y & 0x0F0F0F0Fu);            // codes 4-7
+                    o.z = sext_nibbles((w.x >> 4) & 0x0F0F0F0Fu);     // codes 8-11
+                    o.w = sext_nibbles((w.y >> 4) & 0x0F0F0F0Fu);     // codes 12-15
+                    *reinterpret_cast<uint4 *>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = o;
+                }
+                fence_proxy_async_shared();      // the tensor core reads these stores
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full_bar + 8u * stage);
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
         }
     } else {
@@ -777,7 +848,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------- host side
 
 static void plan_common(GemmPlan *p) {
-    const int stage_bytes = kATileBytes + p->bn * kBlockK;
+    // W4: every stage also holds the packed weight tile it is unpacked from
+    const int stage_bytes = kATileBytes + p->bn * kBlockK + (p->w4 ? (int)kPackedTileBytes : 0);
     int stages = (200 * 1024) / stage_bytes;
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) stages = 2;
@@ -786,8 +858,8 @@ static void plan_common(GemmPlan *p) {
     int cols = 32;
     while (cols < 2 * p->bn) cols <<= 1;
     p->tmem_cols = cols;
-    p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + kExtraBars) + 16 + 16 + 2 * 2 * kBiasStage * 4 +
-                    2 * 16 * kTileA * 2;
+    p->smem_bytes = 1024 + stages * stage_bytes + 8 * (2 * stages + kExtraBars + (p->w4 ? stages : 0)) + 16 + 16 +
+                    2 * 2 * kBiasStage * 4 + 2 * 16 * kTileA * 2;
     // workspace: counters, then INT32 partial tiles [slots][bn][128]
     const size_t cnt = ((size_t)p->slots * 4 + 255) / 256 * 256;
     p->ws_counters_off = 0;
@@ -862,8 +934,10 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
     plan_common(p);
 }
 
-void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p) {
+void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p,
+                     bool w4) {
     *p = GemmPlan{};
+    p->w4 = w4 ? 1 : 0;         // INT4 weights: the swapped orientation only (m <= 256)
     p->njobs = njobs;
     // m <= 256: the weights are the 128-row A operand and the activations
     // one B tile of roundup16(m) rows.  256 < m <= 512: activations are A
@@ -912,6 +986,22 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
+// Byte matrix [rows, cols] -> tensor map with a (box_cols bytes x box_rows)
+// box, no swizzle (packed INT4 weight tiles, unpacked in shared memory).
+static bool make_tmap_plain(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, int box_rows,
+                            int box_cols) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // K-major INT8 matrix [rows, k] -> tensor map with a (128 bytes x box_rows)
 // box and 128-byte swizzle.
 static bool make_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int64_t k, int box_rows) {
@@ -941,6 +1031,7 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
     a.split_ways = p.split_ways;
     a.split_pieces = p.split_pieces;
     a.rep = p.rep > 0 ? p.rep : 1;
+
     a.tail_units = p.tail_units;
     a.stages = p.stages;
     a.acc_cols = p.acc_cols;
@@ -952,7 +1043,13 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
         const GemmProblem &q = probs[j];
         const int8_t *A = p.swap ? q.wq : q.xq;
         const int8_t *B = p.swap ? q.xq : q.wq;
-        if (!make_tmap(&maps.a[j], A, p.rows_a[j], q.k, kTileA)) return cudaErrorInvalidValue;
+        if (p.w4) {
+            // packed INT4 weight [n, k/2] bytes, plain (unswizzled) 64-byte boxes
+            if (!p.swap || !make_tmap_plain(&maps.a[j], A, p.rows_a[j], q.k / 2, kTileA, (int)kPackedTileBytes / kTileA))
+                return cudaErrorInvalidValue;
+        } else if (!make_tmap(&maps.a[j], A, p.rows_a[j], q.k, kTileA)) {
+            return cudaErrorInvalidValue;
+        }
         if (!make_tmap(&maps.b[j], B, p.rows_b[j], q.k, p.bn)) return cudaErrorInvalidValue;
         GemmJob &J = a.job[j];
         J.m = (int)q.m;
@@ -976,7 +1073,9 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(gemm_i8_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        e = cudaFuncSetAttribute(gemm_i8_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(gemm_i8_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev] = true;
     }
@@ -986,12 +1085,13 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3((unsigned)p.grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(p.w4 ? kThreadsW4 : kThreads);
     cfg.dynamicSmemBytes = (size_t)p.smem_bytes;
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel, maps, a);
+    if (p.w4) return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel<true>, maps, a);
+    return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel<false>, maps, a);
 }
 
 }  // namespace convrot

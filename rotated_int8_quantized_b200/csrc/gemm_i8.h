@@ -74,6 +74,7 @@ struct GemmProblem {
 struct GemmPlan {
     int njobs, swap, bn;
     int grid, full_waves, full_tiles, split_ways, split_pieces, stages, acc_cols, tmem_cols, smem_bytes, rep;
+    int w4;             // INT4 weights (packed), unpacked in shared memory
     long long tail_units;
     int tiles_a[kMaxJobs], tiles_b[kMaxJobs], group_a[kMaxJobs], kbpt[kMaxJobs], tile_base[kMaxJobs];
     long long unit0[kMaxJobs];
@@ -88,7 +89,9 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p);
 // Several products with the same m <= kMaxSwapM in one launch: every K
 // block of every (weight tile, activation tile) pair dealt out evenly by
 // stream-K.
-void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p);
+// w4: INT4 weights (packed two codes per byte; m <= 256 only).
+void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p,
+                     bool w4 = false);
 
 cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws, cudaStream_t stream,
                            bool pdl, bool w_prefetch);
@@ -98,8 +101,9 @@ struct RQProblem {
     const void *a;      // BF16 [rows, k]
     int64_t k;
     int group;          // rotation group (power of two, 16 .. 256)
-    int8_t *q;          // int8 [rows, k]
+    int8_t *q;          // int8 [rows, k], or packed INT4 [rows, k/2] (int4)
     float *s;           // fp32 [rows]
+    int int4;           // 1: INT4 weight codes (levels -7..7), packed
 };
 
 // Rotate and quantise `rows` rows of each of `njobs` matrices (same row

@@ -39,6 +39,15 @@ struct RowScale {
     bool fast;      // r is finite, so the rounding test below applies
 };
 
+__device__ __forceinline__ RowScale make_row_scale_levels(float amax, float levels) {
+    RowScale rs;
+    rs.s = __fdiv_rn(amax, levels);
+    rs.zero = (amax == 0.0f);
+    rs.r = rs.zero ? 0.0f : __frcp_rn(rs.s);
+    rs.fast = !rs.zero && isfinite(rs.r);
+    return rs;
+}
+
 __device__ __forceinline__ RowScale make_row_scale(float amax) {
     RowScale rs;
     rs.s = __fdiv_rn(amax, 127.0f);
@@ -101,6 +110,40 @@ __device__ __forceinline__ uint4 quant16(const float (&y)[16], const RowScale &r
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+
+// INT4 weight codes (W4A8): q = clamp(rne(fl(y / s)), -7, 7) with s = a / 7,
+// the same rounding test as quant16 (|y/s| <= 7 here, so the bound holds with
+// room to spare), packed two per byte: byte j of the 8 holds code j in its
+// low nibble and code 8 + j in its high nibble.
+__device__ __forceinline__ uint2 quant16_int4(const float (&y)[16], const RowScale &rs, unsigned mask) {
+    int code[16];
+    bool slow = false;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float t = __fmul_rn(y[e], rs.r);
+        const float big = __fadd_rn(t, kRoundMagic);
+        code[e] = __float_as_int(big) - kRoundMagicBits;
+        slow |= !(fabsf(__fsub_rn(t, __fsub_rn(big, kRoundMagic))) < 0.49997f);
+    }
+    slow = slow || !rs.fast;
+    if (__any_sync(mask, slow) && slow) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float t = __fmul_rn(y[e], rs.r);
+            const float f = __fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic);
+            if (!rs.fast || !(fabsf(__fsub_rn(t, f)) < 0.49997f))
+                code[e] = __float_as_int(__fadd_rn(__fdiv_rn(y[e], rs.s), kRoundMagic)) - kRoundMagicBits;
+        }
+    }
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int lo = rs.zero ? 0 : min(max(code[j], -7), 7);
+        const int hi = rs.zero ? 0 : min(max(code[8 + j], -7), 7);
+        w[j >> 2] |= (uint32_t)((lo & 0xF) | ((hi & 0xF) << 4)) << (8 * (j & 3));
+    }
+    return make_uint2(w[0], w[1]);
+}
 
 // ---------------------------------------------------------------------------
 // Main variant: 16 threads ("a slot") per 256-group, H_256 = H_16 (x) H_16.
@@ -220,9 +263,12 @@ __device__ __forceinline__ void cluster_wait() {
 // 256/G independent groups (butterflies of strides < G only), a row's last
 // chunk may be partial (k % 256 != 0; k is a multiple of G), and the
 // normalisation divides by sqrt(G) in FP64 when G is not a power of four.
-template <int GPS, bool HALF, bool DYN>
+// MODE 0: INT8 codes, groups of 256; 1: INT8, any group (DYN below); 2: INT4
+// weight codes (levels -7..7, scale a/7), packed two per byte, any group.
+template <int GPS, bool HALF, int MODE>
 __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
+    constexpr bool DYN = MODE != 0;
     constexpr int kXchStride = HALF ? kXchHalf : kXchFull;
     extern __shared__ __align__(16) uint8_t rq_smem[];
     __shared__ float red[kMaxSlots / 2];
@@ -343,7 +389,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
         rmax = red[0];
         cluster_arrive();   // this CTA no longer reads its peers; matched by the wait before exit
     }
-    const RowScale rs = make_row_scale(rmax);
+    const RowScale rs = MODE == 2 ? make_row_scale_levels(rmax, 7.0f) : make_row_scale(rmax);
 
     // quantise 16 consecutive outputs per thread, one 16-byte store
     int8_t *qrow = J.q + (size_t)row * k + (size_t)g0 * 256;
@@ -365,7 +411,11 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                 y[4 * i + 2] = f.z;
                 y[4 * i + 3] = f.w;
             }
-            *reinterpret_cast<uint4 *>(qrow + c * 16) = quant16(y, rs, mask);
+            if (MODE == 2)      // packed INT4: row stride k/2 bytes
+                *reinterpret_cast<uint2 *>(J.q + (size_t)row * (k / 2) + (size_t)g0 * 128 + c * 8) =
+                    quant16_int4(y, rs, mask);
+            else
+                *reinterpret_cast<uint4 *>(qrow + c * 16) = quant16(y, rs, mask);
         }
     }
     if (tid == 0 && part == 0) J.s[row] = rs.s;
@@ -375,7 +425,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     }
 }
 
-template <int GPS, bool HALF, bool DYN>
+template <int GPS, bool HALF, int MODE>
 static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int max_slots, int max_local_groups) {
     cfg.blockDim = dim3(max_slots * 16);
     cfg.dynamicSmemBytes =
@@ -385,32 +435,32 @@ static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(rotate_quant_rows_slots<GPS, HALF, DYN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(rotate_quant_rows_slots<GPS, HALF, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSlotsSmemMax);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev] = true;
     }
-    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS, HALF, DYN>, args);
+    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS, HALF, MODE>, args);
 }
 
-template <bool DYN>
+template <int MODE>
 static cudaError_t launch_gps(cudaLaunchConfig_t &cfg, const RQArgs &args, bool half, int max_gps, int max_slots,
                               int max_local) {
-    if (half) {
+    if (half && MODE != 2) {
         switch (max_gps) {
-            case 1: return launch_slots<1, true, DYN>(cfg, args, max_slots, max_local);
-            case 2: return launch_slots<2, true, DYN>(cfg, args, max_slots, max_local);
-            case 3: return launch_slots<3, true, DYN>(cfg, args, max_slots, max_local);
-            case 4: return launch_slots<4, true, DYN>(cfg, args, max_slots, max_local);
-            default: return launch_slots<6, true, DYN>(cfg, args, max_slots, max_local);
+            case 1: return launch_slots<1, true, MODE>(cfg, args, max_slots, max_local);
+            case 2: return launch_slots<2, true, MODE>(cfg, args, max_slots, max_local);
+            case 3: return launch_slots<3, true, MODE>(cfg, args, max_slots, max_local);
+            case 4: return launch_slots<4, true, MODE>(cfg, args, max_slots, max_local);
+            default: return launch_slots<6, true, MODE>(cfg, args, max_slots, max_local);
         }
     }
     switch (max_gps) {
-        case 1: return launch_slots<1, false, DYN>(cfg, args, max_slots, max_local);
-        case 2: return launch_slots<2, false, DYN>(cfg, args, max_slots, max_local);
-        case 3: return launch_slots<3, false, DYN>(cfg, args, max_slots, max_local);
-        case 4: return launch_slots<4, false, DYN>(cfg, args, max_slots, max_local);
-        default: return launch_slots<6, false, DYN>(cfg, args, max_slots, max_local);
+        case 1: return launch_slots<1, false, MODE>(cfg, args, max_slots, max_local);
+        case 2: return launch_slots<2, false, MODE>(cfg, args, max_slots, max_local);
+        case 3: return launch_slots<3, false, MODE>(cfg, args, max_slots, max_local);
+        case 4: return launch_slots<4, false, MODE>(cfg, args, max_slots, max_local);
+        default: return launch_slots<6, false, MODE>(cfg, args, max_slots, max_local);
     }
 }
 
@@ -472,8 +522,10 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         return cudaSuccess;
     }
     // decode-sized launches use the half-size transpose buffer, so that their
-    // CTAs fit beside the GEMM's
-    const bool half = few_rows;
+    // CTAs fit beside the GEMM's (INT4 weight conversion is offline: full)
+    bool int4 = false;
+    for (int j = 0; j < njobs; ++j) int4 = int4 || probs[j].int4;
+    const bool half = few_rows && !int4;
     const int parts = rq_parts(njobs, rows, probs, num_sms, half);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -519,8 +571,9 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
             rq_shape((groups + parts - 1) / parts, &J.gps, &J.slots);
             dyn = dyn || J.group != 256 || (J.k & 255) != 0;
         }
-        if (dyn) return launch_gps<true>(cfg, args, half, max_gps, max_slots, max_local);
-        return launch_gps<false>(cfg, args, half, max_gps, max_slots, max_local);
+        if (int4) return launch_gps<2>(cfg, args, half, max_gps, max_slots, max_local);
+        if (dyn) return launch_gps<1>(cfg, args, half, max_gps, max_slots, max_local);
+        return launch_gps<0>(cfg, args, half, max_gps, max_slots, max_local);
     }
     // unreachable within the shapes the API accepts (k <= 133120 stages in
     // at most 114 KB per CTA with 8 parts)

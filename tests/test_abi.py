@@ -120,6 +120,9 @@ int main(void) {
     printf("convrot_linear_job_t %zu\n", sizeof(convrot_linear_job_t));
     F(convrot_weight_t, group) F(convrot_gemm_job_t, acc) F(convrot_gemm_job_t, bias_bf16)
     F(convrot_linear_job_t, y_bf16) F(convrot_linear_job_t, bias_bf16)
+    printf("convrot_weight4_t %zu\n", sizeof(convrot_weight4_t));
+    printf("convrot_linear4_job_t %zu\n", sizeof(convrot_linear4_job_t));
+    F(convrot_weight4_t, group) F(convrot_linear4_job_t, bias_bf16)
     return 0;
 }
 ''')
@@ -135,6 +138,10 @@ int main(void) {
         "convrot_gemm_job_t.bias_bf16": cr.convrot_gemm_job_t.bias_bf16.offset,
         "convrot_linear_job_t.y_bf16": cr.convrot_linear_job_t.y_bf16.offset,
         "convrot_linear_job_t.bias_bf16": cr.convrot_linear_job_t.bias_bf16.offset,
+        "convrot_weight4_t": ctypes.sizeof(cr.convrot_weight4_t),
+        "convrot_linear4_job_t": ctypes.sizeof(cr.convrot_linear4_job_t),
+        "convrot_weight4_t.group": cr.convrot_weight4_t.group.offset,
+        "convrot_linear4_job_t.bias_bf16": cr.convrot_linear4_job_t.bias_bf16.offset,
     }
     assert {k: int(v) for k, v in got.items()} == want
 
@@ -149,3 +156,18 @@ def test_dynamic_group(lib):
     for k in range(16, 4000, 16):
         g = lib.convrot_dynamic_group(k, 256)
         assert g >= 16 and g <= 256 and k % g == 0 and (g == 256 or k % (2 * g) != 0)
+
+
+def test_weight4_validation(lib):
+    import rotated_int8_quantized_b200 as cr
+    h = cr.convrot_weight4_t()
+    P = ctypes.c_void_p
+    assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10000), P(0x20000), 8, 512, 256) == 0
+    assert h.k == 512 and h.group == 256
+    assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10000), P(0x20000), 8, 48, 16) == 3   # k % 32
+    assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10001), P(0x20000), 8, 512, 256) == 2
+    job = (cr.convrot_linear4_job_t * 1)()
+    job[0].x_bf16, job[0].w, job[0].y_bf16 = P(0x100000), ctypes.pointer(h), P(0x200000)
+    assert lib.convrot_linear_w4a8(257, 1, job, P(0x300000), 1 << 30, P(0)) == 3     # m > 256
+    assert lib.convrot_linear_w4a8(0, 1, job, P(0x300000), 1 << 30, P(0)) == 1
+    assert lib.convrot_linear_w4a8_workspace_bytes(12, 1, job) > 0

@@ -547,3 +547,74 @@ def test_embed_lookup_matches_oracle(cr):
     cr.convrot_device_status()           # cleared by the read
     assert np.array_equal(to_bits(out2[:1]), oracle.embed_lookup(np.array([1], np.int32), q_ref, s_ref))
     assert not to_bits(out2[1:]).any()
+
+
+
+# ---------------------------------------------------------------- INT4 weights (W4A8)
+@pytest.mark.parametrize("n,k,dyn", [(256, 512, False), (1000, 5120, False), (300, 640, True), (150, 25600, False)])
+def test_weight4_quant_bit_exact(cr, n, k, dyn):
+    w_bits = synth.draw_np(synth.stream_key(n + k, 1), n, k, synth.W_SIGMA)
+    w4 = cr.quantize_weight4(from_bits(w_bits), dynamic=dyn)
+    torch.cuda.synchronize()
+    packed_ref, s_ref = oracle.rotate_quantize4(w_bits, w4.group)
+    assert np.array_equal(w4.q.cpu().numpy(), packed_ref)
+    assert np.array_equal(w4.scale.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# (m, [(k, n), ...]): decode sizes, several weights in one launch, a shared
+# input, a bias, a ragged weight tile, K not a multiple of 128 (dynamic group)
+W4_CASES = [
+    (1, [(512, 256)]),
+    (12, [(5120, 1024), (5120, 768), (2560, 512)]),
+    (4, [(640, 384)]),
+    (100, [(1536, 640), (512, 1000)]),
+    (256, [(1024, 512)]),
+]
+
+
+@pytest.mark.parametrize("m,shapes", W4_CASES)
+def test_w4a8_linear_bit_exact(cr, m, shapes):
+    x_by_k, ws4, ys, biases, refs = {}, [], [], [], []
+    for idx, (k, n) in enumerate(shapes):
+        seed = 9000 + 13 * idx + m
+        group = cr.convrot_dynamic_group(k)
+        if k not in x_by_k:
+            cs = synth.outlier_scale_fraction(synth.stream_key(seed, 2), k, 0.01, 30.0)
+            x_by_k[k] = synth.draw_np(synth.stream_key(seed, 0), m, k, 1.0, cs)
+        w_bits = synth.draw_np(synth.stream_key(seed, 1), n, k, synth.W_SIGMA)
+        packed, sw = oracle.rotate_quantize4(w_bits, group)
+        b_bits = _bias_bits(seed, n) if idx == 1 else None
+        refs.append(oracle.linear_w4a8(x_by_k[k], packed, sw, group=group, bias=b_bits))
+        ws4.append(cr.quantize_weight4(from_bits(w_bits), dynamic=True))
+        ys.append(torch.empty((m, n), dtype=torch.bfloat16, device="cuda"))
+        biases.append(None if b_bits is None else from_bits(b_bits))
+    x_dev = {k: from_bits(v) for k, v in x_by_k.items()}
+    batch = cr.LinearBatchW4([x_dev[k] for k, _ in shapes], ws4, ys, biases=biases)
+    batch()
+    batch()                      # the GEMM scratch is left reusable
+    cr.convrot_device_status()
+    for y, ref in zip(ys, refs):
+        yb = to_bits(y)
+        assert rel_err(yb, ref["y"]) <= TOL
+        assert np.array_equal(yb, ref["y"])
+
+
+def test_w4a8_qwen_decode_layer_sampled(cr):
+    lins = synth.qwen_layer(12)
+    xs, ws4, ys = [], [], []
+    for lin in lins:
+        w_bf = lin.w_torch("cuda")
+        ws4.append(cr.quantize_weight4(w_bf))
+        del w_bf
+        xs.append(lin.x_torch("cuda"))
+        ys.append(torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device="cuda"))
+    cr.LinearBatchW4(xs, ws4, ys)()
+    cr.convrot_device_status()
+    rng = np.random.default_rng(21)
+    for lin, w4, y in zip(lins, ws4, ys):
+        rows = np.unique(np.concatenate([[0, lin.n - 1], rng.integers(0, lin.n, 12)]))
+        packed_ref, s_ref = oracle.rotate_quantize4(lin.w_rows_np(rows))
+        rw = torch.as_tensor(rows, device="cuda")
+        assert np.array_equal(w4.q[rw].cpu().numpy(), packed_ref)
+        ref = oracle.linear_w4a8(lin.x_np(), packed_ref, s_ref)
+        assert np.array_equal(to_bits(y[:, rw]), ref["y"])
