@@ -24,6 +24,8 @@ the source pages it follows, is stated in the C file:
   divides k, with rotations of such groups (0539edu.com section 4, item 3)
 * tensor-wise simple INT8 of the embedding table and the lookup from it
   (zskr.cn quantisation configuration and conversion command)
+* 2-D convolutions as the ConvRot layer on their im2col matrix (NHWC input,
+  taps outer, channels inner; the VAE's int8_convrot)
 * INT4 ConvRot weights (levels -7..7, row scale a/7) packed two per byte,
   with INT8 activations: the W4A4 variant's Blackwell route (0539edu.com
   sections 5 and 7)
@@ -86,6 +88,9 @@ def _load():
         lib.oracle_unpack_int4.argtypes = [P, I64, I64, P]
         lib.oracle_rotate_quantize4.argtypes = [P, I64, I64, ctypes.c_int, P, P]
         lib.oracle_rotate_quantize4.restype = I64
+        lib.oracle_im2col_nhwc.argtypes = [P, I64, I64, I64, I64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, I64, I64, P]
+        lib.oracle_conv_weight_rows.argtypes = [P, I64, I64, ctypes.c_int, ctypes.c_int, P]
         lib.oracle_dynamic_group.argtypes = [I64, ctypes.c_int]
         lib.oracle_dynamic_group.restype = ctypes.c_int
         lib.oracle_dequant_bf16_bias.argtypes = [P, P, P, P, I64, I64, P]
@@ -255,6 +260,43 @@ def linear_w4a8(x_bf16: np.ndarray, packed: np.ndarray, sw: np.ndarray, group: i
     codes unpacked from INT4; exact INT32 GEMM; the same dequantisation."""
     wq = unpack_int4(packed)
     return linear_int8(x_bf16, wq, sw, group=group, bias=bias)
+
+
+def conv_out_size(size: int, k: int, stride: int, pad: int, dil: int) -> int:
+    return (size + 2 * pad - dil * (k - 1) - 1) // stride + 1
+
+
+def im2col_nhwc(x_bf16: np.ndarray, kh: int, kw: int, stride: int = 1, pad: int = 0, dil: int = 1) -> np.ndarray:
+    """BF16 bits [n, h, w, c] -> im2col rows [n*oh*ow, kh*kw*c] (taps outer, channels inner)."""
+    x = _bf16_bits(x_bf16)
+    n, h, w, c = x.shape
+    oh, ow = conv_out_size(h, kh, stride, pad, dil), conv_out_size(w, kw, stride, pad, dil)
+    out = np.empty((n * oh * ow, kh * kw * c), dtype=np.uint16)
+    _load().oracle_im2col_nhwc(_ptr(x), n, h, w, c, kh, kw, stride, pad, dil, oh, ow, _ptr(out))
+    return out
+
+
+def conv_weight_rows(w_bf16: np.ndarray) -> np.ndarray:
+    """BF16 bits [o, c, kh, kw] (OIHW) -> rows [o, kh*kw*c] in the im2col order."""
+    w = _bf16_bits(w_bf16)
+    o, c, kh, kw = w.shape
+    out = np.empty((o, kh * kw * c), dtype=np.uint16)
+    _load().oracle_conv_weight_rows(_ptr(w), o, c, kh, kw, _ptr(out))
+    return out
+
+
+def conv2d_int8(x_nhwc_bf16: np.ndarray, w_oihw_bf16: np.ndarray, stride: int = 1, pad: int = 0, dil: int = 1,
+                group: int = 256):
+    """INT8 ConvRot 2-D convolution: the linear layer on the im2col matrix.
+    Returns the linear_int8 dict with ``y`` reshaped to NHWC [n, oh, ow, o]."""
+    n, h, w, c = x_nhwc_bf16.shape
+    o, _, kh, kw = w_oihw_bf16.shape
+    oh, ow = conv_out_size(h, kh, stride, pad, dil), conv_out_size(w, kw, stride, pad, dil)
+    wq, sw = rotate_quantize(conv_weight_rows(w_oihw_bf16), group)
+    out = linear_int8(im2col_nhwc(x_nhwc_bf16, kh, kw, stride, pad, dil), wq, sw, group=group)
+    out["y"] = out["y"].reshape(n, oh, ow, o)
+    out["wq"], out["sw"] = wq, sw
+    return out
 
 
 def gemm_i32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:

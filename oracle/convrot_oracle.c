@@ -418,6 +418,57 @@ int64_t oracle_rotate_quantize4(const uint16_t *a, int64_t rows, int64_t k, int 
 }
 
 /* ------------------------------------------------------------------ */
+/* ConvRot for 2-D convolutions (the VAE's int8_convrot)               */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The pages apply int8_convrot to the VAE's convolutions (a reported ~1.5x
+ * decode speed-up) without describing it further [feinterview.poetries.top
+ * "MiniMax-H3在ComfyUI的W4A8量化与VAE加速实战", the int8_convrot VAE
+ * optimisation paragraph].  Reading: the convolution as the linear layer on its
+ * im2col matrix.  Row (b, oy, ox) of the im2col matrix holds, tap by tap
+ * (ky, kx row-major) and channel by channel inside a tap, the input
+ * x[b, oy*stride - pad + ky*dil, ox*stride - pad + kx*dil, c] (NHWC), zero
+ * outside the image; weight row o holds w[o, c, ky, kx] in the same order.
+ * The rotation groups then lie inside one tap's channels (group | C), so
+ * rotating both sides preserves the convolution tap by tap.
+ *
+ * x is BF16 bits [n, h, w, c]; out is BF16 bits [n*oh*ow, kh*kw*c].
+ */
+void oracle_im2col_nhwc(const uint16_t *x, int64_t n, int64_t h, int64_t w, int64_t c,
+                        int kh, int kw, int stride, int pad, int dil, int64_t oh, int64_t ow,
+                        uint16_t *out)
+{
+    int64_t k = (int64_t)kh * kw * c;
+    for (int64_t b = 0; b < n; ++b)
+        for (int64_t oy = 0; oy < oh; ++oy)
+            for (int64_t ox = 0; ox < ow; ++ox) {
+                int64_t row = (b * oh + oy) * ow + ox;
+                for (int ky = 0; ky < kh; ++ky)
+                    for (int kx = 0; kx < kw; ++kx) {
+                        int64_t iy = oy * stride - pad + (int64_t)ky * dil;
+                        int64_t ix = ox * stride - pad + (int64_t)kx * dil;
+                        int inside = iy >= 0 && iy < h && ix >= 0 && ix < w;
+                        for (int64_t ch = 0; ch < c; ++ch)
+                            out[row * k + ((int64_t)ky * kw + kx) * c + ch] =
+                                inside ? x[((b * h + iy) * w + ix) * c + ch] : 0;
+                    }
+            }
+}
+
+/* Weight w[o, c, ky, kx] (PyTorch OIHW, BF16 bits) -> rows [o, (ky, kx, c)]. */
+void oracle_conv_weight_rows(const uint16_t *w, int64_t o, int64_t c, int kh, int kw, uint16_t *out)
+{
+    int64_t k = (int64_t)kh * kw * c;
+    for (int64_t oo = 0; oo < o; ++oo)
+        for (int ky = 0; ky < kh; ++ky)
+            for (int kx = 0; kx < kw; ++kx)
+                for (int64_t ch = 0; ch < c; ++ch)
+                    out[oo * k + ((int64_t)ky * kw + kx) * c + ch] =
+                        w[((oo * c + ch) * kh + ky) * kw + kx];
+}
+
+/* ------------------------------------------------------------------ */
 /* INT8 GEMM with INT32 result                                         */
 /* ------------------------------------------------------------------ */
 

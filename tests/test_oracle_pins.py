@@ -261,6 +261,60 @@ def test_w4a8_linear_composes():
 
 
 # ---------------------------------------------------------------------------
+# 2-D convolution as the layer on its im2col matrix
+# ---------------------------------------------------------------------------
+def _conv_direct_f64(x, w, stride, pad, dil):
+    """Plain loops: out[b, oy, ox, o] = sum_{c, ky, kx} x[b, iy, ix, c] * w[o, c, ky, kx]."""
+    n, h, wd, c = x.shape
+    o, _, kh, kw = w.shape
+    oh, ow = oracle.conv_out_size(h, kh, stride, pad, dil), oracle.conv_out_size(wd, kw, stride, pad, dil)
+    out = np.zeros((n, oh, ow, o))
+    for b in range(n):
+        for oy in range(oh):
+            for ox in range(ow):
+                for ky in range(kh):
+                    for kx in range(kw):
+                        iy, ix = oy * stride - pad + ky * dil, ox * stride - pad + kx * dil
+                        if 0 <= iy < h and 0 <= ix < wd:
+                            out[b, oy, ox] += w[:, :, ky, kx] @ x[b, iy, ix]
+    return out
+
+
+@pytest.mark.parametrize("stride,pad,dil,kh", [(1, 1, 1, 3), (2, 1, 1, 3), (1, 2, 2, 3), (1, 0, 1, 1), (2, 0, 1, 2)])
+def test_im2col_matches_direct_conv_and_torch(stride, pad, dil, kh):
+    rng = np.random.default_rng(stride * 10 + pad + kh)
+    xf = rng.standard_normal((2, 7, 6, 32)).astype(np.float32)
+    wf = rng.standard_normal((5, 32, kh, kh)).astype(np.float32)
+    xb, wb = synth.f32_to_bf16_bits(xf), synth.f32_to_bf16_bits(wf)
+    x64, w64 = synth.bf16_bits_to_f32(xb).astype(np.float64), synth.bf16_bits_to_f32(wb).astype(np.float64)
+    cols = synth.bf16_bits_to_f32(oracle.im2col_nhwc(xb, kh, kh, stride, pad, dil)).astype(np.float64)
+    rows = synth.bf16_bits_to_f32(oracle.conv_weight_rows(wb)).astype(np.float64)
+    got = cols @ rows.T
+    direct = _conv_direct_f64(x64, w64, stride, pad, dil)
+    assert np.allclose(got, direct.reshape(got.shape), rtol=1e-12, atol=1e-12)
+    ref = torch.nn.functional.conv2d(torch.from_numpy(x64).permute(0, 3, 1, 2), torch.from_numpy(w64),
+                                     stride=stride, padding=pad, dilation=dil).permute(0, 2, 3, 1).numpy()
+    assert np.allclose(got, ref.reshape(got.shape), rtol=1e-10, atol=1e-10)
+
+
+def test_rotation_preserves_the_convolution_and_int8_approximates_it():
+    # groups lie inside a tap's channels, so rotating both sides keeps the product
+    rng = np.random.default_rng(31)
+    xf = rng.standard_normal((1, 6, 6, 256)).astype(np.float32)
+    xf[..., 7] *= 40.0                                   # an outlier channel
+    wf = (rng.standard_normal((16, 256, 3, 3)) * 0.02).astype(np.float32)
+    xb, wb = synth.f32_to_bf16_bits(xf), synth.f32_to_bf16_bits(wf)
+    cols = synth.bf16_bits_to_f32(oracle.im2col_nhwc(xb, 3, 3, 1, 1, 1)).astype(np.float64)
+    rows = synth.bf16_bits_to_f32(oracle.conv_weight_rows(wb)).astype(np.float64)
+    rot = oracle.rotate_rows_f64(cols, 256) @ oracle.rotate_rows_f64(rows, 256).T
+    assert np.max(np.abs(rot - cols @ rows.T)) <= 1e-9 * np.max(np.abs(cols @ rows.T))
+    out = oracle.conv2d_int8(xb, wb, 1, 1, 1)
+    ref = (cols @ rows.T).reshape(out["y"].shape)
+    y = oracle.bf16_bits_to_f64(out["y"])
+    assert np.max(np.abs(y - ref)) / np.max(np.abs(ref)) < 0.05
+
+
+# ---------------------------------------------------------------------------
 # --dynamic-convrot: smaller power-of-two groups
 # ---------------------------------------------------------------------------
 def test_dynamic_group_choice():
