@@ -448,6 +448,43 @@ def w4a8_secondary(cr, lins, device, stream, peaks, steps=2000, warmup=20):
             "weight_stream_gb_s_int8_equivalent": sum(l.n * l.k for l in lins) / t / 1e9}
 
 
+def conv_secondary(cr, device, stream, peaks, steps=10, warmup=3):
+    """VAE-decoder-shaped 3x3 convolutions (int8_convrot): NHWC BF16 in and
+    out, im2col rows gathered by the prologue, INT8 GEMM; TOPS (2MNK)."""
+    out = {}
+    peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    for (h, c) in ((128, 512), (256, 256)):
+        seed = 77 + c
+        x = synth.Linear("conv_x", h * h, c, 1, seed, None).x_torch(device).view(1, h, h, c)
+        w_rows = synth.Linear("conv_w", 1, 9 * c, c, seed, None).w_torch(device)
+        w_oihw = w_rows.view(c, c, 3, 3)
+        wq = cr.quantize_conv_weight(w_oihw)
+        y = torch.empty((1, h, h, c), dtype=torch.bfloat16, device=device)
+        g = cr.conv2d_geometry(x.shape, 3, 3, 1, 1, 1)
+        need = int(cr.load_library().convrot_conv2d_workspace_bytes(ctypes_byref(g), ctypes_byref(wq.handle)))
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        torch.cuda.synchronize()
+        fn = lambda: cr.conv2d_int8(x, wq, 3, 3, 1, 1, 1, y=y, ws=ws, stream=stream)  # noqa: E731
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                fn()
+        torch.cuda.synchronize()
+        keep_busy(stream, 200.0)
+        t = time_region(fn, steps, stream) / steps
+        ops = 2 * (h * h) * c * (9 * c)
+        out["h%d_c%d" % (h, c)] = {"ms": t * 1e3, "tops": ops / t / 1e12, "frac_of_int8_ref": ops / t / 1e12 / peak,
+                                   "m": h * h, "n": c, "k": 9 * c}
+        del x, w_rows, w_oihw, wq, y, ws
+        torch.cuda.empty_cache()
+    out["workload"] = "vae_decoder_conv3x3_nhwc"
+    return out
+
+
+def ctypes_byref(obj):
+    import ctypes
+    return ctypes.byref(obj)
+
+
 def minimax_secondary(cr, device, stream, peaks, steps=5, warmup=2):
     """MiniMax-H3-shaped qkv projection (K = 5376, N = 16128) at M = 8192 and
     32768 video tokens through the single-linear entry point: INT8 TOPS."""
@@ -676,6 +713,7 @@ def run_ours(args):
     cr.convrot_device_status(stream)
     others = {"shared_inputs": shared_input_secondary(cr, layer, lins, device, stream, peaks),
               "w4a8": w4a8_secondary(cr, lins, device, stream, peaks)}
+    others["conv"] = conv_secondary(cr, device, stream, peaks)
     if not args.no_minimax:
         others["minimax_qkv"] = minimax_secondary(cr, device, stream, peaks)
         cr.convrot_device_status(stream)

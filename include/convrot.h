@@ -333,6 +333,49 @@ convrot_status_t convrot_linear_w4a8(int64_t m, int count, const convrot_linear4
 size_t convrot_linear_w4a8_workspace_bytes(int64_t m, int count, const convrot_linear4_job_t *jobs);
 
 /*
+ * ---------------------------------------------------------------- 2-D convolutions (int8_convrot)
+ * The pages apply int8_convrot to the VAE's convolutions (a reported ~1.5x
+ * decode speed-up; feinterview.poetries.top "MiniMax-H3在ComfyUI的W4A8量化与
+ * VAE加速实战", the int8_convrot VAE paragraph) without further detail.
+ * Here a convolution is the ConvRot INT8 layer on its im2col matrix: row
+ * (b, oy, ox) holds, tap by tap (ky, kx row-major) and channel by channel,
+ * x[b, oy*stride - pad + ky*dil, ox*stride - pad + kx*dil, c] (zero outside
+ * the image); the weight row o holds w[o, c, ky, kx] in the same order; the
+ * rotation groups lie inside one tap's channels (group divides C), so
+ * rotating both sides preserves the convolution.  The activation prologue
+ * gathers the im2col rows straight from the NHWC input (no BF16 im2col copy)
+ * and writes their INT8 codes to the workspace.
+ */
+typedef struct {
+    int32_t n, h, w, c;             /* input NHWC: batch, height, width, channels (c % 16 == 0) */
+    int32_t kh, kw;                 /* kernel size */
+    int32_t stride, pad, dilation;  /* the same along both axes */
+} convrot_conv2d_t;
+
+/* Output height and width: (size + 2 pad - dil (k - 1) - 1) / stride + 1. */
+convrot_status_t convrot_conv2d_shape(const convrot_conv2d_t *g, int32_t *oh, int32_t *ow);
+
+/*
+ * Offline: rotate and quantise a BF16 OIHW weight [c_out, c, kh, kw] into
+ * the handle `out` (out->n = c_out, out->k = kh * kw * c, out->group dividing
+ * c; convrot_dynamic_group(c, 256) picks it), rows in the im2col order.
+ */
+convrot_status_t convrot_quantize_conv_weight(const void *w_oihw_bf16, const convrot_conv2d_t *g,
+                                              const convrot_weight_t *out, void *stream);
+
+/* Workspace of convrot_conv2d_int8 (GEMM scratch + the INT8 im2col codes). */
+size_t convrot_conv2d_workspace_bytes(const convrot_conv2d_t *g, const convrot_weight_t *w);
+
+/*
+ * y [n, oh, ow, w->n] (NHWC, BF16) = the INT8 ConvRot convolution of x
+ * [n, h, w, c] (NHWC, BF16) with the handle from convrot_quantize_conv_weight.
+ * Two launches: the gathering activation prologue, then the INT8 GEMM with
+ * M = n * oh * ow, N = c_out, K = kh * kw * c.
+ */
+convrot_status_t convrot_conv2d_int8(const void *x_nhwc_bf16, const convrot_conv2d_t *g, const convrot_weight_t *w,
+                                     void *y_nhwc_bf16, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Tensor-wise "simple" INT8 of a BF16 tensor of `count` elements (the
  * word-embedding table [vocab, dim]): no rotation, ONE scale for the whole
  * tensor, round-to-nearest-even --

@@ -62,6 +62,11 @@ class convrot_linear4_job_t(ctypes.Structure):
                 ("y_bf16", ctypes.c_void_p), ("bias_bf16", ctypes.c_void_p)]
 
 
+class convrot_conv2d_t(ctypes.Structure):
+    """Mirror of the C struct: convolution geometry (NHWC input)."""
+    _fields_ = [(f, ctypes.c_int32) for f in ("n", "h", "w", "c", "kh", "kw", "stride", "pad", "dilation")]
+
+
 class convrot_gemm_job_t(ctypes.Structure):
     """Mirror of the C struct: one product of a batched GEMM call."""
     _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight_t)),
@@ -76,6 +81,10 @@ SIGNATURES = {
     "convrot_version": ([], ctypes.c_int),
     "convrot_dynamic_group": ([_I64, _I32], _I32),
     "convrot_quantize_tensor": ([_P, _I64, _P, _P, _P], ctypes.c_int),
+    "convrot_conv2d_shape": ([_P, _P, _P], ctypes.c_int),
+    "convrot_quantize_conv_weight": ([_P, _P, _WP, _P], ctypes.c_int),
+    "convrot_conv2d_workspace_bytes": ([_P, _WP], _SZ),
+    "convrot_conv2d_int8": ([_P, _P, _WP, _P, _P, _SZ, _P], ctypes.c_int),
     "convrot_weight4_init": ([ctypes.POINTER(convrot_weight4_t), _P, _P, _I64, _I64, _I32], ctypes.c_int),
     "convrot_quantize_weight4": ([_P, ctypes.POINTER(convrot_weight4_t), _P], ctypes.c_int),
     "convrot_linear_w4a8": ([_I64, ctypes.c_int, _P, _P, _SZ, _P], ctypes.c_int),
@@ -370,6 +379,48 @@ class LinearBatchW4:
     def __call__(self, stream=None) -> None:
         _check(load_library().convrot_linear_w4a8(self.m, len(self.jobs), self.jobs, _ptr(self.ws),
                                                   self.ws.numel(), _stream(stream)), "convrot_linear_w4a8")
+
+
+# ---------------------------------------------------------------- convolutions
+def conv2d_geometry(x_shape, kh: int, kw: int, stride: int = 1, pad: int = 0, dilation: int = 1) -> convrot_conv2d_t:
+    n, h, w, c = x_shape
+    return convrot_conv2d_t(n, h, w, c, kh, kw, stride, pad, dilation)
+
+
+def quantize_conv_weight(w_oihw_bf16: torch.Tensor, stride: int = 1, pad: int = 0, dilation: int = 1,
+                         group: Optional[int] = None, stream=None) -> QuantizedWeight:
+    """Offline INT8 ConvRot conversion of a BF16 OIHW weight; the group
+    defaults to the largest power of two <= 256 dividing the channels."""
+    o, c, kh, kw = w_oihw_bf16.shape
+    group = group or convrot_dynamic_group(c)
+    k = kh * kw * c
+    q = torch.empty((o, k), dtype=torch.int8, device=w_oihw_bf16.device)
+    scale = torch.empty((o,), dtype=torch.float32, device=w_oihw_bf16.device)
+    wt = convrot_weight_init(q, scale, group)
+    g = convrot_conv2d_t(1, kh, kw, c, kh, kw, 1, 0, 1)      # only c, kh, kw matter for the weight
+    _check(load_library().convrot_quantize_conv_weight(_ptr(w_oihw_bf16), ctypes.byref(g), ctypes.byref(wt.handle),
+                                                       _stream(stream)), "convrot_quantize_conv_weight")
+    return wt
+
+
+def conv2d_int8(x_nhwc: torch.Tensor, w: QuantizedWeight, kh: int, kw: int, stride: int = 1, pad: int = 0,
+                dilation: int = 1, y: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """INT8 ConvRot convolution: NHWC BF16 in, NHWC BF16 out."""
+    g = conv2d_geometry(x_nhwc.shape, kh, kw, stride, pad, dilation)
+    lib = load_library()
+    oh, ow = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib.convrot_conv2d_shape(ctypes.byref(g), ctypes.byref(oh), ctypes.byref(ow)), "convrot_conv2d_shape")
+    if y is None:
+        y = torch.empty((g.n, oh.value, ow.value, w.n), dtype=torch.bfloat16, device=x_nhwc.device)
+    if ws is None:
+        need = int(lib.convrot_conv2d_workspace_bytes(ctypes.byref(g), ctypes.byref(w.handle)))
+        if need == 0:
+            raise ConvrotError(3, "convrot_conv2d_workspace_bytes")
+        ws = torch.zeros(need, dtype=torch.uint8, device=x_nhwc.device)
+    _check(lib.convrot_conv2d_int8(_ptr(x_nhwc), ctypes.byref(g), ctypes.byref(w.handle), _ptr(y), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "convrot_conv2d_int8")
+    return y
 
 
 def convrot_device_status(stream=None) -> None:

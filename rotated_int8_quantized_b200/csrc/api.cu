@@ -481,6 +481,104 @@ convrot_status_t convrot_linear_w4a8(int64_t m, int count, const convrot_linear4
     return run_linear(m, count, lj, true, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------- convolutions
+namespace {
+convrot_status_t conv_geom(const convrot_conv2d_t *g, convrot::ConvGeom *cg) {
+    if (!g || g->n < 1 || g->h < 1 || g->w < 1 || g->c < 1 || g->kh < 1 || g->kw < 1 || g->stride < 1 ||
+        g->pad < 0 || g->dilation < 1)
+        return CONVROT_ERR_INVALID_ARG;
+    if (g->c % 16 != 0) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    const int64_t oh = ((int64_t)g->h + 2 * g->pad - (int64_t)g->dilation * (g->kh - 1) - 1) / g->stride + 1;
+    const int64_t ow = ((int64_t)g->w + 2 * g->pad - (int64_t)g->dilation * (g->kw - 1) - 1) / g->stride + 1;
+    if (oh < 1 || ow < 1) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    if ((int64_t)g->n * oh * ow > 0x7FFFFFFF || (int64_t)g->kh * g->kw * g->c > kMaxK ||
+        (int64_t)g->n * g->h * g->w * g->c > ((int64_t)1 << 40))
+        return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    *cg = {0, g->n, g->h, g->w, g->c, g->kh, g->kw, g->stride, g->pad, g->dilation, (int)oh, (int)ow};
+    return CONVROT_OK;
+}
+
+convrot_status_t check_conv_weight(const convrot_conv2d_t *g, const convrot_weight_t *w, convrot::ConvGeom *cg) {
+    convrot_status_t s = conv_geom(g, cg);
+    if (s != CONVROT_OK) return s;
+    if ((s = check_weight(w)) != CONVROT_OK) return s;
+    if (w->k != (int64_t)g->kh * g->kw * g->c || g->c % w->group != 0) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    return CONVROT_OK;
+}
+}  // namespace
+
+convrot_status_t convrot_conv2d_shape(const convrot_conv2d_t *g, int32_t *oh, int32_t *ow) {
+    convrot::ConvGeom cg;
+    convrot_status_t s = conv_geom(g, &cg);
+    if (s != CONVROT_OK) return s;
+    if (oh) *oh = cg.oh;
+    if (ow) *ow = cg.ow;
+    return CONVROT_OK;
+}
+
+convrot_status_t convrot_quantize_conv_weight(const void *w_oihw_bf16, const convrot_conv2d_t *g,
+                                              const convrot_weight_t *out, void *stream) {
+    if (!w_oihw_bf16) return CONVROT_ERR_INVALID_ARG;
+    convrot::ConvGeom cg;
+    convrot_status_t s = check_conv_weight(g, out, &cg);
+    if (s != CONVROT_OK) return s;
+    if ((reinterpret_cast<uintptr_t>(w_oihw_bf16) & 1u) != 0) return CONVROT_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    if ((s = current_device(&dev)) != CONVROT_OK) return s;
+    cg.mode = 4;
+    convrot::RQProblem prob = {w_oihw_bf16, out->k, out->group, out->q, out->scale, 0};
+    return from_cuda(convrot::launch_rotate_quant(1, out->n, &prob, static_cast<cudaStream_t>(stream), false, &cg));
+}
+
+namespace {
+size_t conv_layout(const convrot::ConvGeom &cg, const convrot_weight_t *w, int sms, convrot::GemmPlan *p,
+                   size_t *gemm_bytes) {
+    const int64_t m = (int64_t)cg.n * cg.oh * cg.ow;
+    convrot::plan_gemm(m, w->n, w->k, sms, p);
+    *gemm_bytes = round256(p->ws_bytes);
+    return *gemm_bytes + round256((size_t)m * (size_t)w->k) + round256((size_t)m * 4);
+}
+}  // namespace
+
+size_t convrot_conv2d_workspace_bytes(const convrot_conv2d_t *g, const convrot_weight_t *w) {
+    convrot::ConvGeom cg;
+    if (check_conv_weight(g, w, &cg) != CONVROT_OK) return 0;
+    convrot::GemmPlan p;
+    size_t gb;
+    return conv_layout(cg, w, sms_for_sizing(), &p, &gb);
+}
+
+convrot_status_t convrot_conv2d_int8(const void *x_nhwc_bf16, const convrot_conv2d_t *g, const convrot_weight_t *w,
+                                     void *y_nhwc_bf16, void *ws, size_t ws_bytes, void *stream) {
+    if (!x_nhwc_bf16 || !y_nhwc_bf16) return CONVROT_ERR_INVALID_ARG;
+    convrot::ConvGeom cg;
+    convrot_status_t s = check_conv_weight(g, w, &cg);
+    if (s != CONVROT_OK) return s;
+    if (!aligned16(x_nhwc_bf16) || !aligned16(y_nhwc_bf16)) return CONVROT_ERR_ALIGNMENT;
+    if (!ws) return CONVROT_ERR_WORKSPACE;
+    if (!aligned16(ws)) return CONVROT_ERR_ALIGNMENT;
+    const int64_t m = (int64_t)cg.n * cg.oh * cg.ow;
+    if (ranges_overlap(y_nhwc_bf16, (size_t)m * (size_t)w->n * 2, x_nhwc_bf16,
+                       (size_t)g->n * g->h * g->w * g->c * 2))
+        return CONVROT_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if ((s = current_device(&dev)) != CONVROT_OK) return s;
+    convrot::GemmPlan p;
+    size_t gb;
+    if (ws_bytes < conv_layout(cg, w, dev.num_sms, &p, &gb)) return CONVROT_ERR_WORKSPACE;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    int8_t *xq = reinterpret_cast<int8_t *>(base + gb);
+    float *sx = reinterpret_cast<float *>(base + gb + round256((size_t)m * (size_t)w->k));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cg.mode = 3;
+    convrot::RQProblem rq = {x_nhwc_bf16, w->k, w->group, xq, sx, 0};
+    cudaError_t e = convrot::launch_rotate_quant(1, m, &rq, st, true, &cg);
+    if (e != cudaSuccess) return from_cuda(e);
+    convrot::GemmProblem gp = {m, w->n, w->k, xq, sx, w->q, w->scale, static_cast<__nv_bfloat16 *>(y_nhwc_bf16),
+                               nullptr, nullptr};
+    return from_cuda(convrot::launch_gemm_i8(p, &gp, base, st, true, true));
+}
+
 convrot_status_t convrot_quantize_tensor(const void *w_bf16, int64_t count, int8_t *q, float *scale,
                                          void *stream) {
     if (!w_bf16 || !q || !scale || count < 16) return CONVROT_ERR_INVALID_ARG;

@@ -106,9 +106,19 @@ struct RQProblem {
     int int4;           // 1: INT4 weight codes (levels -7..7), packed
 };
 
+// Geometry of a convolution whose im2col rows (mode 3) or OIHW weight rows
+// (mode 4) the rotation kernel gathers.
+struct ConvGeom {
+    int mode;           // 3: activations (NHWC input), 4: weights (OIHW)
+    int n, h, w, c;     // input batch, height, width, channels
+    int kh, kw, stride, pad, dil;
+    int oh, ow;         // output height and width
+};
+
 // Rotate and quantise `rows` rows of each of `njobs` matrices (same row
-// count) in one launch.
-cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl);
+// count) in one launch; `conv`: the rows are gathered from a convolution.
+cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl,
+                                const ConvGeom *conv = nullptr);
 
 // ------------------------------------------------------------------ tensor-wise INT8 (embedding table)
 cudaError_t launch_quantize_tensor(const void *a, int64_t count, int8_t *q, float *scale, cudaStream_t stream);

@@ -221,6 +221,7 @@ struct RQJobDev {
 struct RQArgs {
     int njobs, rows;
     int parts;              // CTAs (a thread-block cluster) per row
+    ConvGeom conv;          // MODE 3 / 4: the convolution the rows come from
     RQJobDev job[kMaxJobs];
 };
 
@@ -264,7 +265,9 @@ __device__ __forceinline__ void cluster_wait() {
 // chunk may be partial (k % 256 != 0; k is a multiple of G), and the
 // normalisation divides by sqrt(G) in FP64 when G is not a power of four.
 // MODE 0: INT8 codes, groups of 256; 1: INT8, any group (DYN below); 2: INT4
-// weight codes (levels -7..7, scale a/7), packed two per byte, any group.
+// weight codes (levels -7..7, scale a/7), packed two per byte, any group;
+// 3: INT8 codes of the im2col rows of a convolution, gathered from NHWC
+// input; 4: INT8 codes of a convolution's OIHW weight in the im2col order.
 template <int GPS, bool HALF, int MODE>
 __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
@@ -293,19 +296,59 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     const unsigned half_mask = 0xFFFFu << (16 * (slot & 1));
     const __nv_bfloat16 *arow = J.a + (size_t)row * k;
 
+    // MODE 3: the row is output pixel (b, oy, ox) of the convolution
+    int cb = 0, coy = 0, cox = 0;
+    if (MODE == 3) {
+        const int hw = args.conv.oh * args.conv.ow;
+        cb = row / hw;
+        coy = (row - cb * hw) / args.conv.ow;
+        cox = row - cb * hw - coy * args.conv.ow;
+    }
+
     // issue every load of this thread first
     uint4 raw[GPS][2];
 #pragma unroll
     for (int gi = 0; gi < GPS; ++gi) {
         const int g = g0 + slot + gi * slots;
         if (gi < gps && slot < slots && g < g1) {
-            if (!DYN || g * 256 + t * 16 < k) {
+            const int kel = g * 256 + t * 16;            // first of this thread's 16 elements
+            raw[gi][0] = make_uint4(0u, 0u, 0u, 0u);     // zeros past the row / outside the image
+            raw[gi][1] = make_uint4(0u, 0u, 0u, 0u);
+            if (MODE == 3) {
+                // im2col gather from NHWC: tap (ky, kx), 16 channels from c0
+                const ConvGeom &cg = args.conv;
+                if (kel < k) {
+                    const int tap = kel / cg.c, c0 = kel - tap * cg.c;
+                    const int ky = tap / cg.kw, kx = tap - ky * cg.kw;
+                    const int iy = coy * cg.stride - cg.pad + ky * cg.dil;
+                    const int ix = cox * cg.stride - cg.pad + kx * cg.dil;
+                    if (iy >= 0 && iy < cg.h && ix >= 0 && ix < cg.w) {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(
+                            J.a + (((size_t)cb * cg.h + iy) * cg.w + ix) * cg.c + c0);
+                        raw[gi][0] = __ldg(src);
+                        raw[gi][1] = __ldg(src + 1);
+                    }
+                }
+            } else if (MODE == 4) {
+                // weight row o in the im2col order from OIHW: w[o, c0 + e, ky, kx]
+                const ConvGeom &cg = args.conv;
+                if (kel < k) {
+                    const int tap = kel / cg.c, c0 = kel - tap * cg.c;
+                    const int taps = cg.kh * cg.kw;
+                    const unsigned short *w = reinterpret_cast<const unsigned short *>(J.a) +
+                                              ((size_t)row * cg.c + c0) * taps + tap;
+                    uint32_t v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        v[e] = (uint32_t)__ldg(w + (size_t)(2 * e) * taps) |
+                               ((uint32_t)__ldg(w + (size_t)(2 * e + 1) * taps) << 16);
+                    raw[gi][0] = make_uint4(v[0], v[1], v[2], v[3]);
+                    raw[gi][1] = make_uint4(v[4], v[5], v[6], v[7]);
+                }
+            } else if (!DYN || kel < k) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(arow + (size_t)g * 256 + t * 16);
                 raw[gi][0] = __ldg(src);
                 raw[gi][1] = __ldg(src + 1);
-            } else {        // past the end of the row: zeros rotate to zeros
-                raw[gi][0] = make_uint4(0u, 0u, 0u, 0u);
-                raw[gi][1] = make_uint4(0u, 0u, 0u, 0u);
             }
         }
     }
@@ -446,7 +489,7 @@ static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int
 template <int MODE>
 static cudaError_t launch_gps(cudaLaunchConfig_t &cfg, const RQArgs &args, bool half, int max_gps, int max_slots,
                               int max_local) {
-    if (half && MODE != 2) {
+    if (half && MODE < 2) {
         switch (max_gps) {
             case 1: return launch_slots<1, true, MODE>(cfg, args, max_slots, max_local);
             case 2: return launch_slots<2, true, MODE>(cfg, args, max_slots, max_local);
@@ -506,7 +549,8 @@ static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, bool h
     return (size_t)ms * (half ? kXchHalf : kXchFull) * 8 + (size_t)ml * y_group_stride(half) * 4;
 }
 
-cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl) {
+cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl,
+                                const ConvGeom *conv) {
     int dev = 0, num_sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
@@ -516,7 +560,7 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         // its own row length (a shared shape would size every CTA for the
         // longest rows)
         for (int jj = 0; jj < njobs; ++jj) {
-            cudaError_t e = launch_rotate_quant(1, rows, probs + jj, stream, pdl);
+            cudaError_t e = launch_rotate_quant(1, rows, probs + jj, stream, pdl, conv);
             if (e != cudaSuccess) return e;
         }
         return cudaSuccess;
@@ -525,7 +569,8 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
     // CTAs fit beside the GEMM's (INT4 weight conversion is offline: full)
     bool int4 = false;
     for (int j = 0; j < njobs; ++j) int4 = int4 || probs[j].int4;
-    const bool half = few_rows && !int4;
+    const int conv_mode = conv ? conv->mode : 0;
+    const bool half = few_rows && !int4 && conv_mode == 0;
     const int parts = rq_parts(njobs, rows, probs, num_sms, half);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -551,6 +596,7 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         rq_smem_bytes(njobs, probs, parts, half, &max_slots, &max_gps, &max_local) <= (size_t)kSlotsSmemMax) {
         RQArgs args;
         memset(&args, 0, sizeof(args));
+        if (conv) args.conv = *conv;
         bool dyn = false;
         args.njobs = njobs;
         args.rows = (int)rows;
@@ -571,6 +617,8 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
             rq_shape((groups + parts - 1) / parts, &J.gps, &J.slots);
             dyn = dyn || J.group != 256 || (J.k & 255) != 0;
         }
+        if (conv_mode == 3) return launch_gps<3>(cfg, args, false, max_gps, max_slots, max_local);
+        if (conv_mode == 4) return launch_gps<4>(cfg, args, false, max_gps, max_slots, max_local);
         if (int4) return launch_gps<2>(cfg, args, half, max_gps, max_slots, max_local);
         if (dyn) return launch_gps<1>(cfg, args, half, max_gps, max_slots, max_local);
         return launch_gps<0>(cfg, args, half, max_gps, max_slots, max_local);

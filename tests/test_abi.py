@@ -171,3 +171,25 @@ def test_weight4_validation(lib):
     assert lib.convrot_linear_w4a8(257, 1, job, P(0x300000), 1 << 30, P(0)) == 3     # m > 256
     assert lib.convrot_linear_w4a8(0, 1, job, P(0x300000), 1 << 30, P(0)) == 1
     assert lib.convrot_linear_w4a8_workspace_bytes(12, 1, job) > 0
+
+
+def test_conv2d_shape_and_validation(lib):
+    import rotated_int8_quantized_b200 as cr
+    g = cr.convrot_conv2d_t(1, 64, 64, 512, 3, 3, 1, 1, 1)
+    oh, ow = ctypes.c_int32(), ctypes.c_int32()
+    assert lib.convrot_conv2d_shape(ctypes.byref(g), ctypes.byref(oh), ctypes.byref(ow)) == 0
+    assert (oh.value, ow.value) == (64, 64)
+    g2 = cr.convrot_conv2d_t(2, 9, 7, 128, 3, 3, 2, 1, 1)
+    assert lib.convrot_conv2d_shape(ctypes.byref(g2), ctypes.byref(oh), ctypes.byref(ow)) == 0
+    assert (oh.value, ow.value) == (5, 4)
+    bad = cr.convrot_conv2d_t(1, 8, 8, 24, 3, 3, 1, 1, 1)      # channels not a multiple of 16
+    assert lib.convrot_conv2d_shape(ctypes.byref(bad), None, None) == 3
+    h = cr.convrot_weight_t()
+    P = ctypes.c_void_p
+    assert lib.convrot_weight_init(ctypes.byref(h), P(0x10000), P(0x20000), 64, 3 * 3 * 512, 256) == 0
+    assert lib.convrot_conv2d_workspace_bytes(ctypes.byref(g), ctypes.byref(h)) > 64 * 64 * 4608
+    assert lib.convrot_weight_init(ctypes.byref(h), P(0x10000), P(0x20000), 64, 3 * 3 * 96, 32) == 0
+    g3 = cr.convrot_conv2d_t(1, 8, 8, 96, 3, 3, 1, 1, 1)
+    assert lib.convrot_conv2d_workspace_bytes(ctypes.byref(g3), ctypes.byref(h)) > 0
+    g4 = cr.convrot_conv2d_t(1, 8, 8, 96, 1, 1, 1, 0, 1)         # k mismatch
+    assert lib.convrot_conv2d_workspace_bytes(ctypes.byref(g4), ctypes.byref(h)) == 0

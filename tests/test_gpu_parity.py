@@ -618,3 +618,38 @@ def test_w4a8_qwen_decode_layer_sampled(cr):
         assert np.array_equal(w4.q[rw].cpu().numpy(), packed_ref)
         ref = oracle.linear_w4a8(lin.x_np(), packed_ref, s_ref)
         assert np.array_equal(to_bits(y[:, rw]), ref["y"])
+
+
+
+# ---------------------------------------------------------------- convolutions (int8_convrot)
+# (n, h, w, c, o, k, stride, pad, dil): 3x3 with padding, stride 2, dilation,
+# a 1x1, channels below 256 (dynamic group), a ragged last chunk, enough rows
+# for the large-M GEMM path, and a few rows (stream-K path)
+CONV_CASES = [
+    (1, 8, 8, 256, 64, 3, 1, 1, 1),
+    (2, 9, 7, 128, 96, 3, 2, 1, 1),
+    (1, 10, 10, 64, 32, 3, 1, 2, 2),
+    (1, 16, 16, 512, 256, 1, 1, 0, 1),
+    (1, 12, 12, 96, 48, 3, 1, 1, 1),
+    (1, 32, 32, 128, 128, 3, 1, 1, 1),
+    (1, 3, 3, 256, 64, 3, 1, 0, 1),
+]
+
+
+@pytest.mark.parametrize("n,h,w,c,o,k,stride,pad,dil", CONV_CASES)
+def test_conv2d_int8_bit_exact(cr, n, h, w, c, o, k, stride, pad, dil):
+    seed = n * 1000 + h * 10 + c + o + k
+    cs = synth.outlier_scale_fraction(synth.stream_key(seed, 2), c, 0.02, 30.0)
+    x_bits = synth.draw_np(synth.stream_key(seed, 0), n * h * w, c, 1.0, cs).reshape(n, h, w, c)
+    w_bits = synth.draw_np(synth.stream_key(seed, 1), o, c * k * k, synth.W_SIGMA).reshape(o, c, k, k)
+    group = cr.convrot_dynamic_group(c)
+    ref = oracle.conv2d_int8(x_bits, w_bits, stride, pad, dil, group=group)
+    wq = cr.quantize_conv_weight(from_bits(w_bits))
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.q.cpu().numpy(), ref["wq"]) and np.array_equal(wq.scale.cpu().numpy(), ref["sw"])
+    y = cr.conv2d_int8(from_bits(x_bits), wq, k, k, stride, pad, dil)
+    cr.convrot_device_status()
+    yb = to_bits(y)
+    assert yb.shape == ref["y"].shape
+    assert rel_err(yb, ref["y"]) <= TOL
+    assert np.array_equal(yb, ref["y"])
