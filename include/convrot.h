@@ -342,9 +342,11 @@ size_t convrot_linear_w4a8_workspace_bytes(int64_t m, int count, const convrot_l
  * x[b, oy*stride - pad + ky*dil, ox*stride - pad + kx*dil, c] (zero outside
  * the image); the weight row o holds w[o, c, ky, kx] in the same order; the
  * rotation groups lie inside one tap's channels (group divides C), so
- * rotating both sides preserves the convolution.  The activation prologue
- * gathers the im2col rows straight from the NHWC input (no BF16 im2col copy)
- * and writes their INT8 codes to the workspace.
+ * rotating both sides preserves the convolution.  For kernels larger than
+ * 1x1 every input pixel is rotated once (FP32 copy and its maximum in the
+ * workspace) and a second kernel gathers the im2col rows from those pixels
+ * and quantises them (a row's maximum is the maximum of its pixels'); a 1x1
+ * convolution gathers and rotates in one step.  No BF16 im2col copy exists.
  */
 typedef struct {
     int32_t n, h, w, c;             /* input NHWC: batch, height, width, channels (c % 16 == 0) */
@@ -369,8 +371,8 @@ size_t convrot_conv2d_workspace_bytes(const convrot_conv2d_t *g, const convrot_w
 /*
  * y [n, oh, ow, w->n] (NHWC, BF16) = the INT8 ConvRot convolution of x
  * [n, h, w, c] (NHWC, BF16) with the handle from convrot_quantize_conv_weight.
- * Two launches: the gathering activation prologue, then the INT8 GEMM with
- * M = n * oh * ow, N = c_out, K = kh * kw * c.
+ * Launches: the activation prologue (two kernels, one for 1x1), then the
+ * INT8 GEMM with M = n * oh * ow, N = c_out, K = kh * kw * c.
  */
 convrot_status_t convrot_conv2d_int8(const void *x_nhwc_bf16, const convrot_conv2d_t *g, const convrot_weight_t *w,
                                      void *y_nhwc_bf16, void *ws, size_t ws_bytes, void *stream);

@@ -531,12 +531,21 @@ convrot_status_t convrot_quantize_conv_weight(const void *w_oihw_bf16, const con
 }
 
 namespace {
+// Workspace: [GEMM scratch][xq M x K][sx M] and, for kernels larger than
+// 1x1, [every pixel rotated once: FP32 n*h*w x c][the pixels' maxima].
+bool conv_two_pass(const convrot::ConvGeom &cg) { return cg.kh * cg.kw > 1; }
+
 size_t conv_layout(const convrot::ConvGeom &cg, const convrot_weight_t *w, int sms, convrot::GemmPlan *p,
                    size_t *gemm_bytes) {
     const int64_t m = (int64_t)cg.n * cg.oh * cg.ow;
     convrot::plan_gemm(m, w->n, w->k, sms, p);
     *gemm_bytes = round256(p->ws_bytes);
-    return *gemm_bytes + round256((size_t)m * (size_t)w->k) + round256((size_t)m * 4);
+    size_t t = *gemm_bytes + round256((size_t)m * (size_t)w->k) + round256((size_t)m * 4);
+    if (conv_two_pass(cg)) {
+        const size_t pix = (size_t)cg.n * cg.h * cg.w;
+        t += round256(pix * (size_t)cg.c * 4) + round256(pix * 4);
+    }
+    return t;
 }
 }  // namespace
 
@@ -570,10 +579,25 @@ convrot_status_t convrot_conv2d_int8(const void *x_nhwc_bf16, const convrot_conv
     int8_t *xq = reinterpret_cast<int8_t *>(base + gb);
     float *sx = reinterpret_cast<float *>(base + gb + round256((size_t)m * (size_t)w->k));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cg.mode = 3;
-    convrot::RQProblem rq = {x_nhwc_bf16, w->k, w->group, xq, sx, 0};
-    cudaError_t e = convrot::launch_rotate_quant(1, m, &rq, st, true, &cg);
-    if (e != cudaSuccess) return from_cuda(e);
+    cudaError_t e;
+    if (conv_two_pass(cg)) {
+        // every input pixel rotated once (its C channels, FP32) with its
+        // maximum; then the im2col rows gathered from them and quantised
+        const size_t pix = (size_t)cg.n * cg.h * cg.w;
+        float *yrot = reinterpret_cast<float *>(base + gb + round256((size_t)m * (size_t)w->k) + round256((size_t)m * 4));
+        float *pmax = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(yrot) + round256(pix * (size_t)cg.c * 4));
+        cg.mode = 5;
+        convrot::RQProblem rq = {x_nhwc_bf16, g->c, w->group, reinterpret_cast<int8_t *>(yrot), pmax, 0};
+        e = convrot::launch_rotate_quant(1, (int64_t)pix, &rq, st, true, &cg);
+        if (e != cudaSuccess) return from_cuda(e);
+        e = convrot::launch_conv_gather_quant(yrot, pmax, cg, m, xq, sx, st);
+        if (e != cudaSuccess) return from_cuda(e);
+    } else {
+        cg.mode = 3;
+        convrot::RQProblem rq = {x_nhwc_bf16, w->k, w->group, xq, sx, 0};
+        e = convrot::launch_rotate_quant(1, m, &rq, st, true, &cg);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
     convrot::GemmProblem gp = {m, w->n, w->k, xq, sx, w->q, w->scale, static_cast<__nv_bfloat16 *>(y_nhwc_bf16),
                                nullptr, nullptr};
     return from_cuda(convrot::launch_gemm_i8(p, &gp, base, st, true, true));

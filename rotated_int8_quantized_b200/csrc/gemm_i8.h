@@ -109,7 +109,7 @@ struct RQProblem {
 // Geometry of a convolution whose im2col rows (mode 3) or OIHW weight rows
 // (mode 4) the rotation kernel gathers.
 struct ConvGeom {
-    int mode;           // 3: activations (NHWC input), 4: weights (OIHW)
+    int mode;           // 3: activations (NHWC input), 4: weights (OIHW), 5: pixels rotated once
     int n, h, w, c;     // input batch, height, width, channels
     int kh, kw, stride, pad, dil;
     int oh, ow;         // output height and width
@@ -119,6 +119,11 @@ struct ConvGeom {
 // count) in one launch; `conv`: the rows are gathered from a convolution.
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl,
                                 const ConvGeom *conv = nullptr);
+
+// Convolution im2col codes from pixels rotated once (yrot FP32 [n*h*w, c],
+// pmax [n*h*w]): codes xq [rows, kh*kw*c] and scales sx [rows].
+cudaError_t launch_conv_gather_quant(const float *yrot, const float *pmax, const ConvGeom &g, int64_t rows,
+                                     int8_t *xq, float *sx, cudaStream_t stream);
 
 // ------------------------------------------------------------------ tensor-wise INT8 (embedding table)
 cudaError_t launch_quantize_tensor(const void *a, int64_t count, int8_t *q, float *scale, cudaStream_t stream);

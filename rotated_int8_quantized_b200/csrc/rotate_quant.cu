@@ -267,7 +267,9 @@ __device__ __forceinline__ void cluster_wait() {
 // MODE 0: INT8 codes, groups of 256; 1: INT8, any group (DYN below); 2: INT4
 // weight codes (levels -7..7, scale a/7), packed two per byte, any group;
 // 3: INT8 codes of the im2col rows of a convolution, gathered from NHWC
-// input; 4: INT8 codes of a convolution's OIHW weight in the im2col order.
+// input; 4: INT8 codes of a convolution's OIHW weight in the im2col order;
+// 5: the rotated FP32 rows themselves and their maxima (no quantisation):
+// every input pixel of a convolution rotated once, for conv_gather_quant.
 template <int GPS, bool HALF, int MODE>
 __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
@@ -454,14 +456,21 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                 y[4 * i + 2] = f.z;
                 y[4 * i + 3] = f.w;
             }
-            if (MODE == 2)      // packed INT4: row stride k/2 bytes
+            if (MODE == 5) {    // rotated values themselves (FP32 [rows, k], in J.q)
+                float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(J.q) + (size_t)row * k +
+                                                         (size_t)g0 * 256 + c * 16);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+            } else if (MODE == 2) {     // packed INT4: row stride k/2 bytes
                 *reinterpret_cast<uint2 *>(J.q + (size_t)row * (k / 2) + (size_t)g0 * 128 + c * 8) =
                     quant16_int4(y, rs, mask);
-            else
+            } else {
                 *reinterpret_cast<uint4 *>(qrow + c * 16) = quant16(y, rs, mask);
+            }
         }
     }
-    if (tid == 0 && part == 0) J.s[row] = rs.s;
+    // MODE 5 keeps the row maximum (the scale is a later, per-im2col-row step)
+    if (tid == 0 && part == 0) J.s[row] = MODE == 5 ? rmax : rs.s;
     if (C > 1) {
         __syncwarp();
         cluster_wait();   // peers may still read part_max until they arrive
@@ -617,6 +626,7 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
             rq_shape((groups + parts - 1) / parts, &J.gps, &J.slots);
             dyn = dyn || J.group != 256 || (J.k & 255) != 0;
         }
+        if (conv_mode == 5) return launch_gps<5>(cfg, args, false, max_gps, max_slots, max_local);
         if (conv_mode == 3) return launch_gps<3>(cfg, args, false, max_gps, max_slots, max_local);
         if (conv_mode == 4) return launch_gps<4>(cfg, args, false, max_gps, max_slots, max_local);
         if (int4) return launch_gps<2>(cfg, args, half, max_gps, max_slots, max_local);
@@ -626,6 +636,90 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
     // unreachable within the shapes the API accepts (k <= 133120 stages in
     // at most 114 KB per CTA with 8 parts)
     return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------
+// Convolutions, second pass: the INT8 codes of im2col row m from the pixels'
+// rotated values (rotate_quant_rows_slots MODE 5).  A row's maximum is the
+// maximum over its taps of the pixels' maxima (padding taps are zeros), so
+// the scale and codes equal those of rotating and quantising the gathered
+// row directly; each pixel is rotated once instead of kh * kw times.
+// One warp per row (grid-stride over warps), 16 codes per lane per step.
+// ---------------------------------------------------------------------------
+constexpr int kGatherThreads = 256;
+
+__global__ void __launch_bounds__(kGatherThreads) conv_gather_quant_kernel(const float *yrot, const float *pmax,
+                                                                          const __grid_constant__ ConvGeom g,
+                                                                          int64_t rows, int8_t *xq, float *sx) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int taps = g.kh * g.kw;
+    const int k = taps * g.c;
+    const int chunks = k / 16;
+    const int hw = g.oh * g.ow;
+    const int64_t nwarps = (int64_t)gridDim.x * (kGatherThreads / 32);
+    for (int64_t row = (int64_t)blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5); row < rows; row += nwarps) {
+        const int b = (int)(row / hw);
+        const int oy = (int)(row - (int64_t)b * hw) / g.ow;
+        const int ox = (int)(row - (int64_t)b * hw) - oy * g.ow;
+        float m = 0.f;
+        for (int t = lane; t < taps; t += 32) {
+            const int ky = t / g.kw, kx = t - ky * g.kw;
+            const int iy = oy * g.stride - g.pad + ky * g.dil, ix = ox * g.stride - g.pad + kx * g.dil;
+            if (iy >= 0 && iy < g.h && ix >= 0 && ix < g.w)
+                m = fmaxf(m, __ldg(pmax + ((size_t)b * g.h + iy) * g.w + ix));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const RowScale rs = make_row_scale(m);
+        for (int c0 = 0; c0 < chunks; c0 += 32) {
+            const int c = c0 + lane;
+            const unsigned mask = __ballot_sync(0xffffffffu, c < chunks);
+            if (c < chunks) {
+                const int kel = c * 16;
+                const int tap = kel / g.c, ch = kel - tap * g.c;
+                const int ky = tap / g.kw, kx = tap - ky * g.kw;
+                const int iy = oy * g.stride - g.pad + ky * g.dil, ix = ox * g.stride - g.pad + kx * g.dil;
+                float y[16];
+                if (iy >= 0 && iy < g.h && ix >= 0 && ix < g.w) {
+                    const float4 *src =
+                        reinterpret_cast<const float4 *>(yrot + (((size_t)b * g.h + iy) * g.w + ix) * g.c + ch);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float4 f = __ldg(src + i);
+                        y[4 * i] = f.x;
+                        y[4 * i + 1] = f.y;
+                        y[4 * i + 2] = f.z;
+                        y[4 * i + 3] = f.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) y[e] = 0.f;
+                }
+                *reinterpret_cast<uint4 *>(xq + row * (int64_t)k + kel) = quant16(y, rs, mask);
+            }
+        }
+        if (lane == 0) sx[row] = rs.s;
+    }
+}
+
+cudaError_t launch_conv_gather_quant(const float *yrot, const float *pmax, const ConvGeom &g, int64_t rows,
+                                     int8_t *xq, float *sx, cudaStream_t stream) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = (int64_t)sms * 8;
+    const int64_t blocks = (rows + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)(blocks < cap ? blocks : cap));
+    cfg.blockDim = dim3(kGatherThreads);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, conv_gather_quant_kernel, yrot, pmax, g, rows, xq, sx);
 }
 
 }  // namespace convrot
