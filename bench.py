@@ -68,11 +68,15 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
-def kernel_source_hash() -> str:
+GEMM_SOURCES = ("common.cuh", "gemm_i8.cu", "gemm_i8.h")
+
+
+def kernel_source_hash(only=None) -> str:
+    """Hash of the CUDA sources (all of them, or the named files)."""
     csrc = os.path.join(ROOT, "rotated_int8_quantized_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
+        if f.endswith((".cu", ".cuh", ".h")) and (only is None or f in only):
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
@@ -80,11 +84,12 @@ def kernel_source_hash() -> str:
 
 def profiled_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
-    summary, if it was taken on the current kernel sources (else None)."""
+    summary, if it was taken on the current sources of that kernel (the GEMM's
+    files; else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.tsv")
     if not os.path.exists(path):
         return None
-    want = kernel_source_hash()
+    want = kernel_source_hash(GEMM_SOURCES)
     with open(path) as f:
         for line in f:
             if line.startswith("#") or not line.strip():
@@ -746,6 +751,7 @@ def run_ours(args):
                                        "value": bytes_step / per_linear_t / 1e9,
                                        "launches_per_step": 2 * len(lins)},
             "secondary": secondary, "more": others or None, "kernel_sources": kernel_source_hash(),
+            "gemm_sources": kernel_source_hash(GEMM_SOURCES),
         }
         print(json.dumps(line), flush=True)
     del graph

@@ -53,8 +53,15 @@ __device__ __forceinline__ RowScale make_row_scale(float amax) {
     rs.s = __fdiv_rn(amax, 127.0f);
     rs.zero = (amax == 0.0f);
     rs.r = rs.zero ? 0.0f : __frcp_rn(rs.s);
-    rs.fast = !rs.zero && isfinite(rs.r);
+    // a subnormal s carries less than 24 bits, so the bound below needs a
+    // normal one; rows that small take the division
+    rs.fast = !rs.zero && isfinite(rs.r) && rs.s >= 1.17549435e-38f;
     return rs;
+}
+
+// The low bytes of a, b, c, d as one word (a in byte 0).
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 // q = clamp(rne(fl(y / s)), -127, 127) for 16 consecutive values y: the
@@ -71,43 +78,93 @@ __device__ __forceinline__ RowScale make_row_scale(float amax) {
 // |t - fl(y/s)| < 2.3e-5.  When t is more than 3e-5 away from every
 // half-integer, fl(y/s) rounds to the same integer as t; otherwise (about
 // 6e-5 of the elements) the IEEE division is evaluated.
-// The fast path is straight-line code over the 16 values (independent work
-// for the scheduler); the division runs only where some thread of the warp
-// needs it.  Every thread of `mask` (the active threads) must call it.
 // Rounding to the nearest integer, ties to even, on the FP32 pipe instead of
 // the conversion unit: for |t| < 2^22 the sum fl(t + 1.5 * 2^23) has an ulp
 // of 1, so the addition itself rounds t to an integer (round-to-nearest-even
-// is the FP32 mode) and that integer sits in the low mantissa bits of the sum.
+// is the FP32 mode), and the sum's low byte is that integer's two's
+// complement byte (1.5 * 2^23 has a zero low byte).  With a normal s,
+// |t| <= 127 (1 + 3 * 2^-24), so the fast path needs no clamp.
+// The fast path is straight-line code over the 16 values (independent work
+// for the scheduler), with one predicate accumulating "near a half-integer
+// (or NaN)"; the division runs only where some thread of the warp needs
+// it.  Every thread of `mask` (the active threads) must call it.
 constexpr float kRoundMagic = 12582912.0f;          // 1.5 * 2^23
 constexpr int kRoundMagicBits = 0x4B400000;         // its bit pattern
 
 __device__ __forceinline__ uint4 quant16(const float (&y)[16], const RowScale &rs, unsigned mask) {
-    int code[16];
-    bool slow = false;
+    uint32_t b[16];
+    bool near = false;
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const float t = __fmul_rn(y[e], rs.r);
         const float big = __fadd_rn(t, kRoundMagic);
-        code[e] = __float_as_int(big) - kRoundMagicBits;            // rne(t)
-        slow |= !(fabsf(__fsub_rn(t, __fsub_rn(big, kRoundMagic))) < 0.49997f);
+        b[e] = __float_as_uint(big);                                 // low byte: rne(t)
+        near |= !(fabsf(__fsub_rn(t, __fsub_rn(big, kRoundMagic))) < 0.49997f);   // NaN too
     }
-    slow = slow || !rs.fast;
+    const bool slow = near || !rs.fast;      // zero rows too (their codes are set below)
     if (__any_sync(mask, slow) && slow) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const float t = __fmul_rn(y[e], rs.r);
             const float f = __fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic);
-            if (!rs.fast || !(fabsf(__fsub_rn(t, f)) < 0.49997f))
-                code[e] = __float_as_int(__fadd_rn(__fdiv_rn(y[e], rs.s), kRoundMagic)) - kRoundMagicBits;
+            if (!rs.fast || !(fabsf(__fsub_rn(t, f)) < 0.49997f)) {
+                const int c = __float_as_int(__fadd_rn(__fdiv_rn(y[e], rs.s), kRoundMagic)) - kRoundMagicBits;
+                b[e] = (uint32_t)min(max(c, -127), 127);
+            }
         }
     }
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (rs.zero) return make_uint4(0u, 0u, 0u, 0u);
+    return make_uint4(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]),
+                      pack_low_bytes(b[8], b[9], b[10], b[11]), pack_low_bytes(b[12], b[13], b[14], b[15]));
+}
+
+
+// The same codes with the FP32 pair instructions of sm_100 (two values per
+// multiply or add): identical arithmetic, each operation still rounded to
+// nearest even per value, half the instructions on the FP32 pipe.
+__device__ __forceinline__ uint64_t pack_f32x2(float a, float b) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(a), "f"(b));
+    return d;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t d, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(d));
+}
+
+__device__ __forceinline__ uint4 quant16x2(const float (&y)[16], const RowScale &rs, unsigned mask) {
+    uint32_t b[16];
+    bool near = false;
+    const uint64_t r2 = pack_f32x2(rs.r, rs.r), m2 = pack_f32x2(kRoundMagic, kRoundMagic);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        const int c = rs.zero ? 0 : min(max(code[e], -127), 127);
-        w[e >> 2] |= (uint32_t)(c & 0xFF) << (8 * (e & 3));
+    for (int i = 0; i < 8; ++i) {
+        uint64_t t2, big2, rnd2, d2;
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(pack_f32x2(y[2 * i], y[2 * i + 1])), "l"(r2));
+        asm("add.rn.f32x2 %0, %1, %2;" : "=l"(big2) : "l"(t2), "l"(m2));
+        asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rnd2) : "l"(big2), "l"(m2));
+        asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d2) : "l"(t2), "l"(rnd2));
+        float d0, d1, b0, b1;
+        unpack_f32x2(d2, d0, d1);
+        unpack_f32x2(big2, b0, b1);
+        b[2 * i] = __float_as_uint(b0);                               // low byte: rne(t)
+        b[2 * i + 1] = __float_as_uint(b1);
+        near |= !(fabsf(d0) < 0.49997f);                              // NaN too
+        near |= !(fabsf(d1) < 0.49997f);
     }
-    return make_uint4(w[0], w[1], w[2], w[3]);
+    const bool slow = near || !rs.fast;      // zero rows too (their codes are set below)
+    if (__any_sync(mask, slow) && slow) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float t = __fmul_rn(y[e], rs.r);
+            const float f = __fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic);
+            if (!rs.fast || !(fabsf(__fsub_rn(t, f)) < 0.49997f)) {
+                const int c = __float_as_int(__fadd_rn(__fdiv_rn(y[e], rs.s), kRoundMagic)) - kRoundMagicBits;
+                b[e] = (uint32_t)min(max(c, -127), 127);
+            }
+        }
+    }
+    if (rs.zero) return make_uint4(0u, 0u, 0u, 0u);
+    return make_uint4(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]),
+                      pack_low_bytes(b[8], b[9], b[10], b[11]), pack_low_bytes(b[12], b[13], b[14], b[15]));
 }
 
 
@@ -221,6 +278,7 @@ struct RQJobDev {
 struct RQArgs {
     int njobs, rows;
     int parts;              // CTAs (a thread-block cluster) per row
+    int rpc;                // rows per CTA: 1, or several short rows (parts == 1, at most 2 slots a row)
     ConvGeom conv;          // MODE 3 / 4: the convolution the rows come from
     RQJobDev job[kMaxJobs];
 };
@@ -251,6 +309,12 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Layout of the rotated pixels (MODE 5): FP32 [pixels, c], and inside each
+// 16-value chunk ci of a pixel, float4 part j stored at position
+// j ^ yrot_swizzle(ci), so that 8 lanes reading 8 consecutive chunks one
+// float4 part at a time hit 8 different 16-byte bank groups.
+__host__ __device__ __forceinline__ int yrot_swizzle(int ci) { return (ci >> 1) & 3; }
+
 // One row per CTA (parts == 1) or per cluster of `parts` CTAs: CTA p of the
 // cluster rotates groups [p*G/parts, (p+1)*G/parts) of the row, the row
 // maximum is combined through distributed shared memory, then each CTA
@@ -270,7 +334,7 @@ __device__ __forceinline__ void cluster_wait() {
 // input; 4: INT8 codes of a convolution's OIHW weight in the im2col order;
 // 5: the rotated FP32 rows themselves and their maxima (no quantisation):
 // every input pixel of a convolution rotated once, for conv_gather_quant.
-template <int GPS, bool HALF, int MODE>
+template <int GPS, bool HALF, int MODE, bool MR = false>
 __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
     constexpr bool DYN = MODE != 0;
@@ -282,8 +346,13 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     pdl_launch_dependents();
 
     const int C = args.parts;
-    const int part = (int)(blockIdx.x % (unsigned)C);
-    const int rowid = (int)(blockIdx.x / (unsigned)C);
+    // several short rows per CTA: 16 or 32 threads a row, each row inside one warp
+    const int R = MR ? args.rpc : 1;
+    const int row_threads = (int)blockDim.x / R;
+    const int rloc = R > 1 ? (int)threadIdx.x / row_threads : 0;
+    const int part = R > 1 ? 0 : (int)(blockIdx.x % (unsigned)C);
+    const int rowid = R > 1 ? (int)blockIdx.x * R + rloc : (int)(blockIdx.x / (unsigned)C);
+    if (R > 1 && rowid >= args.rows * args.njobs) return;     // the last CTA's missing rows (whole warps or half-warps)
     const int jb = rowid / args.rows;
     const int row = rowid - jb * args.rows;
     const RQJobDev &J = args.job[jb];
@@ -291,11 +360,13 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     const int groups = DYN ? (k + 255) >> 8 : k >> 8;     // 256-element chunks
     const int g0 = part * groups / C, g1 = (part + 1) * groups / C;
     double *xch = reinterpret_cast<double *>(rq_smem);                    // slots * 272 doubles
-    float *ybuf = reinterpret_cast<float *>(rq_smem + (size_t)(blockDim.x >> 4) * kXchStride * 8);
+    float *ybuf = reinterpret_cast<float *>(rq_smem + (size_t)(blockDim.x >> 4) * kXchStride * 8) +
+                  (size_t)rloc * (g1 - g0) * y_group_stride(HALF);
 
-    const int tid = threadIdx.x;
+    const int tid = (int)threadIdx.x - rloc * row_threads;     // thread within its row
     const int slot = tid >> 4, t = tid & 15;
-    const unsigned half_mask = 0xFFFFu << (16 * (slot & 1));
+    const int cta_slot = R > 1 ? (int)(threadIdx.x >> 4) : slot;      // half-warp within the CTA
+    const unsigned half_mask = 0xFFFFu << (16 * (cta_slot & 1));
     const __nv_bfloat16 *arow = J.a + (size_t)row * k;
 
     // MODE 3: the row is output pixel (b, oy, ox) of the convolution
@@ -355,7 +426,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
         }
     }
 
-    double *xb = xch + slot * kXchStride;
+    double *xb = xch + cta_slot * kXchStride;
     float amax = 0.f;
 #pragma unroll
     for (int gi = 0; gi < GPS; ++gi) {
@@ -412,13 +483,20 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     }
 
     // maximum over this CTA's part of the row
+    float rmax;
+    if (R > 1) {
+        const unsigned row_mask = row_threads == 32 ? 0xffffffffu : half_mask;
+        for (int o = row_threads >> 1; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(row_mask, amax, o));
+        rmax = amax;
+    } else {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const int warp = tid >> 5, lane = tid & 31, nwarps = (blockDim.x + 31) >> 5;
-    if (lane == 0) red[warp] = amax;
-    __syncthreads();
-    float rmax = red[0];
-    for (int w = 1; w < nwarps; ++w) rmax = fmaxf(rmax, red[w]);
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const int warp = tid >> 5, lane = tid & 31, nwarps = (blockDim.x + 31) >> 5;
+        if (lane == 0) red[warp] = amax;
+        __syncthreads();
+        rmax = red[0];
+        for (int w = 1; w < nwarps; ++w) rmax = fmaxf(rmax, red[w]);
+    }
     if (C > 1) {
         // combine the parts of the row across the cluster
         if (tid == 0) part_max = rmax;
@@ -440,7 +518,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     int8_t *qrow = J.q + (size_t)row * k + (size_t)g0 * 256;
     int chunks = (g1 - g0) * 16;
     if (DYN && g0 * 256 + chunks * 16 > k) chunks = (k - g0 * 256) / 16;     // partial last chunk
-    for (int c0 = 0; c0 < chunks; c0 += blockDim.x) {
+    for (int c0 = 0; c0 < chunks; c0 += (R > 1 ? (unsigned)row_threads : blockDim.x)) {
         const int c = c0 + tid;
         const unsigned mask = __ballot_sync(__activemask(), c < chunks);
         if (c < chunks) {
@@ -456,11 +534,13 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                 y[4 * i + 2] = f.z;
                 y[4 * i + 3] = f.w;
             }
-            if (MODE == 5) {    // rotated values themselves (FP32 [rows, k], in J.q)
+            if (MODE == 5) {    // rotated values themselves (FP32 [rows, k], in J.q), float4 parts swizzled
                 float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(J.q) + (size_t)row * k +
                                                          (size_t)g0 * 256 + c * 16);
+                const int sw = yrot_swizzle(c);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+                for (int i = 0; i < 4; ++i)
+                    dst[i ^ sw] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
             } else if (MODE == 2) {     // packed INT4: row stride k/2 bytes
                 *reinterpret_cast<uint2 *>(J.q + (size_t)row * (k / 2) + (size_t)g0 * 128 + c * 8) =
                     quant16_int4(y, rs, mask);
@@ -477,27 +557,30 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     }
 }
 
-template <int GPS, bool HALF, int MODE>
+template <int GPS, bool HALF, int MODE, bool MR = false>
 static cudaError_t launch_slots(cudaLaunchConfig_t &cfg, const RQArgs &args, int max_slots, int max_local_groups) {
-    cfg.blockDim = dim3(max_slots * 16);
-    cfg.dynamicSmemBytes =
-        (size_t)max_slots * (HALF ? kXchHalf : kXchFull) * 8 + (size_t)max_local_groups * y_group_stride(HALF) * 4;
+    cfg.blockDim = dim3(max_slots * 16 * args.rpc);
+    cfg.dynamicSmemBytes = ((size_t)max_slots * (HALF ? kXchHalf : kXchFull) * 8 +
+                            (size_t)max_local_groups * y_group_stride(HALF) * 4) * args.rpc;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(rotate_quant_rows_slots<GPS, HALF, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(rotate_quant_rows_slots<GPS, HALF, MODE, MR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSlotsSmemMax);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev] = true;
     }
-    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS, HALF, MODE>, args);
+    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_slots<GPS, HALF, MODE, MR>, args);
 }
 
 template <int MODE>
 static cudaError_t launch_gps(cudaLaunchConfig_t &cfg, const RQArgs &args, bool half, int max_gps, int max_slots,
                               int max_local) {
+    if constexpr (MODE != 2 && MODE != 4) {
+        if (args.rpc > 1) return launch_slots<1, false, MODE, true>(cfg, args, max_slots, max_local);
+    }
     if (half && MODE < 2) {
         switch (max_gps) {
             case 1: return launch_slots<1, true, MODE>(cfg, args, max_slots, max_local);
@@ -596,7 +679,6 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         attr[na].val.clusterDim.z = 1;
         ++na;
     }
-    cfg.gridDim = dim3((unsigned)(rows * njobs * parts));
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = na;
@@ -610,6 +692,11 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         args.njobs = njobs;
         args.rows = (int)rows;
         args.parts = parts;
+        // short rows (one or two 256-chunks) of a matrix that fills the GPU:
+        // 256 threads per CTA, a row per half-warp or warp
+        args.rpc = (!int4 && conv_mode != 4 && parts == 1 && njobs == 1 && !half && max_gps == 1 &&
+                    max_slots <= 2 && rows >= 8 * (int64_t)num_sms) ? 16 / max_slots : 1;
+        cfg.gridDim = dim3((unsigned)((rows * njobs * parts + args.rpc - 1) / args.rpc));
         for (int j = 0; j < njobs; ++j) {
             RQJobDev &J = args.job[j];
             J.a = static_cast<const __nv_bfloat16 *>(probs[j].a);
@@ -685,9 +772,10 @@ __global__ void __launch_bounds__(kGatherThreads) conv_gather_quant_kernel(const
                 if (iy >= 0 && iy < g.h && ix >= 0 && ix < g.w) {
                     const float4 *src =
                         reinterpret_cast<const float4 *>(yrot + (((size_t)b * g.h + iy) * g.w + ix) * g.c + ch);
+                    const int sw = yrot_swizzle(ch >> 4);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const float4 f = __ldg(src + i);
+                        const float4 f = __ldg(src + (i ^ sw));
                         y[4 * i] = f.x;
                         y[4 * i + 1] = f.y;
                         y[4 * i + 2] = f.z;
@@ -704,21 +792,282 @@ __global__ void __launch_bounds__(kGatherThreads) conv_gather_quant_kernel(const
     }
 }
 
+// ---------------------------------------------------------------------------
+// Tiled variant of the same pass: a CTA takes a th x tw tile of output pixels
+// of one image, brings the rotated values of the input pixels the tile reads
+// (its region, rh x rw pixels) into shared memory with one bulk copy per
+// region row, and the pixels' maxima with 4-byte asynchronous copies, then
+// quantises the tile's im2col rows from shared memory.  Two region buffers:
+// the next tile's copies run while this tile is quantised.  A rotated pixel
+// crosses from L2 once per tile that reads it instead of once per tap, and
+// no warp waits on a global load between the row scale and its codes.
+// One warp per row; lane l takes 16-value chunk base + l of the row (one
+// 16-byte store of codes; a warp stores 512 contiguous bytes), reading its
+// four float4 parts in the swizzled order of the rotated pixels, so that
+// the warp's shared-memory reads are free of bank conflicts.
+// ---------------------------------------------------------------------------
+constexpr int kTileThreads = 512;
+constexpr int kTileMaxTaps = 32;                      // a row's taps, one per lane
+constexpr size_t kTileSmemMax = 226 * 1024;           // both region buffers
+
+struct ConvTileArgs {
+    ConvGeom g;
+    int th, tw, rh, rw;         // tile (output pixels) and its region (input pixels)
+    int tiles_y, tiles_x;       // tiles per image
+    int64_t ntiles;
+    uint32_t buf_bytes;         // one buffer: rh*rw*c FP32 values, a zero pixel (c values), rh*rw maxima; 16-byte multiple
+    int cc;                     // 16-value chunks per pixel (c / 16)
+    int adv_t, adv_c;           // 32 chunks = adv_t pixels + adv_c chunks
+};
+
+struct TilePos {
+    int b, oy0, ox0, iy0, ix0;
+};
+
+__device__ __forceinline__ TilePos tile_pos(const ConvTileArgs &A, int64_t tile) {
+    const int per_img = A.tiles_y * A.tiles_x;
+    TilePos p;
+    p.b = (int)(tile / per_img);
+    const int r = (int)(tile - (int64_t)p.b * per_img);
+    const int ty = r / A.tiles_x;
+    p.oy0 = ty * A.th;
+    p.ox0 = (r - ty * A.tiles_x) * A.tw;
+    p.iy0 = p.oy0 * A.g.stride - A.g.pad;
+    p.ix0 = p.ox0 * A.g.stride - A.g.pad;
+    return p;
+}
+
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Start the copies of `tile`'s region into `buf` (every thread calls it; it
+// always commits one group of asynchronous copies, empty past the last tile).
+// Returns whether a bulk copy phase was started on `bar`.
+__device__ __forceinline__ bool tile_issue(const ConvTileArgs &A, const float *yrot, const float *pmax,
+                                           int64_t tile, uint8_t *buf, uint32_t bar) {
+    bool started = false;
+    if (tile < A.ntiles) {
+        const ConvGeom &g = A.g;
+        const TilePos p = tile_pos(A, tile);
+        const int cx0 = max(p.ix0, 0), cx1 = min(p.ix0 + A.rw, g.w);
+        const uint32_t row_bytes = cx1 > cx0 ? (uint32_t)(cx1 - cx0) * (uint32_t)g.c * 4u : 0u;
+        float *pm = reinterpret_cast<float *>(buf + (size_t)(A.rh * A.rw + 1) * g.c * 4);
+        if (threadIdx.x == 0) {
+            uint32_t bytes = 0;
+            for (int r = 0; r < A.rh; ++r) {
+                const int iy = p.iy0 + r;
+                if (iy >= 0 && iy < g.h) bytes += row_bytes;
+            }
+            fence_proxy_async_shared();      // the buffer's earlier reads (ordered by the CTA barrier) first
+            mbar_arrive_expect_tx(bar, bytes);
+            if (row_bytes != 0) {
+                for (int r = 0; r < A.rh; ++r) {
+                    const int iy = p.iy0 + r;
+                    if (iy < 0 || iy >= g.h) continue;
+                    bulk_load_1d(smem_addr(buf) + (uint32_t)(r * A.rw + (cx0 - p.ix0)) * (uint32_t)g.c * 4u,
+                                 yrot + (((size_t)p.b * g.h + iy) * g.w + cx0) * g.c, row_bytes, bar);
+                }
+            }
+        }
+        for (int i = threadIdx.x; i < A.rh * A.rw; i += blockDim.x) {
+            const int r = i / A.rw, cc = i - r * A.rw;
+            const int iy = p.iy0 + r, ix = p.ix0 + cc;
+            if (iy >= 0 && iy < g.h && ix >= 0 && ix < g.w)
+                cp_async_4(smem_addr(pm + i), pmax + ((size_t)p.b * g.h + iy) * g.w + ix);
+            else
+                pm[i] = 0.f;                 // padding: contributes 0 to a row maximum
+        }
+        started = true;
+    }
+    cp_async_commit();
+    return started;
+}
+
+// Quantise the im2col rows of `tile` from its region in `buf`.
+__device__ __forceinline__ void tile_emit(const ConvTileArgs &A, int64_t tile, const uint8_t *buf, int8_t *xq,
+                                          float *sx) {
+    const ConvGeom &g = A.g;
+    const TilePos p = tile_pos(A, tile);
+    const float4 *reg4 = reinterpret_cast<const float4 *>(buf);
+    const float *pm = reinterpret_cast<const float *>(buf + (size_t)(A.rh * A.rw + 1) * g.c * 4);
+    const int zero_pixel = A.rh * A.rw * (g.c / 4);     // float4 offset of the buffer's zero pixel
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int taps = g.kh * g.kw;
+    const int kc = taps * A.cc;                         // 16-value chunks per row
+    const int64_t kbytes = (int64_t)taps * g.c;
+    const int tky = lane < taps ? lane / g.kw : 0;      // this lane's tap, for the row's tap table
+    const int tkx = lane < taps ? lane - tky * g.kw : 0;
+    const int t0 = lane / A.cc, c0 = lane - t0 * A.cc;  // tap and chunk-in-pixel of chunk `lane`
+    for (int q = warp; q < A.th * A.tw; q += nwarps) {
+        const int ty = q / A.tw, tx = q - ty * A.tw;
+        const int oy = p.oy0 + ty, ox = p.ox0 + tx;
+        if (oy >= g.oh || ox >= g.ow) continue;        // ragged tile (warp-uniform)
+        const int64_t row = ((int64_t)p.b * g.oh + oy) * g.ow + ox;
+        // tap `lane` of the row: its pixel's first float4 in the region; the
+        // zero pixel outside the image (and for lanes past the taps)
+        int off = zero_pixel;
+        float m = 0.f;
+        if (lane < taps) {
+            const int ry = ty * g.stride + tky * g.dil, rx = tx * g.stride + tkx * g.dil;
+            const int iy = p.iy0 + ry, ix = p.ix0 + rx;
+            if (iy >= 0 && iy < g.h && ix >= 0 && ix < g.w) {
+                off = (ry * A.rw + rx) * (g.c / 4);
+                m = pm[ry * A.rw + rx];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const RowScale rs = make_row_scale(m);
+        uint4 *qrow = reinterpret_cast<uint4 *>(xq + row * kbytes);
+        int t = t0, ci = c0;                            // chunk base + lane: tap t, chunk ci of its pixel
+        for (int base = 0; base < kc; base += 32) {
+            // (past the row's end, t may name any lane: the values read are not stored)
+            const int o = __shfl_sync(0xffffffffu, off, t & 31);
+            const float4 *src = reg4 + o + 4 * ci;
+            const int sw = yrot_swizzle(ci);
+            float y[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 v = src[j ^ sw];
+                y[4 * j] = v.x;
+                y[4 * j + 1] = v.y;
+                y[4 * j + 2] = v.z;
+                y[4 * j + 3] = v.w;
+            }
+            const uint4 w = quant16x2(y, rs, 0xffffffffu);
+            if (base + lane < kc) qrow[base + lane] = w;
+            ci += A.adv_c;
+            t += A.adv_t;
+            if (ci >= A.cc) {
+                ci -= A.cc;
+                ++t;
+            }
+        }
+        if (lane == 0) sx[row] = rs.s;
+    }
+}
+
+__global__ void __launch_bounds__(kTileThreads, 1) conv_gather_tile_kernel(const float *yrot, const float *pmax,
+                                                                          const __grid_constant__ ConvTileArgs A,
+                                                                          int8_t *xq, float *sx) {
+    extern __shared__ __align__(128) uint8_t tsmem[];
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bars[0]), 1);
+        mbar_init(smem_addr(&bars[1]), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    uint8_t *bufs[2] = {tsmem, tsmem + A.buf_bytes};
+    for (int b = 0; b < 2; ++b) {
+        float4 *zp = reinterpret_cast<float4 *>(bufs[b] + (size_t)A.rh * A.rw * A.g.c * 4);
+        for (int i = threadIdx.x; i < A.g.c / 4; i += blockDim.x) zp[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
+    int issued[2] = {0, 0}, consumed[2] = {0, 0};     // bulk phases started / waited for, per buffer
+    const int64_t stride = gridDim.x;
+    issued[0] += tile_issue(A, yrot, pmax, blockIdx.x, bufs[0], smem_addr(&bars[0]));
+    issued[1] += tile_issue(A, yrot, pmax, blockIdx.x + stride, bufs[1], smem_addr(&bars[1]));
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < A.ntiles; tile += stride, ++it) {
+        const int b = it & 1;
+        mbar_wait_bounded(smem_addr(&bars[b]), (uint32_t)(consumed[b] & 1), &abort_flag);
+        ++consumed[b];
+        cp_async_wait_1();
+        __syncthreads();
+        if (*(volatile int *)&abort_flag) break;       // a copy never arrived: the status word says so
+        tile_emit(A, tile, bufs[b], xq, sx);
+        __syncthreads();                                // every warp is done with this buffer
+        issued[b] += tile_issue(A, yrot, pmax, tile + 2 * stride, bufs[b], smem_addr(&bars[b]));
+    }
+    cp_async_wait_all();
+    // after an early exit, let the bulk copies still in flight land (bounded)
+    for (int b = 0; b < 2; ++b)
+        if (issued[b] > consumed[b]) mbar_wait_bounded(smem_addr(&bars[b]), (uint32_t)(consumed[b] & 1), &abort_flag);
+}
+
+// Tile shape for the tiled pass, or false when no tile of at most 32 taps
+// fits its two region buffers in shared memory.  Prefers a multiple of the
+// warp count in rows, then the fewest region pixels copied per output pixel,
+// with enough tiles for every SM.
+static bool conv_tile_shape(const ConvGeom &g, int sms, ConvTileArgs *A) {
+    const int taps = g.kh * g.kw;
+    if (taps > kTileMaxTaps) return false;
+    const size_t budget = kTileSmemMax / 2;
+    double best = 0.0;
+    bool found = false;
+    for (int th = 1; th <= 64 && th <= g.oh; ++th) {
+        for (int tw = 1; tw <= 128 && tw <= g.ow; ++tw) {
+            const int64_t rh = (int64_t)(th - 1) * g.stride + (int64_t)(g.kh - 1) * g.dil + 1;
+            const int64_t rw = (int64_t)(tw - 1) * g.stride + (int64_t)(g.kw - 1) * g.dil + 1;
+            const size_t bytes = ((size_t)(rh * rw + 1) * g.c * 4 + (size_t)(rh * rw) * 4 + 15) / 16 * 16;
+            if (bytes > budget) break;              // wider tiles only grow
+            const int64_t ty = (g.oh + th - 1) / th, tx = (g.ow + tw - 1) / tw;
+            const int64_t tiles = (int64_t)g.n * ty * tx;
+            // quantising dominates: whole rows per warp first, then the
+            // region pixels copied per row
+            const int rows = th * tw, warps = kTileThreads / 32;
+            double score = (double)((rows + warps - 1) / warps * warps) / rows *
+                           (1.0 + 0.25 * ((double)(rh * rw) / rows - 1.0));
+            if (tiles < sms) score *= (double)sms / (double)tiles;
+            if (!found || score < best) {
+                found = true;
+                best = score;
+                A->th = th;
+                A->tw = tw;
+                A->rh = (int)rh;
+                A->rw = (int)rw;
+                A->tiles_y = (int)ty;
+                A->tiles_x = (int)tx;
+                A->ntiles = tiles;
+                A->buf_bytes = (uint32_t)bytes;
+            }
+        }
+    }
+    if (!found) return false;
+    A->g = g;
+    A->cc = g.c / 16;
+    A->adv_t = 32 / A->cc;
+    A->adv_c = 32 % A->cc;
+    return true;
+}
+
 cudaError_t launch_conv_gather_quant(const float *yrot, const float *pmax, const ConvGeom &g, int64_t rows,
                                      int8_t *xq, float *sx, cudaStream_t stream) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t cap = (int64_t)sms * 8;
-    const int64_t blocks = (rows + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3((unsigned)(blocks < cap ? blocks : cap));
-    cfg.blockDim = dim3(kGatherThreads);
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    ConvTileArgs A;
+    if (conv_tile_shape(g, sms, &A)) {
+        static bool configured[64] = {};
+        if (dev >= 64 || !configured[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(conv_gather_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)kTileSmemMax);
+            if (e != cudaSuccess) return e;
+            if (dev < 64) configured[dev] = true;
+        }
+        cfg.gridDim = dim3((unsigned)(A.ntiles < sms ? A.ntiles : sms));
+        cfg.blockDim = dim3(kTileThreads);
+        cfg.dynamicSmemBytes = 2 * (size_t)A.buf_bytes;
+        return cudaLaunchKernelEx(&cfg, conv_gather_tile_kernel, yrot, pmax, A, xq, sx);
+    }
+    const int64_t cap = (int64_t)sms * 8;
+    const int64_t blocks = (rows + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
+    cfg.gridDim = dim3((unsigned)(blocks < cap ? blocks : cap));
+    cfg.blockDim = dim3(kGatherThreads);
     return cudaLaunchKernelEx(&cfg, conv_gather_quant_kernel, yrot, pmax, g, rows, xq, sx);
 }
 

@@ -61,11 +61,13 @@ def test_weight_quant_tiny_bit_exact(cr):
 # m and k span every launch shape of the kernel: rows split over a cluster of
 # up to 8 CTAs (few rows, or rows of more than 32 groups), one CTA per row
 # (>= 148 rows), one or several groups per slot and a ragged last slot, and
-# the longest rows the API accepts
+# the longest rows the API accepts; short rows of a tall matrix packed 16 or 8
+# to a CTA (a ragged last CTA included)
 @pytest.mark.parametrize("m,k", [(1, 256), (4, 512), (3, 768), (17, 5120), (2, 8448), (3, 16384),
                                  (2, 24576), (5, 25600), (2, 38912), (2, 40960), (2, 65536),
                                  (150, 512), (160, 8448), (148, 25600), (149, 40960), (200, 65536),
-                                 (3, 133120), (150, 133120)])
+                                 (3, 133120), (150, 133120), (1200, 256), (1187, 256), (1190, 512),
+                                 (2048, 512)])
 def test_act_quant_bit_exact(cr, m, k):
     cs = synth.outlier_scale_fraction(synth.stream_key(m * 7 + k, 2), k, 0.01, 30.0)
     x_bits = synth.draw_np(synth.stream_key(m * 7 + k, 0), m, k, 1.0, cs)
@@ -119,6 +121,23 @@ def test_act_quant_exact_ties(cr):
     assert np.array_equal(got, q_ref)
     assert np.array_equal(sx.cpu().numpy(), s_ref)
     assert list(got[0, 256::256]) == [2, 4, -4, 0, -126, 2, 0, 6]
+
+
+def test_act_quant_subnormal_scale(cr):
+    # rows so small that s = amax / 127 is subnormal in FP32 (amax < 127 * 2^-126):
+    # the codes still follow q = clamp(rne(fl(y / s))) exactly
+    m, k = 6, 512
+    x = np.random.default_rng(5).standard_normal((m, k)).astype(np.float32)
+    x *= np.float32(2.0 ** -125) * np.array([1, 2, 4, 0.5, 8, 16], dtype=np.float32)[:, None]
+    bits = synth.f32_to_bf16_bits(x)
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+    cr.convrot_quantize_act(from_bits(bits), xq, sx)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.rotate_quantize(bits)
+    assert np.all(s_ref < np.float32(1.17549435e-38)) and np.all(s_ref > 0)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
 # ---------------------------------------------------------------- K2
@@ -449,7 +468,8 @@ def test_gemm_batch_bias(cr, m):
 # chunk, rows shorter than 256, decode-sized launches (rows over a cluster)
 # and one-CTA-per-row launches, the FP64 division by sqrt(G) for G = 32, 128
 DYN_ACT = [(3, 640, 128), (150, 640, 128), (4, 48, 16), (160, 48, 16), (2, 5440, 64), (150, 5440, 64),
-           (5, 1376, 32), (149, 1376, 32), (3, 1024, 128), (2, 25600, 128), (148, 8192, 32)]
+           (5, 1376, 32), (149, 1376, 32), (3, 1024, 128), (2, 25600, 128), (148, 8192, 32),
+           (1300, 384, 128), (1250, 48, 16), (1203, 160, 32)]
 
 
 @pytest.mark.parametrize("m,k,group", DYN_ACT)
@@ -633,6 +653,14 @@ CONV_CASES = [
     (1, 12, 12, 96, 48, 3, 1, 1, 1),
     (1, 32, 32, 128, 128, 3, 1, 1, 1),
     (1, 3, 3, 256, 64, 3, 1, 0, 1),
+    # enough pixels that the pixel rotation packs 16 / 8 / 16 rows to a CTA
+    (1, 40, 40, 256, 64, 3, 1, 1, 1),
+    (1, 36, 36, 512, 64, 3, 1, 1, 1),
+    (1, 48, 48, 128, 64, 3, 1, 1, 1),
+    (2, 20, 13, 16, 32, 3, 1, 1, 1),
+    (1, 9, 9, 48, 32, 5, 1, 2, 1),
+    # 49 taps: more than a warp's lanes, so the untiled gather
+    (1, 12, 12, 32, 16, 7, 1, 3, 1),
 ]
 
 
