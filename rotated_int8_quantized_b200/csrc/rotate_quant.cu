@@ -545,7 +545,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                 *reinterpret_cast<uint2 *>(J.q + (size_t)row * (k / 2) + (size_t)g0 * 128 + c * 8) =
                     quant16_int4(y, rs, mask);
             } else {
-                *reinterpret_cast<uint4 *>(qrow + c * 16) = quant16(y, rs, mask);
+                *reinterpret_cast<uint4 *>(qrow + c * 16) = HALF ? quant16(y, rs, mask) : quant16x2(y, rs, mask);
             }
         }
     }
@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(kGatherThreads) conv_gather_quant_kernel(const
 #pragma unroll
                     for (int e = 0; e < 16; ++e) y[e] = 0.f;
                 }
-                *reinterpret_cast<uint4 *>(xq + row * (int64_t)k + kel) = quant16(y, rs, mask);
+                *reinterpret_cast<uint4 *>(xq + row * (int64_t)k + kel) = quant16x2(y, rs, mask);
             }
         }
         if (lane == 0) sx[row] = rs.s;
@@ -963,9 +963,8 @@ __global__ void __launch_bounds__(kTileThreads, 1) conv_gather_tile_kernel(const
         abort_flag = 0;
         fence_mbar_init();
     }
-    uint8_t *bufs[2] = {tsmem, tsmem + A.buf_bytes};
     for (int b = 0; b < 2; ++b) {
-        float4 *zp = reinterpret_cast<float4 *>(bufs[b] + (size_t)A.rh * A.rw * A.g.c * 4);
+        float4 *zp = reinterpret_cast<float4 *>(tsmem + (size_t)b * A.buf_bytes + (size_t)A.rh * A.rw * A.g.c * 4);
         for (int i = threadIdx.x; i < A.g.c / 4; i += blockDim.x) zp[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
@@ -973,8 +972,8 @@ __global__ void __launch_bounds__(kTileThreads, 1) conv_gather_tile_kernel(const
     pdl_launch_dependents();
     int issued[2] = {0, 0}, consumed[2] = {0, 0};     // bulk phases started / waited for, per buffer
     const int64_t stride = gridDim.x;
-    issued[0] += tile_issue(A, yrot, pmax, blockIdx.x, bufs[0], smem_addr(&bars[0]));
-    issued[1] += tile_issue(A, yrot, pmax, blockIdx.x + stride, bufs[1], smem_addr(&bars[1]));
+    issued[0] += tile_issue(A, yrot, pmax, blockIdx.x, tsmem, smem_addr(&bars[0]));
+    issued[1] += tile_issue(A, yrot, pmax, blockIdx.x + stride, tsmem + A.buf_bytes, smem_addr(&bars[1]));
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < A.ntiles; tile += stride, ++it) {
         const int b = it & 1;
@@ -983,9 +982,10 @@ __global__ void __launch_bounds__(kTileThreads, 1) conv_gather_tile_kernel(const
         cp_async_wait_1();
         __syncthreads();
         if (*(volatile int *)&abort_flag) break;       // a copy never arrived: the status word says so
-        tile_emit(A, tile, bufs[b], xq, sx);
+        uint8_t *buf = tsmem + (b ? A.buf_bytes : 0u);   // (not an indexed array: keeps the shared state space)
+        tile_emit(A, tile, buf, xq, sx);
         __syncthreads();                                // every warp is done with this buffer
-        issued[b] += tile_issue(A, yrot, pmax, tile + 2 * stride, bufs[b], smem_addr(&bars[b]));
+        issued[b] += tile_issue(A, yrot, pmax, tile + 2 * stride, buf, smem_addr(&bars[b]));
     }
     cp_async_wait_all();
     // after an early exit, let the bulk copies still in flight land (bounded)
