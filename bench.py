@@ -581,6 +581,19 @@ def run_profile(args):
     cr.load_library()
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
+    if args.profile == "conv":
+        # the VAE-decoder-shaped 3x3 convolution, 256 x 256 x 256 -> 256
+        h, c = 256, 256
+        x = synth.Linear("conv_x", h * h, c, 1, 77 + c, None).x_torch(device).view(1, h, h, c)
+        w = synth.Linear("conv_w", 1, 9 * c, c, 77 + c, None).w_torch(device).view(c, c, 3, 3)
+        wq = cr.quantize_conv_weight(w)
+        torch.cuda.synchronize()
+        for _ in range(args.steps):
+            cr.conv2d_int8(x, wq, 3, 3, 1, 1, 1)
+        torch.cuda.synchronize()
+        cr.convrot_device_status()
+        print("profile run ok: conv, %d steps" % args.steps)
+        return
     m = {"decode": 12, "prefill": 4096}[args.profile]
     lins = synth.qwen_layer(m)
     layer = Layer(cr, lins, device)
@@ -808,7 +821,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-minimax", action="store_true", help="skip the MiniMax qkv TOPS measurement")
     ap.add_argument("--no-stack", action="store_true", help="skip the 50-layer stack measurement")
-    ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill", "conv"], default=None,
                     help="run a few eager steps of one workload for ncu (no timing)")
     args = ap.parse_args()
     if args.profile:
