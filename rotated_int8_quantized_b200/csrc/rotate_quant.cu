@@ -133,7 +133,7 @@ __device__ __forceinline__ void unpack_f32x2(uint64_t d, float &a, float &b) {
 
 __device__ __forceinline__ uint4 quant16x2(const float (&y)[16], const RowScale &rs, unsigned mask) {
     uint32_t b[16];
-    bool near = false;
+    bool nr[4] = {false, false, false, false};     // four short "near" chains instead of one of 16
     const uint64_t r2 = pack_f32x2(rs.r, rs.r), m2 = pack_f32x2(kRoundMagic, kRoundMagic);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -147,10 +147,10 @@ __device__ __forceinline__ uint4 quant16x2(const float (&y)[16], const RowScale 
         unpack_f32x2(big2, b0, b1);
         b[2 * i] = __float_as_uint(b0);                               // low byte: rne(t)
         b[2 * i + 1] = __float_as_uint(b1);
-        near |= !(fabsf(d0) < 0.49997f);                              // NaN too
-        near |= !(fabsf(d1) < 0.49997f);
+        nr[i & 3] |= !(fabsf(d0) < 0.49997f);                         // NaN too
+        nr[i & 3] |= !(fabsf(d1) < 0.49997f);
     }
-    const bool slow = near || !rs.fast;      // zero rows too (their codes are set below)
+    const bool slow = (nr[0] || nr[1]) || (nr[2] || nr[3]) || !rs.fast;   // zero rows too (codes set below)
     if (__any_sync(mask, slow) && slow) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -794,19 +794,22 @@ __global__ void __launch_bounds__(kGatherThreads) conv_gather_quant_kernel(const
 
 // ---------------------------------------------------------------------------
 // Tiled variant of the same pass: a CTA takes a th x tw tile of output pixels
-// of one image, brings the rotated values of the input pixels the tile reads
-// (its region, rh x rw pixels) into shared memory with one bulk copy per
-// region row, and the pixels' maxima with 4-byte asynchronous copies, then
-// quantises the tile's im2col rows from shared memory.  Two region buffers:
-// the next tile's copies run while this tile is quantised.  A rotated pixel
-// crosses from L2 once per tile that reads it instead of once per tap, and
-// no warp waits on a global load between the row scale and its codes.
+// of one image at a time.  A producer warp brings the rotated values of the
+// input pixels the tile reads (its region, rh x rw pixels) into shared memory
+// with one bulk copy per region row, and the pixels' maxima with 4-byte
+// asynchronous copies, into one of two region buffers (full / empty
+// mbarriers per buffer); sixteen warps quantise the tile's im2col rows from
+// shared memory, each moving on to the next buffer as soon as its own rows
+// are done.  A rotated pixel crosses from L2 once per tile that reads it
+// instead of once per tap, and no warp waits on a global load between the
+// row scale and its codes.
 // One warp per row; lane l takes 16-value chunk base + l of the row (one
 // 16-byte store of codes; a warp stores 512 contiguous bytes), reading its
 // four float4 parts in the swizzled order of the rotated pixels, so that
 // the warp's shared-memory reads are free of bank conflicts.
 // ---------------------------------------------------------------------------
-constexpr int kTileThreads = 512;
+constexpr int kTileConsumers = 16;                    // quantising warps
+constexpr int kTileThreads = 32 * kTileConsumers + 32;  // and one producer warp
 constexpr int kTileMaxTaps = 32;                      // a row's taps, one per lane
 constexpr size_t kTileSmemMax = 226 * 1024;           // both region buffers
 
@@ -840,51 +843,50 @@ __device__ __forceinline__ TilePos tile_pos(const ConvTileArgs &A, int64_t tile)
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Start the copies of `tile`'s region into `buf` (every thread calls it; it
-// always commits one group of asynchronous copies, empty past the last tile).
-// Returns whether a bulk copy phase was started on `bar`.
-__device__ __forceinline__ bool tile_issue(const ConvTileArgs &A, const float *yrot, const float *pmax,
-                                           int64_t tile, uint8_t *buf, uint32_t bar) {
-    bool started = false;
-    if (tile < A.ntiles) {
-        const ConvGeom &g = A.g;
-        const TilePos p = tile_pos(A, tile);
-        const int cx0 = max(p.ix0, 0), cx1 = min(p.ix0 + A.rw, g.w);
-        const uint32_t row_bytes = cx1 > cx0 ? (uint32_t)(cx1 - cx0) * (uint32_t)g.c * 4u : 0u;
-        float *pm = reinterpret_cast<float *>(buf + (size_t)(A.rh * A.rw + 1) * g.c * 4);
-        if (threadIdx.x == 0) {
-            uint32_t bytes = 0;
+// Start the copies of `tile`'s region into `buf` (the producer warp): lane
+// 0 posts the byte count on `bar` and issues one bulk copy per region row;
+// every lane copies its share of the maxima with 4-byte asynchronous copies
+// (zero-filled outside the image) and arrives on `bar` when they complete.
+__device__ __forceinline__ void cp_async_4_zfill(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tile_issue(const ConvTileArgs &A, const float *yrot, const float *pmax,
+                                           int64_t tile, uint8_t *buf, uint32_t bar, int lane) {
+    const ConvGeom &g = A.g;
+    const TilePos p = tile_pos(A, tile);
+    const int cx0 = max(p.ix0, 0), cx1 = min(p.ix0 + A.rw, g.w);
+    const uint32_t row_bytes = cx1 > cx0 ? (uint32_t)(cx1 - cx0) * (uint32_t)g.c * 4u : 0u;
+    float *pm = reinterpret_cast<float *>(buf + (size_t)(A.rh * A.rw + 1) * g.c * 4);
+    if (lane == 0) {
+        uint32_t bytes = 0;
+        for (int r = 0; r < A.rh; ++r) {
+            const int iy = p.iy0 + r;
+            if (iy >= 0 && iy < g.h) bytes += row_bytes;
+        }
+        fence_proxy_async_shared();      // the buffer's earlier reads (released through `empty`) first
+        mbar_arrive_expect_tx(bar, bytes);
+        if (row_bytes != 0) {
             for (int r = 0; r < A.rh; ++r) {
                 const int iy = p.iy0 + r;
-                if (iy >= 0 && iy < g.h) bytes += row_bytes;
-            }
-            fence_proxy_async_shared();      // the buffer's earlier reads (ordered by the CTA barrier) first
-            mbar_arrive_expect_tx(bar, bytes);
-            if (row_bytes != 0) {
-                for (int r = 0; r < A.rh; ++r) {
-                    const int iy = p.iy0 + r;
-                    if (iy < 0 || iy >= g.h) continue;
-                    bulk_load_1d(smem_addr(buf) + (uint32_t)(r * A.rw + (cx0 - p.ix0)) * (uint32_t)g.c * 4u,
-                                 yrot + (((size_t)p.b * g.h + iy) * g.w + cx0) * g.c, row_bytes, bar);
-                }
+                if (iy < 0 || iy >= g.h) continue;
+                bulk_load_1d(smem_addr(buf) + (uint32_t)(r * A.rw + (cx0 - p.ix0)) * (uint32_t)g.c * 4u,
+                             yrot + (((size_t)p.b * g.h + iy) * g.w + cx0) * g.c, row_bytes, bar);
             }
         }
-        for (int i = threadIdx.x; i < A.rh * A.rw; i += blockDim.x) {
-            const int r = i / A.rw, cc = i - r * A.rw;
-            const int iy = p.iy0 + r, ix = p.ix0 + cc;
-            if (iy >= 0 && iy < g.h && ix >= 0 && ix < g.w)
-                cp_async_4(smem_addr(pm + i), pmax + ((size_t)p.b * g.h + iy) * g.w + ix);
-            else
-                pm[i] = 0.f;                 // padding: contributes 0 to a row maximum
-        }
-        started = true;
     }
-    cp_async_commit();
-    return started;
+    for (int i = lane; i < A.rh * A.rw; i += 32) {
+        const int r = i / A.rw, cc = i - r * A.rw;
+        const int iy = p.iy0 + r, ix = p.ix0 + cc;
+        const bool in = iy >= 0 && iy < g.h && ix >= 0 && ix < g.w;     // padding: 0 in a row maximum
+        cp_async_4_zfill(smem_addr(pm + i), in ? pmax + ((size_t)p.b * g.h + iy) * g.w + ix : pmax, in);
+    }
+    cp_async_arrive_noinc(bar);
 }
 
 // Quantise the im2col rows of `tile` from its region in `buf`.
@@ -895,7 +897,7 @@ __device__ __forceinline__ void tile_emit(const ConvTileArgs &A, int64_t tile, c
     const float4 *reg4 = reinterpret_cast<const float4 *>(buf);
     const float *pm = reinterpret_cast<const float *>(buf + (size_t)(A.rh * A.rw + 1) * g.c * 4);
     const int zero_pixel = A.rh * A.rw * (g.c / 4);     // float4 offset of the buffer's zero pixel
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = kTileConsumers;
     const int taps = g.kh * g.kw;
     const int kc = taps * A.cc;                         // 16-value chunks per row
     const int64_t kbytes = (int64_t)taps * g.c;
@@ -955,11 +957,13 @@ __global__ void __launch_bounds__(kTileThreads, 1) conv_gather_tile_kernel(const
                                                                           const __grid_constant__ ConvTileArgs A,
                                                                           int8_t *xq, float *sx) {
     extern __shared__ __align__(128) uint8_t tsmem[];
-    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ __align__(8) uint64_t full[2], empty[2];
     __shared__ int abort_flag;
     if (threadIdx.x == 0) {
-        mbar_init(smem_addr(&bars[0]), 1);
-        mbar_init(smem_addr(&bars[1]), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_addr(&full[b]), 1 + 32);           // byte count + the producer lanes' copies
+            mbar_init(smem_addr(&empty[b]), kTileConsumers);  // one arrival per quantising warp
+        }
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -970,27 +974,29 @@ __global__ void __launch_bounds__(kTileThreads, 1) conv_gather_tile_kernel(const
     __syncthreads();
     pdl_wait();
     pdl_launch_dependents();
-    int issued[2] = {0, 0}, consumed[2] = {0, 0};     // bulk phases started / waited for, per buffer
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t stride = gridDim.x;
-    issued[0] += tile_issue(A, yrot, pmax, blockIdx.x, tsmem, smem_addr(&bars[0]));
-    issued[1] += tile_issue(A, yrot, pmax, blockIdx.x + stride, tsmem + A.buf_bytes, smem_addr(&bars[1]));
+    if (warp == kTileConsumers) {
+        // producer: fill buffer it & 1 with tile `it` once its previous use is released
+        int it = 0;
+        for (int64_t tile = blockIdx.x; tile < A.ntiles; tile += stride, ++it) {
+            const int b = it & 1, use = it >> 1;
+            if (use > 0 && !mbar_wait_bounded(smem_addr(&empty[b]), (uint32_t)((use - 1) & 1), &abort_flag)) break;
+            tile_issue(A, yrot, pmax, tile, tsmem + (b ? A.buf_bytes : 0u), smem_addr(&full[b]), lane);
+        }
+        cp_async_wait_all();
+        return;
+    }
+    // quantising warps: no CTA-wide barrier, a warp that finishes its rows of
+    // one tile goes on to the next tile's buffer
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < A.ntiles; tile += stride, ++it) {
-        const int b = it & 1;
-        mbar_wait_bounded(smem_addr(&bars[b]), (uint32_t)(consumed[b] & 1), &abort_flag);
-        ++consumed[b];
-        cp_async_wait_1();
-        __syncthreads();
-        if (*(volatile int *)&abort_flag) break;       // a copy never arrived: the status word says so
-        uint8_t *buf = tsmem + (b ? A.buf_bytes : 0u);   // (not an indexed array: keeps the shared state space)
-        tile_emit(A, tile, buf, xq, sx);
-        __syncthreads();                                // every warp is done with this buffer
-        issued[b] += tile_issue(A, yrot, pmax, tile + 2 * stride, buf, smem_addr(&bars[b]));
+        const int b = it & 1, use = it >> 1;
+        if (!mbar_wait_bounded(smem_addr(&full[b]), (uint32_t)(use & 1), &abort_flag)) break;
+        tile_emit(A, tile, tsmem + (b ? A.buf_bytes : 0u), xq, sx);   // (not an indexed array: shared state space)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&empty[b]));
     }
-    cp_async_wait_all();
-    // after an early exit, let the bulk copies still in flight land (bounded)
-    for (int b = 0; b < 2; ++b)
-        if (issued[b] > consumed[b]) mbar_wait_bounded(smem_addr(&bars[b]), (uint32_t)(consumed[b] & 1), &abort_flag);
 }
 
 // Tile shape for the tiled pass, or false when no tile of at most 32 taps
@@ -1013,7 +1019,7 @@ static bool conv_tile_shape(const ConvGeom &g, int sms, ConvTileArgs *A) {
             const int64_t tiles = (int64_t)g.n * ty * tx;
             // quantising dominates: whole rows per warp first, then the
             // region pixels copied per row
-            const int rows = th * tw, warps = kTileThreads / 32;
+            const int rows = th * tw, warps = kTileConsumers;
             double score = (double)((rows + warps - 1) / warps * warps) / rows *
                            (1.0 + 0.25 * ((double)(rh * rw) / rows - 1.0));
             if (tiles < sms) score *= (double)sms / (double)tiles;
