@@ -798,7 +798,7 @@ __global__ void __launch_bounds__(kGatherThreads) conv_gather_quant_kernel(const
 // input pixels the tile reads (its region, rh x rw pixels) into shared memory
 // with one bulk copy per region row, and the pixels' maxima with 4-byte
 // asynchronous copies, into one of two region buffers (full / empty
-// mbarriers per buffer); sixteen warps quantise the tile's im2col rows from
+// mbarriers per buffer); the quantising warps take the tile's im2col rows from
 // shared memory, each moving on to the next buffer as soon as its own rows
 // are done.  A rotated pixel crosses from L2 once per tile that reads it
 // instead of once per tap, and no warp waits on a global load between the
