@@ -333,11 +333,13 @@ __host__ __device__ __forceinline__ int yrot_swizzle(int ci) { return (ci >> 1) 
 // 3: INT8 codes of the im2col rows of a convolution, gathered from NHWC
 // input; 4: INT8 codes of a convolution's OIHW weight in the im2col order;
 // 5: the rotated FP32 rows themselves and their maxima (no quantisation):
-// every input pixel of a convolution rotated once, for conv_gather_quant.
+// every input pixel of a convolution rotated once, for conv_gather_quant;
+// 6: the same with groups of 256 and whole 256-chunks (no DYN paths).
 template <int GPS, bool HALF, int MODE, bool MR = false>
 __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
     rotate_quant_rows_slots(const __grid_constant__ RQArgs args) {
-    constexpr bool DYN = MODE != 0;
+    constexpr bool ROT = MODE == 5 || MODE == 6;    // rotated values only
+    constexpr bool DYN = MODE != 0 && MODE != 6;
     constexpr int kXchStride = HALF ? kXchHalf : kXchFull;
     extern __shared__ __align__(16) uint8_t rq_smem[];
     __shared__ float red[kMaxSlots / 2];
@@ -534,7 +536,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
                 y[4 * i + 2] = f.z;
                 y[4 * i + 3] = f.w;
             }
-            if (MODE == 5) {    // rotated values themselves (FP32 [rows, k], in J.q), float4 parts swizzled
+            if (ROT) {    // rotated values themselves (FP32 [rows, k], in J.q), float4 parts swizzled
                 float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(J.q) + (size_t)row * k +
                                                          (size_t)g0 * 256 + c * 16);
                 const int sw = yrot_swizzle(c);
@@ -549,8 +551,8 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
             }
         }
     }
-    // MODE 5 keeps the row maximum (the scale is a later, per-im2col-row step)
-    if (tid == 0 && part == 0) J.s[row] = MODE == 5 ? rmax : rs.s;
+    // MODE 5 / 6 keep the row maximum (the scale is a later, per-im2col-row step)
+    if (tid == 0 && part == 0) J.s[row] = ROT ? rmax : rs.s;
     if (C > 1) {
         __syncwarp();
         cluster_wait();   // peers may still read part_max until they arrive
@@ -581,13 +583,15 @@ static cudaError_t launch_gps(cudaLaunchConfig_t &cfg, const RQArgs &args, bool 
     if constexpr (MODE != 2 && MODE != 4) {
         if (args.rpc > 1) return launch_slots<1, false, MODE, true>(cfg, args, max_slots, max_local);
     }
-    if (half && MODE < 2) {
-        switch (max_gps) {
-            case 1: return launch_slots<1, true, MODE>(cfg, args, max_slots, max_local);
-            case 2: return launch_slots<2, true, MODE>(cfg, args, max_slots, max_local);
-            case 3: return launch_slots<3, true, MODE>(cfg, args, max_slots, max_local);
-            case 4: return launch_slots<4, true, MODE>(cfg, args, max_slots, max_local);
-            default: return launch_slots<6, true, MODE>(cfg, args, max_slots, max_local);
+    if constexpr (MODE < 2) {       // the half-size transpose: decode-sized activations only
+        if (half) {
+            switch (max_gps) {
+                case 1: return launch_slots<1, true, MODE>(cfg, args, max_slots, max_local);
+                case 2: return launch_slots<2, true, MODE>(cfg, args, max_slots, max_local);
+                case 3: return launch_slots<3, true, MODE>(cfg, args, max_slots, max_local);
+                case 4: return launch_slots<4, true, MODE>(cfg, args, max_slots, max_local);
+                default: return launch_slots<6, true, MODE>(cfg, args, max_slots, max_local);
+            }
         }
     }
     switch (max_gps) {
@@ -713,6 +717,7 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
             rq_shape((groups + parts - 1) / parts, &J.gps, &J.slots);
             dyn = dyn || J.group != 256 || (J.k & 255) != 0;
         }
+        if (conv_mode == 5 && !dyn) return launch_gps<6>(cfg, args, false, max_gps, max_slots, max_local);
         if (conv_mode == 5) return launch_gps<5>(cfg, args, false, max_gps, max_slots, max_local);
         if (conv_mode == 3) return launch_gps<3>(cfg, args, false, max_gps, max_slots, max_local);
         if (conv_mode == 4) return launch_gps<4>(cfg, args, false, max_gps, max_slots, max_local);
