@@ -661,6 +661,9 @@ CONV_CASES = [
     (1, 9, 9, 48, 32, 5, 1, 2, 1),
     # 49 taps: more than a warp's lanes, so the untiled gather
     (1, 12, 12, 32, 16, 7, 1, 3, 1),
+    # 1x1 with enough pixels that the one-step gather packs 16 rows to a CTA, and strided
+    (1, 40, 40, 256, 64, 1, 1, 0, 1),
+    (2, 50, 50, 128, 32, 1, 2, 0, 1),
 ]
 
 
