@@ -984,12 +984,20 @@ __global__ void __launch_bounds__(kTileThreads, 1) conv_gather_tile_kernel(const
     if (warp == kTileConsumers) {
         // producer: fill buffer it & 1 with tile `it` once its previous use is released
         int it = 0;
+        int issued[2] = {0, 0};
         for (int64_t tile = blockIdx.x; tile < A.ntiles; tile += stride, ++it) {
             const int b = it & 1, use = it >> 1;
             if (use > 0 && !mbar_wait_bounded(smem_addr(&empty[b]), (uint32_t)((use - 1) & 1), &abort_flag)) break;
             tile_issue(A, yrot, pmax, tile, tsmem + (b ? A.buf_bytes : 0u), smem_addr(&full[b]), lane);
+            ++issued[b];
         }
         cp_async_wait_all();
+        // this warp keeps the CTA (and its shared memory) alive until every
+        // copy it started has landed, even when the quantising warps gave up
+        // early (a wait that ran out); normally these return at once
+        volatile int no_abort = 0;
+        for (int b = 0; b < 2; ++b)
+            if (issued[b] > 0) mbar_wait_bounded(smem_addr(&full[b]), (uint32_t)((issued[b] - 1) & 1), &no_abort);
         return;
     }
     // quantising warps: no CTA-wide barrier, a warp that finishes its rows of
