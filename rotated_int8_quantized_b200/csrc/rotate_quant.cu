@@ -645,6 +645,102 @@ static size_t rq_smem_bytes(int njobs, const RQProblem *probs, int parts, bool h
     return (size_t)ms * (half ? kXchHalf : kXchFull) * 8 + (size_t)ml * y_group_stride(half) * 4;
 }
 
+// ---------------------------------------------------------------------------
+// Every input pixel of a convolution rotated once, for pixels of CH = 1 or 2
+// chunks of 256 channels (groups of 256): the same values and layout as
+// rotate_quant_rows_slots MODE 6 with none of its row bookkeeping.  A half-
+// warp per 256-chunk (two pixels per warp, or one pixel of two chunks),
+// persistent warps striding over the pixels with the next pixel's 32 bytes
+// per thread loaded while the current one is transformed; each thread stores
+// its 16 rotated values straight to their swizzled places (a half-warp
+// writes one 64-byte chunk per store) and the pixel maximum is reduced by
+// shuffles.
+// ---------------------------------------------------------------------------
+constexpr int kPixThreads = 256;
+
+template <int CH>
+__global__ void __launch_bounds__(kPixThreads) rotate_pixels_kernel(const __nv_bfloat16 *x, int64_t pixels,
+                                                                   float *yrot, float *pmax) {
+    __shared__ double xch[kPixThreads / 16][kXchFull];
+    pdl_wait();
+    pdl_launch_dependents();
+    constexpr int kPPW = 2 / CH;                         // pixels per warp
+    constexpr int kC = 256 * CH;
+    const int slot = threadIdx.x >> 4, t = threadIdx.x & 15, hw = slot & 1;
+    const unsigned half_mask = 0xFFFFu << (16 * hw);
+    const unsigned pix_mask = CH == 1 ? half_mask : 0xffffffffu;
+    const int chunk = CH == 1 ? 0 : hw;                  // this half-warp's 256-chunk of the pixel
+    const int64_t stride = (int64_t)gridDim.x * (kPixThreads / 32) * kPPW;
+    int64_t p = ((int64_t)blockIdx.x * (kPixThreads / 32) + (threadIdx.x >> 5)) * kPPW + (CH == 1 ? hw : 0);
+    double *xb = &xch[slot][0];
+    uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0;
+    if (p < pixels) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + p * kC + chunk * 256 + t * 16);
+        r0 = __ldg(src);
+        r1 = __ldg(src + 1);
+    }
+    for (; p < pixels; p += stride) {
+        const int64_t pn = p + stride;
+        uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
+        if (pn < pixels) {                               // the next pixel's load overlaps this transform
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + pn * kC + chunk * 256 + t * 16);
+            n0 = __ldg(src);
+            n1 = __ldg(src + 1);
+        }
+        double v[16];
+        const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
+        fwht16_regs(v);                                  // index bits 0-3
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xb[17 * t + i] = v[i];
+        __syncwarp(half_mask);
+        double xx[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xx[i] = xb[t + 17 * i];
+        __syncwarp(half_mask);
+        fwht16_regs(xx);                                 // index bits 4-7: xx[i] is output 16 i + t
+        float *dst = yrot + p * kC + chunk * 256 + (t & 3);
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float y = __double2float_rn(xx[i] * 0.0625);     // / sqrt(256), exact
+            dst[16 * i + 4 * ((t >> 2) ^ yrot_swizzle(i))] = y;
+            amax = fmaxf(amax, fabsf(y));
+        }
+#pragma unroll
+        for (int o = 8 * CH; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(pix_mask, amax, o));
+        if (t == 0 && chunk == 0) pmax[p] = amax;
+        r0 = n0;
+        r1 = n1;
+    }
+}
+
+static cudaError_t launch_rotate_pixels(const void *x, int64_t pixels, int c, float *yrot, float *pmax,
+                                        cudaStream_t stream, bool pdl) {
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const bool two = c == 512;
+    cudaError_t e = two ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_pixels_kernel<2>, kPixThreads, 0)
+                        : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_pixels_kernel<1>, kPixThreads, 0);
+    if (e != cudaSuccess) return e;
+    const int64_t per_cta = (kPixThreads / 32) * (two ? 1 : 2);
+    const int64_t need = (pixels + per_cta - 1) / per_cta;
+    const int64_t cap = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)(need < cap ? need : cap));
+    cfg.blockDim = dim3(kPixThreads);
+    cfg.stream = stream;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+    return two ? cudaLaunchKernelEx(&cfg, rotate_pixels_kernel<2>, xb, pixels, yrot, pmax)
+               : cudaLaunchKernelEx(&cfg, rotate_pixels_kernel<1>, xb, pixels, yrot, pmax);
+}
+
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl,
                                 const ConvGeom *conv) {
     int dev = 0, num_sms = 148;
@@ -666,6 +762,9 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
     bool int4 = false;
     for (int j = 0; j < njobs; ++j) int4 = int4 || probs[j].int4;
     const int conv_mode = conv ? conv->mode : 0;
+    if (conv_mode == 5 && njobs == 1 && probs[0].group == 256 && (probs[0].k == 256 || probs[0].k == 512))
+        return launch_rotate_pixels(probs[0].a, rows, (int)probs[0].k, reinterpret_cast<float *>(probs[0].q),
+                                    probs[0].s, stream, pdl);
     const bool half = few_rows && !int4 && conv_mode == 0;
     const int parts = rq_parts(njobs, rows, probs, num_sms, half);
     cudaLaunchConfig_t cfg = {};
