@@ -741,6 +741,145 @@ static cudaError_t launch_rotate_pixels(const void *x, int64_t pixels, int c, fl
                : cudaLaunchKernelEx(&cfg, rotate_pixels_kernel<1>, xb, pixels, yrot, pmax);
 }
 
+// ---------------------------------------------------------------------------
+// Many long rows with groups of 256 (activations at prefill, weights
+// offline): persistent CTAs of S slots (one per group, in whole warps, or 32
+// when a slot takes several groups) walk the rows, the same arithmetic as
+// rotate_quant_rows_slots MODE 0 without its per-row bookkeeping (no job
+// table, parts or row packing), and each row's loads are issued while the
+// previous row is reduced and quantised.  Slot s takes groups s, s + S, ...
+// ---------------------------------------------------------------------------
+constexpr int kLeanThreads = 512;
+constexpr int kLeanMinGroups = 16;      // below this most slots would idle
+constexpr int kLeanMaxGps = 4;
+
+template <int GPS, bool DYNS>
+__global__ void __launch_bounds__(kLeanThreads, GPS == 1 ? 2 : 1)
+    rotate_quant_rows_lean(const __nv_bfloat16 *a, int64_t rows, int k, int8_t *q, float *s) {
+    extern __shared__ __align__(16) uint8_t lsm[];
+    __shared__ float red[kLeanThreads / 32];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, slot = tid >> 4, t = tid & 15, lane = tid & 31, warp = tid >> 5;
+    // DYNS: as many slots as the launch has; otherwise 32, a constant for the compiler
+    const int S = DYNS ? (int)blockDim.x >> 4 : kLeanThreads / 16;
+    const int nthreads = S * 16, nwarps = nthreads >> 5;
+    const unsigned half_mask = 0xFFFFu << (16 * (slot & 1));
+    const int groups = k >> 8, chunks = k >> 4;
+    double *xb = reinterpret_cast<double *>(lsm) + slot * kXchFull;
+    float *ybuf = reinterpret_cast<float *>(lsm + (size_t)S * kXchFull * 8);
+    uint4 raw[GPS][2];
+    auto load = [&](int64_t r) {
+#pragma unroll
+        for (int gi = 0; gi < GPS; ++gi) {
+            const int g = slot + S * gi;
+            if (g < groups) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(a + r * k + g * 256 + t * 16);
+                raw[gi][0] = __ldg(src);
+                raw[gi][1] = __ldg(src + 1);
+            }
+        }
+    };
+    int64_t row = blockIdx.x;
+    if (row < rows) load(row);
+    for (; row < rows; row += gridDim.x) {
+        float amax = 0.f;
+#pragma unroll
+        for (int gi = 0; gi < GPS; ++gi) {
+            const int g = slot + S * gi;
+            if (g < groups) {
+                double v[16];
+                const uint32_t w[8] = {raw[gi][0].x, raw[gi][0].y, raw[gi][0].z, raw[gi][0].w,
+                                       raw[gi][1].x, raw[gi][1].y, raw[gi][1].z, raw[gi][1].w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
+                fwht16_regs(v);                              // index bits 0-3
+#pragma unroll
+                for (int i = 0; i < 16; ++i) xb[17 * t + i] = v[i];
+                __syncwarp(half_mask);
+                double x[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = xb[t + 17 * i];
+                __syncwarp(half_mask);
+                fwht16_regs(x);                              // index bits 4-7: x[i] is output 16 i + t
+                float *yg = ybuf + (size_t)g * kYGroupStride + (t & 3);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float y = __double2float_rn(x[i] * 0.0625);     // / sqrt(256), exact
+                    yg[16 * i + 4 * ((t >> 2) ^ ((i >> 1) & 3))] = y;
+                    amax = fmaxf(amax, fabsf(y));
+                }
+            }
+        }
+        const int64_t nrow = row + gridDim.x;
+        if (nrow < rows) load(nrow);         // in flight during this row's reduction and quantisation
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0) red[warp] = amax;
+        __syncthreads();
+        float rmax = red[0];
+        for (int w = 1; w < nwarps; ++w) rmax = fmaxf(rmax, red[w]);
+        const RowScale rs = make_row_scale(rmax);
+        int8_t *qrow = q + row * k;
+        for (int c0 = 0; c0 < chunks; c0 += nthreads) {
+            const int c = c0 + tid;
+            const unsigned mask = __ballot_sync(0xffffffffu, c < chunks);
+            if (c < chunks) {
+                const int ci = c & 15;
+                const float4 *src = reinterpret_cast<const float4 *>(ybuf + (size_t)(c >> 4) * kYGroupStride + ci * 16);
+                float y[16];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 f = src[i ^ ((ci >> 1) & 3)];
+                    y[4 * i] = f.x;
+                    y[4 * i + 1] = f.y;
+                    y[4 * i + 2] = f.z;
+                    y[4 * i + 3] = f.w;
+                }
+                *reinterpret_cast<uint4 *>(qrow + c * 16) = quant16x2(y, rs, mask);
+            }
+        }
+        if (tid == 0) s[row] = rs.s;
+        __syncthreads();                     // ybuf and red are written again by the next row
+    }
+}
+
+template <int GPS, bool DYNS>
+static cudaError_t launch_lean(const RQProblem &pr, int64_t rows, int sms, cudaStream_t stream, bool pdl) {
+    const int groups = (int)(pr.k >> 8);
+    // one group per slot: as many slots as groups (whole warps); several:
+    // all 32 slots (more warps per SM measured faster for the longest rows)
+    const int slots = DYNS ? (groups + 1) & ~1 : kLeanThreads / 16;
+    const size_t smem = (size_t)slots * kXchFull * 8 + (size_t)groups * kYGroupStride * 4;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(rotate_quant_rows_lean<GPS, DYNS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSlotsSmemMax);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured[dev] = true;
+    }
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_rows_lean<GPS, DYNS>, slots * 16, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t cap = (int64_t)sms * per_sm;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)(rows < cap ? rows : cap));
+    cfg.blockDim = dim3(slots * 16);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_lean<GPS, DYNS>, static_cast<const __nv_bfloat16 *>(pr.a), rows,
+                              (int)pr.k, pr.q, pr.s);
+}
+
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl,
                                 const ConvGeom *conv) {
     int dev = 0, num_sms = 148;
@@ -765,6 +904,21 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
     if (conv_mode == 5 && njobs == 1 && probs[0].group == 256 && (probs[0].k == 256 || probs[0].k == 512))
         return launch_rotate_pixels(probs[0].a, rows, (int)probs[0].k, reinterpret_cast<float *>(probs[0].q),
                                     probs[0].s, stream, pdl);
+    if (conv_mode == 0 && !int4 && njobs == 1 && probs[0].group == 256 && (probs[0].k & 255) == 0 &&
+        rows >= 2 * (int64_t)num_sms) {
+        const int groups = (int)(probs[0].k >> 8);
+        const int gps = (groups + 31) / 32;
+        if (groups >= kLeanMinGroups && gps <= kLeanMaxGps) {
+            switch (gps) {
+                case 1:
+                    return groups >= 31 ? launch_lean<1, false>(probs[0], rows, num_sms, stream, pdl)
+                                        : launch_lean<1, true>(probs[0], rows, num_sms, stream, pdl);
+                case 2: return launch_lean<2, false>(probs[0], rows, num_sms, stream, pdl);
+                case 3: return launch_lean<3, false>(probs[0], rows, num_sms, stream, pdl);
+                default: return launch_lean<4, false>(probs[0], rows, num_sms, stream, pdl);
+            }
+        }
+    }
     const bool half = few_rows && !int4 && conv_mode == 0;
     const int parts = rq_parts(njobs, rows, probs, num_sms, half);
     cudaLaunchConfig_t cfg = {};

@@ -62,12 +62,15 @@ def test_weight_quant_tiny_bit_exact(cr):
 # up to 8 CTAs (few rows, or rows of more than 32 groups), one CTA per row
 # (>= 148 rows), one or several groups per slot and a ragged last slot, and
 # the longest rows the API accepts; short rows of a tall matrix packed 16 or 8
-# to a CTA (a ragged last CTA included)
+# to a CTA (a ragged last CTA included); tall matrices of 16 to 128 groups
 @pytest.mark.parametrize("m,k", [(1, 256), (4, 512), (3, 768), (17, 5120), (2, 8448), (3, 16384),
                                  (2, 24576), (5, 25600), (2, 38912), (2, 40960), (2, 65536),
                                  (150, 512), (160, 8448), (148, 25600), (149, 40960), (200, 65536),
                                  (3, 133120), (150, 133120), (1200, 256), (1187, 256), (1190, 512),
-                                 (2048, 512)])
+                                 (2048, 512),
+                                 # tall matrices of long rows: persistent CTAs walking the rows
+                                 (300, 4096), (597, 5120), (1000, 8192), (320, 6144), (400, 25600),
+                                 (350, 32768)])
 def test_act_quant_bit_exact(cr, m, k):
     cs = synth.outlier_scale_fraction(synth.stream_key(m * 7 + k, 2), k, 0.01, 30.0)
     x_bits = synth.draw_np(synth.stream_key(m * 7 + k, 0), m, k, 1.0, cs)
