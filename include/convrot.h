@@ -365,14 +365,19 @@ convrot_status_t convrot_conv2d_shape(const convrot_conv2d_t *g, int32_t *oh, in
 convrot_status_t convrot_quantize_conv_weight(const void *w_oihw_bf16, const convrot_conv2d_t *g,
                                               const convrot_weight_t *out, void *stream);
 
-/* Workspace of convrot_conv2d_int8 (GEMM scratch + the INT8 im2col codes). */
+/* Workspace of convrot_conv2d_int8: GEMM scratch + the INT8 im2col codes and
+ * their row scales, and for kernels larger than 1x1 every input pixel's
+ * rotated FP32 values (n*h*w x c) and maxima.  0 for an invalid argument. */
 size_t convrot_conv2d_workspace_bytes(const convrot_conv2d_t *g, const convrot_weight_t *w);
 
 /*
  * y [n, oh, ow, w->n] (NHWC, BF16) = the INT8 ConvRot convolution of x
  * [n, h, w, c] (NHWC, BF16) with the handle from convrot_quantize_conv_weight.
- * Launches: the activation prologue (two kernels, one for 1x1), then the
- * INT8 GEMM with M = n * oh * ow, N = c_out, K = kh * kw * c.
+ * Launches: the activation prologue (two kernels, one for 1x1: every input
+ * pixel rotated once, then the im2col rows gathered from the rotated pixels
+ * and quantised), then the INT8 GEMM with M = n * oh * ow, N = c_out,
+ * K = kh * kw * c.  The codes equal those of rotating and quantising each
+ * im2col row directly.
  */
 convrot_status_t convrot_conv2d_int8(const void *x_nhwc_bf16, const convrot_conv2d_t *g, const convrot_weight_t *w,
                                      void *y_nhwc_bf16, void *ws, size_t ws_bytes, void *stream);
