@@ -878,7 +878,12 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
     *p = GemmPlan{};
     p->njobs = 1;
     p->swap = (m <= 256) ? 1 : 0;
-    p->bn = p->swap ? (int)((m + 15) / 16 * 16) : 256;
+    // an A operand streamed once from HBM against a single B tile (a
+    // convolution's im2col rows with few output channels): 128-row B tiles
+    // halve the ring stage, so twice the stages keep A in flight; the two
+    // B tiles of an A tile run in the same wave and share its rows in L2
+    const bool narrow = !p->swap && n <= 256 && (long long)m * k > kGroupABytes;
+    p->bn = p->swap ? (int)((m + 15) / 16 * 16) : (narrow ? 128 : 256);
     p->rows_a[0] = p->swap ? n : m;
     p->rows_b[0] = p->swap ? m : n;
     const int tiles_a = (int)((p->rows_a[0] + kTileA - 1) / kTileA);

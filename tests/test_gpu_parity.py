@@ -298,6 +298,17 @@ def test_minimax_qkv_m32768_sampled(cr):
     _sampled_layer_check(cr, lin, rows_w, rows_x)
 
 
+@pytest.mark.parametrize("n", [256, 200])
+def test_narrow_n_large_m_sampled(cr, n):
+    # 64 MB of INT8 activations against at most 256 weight rows: 128-row B
+    # tiles (two per A tile, the second ragged for n = 200), A in groups of 16
+    lin = synth.Linear("narrow", 65536, 1024, n, 31 + n)
+    rng = np.random.default_rng(n)
+    rows_w = np.unique(np.concatenate([[0, 127, 128, n - 1], rng.integers(0, n, 8)]))
+    rows_x = np.unique(np.concatenate([[0, 127, 128, 2047, 2048, lin.m - 1], rng.integers(0, lin.m, 10)]))
+    _sampled_layer_check(cr, lin, rows_w, rows_x)
+
+
 def test_grouped_tile_order_ragged_sampled(cr):
     # 79 A tiles = 4 groups of 16 + a ragged group of 15, 4 B tiles (the last
     # ragged), 316 tiles = 2 full waves + 20 tail tiles split along K
