@@ -376,6 +376,24 @@ def test_quantize_golden_ties():
         assert ties == sum(1 for v in ys.split() if float(v) % 1 == 0.5)
 
 
+def test_quantize_subnormal_scale_matches_numpy_definition():
+    # rows whose scale a / 127 is subnormal in FP32 (a < 127 * 2^-126): numpy's
+    # FP32 division (IEEE, gradual underflow) gives s and y / s; the codes
+    # stay in [-127, 127] and the row maximum still maps to +-127
+    rng = np.random.default_rng(11)
+    y = (rng.standard_normal((6, 256)) * np.float32(2.0 ** -126)).astype(np.float32)
+    y *= np.array([1, 4, 16, 0.25, 8, 0.03], dtype=np.float32)[:, None]
+    q, s, _ = oracle.quantize_rows(y)
+    a = np.max(np.abs(y), axis=1)
+    s_ref = (a / np.float32(127.0)).astype(np.float32)
+    assert np.all(s_ref < np.float32(1.17549435e-38)) and np.all(s_ref > 0)
+    assert np.array_equal(s.view(np.uint32), s_ref.view(np.uint32))
+    t = (y / s_ref[:, None]).astype(np.float32)
+    q_ref = np.clip(np.rint(t), -127, 127).astype(np.int8)
+    assert np.array_equal(q, q_ref)
+    assert np.all(np.abs(q[np.arange(6), np.argmax(np.abs(y), axis=1)]) == 127)
+
+
 def test_quantize_matches_numpy_definition():
     rng = np.random.default_rng(2)
     y = (rng.standard_normal((16, 1024)) * rng.uniform(0.01, 100, (16, 1))).astype(np.float32)
