@@ -358,6 +358,28 @@ typedef struct {
 convrot_status_t convrot_conv2d_shape(const convrot_conv2d_t *g, int32_t *oh, int32_t *ow);
 
 /*
+ * How convrot_conv2d_int8 gathers the im2col rows of a kernel larger than
+ * 1x1 on a GPU of `sms` SMs (host arithmetic only: no device is touched;
+ * for tests and tuning).  tiled = 1: persistent CTAs (one per SM, at most
+ * `tiles`) quantise th x tw tiles of output pixels of one image from the
+ * rotated pixels of the tile's input region, rh x rw pixels, staged in one of
+ * two shared-memory buffers of buf_bytes each (the region's FP32 values, one
+ * zero pixel, then the region's pixel maxima).  tiled = 0: more than 32 taps
+ * or no tile fits, and a warp per row gathers straight from global memory
+ * (the other fields are 0).  Errors: CONVROT_ERR_INVALID_ARG for a null
+ * pointer, sms < 1 or an invalid geometry, CONVROT_ERR_UNSUPPORTED_SHAPE for
+ * a 1x1 kernel (its rows are gathered and rotated in one step).
+ */
+typedef struct {
+    int32_t tiled;
+    int32_t th, tw;                 /* output pixels per tile (rows x columns) */
+    int32_t rh, rw;                 /* input pixels the tile reads */
+    int64_t tiles;                  /* n * ceil(oh / th) * ceil(ow / tw) */
+    int64_t buf_bytes;              /* one region buffer */
+} convrot_conv2d_plan_t;
+convrot_status_t convrot_conv2d_gather_plan(const convrot_conv2d_t *g, int32_t sms, convrot_conv2d_plan_t *out);
+
+/*
  * Offline: rotate and quantise a BF16 OIHW weight [c_out, c, kh, kw] into
  * the handle `out` (out->n = c_out, out->k = kh * kw * c, out->group dividing
  * c; convrot_dynamic_group(c, 256) picks it), rows in the im2col order.

@@ -67,6 +67,12 @@ class convrot_conv2d_t(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int32) for f in ("n", "h", "w", "c", "kh", "kw", "stride", "pad", "dilation")]
 
 
+class convrot_conv2d_plan_t(ctypes.Structure):
+    """Mirror of the C struct: how the im2col gather of a convolution runs."""
+    _fields_ = [("tiled", ctypes.c_int32), ("th", ctypes.c_int32), ("tw", ctypes.c_int32), ("rh", ctypes.c_int32),
+                ("rw", ctypes.c_int32), ("tiles", ctypes.c_int64), ("buf_bytes", ctypes.c_int64)]
+
+
 class convrot_gemm_job_t(ctypes.Structure):
     """Mirror of the C struct: one product of a batched GEMM call."""
     _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight_t)),
@@ -82,6 +88,7 @@ SIGNATURES = {
     "convrot_dynamic_group": ([_I64, _I32], _I32),
     "convrot_quantize_tensor": ([_P, _I64, _P, _P, _P], ctypes.c_int),
     "convrot_conv2d_shape": ([_P, _P, _P], ctypes.c_int),
+    "convrot_conv2d_gather_plan": ([_P, _I32, _P], ctypes.c_int),
     "convrot_quantize_conv_weight": ([_P, _P, _WP, _P], ctypes.c_int),
     "convrot_conv2d_workspace_bytes": ([_P, _WP], _SZ),
     "convrot_conv2d_int8": ([_P, _P, _WP, _P, _P, _SZ, _P], ctypes.c_int),
@@ -385,6 +392,16 @@ class LinearBatchW4:
 def conv2d_geometry(x_shape, kh: int, kw: int, stride: int = 1, pad: int = 0, dilation: int = 1) -> convrot_conv2d_t:
     n, h, w, c = x_shape
     return convrot_conv2d_t(n, h, w, c, kh, kw, stride, pad, dilation)
+
+
+def conv2d_gather_plan(x_shape, kh: int, kw: int, stride: int = 1, pad: int = 0, dilation: int = 1,
+                       sms: int = 148) -> convrot_conv2d_plan_t:
+    """The im2col gather's launch plan for a convolution (host only)."""
+    g = conv2d_geometry(x_shape, kh, kw, stride, pad, dilation)
+    out = convrot_conv2d_plan_t()
+    _check(load_library().convrot_conv2d_gather_plan(ctypes.byref(g), sms, ctypes.byref(out)),
+           "convrot_conv2d_gather_plan")
+    return out
 
 
 def quantize_conv_weight(w_oihw_bf16: torch.Tensor, stride: int = 1, pad: int = 0, dilation: int = 1,

@@ -516,6 +516,27 @@ convrot_status_t convrot_conv2d_shape(const convrot_conv2d_t *g, int32_t *oh, in
     return CONVROT_OK;
 }
 
+convrot_status_t convrot_conv2d_gather_plan(const convrot_conv2d_t *g, int32_t sms, convrot_conv2d_plan_t *out) {
+    if (!out || sms < 1) return CONVROT_ERR_INVALID_ARG;
+    convrot::ConvGeom cg;
+    convrot_status_t s = conv_geom(g, &cg);
+    if (s != CONVROT_OK) return s;
+    if (cg.kh * cg.kw == 1) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    *out = convrot_conv2d_plan_t{};
+    int th, tw, rh, rw;
+    int64_t tiles, bytes;
+    if (convrot::conv_gather_tile_plan(cg, sms, &th, &tw, &rh, &rw, &tiles, &bytes)) {
+        out->tiled = 1;
+        out->th = th;
+        out->tw = tw;
+        out->rh = rh;
+        out->rw = rw;
+        out->tiles = tiles;
+        out->buf_bytes = bytes;
+    }
+    return CONVROT_OK;
+}
+
 convrot_status_t convrot_quantize_conv_weight(const void *w_oihw_bf16, const convrot_conv2d_t *g,
                                               const convrot_weight_t *out, void *stream) {
     if (!w_oihw_bf16) return CONVROT_ERR_INVALID_ARG;

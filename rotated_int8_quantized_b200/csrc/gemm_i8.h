@@ -120,6 +120,10 @@ struct ConvGeom {
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl,
                                 const ConvGeom *conv = nullptr);
 
+// The tiled gather's shape for a geometry (false: the untiled gather runs).
+bool conv_gather_tile_plan(const ConvGeom &g, int sms, int *th, int *tw, int *rh, int *rw, int64_t *tiles,
+                           int64_t *buf_bytes);
+
 // Convolution im2col codes from pixels rotated once (yrot FP32 [n*h*w, c],
 // pmax [n*h*w]): codes xq [rows, kh*kw*c] and scales sx [rows].
 cudaError_t launch_conv_gather_quant(const float *yrot, const float *pmax, const ConvGeom &g, int64_t rows,

@@ -1311,6 +1311,19 @@ static bool conv_tile_shape(const ConvGeom &g, int sms, ConvTileArgs *A) {
     return true;
 }
 
+bool conv_gather_tile_plan(const ConvGeom &g, int sms, int *th, int *tw, int *rh, int *rw, int64_t *tiles,
+                           int64_t *buf_bytes) {
+    ConvTileArgs A;
+    if (!conv_tile_shape(g, sms, &A)) return false;
+    *th = A.th;
+    *tw = A.tw;
+    *rh = A.rh;
+    *rw = A.rw;
+    *tiles = A.ntiles;
+    *buf_bytes = A.buf_bytes;
+    return true;
+}
+
 cudaError_t launch_conv_gather_quant(const float *yrot, const float *pmax, const ConvGeom &g, int64_t rows,
                                      int8_t *xq, float *sx, cudaStream_t stream) {
     int dev = 0, sms = 148;

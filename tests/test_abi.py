@@ -123,6 +123,9 @@ int main(void) {
     printf("convrot_weight4_t %zu\n", sizeof(convrot_weight4_t));
     printf("convrot_linear4_job_t %zu\n", sizeof(convrot_linear4_job_t));
     F(convrot_weight4_t, group) F(convrot_linear4_job_t, bias_bf16)
+    printf("convrot_conv2d_t %zu\n", sizeof(convrot_conv2d_t));
+    printf("convrot_conv2d_plan_t %zu\n", sizeof(convrot_conv2d_plan_t));
+    F(convrot_conv2d_t, dilation) F(convrot_conv2d_plan_t, tiles) F(convrot_conv2d_plan_t, buf_bytes)
     return 0;
 }
 ''')
@@ -142,6 +145,11 @@ int main(void) {
         "convrot_linear4_job_t": ctypes.sizeof(cr.convrot_linear4_job_t),
         "convrot_weight4_t.group": cr.convrot_weight4_t.group.offset,
         "convrot_linear4_job_t.bias_bf16": cr.convrot_linear4_job_t.bias_bf16.offset,
+        "convrot_conv2d_t": ctypes.sizeof(cr.convrot_conv2d_t),
+        "convrot_conv2d_plan_t": ctypes.sizeof(cr.convrot_conv2d_plan_t),
+        "convrot_conv2d_t.dilation": cr.convrot_conv2d_t.dilation.offset,
+        "convrot_conv2d_plan_t.tiles": cr.convrot_conv2d_plan_t.tiles.offset,
+        "convrot_conv2d_plan_t.buf_bytes": cr.convrot_conv2d_plan_t.buf_bytes.offset,
     }
     assert {k: int(v) for k, v in got.items()} == want
 
