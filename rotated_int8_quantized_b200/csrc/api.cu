@@ -9,6 +9,7 @@
 #include "../../include/convrot.h"
 #include "common.cuh"
 #include "gemm_i8.h"
+#include "rotate_quant.h"
 
 namespace {
 

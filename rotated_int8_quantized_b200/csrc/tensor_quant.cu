@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "gemm_i8.h"
+#include "rotate_quant.h"
 
 namespace convrot {
 
