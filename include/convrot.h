@@ -148,6 +148,36 @@ convrot_status_t convrot_quantize_act(const void *x_bf16, int64_t m, int64_t k, 
  */
 size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
+/*
+ * How the GEMM kernel would tile a product (host arithmetic only: no device
+ * is touched; for tests and tuning).  count == 1: the single-product entry
+ * points (convrot_gemm_i8 / convrot_linear_int8) for m x k against n x k;
+ * count in 2..8 (m <= 512): one batched launch of `count` products with the
+ * same m (convrot_gemm_i8_batch / convrot_linear_int8_batch), w4 = 1 for
+ * INT4 weights (m <= 256).  A CTA c of the `grid` takes, in order: whole
+ * tiles wave * grid + c for wave < full_waves while below full_tiles; piece
+ * c of the split tail when c < split_pieces (tile full_tiles + c / split_ways,
+ * K blocks [s * kbpt / ways, (s + 1) * kbpt / ways) with s = c % ways); then
+ * the stream-K units [tail_units * q / Q, tail_units * (q + 1) / Q) with
+ * q = c / rep, Q = grid / rep, where unit u of job j (u - unit0[j] = t * kbpt
+ * + kb) is K block kb of tile tile_base[j] + t * rep + c % rep.  A tile of
+ * job j is (A tile, B tile) with tiles_a[j] x tiles_b[j] tiles; 128-byte K
+ * blocks, kbpt[j] per tile.  swap = 1: the weights are the 128-row A operand.
+ * Errors: CONVROT_ERR_INVALID_ARG (null pointers, count out of range, sizes
+ * < 1, sms < 1), CONVROT_ERR_UNSUPPORTED_SHAPE (a batch with m > 512, INT4
+ * with m > 256).
+ */
+typedef struct {
+    int32_t njobs, swap, bn, grid;
+    int32_t full_waves, full_tiles, split_ways, split_pieces;
+    int32_t rep, stages, tmem_cols, slots;
+    int64_t tail_units, smem_bytes, ws_bytes;
+    int32_t tiles_a[8], tiles_b[8], group_a[8], kbpt[8], tile_base[8];
+    int64_t unit0[8];
+} convrot_gemm_plan_t;
+convrot_status_t convrot_gemm_plan(int64_t m, int32_t count, const int64_t *n, const int64_t *k, int32_t w4,
+                                   int32_t sms, convrot_gemm_plan_t *out);
+
 /* Scratch bytes convrot_linear_int8 needs: the GEMM scratch followed by the
    quantised activations xq [m, k] and their scales sx [m]. */
 size_t convrot_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);

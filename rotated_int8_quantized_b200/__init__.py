@@ -73,6 +73,16 @@ class convrot_conv2d_plan_t(ctypes.Structure):
                 ("rw", ctypes.c_int32), ("tiles", ctypes.c_int64), ("buf_bytes", ctypes.c_int64)]
 
 
+class convrot_gemm_plan_t(ctypes.Structure):
+    """Mirror of the C struct: how the GEMM kernel tiles a product."""
+    _fields_ = [(f, ctypes.c_int32) for f in ("njobs", "swap", "bn", "grid", "full_waves", "full_tiles",
+                                               "split_ways", "split_pieces", "rep", "stages", "tmem_cols",
+                                               "slots")] + \
+               [(f, ctypes.c_int64) for f in ("tail_units", "smem_bytes", "ws_bytes")] + \
+               [(f, ctypes.c_int32 * 8) for f in ("tiles_a", "tiles_b", "group_a", "kbpt", "tile_base")] + \
+               [("unit0", ctypes.c_int64 * 8)]
+
+
 class convrot_gemm_job_t(ctypes.Structure):
     """Mirror of the C struct: one product of a batched GEMM call."""
     _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("w", ctypes.POINTER(convrot_weight_t)),
@@ -89,6 +99,7 @@ SIGNATURES = {
     "convrot_quantize_tensor": ([_P, _I64, _P, _P, _P], ctypes.c_int),
     "convrot_conv2d_shape": ([_P, _P, _P], ctypes.c_int),
     "convrot_conv2d_gather_plan": ([_P, _I32, _P], ctypes.c_int),
+    "convrot_gemm_plan": ([_I64, _I32, _P, _P, _I32, _I32, _P], ctypes.c_int),
     "convrot_quantize_conv_weight": ([_P, _P, _WP, _P], ctypes.c_int),
     "convrot_conv2d_workspace_bytes": ([_P, _WP], _SZ),
     "convrot_conv2d_int8": ([_P, _P, _WP, _P, _P, _SZ, _P], ctypes.c_int),
@@ -392,6 +403,18 @@ class LinearBatchW4:
 def conv2d_geometry(x_shape, kh: int, kw: int, stride: int = 1, pad: int = 0, dilation: int = 1) -> convrot_conv2d_t:
     n, h, w, c = x_shape
     return convrot_conv2d_t(n, h, w, c, kh, kw, stride, pad, dilation)
+
+
+def gemm_plan(m: int, ns, ks, w4: bool = False, sms: int = 148) -> convrot_gemm_plan_t:
+    """How the GEMM kernel tiles one product (len(ns) == 1) or a batched
+    launch of several (host only)."""
+    count = len(ns)
+    n_arr = (ctypes.c_int64 * count)(*ns)
+    k_arr = (ctypes.c_int64 * count)(*ks)
+    out = convrot_gemm_plan_t()
+    _check(load_library().convrot_gemm_plan(m, count, n_arr, k_arr, 1 if w4 else 0, sms, ctypes.byref(out)),
+           "convrot_gemm_plan")
+    return out
 
 
 def conv2d_gather_plan(x_shape, kh: int, kw: int, stride: int = 1, pad: int = 0, dilation: int = 1,

@@ -181,6 +181,44 @@ size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
 }
 
 
+convrot_status_t convrot_gemm_plan(int64_t m, int32_t count, const int64_t *n, const int64_t *k, int32_t w4,
+                                   int32_t sms, convrot_gemm_plan_t *out) {
+    if (!out || !n || !k || count < 1 || count > kMaxBatch || m < 1 || sms < 1) return CONVROT_ERR_INVALID_ARG;
+    for (int j = 0; j < count; ++j)
+        if (n[j] < 1 || k[j] < 1) return CONVROT_ERR_INVALID_ARG;
+    if ((count > 1 && m > convrot::kMaxSwapM) || (w4 && m > 256)) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    convrot::GemmPlan p;
+    if (count == 1 && !w4)
+        convrot::plan_gemm(m, n[0], k[0], sms, &p);
+    else
+        convrot::plan_gemm_batch(m, count, n, k, sms, &p, w4 != 0);
+    *out = convrot_gemm_plan_t{};
+    out->njobs = p.njobs;
+    out->swap = p.swap;
+    out->bn = p.bn;
+    out->grid = p.grid;
+    out->full_waves = p.full_waves;
+    out->full_tiles = p.full_tiles;
+    out->split_ways = p.split_ways;
+    out->split_pieces = p.split_pieces;
+    out->rep = p.rep > 0 ? p.rep : 1;   // as the launch passes it
+    out->stages = p.stages;
+    out->tmem_cols = p.tmem_cols;
+    out->slots = p.slots;
+    out->tail_units = p.tail_units;
+    out->smem_bytes = p.smem_bytes;
+    out->ws_bytes = (int64_t)p.ws_bytes;
+    for (int j = 0; j < p.njobs; ++j) {
+        out->tiles_a[j] = p.tiles_a[j];
+        out->tiles_b[j] = p.tiles_b[j];
+        out->group_a[j] = p.group_a[j];
+        out->kbpt[j] = p.kbpt[j];
+        out->tile_base[j] = p.tile_base[j];
+        out->unit0[j] = p.unit0[j];
+    }
+    return CONVROT_OK;
+}
+
 convrot_status_t convrot_workspace_init(void *ws, size_t ws_bytes, void *stream) {
     if (!ws && ws_bytes) return CONVROT_ERR_INVALID_ARG;
     if (!ws_bytes) return CONVROT_OK;

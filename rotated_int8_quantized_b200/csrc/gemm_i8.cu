@@ -966,7 +966,8 @@ void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, i
         p->unit0[j] = units;
         units += (long long)(p->swap ? p->tiles_a[j] : p->tiles_b[j]) * p->kbpt[j];
     }
-    const long long groups = num_sms / p->rep;
+    // (at least one group: a GPU with fewer SMs than replicas still runs)
+    const long long groups = num_sms >= p->rep ? num_sms / p->rep : 1;
     p->grid = (int)(units < groups ? units : groups) * p->rep;
     p->full_waves = 0;
     p->slots = p->grid;

@@ -1,0 +1,120 @@
+"""The GEMM launch plan (host arithmetic, no GPU): every (job, tile, K block)
+of a product is processed by exactly one CTA, and each plan fits the SM.
+
+The coverage model restates, in plain Python, the order in which a CTA takes
+its work (as the header documents for convrot_gemm_plan): whole tiles in
+full waves, a piece of the split tail, then a contiguous range of stream-K
+units.
+"""
+import collections
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+SMS = 148
+SMEM_PER_CTA = 227 * 1024
+
+
+def covered_units(p):
+    """(job, tile, kb) -> how many CTAs process it."""
+    seen = collections.Counter()
+    for c in range(p.grid):
+        wave = 0
+        while wave < p.full_waves and wave * p.grid + c < p.full_tiles:
+            tile = wave * p.grid + c
+            for kb in range(p.kbpt[0]):
+                seen[(0, tile, kb)] += 1
+            wave += 1
+        if p.split_ways > 1 and c < p.split_pieces:
+            slot, piece = divmod(c, p.split_ways)
+            kbpt = p.kbpt[0]
+            for kb in range(piece * kbpt // p.split_ways, (piece + 1) * kbpt // p.split_ways):
+                seen[(0, p.full_tiles + slot, kb)] += 1
+        rep = p.rep
+        q, r = divmod(c, rep)
+        groups = p.grid // rep
+        u, u_end = p.tail_units * q // groups, p.tail_units * (q + 1) // groups
+        j = 0
+        while u < u_end:
+            while j + 1 < p.njobs and u >= p.unit0[j + 1]:
+                j += 1
+            lu = u - p.unit0[j]
+            t, kb0 = divmod(lu, p.kbpt[j])
+            kb1 = min(kb0 + (u_end - u), p.kbpt[j])
+            tile = p.tile_base[j] + t * rep + r
+            for kb in range(kb0, kb1):
+                seen[(j, tile, kb)] += 1
+            u += kb1 - kb0
+    return seen
+
+
+def check(p, m, ns, ks):
+    assert p.njobs == len(ns)
+    assert p.grid >= 1 and p.grid <= SMS and p.grid % p.rep == 0
+    assert 2 <= p.stages <= 8 and p.smem_bytes <= SMEM_PER_CTA
+    assert p.tmem_cols <= 512 and p.tmem_cols & (p.tmem_cols - 1) == 0 and p.tmem_cols >= 2 * p.bn
+    want = set()
+    for j, (n, k) in enumerate(zip(ns, ks)):
+        rows_a, rows_b = (n, m) if p.swap else (m, n)
+        assert p.tiles_a[j] == -(-rows_a // 128) and p.tiles_b[j] == -(-rows_b // p.bn)
+        assert p.kbpt[j] == -(-k // 128)
+        for tile in range(p.tiles_a[j] * p.tiles_b[j]):
+            for kb in range(p.kbpt[j]):
+                want.add((j, tile, kb))
+    seen = covered_units(p)
+    assert set(seen) == want
+    assert max(seen.values()) == 1
+
+
+QWEN_N = [8192, 1024, 1024, 5120, 25600, 25600, 5120]
+QWEN_K = [5120, 5120, 5120, 8192, 5120, 5120, 25600]
+
+
+@pytest.mark.parametrize("m,n,k", [
+    (4, 256, 512), (12, 8192, 5120), (12, 1024, 5120), (17, 5120, 25600), (256, 768, 1024),
+    (300, 768, 1024), (400, 5120, 5120), (512, 25600, 5120),                  # a few hundred rows
+    (4096, 8192, 5120), (4096, 1024, 5120), (4096, 25600, 5120), (4096, 5120, 25600),
+    (8192, 16128, 5376), (32768, 16128, 5376),                                  # A in groups of 16 tiles
+    (65536, 256, 2304), (65536, 200, 1024), (10112, 1000, 5376),                # narrow B, ragged
+])
+def test_single_product_covers_every_block_once(m, n, k):
+    import rotated_int8_quantized_b200 as cr
+    p = cr.gemm_plan(m, [n], [k], sms=SMS)
+    check(p, m, [n], [k])
+    if m <= 256:
+        assert p.swap == 1
+    if m > 512:
+        assert p.swap == 0 and p.rep == 1
+
+
+@pytest.mark.parametrize("m", [1, 12, 100, 256, 257, 400, 512])
+def test_batched_layer_covers_every_block_once(m):
+    import rotated_int8_quantized_b200 as cr
+    p = cr.gemm_plan(m, QWEN_N, QWEN_K, sms=SMS)
+    check(p, m, QWEN_N, QWEN_K)
+    assert p.full_waves == 0 and p.tail_units == sum(
+        (p.tiles_a[j] if p.swap else p.tiles_b[j]) * p.kbpt[j] for j in range(7))
+
+
+def test_int4_batch_and_other_gpu_sizes():
+    import rotated_int8_quantized_b200 as cr
+    p = cr.gemm_plan(12, QWEN_N, QWEN_K, w4=True, sms=SMS)
+    check(p, 12, QWEN_N, QWEN_K)
+    for sms in (1, 7, 64, 132):
+        for (m, n, k) in ((12, 5120, 8192), (4096, 8192, 5120), (400, 5120, 5120)):
+            check(cr.gemm_plan(m, [n], [k], sms=sms), m, [n], [k])
+
+
+def test_plan_rejections():
+    import rotated_int8_quantized_b200 as cr
+    with pytest.raises(cr.ConvrotError):
+        cr.gemm_plan(600, [1024, 1024], [512, 512])      # batches are for m <= 512
+    with pytest.raises(cr.ConvrotError):
+        cr.gemm_plan(300, [1024], [512], w4=True)        # INT4 weights: m <= 256
+    with pytest.raises(cr.ConvrotError):
+        cr.gemm_plan(12, [1024], [512], sms=0)
