@@ -125,3 +125,27 @@ def test_untiled_and_rejected_plans():
         cr.conv2d_gather_plan((1, 16, 16, 64), 1, 1)                              # 1x1: one-step gather
     with pytest.raises(cr.ConvrotError):
         cr.conv2d_gather_plan((1, 16, 16, 64), 3, 3, sms=0)
+
+
+def test_random_geometries_stay_in_bounds():
+    # seeded sweep: small images (so every code is modelled) over channel
+    # counts, kernel sizes, strides, paddings and dilations
+    import rotated_int8_quantized_b200 as cr
+    rng = np.random.default_rng(7)
+    tried = 0
+    while tried < 60:
+        k = int(rng.choice([2, 3, 4, 5]))
+        stride, dil = int(rng.integers(1, 3)), int(rng.integers(1, 3))
+        pad = int(rng.integers(0, k))
+        n, h, w = int(rng.integers(1, 3)), int(rng.integers(k, 14)), int(rng.integers(k, 14))
+        c = int(rng.choice([16, 32, 48, 64, 128, 256, 512]))
+        if out_size(h, k, stride, pad, dil) < 1 or out_size(w, k, stride, pad, dil) < 1:
+            continue
+        plan = cr.conv2d_gather_plan((n, h, w, c), k, k, stride, pad, dil, int(rng.choice([1, 8, 148])))
+        if plan.tiled == 0:
+            # only when not even one output pixel's region fits a buffer
+            r1 = (k - 1) * dil + 1
+            assert (r1 * r1 + 1) * c * 4 + r1 * r1 * 4 > SMEM_TWO_BUFFERS // 2
+            continue
+        check_plan(n, h, w, c, k, stride, pad, dil, plan)
+        tried += 1

@@ -118,3 +118,25 @@ def test_plan_rejections():
         cr.gemm_plan(300, [1024], [512], w4=True)        # INT4 weights: m <= 256
     with pytest.raises(cr.ConvrotError):
         cr.gemm_plan(12, [1024], [512], sms=0)
+
+
+def test_random_shapes_cover_every_block_once():
+    # seeded sweep over shapes and SM counts (single products and batches),
+    # sized so the coverage model stays quick
+    import numpy as np
+    import rotated_int8_quantized_b200 as cr
+    rng = np.random.default_rng(2024)
+    for _ in range(150):
+        sms = int(rng.choice([1, 3, 8, 37, 132, 148]))
+        if rng.random() < 0.5:
+            m = int(rng.choice([1, 5, 12, 100, 256, 257, 300, 511, 512, 513, 1000, 3000, 9000]))
+            n = int(rng.integers(1, 40)) * 16 * int(rng.choice([1, 4, 16]))
+            k = int(rng.integers(1, 64)) * 16 * int(rng.choice([1, 2, 8]))
+            check(cr.gemm_plan(m, [n], [k], sms=sms), m, [n], [k])
+        else:
+            m = int(rng.choice([1, 7, 12, 64, 200, 256, 300, 512]))
+            count = int(rng.integers(2, 9))
+            ns = [int(rng.integers(1, 50)) * 64 for _ in range(count)]
+            ks = [int(rng.integers(1, 40)) * 128 for _ in range(count)]
+            w4 = bool(m <= 256 and rng.random() < 0.3)
+            check(cr.gemm_plan(m, ns, ks, w4=w4, sms=sms), m, ns, ks)
