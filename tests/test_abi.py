@@ -201,3 +201,47 @@ def test_conv2d_shape_and_validation(lib):
     assert lib.convrot_conv2d_workspace_bytes(ctypes.byref(g3), ctypes.byref(h)) > 0
     g4 = cr.convrot_conv2d_t(1, 8, 8, 96, 1, 1, 1, 0, 1)         # k mismatch
     assert lib.convrot_conv2d_workspace_bytes(ctypes.byref(g4), ctypes.byref(h)) == 0
+
+
+def test_plain_c_program_uses_the_library(tmp_path):
+    """The C ABI needs no Python: a C99 program compiled against
+    include/convrot.h and linked with libconvrot.so calls the host-only
+    entry points (version, status strings, argument checks, dynamic group,
+    plan queries) and checks their answers."""
+    import subprocess
+    import rotated_int8_quantized_b200 as cr
+    lib_dir = os.path.dirname(cr.LIB_PATH)
+    src = tmp_path / "use.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "convrot.h"
+#define CHECK(c) do { if (!(c)) { printf("FAIL %s:%d %s\n", __FILE__, __LINE__, #c); return 1; } } while (0)
+int main(void) {
+    CHECK(convrot_version() >= 100);
+    CHECK(strcmp(convrot_status_string(CONVROT_OK), "CONVROT_OK") == 0);
+    CHECK(convrot_dynamic_group(5376, 256) == 256 && convrot_dynamic_group(640, 256) == 128);
+    convrot_weight_t w;
+    CHECK(convrot_weight_init(&w, NULL, NULL, 256, 512, 256) != CONVROT_OK);      /* null storage */
+    int64_t n[7] = {8192, 1024, 1024, 5120, 25600, 25600, 5120};
+    int64_t k[7] = {5120, 5120, 5120, 8192, 5120, 5120, 25600};
+    convrot_gemm_plan_t p;
+    CHECK(convrot_gemm_plan(12, 7, n, k, 0, 148, &p) == CONVROT_OK);
+    CHECK(p.njobs == 7 && p.swap == 1 && p.bn == 16 && p.grid == 148);
+    CHECK(p.tail_units == 29760 && p.full_waves == 0);
+    CHECK(convrot_gemm_plan(600, 2, n, k, 0, 148, &p) == CONVROT_ERR_UNSUPPORTED_SHAPE);
+    convrot_conv2d_t g = {1, 256, 256, 256, 3, 3, 1, 1, 1};
+    int32_t oh = 0, ow = 0;
+    CHECK(convrot_conv2d_shape(&g, &oh, &ow) == CONVROT_OK && oh == 256 && ow == 256);
+    convrot_conv2d_plan_t cp;
+    CHECK(convrot_conv2d_gather_plan(&g, 148, &cp) == CONVROT_OK && cp.tiled == 1);
+    CHECK(cp.tiles == (int64_t)(256 / cp.th + (256 % cp.th != 0)) * (256 / cp.tw + (256 % cp.tw != 0)));
+    printf("ok\n");
+    return 0;
+}
+''')
+    exe = tmp_path / "use"
+    subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                           "-L", lib_dir, "-l:libconvrot.so", "-Wl,-rpath," + lib_dir])
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
