@@ -310,8 +310,9 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Layout of the rotated pixels (MODE 5): FP32 [pixels, c], and inside each
-// 16-value chunk ci of a pixel, float4 part j stored at position
+// Layout of the rotated pixels (MODE 5 / 6, rotate_pixels_kernel): FP32
+// [pixels, c], and inside each 16-value chunk ci of a pixel, float4 part j
+// stored at position
 // j ^ yrot_swizzle(ci), so that 8 lanes reading 8 consecutive chunks one
 // float4 part at a time hit 8 different 16-byte bank groups.
 __host__ __device__ __forceinline__ int yrot_swizzle(int ci) { return (ci >> 1) & 3; }
@@ -334,7 +335,7 @@ __host__ __device__ __forceinline__ int yrot_swizzle(int ci) { return (ci >> 1) 
 // 3: INT8 codes of the im2col rows of a convolution, gathered from NHWC
 // input; 4: INT8 codes of a convolution's OIHW weight in the im2col order;
 // 5: the rotated FP32 rows themselves and their maxima (no quantisation):
-// every input pixel of a convolution rotated once, for conv_gather_quant;
+// every input pixel of a convolution rotated once, for the im2col gather;
 // 6: the same with groups of 256 and whole 256-chunks (no DYN paths).
 template <int GPS, bool HALF, int MODE, bool MR = false>
 __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
