@@ -189,6 +189,30 @@ def test_gemm_acc_and_y_bit_exact(cr, m, n, k):
     assert int(ws.count_nonzero()) == 0      # workspace returned to zero
 
 
+@pytest.mark.parametrize("m,n,k", [(32, 1024, 5120), (64, 512, 768), (400, 640, 5120), (4096, 1024, 5120)])
+def test_int32_accumulators_match_a_vendor_int8_gemm(cr, m, n, k):
+    # a second opinion, run not read: a library INT8 GEMM (torch._int_mm,
+    # cuBLASLt) on the same INT8 operands; both INT32 products are exact
+    if not hasattr(torch, "_int_mm"):
+        pytest.skip("torch._int_mm unavailable")
+    gen = torch.Generator(device="cuda").manual_seed(m * 7 + n * 3 + k)
+    xq = torch.randint(-127, 128, (m, k), generator=gen, device="cuda", dtype=torch.int32).to(torch.int8)
+    wq = torch.randint(-127, 128, (n, k), generator=gen, device="cuda", dtype=torch.int32).to(torch.int8)
+    sx = torch.ones(m, dtype=torch.float32, device="cuda")
+    sw = torch.ones(n, dtype=torch.float32, device="cuda")
+    w = cr.convrot_weight_init(wq, sw)
+    acc = torch.empty((m, n), dtype=torch.int32, device="cuda")
+    ws = cr.make_workspace(m, w, linear=False)
+    cr.convrot_gemm_i8(xq, sx, w, None, acc, ws)
+    cr.convrot_device_status()
+    try:
+        ref = torch._int_mm(xq, wq.t())
+    except RuntimeError as e:
+        pytest.skip("torch._int_mm does not take this shape here: %s" % e)
+    torch.cuda.synchronize()
+    assert torch.equal(acc, ref)
+
+
 @pytest.mark.parametrize("m,n,k", [(4, 256, 512), (12, 1024, 5120), (300, 768, 1024)])
 def test_linear_end_to_end(cr, m, n, k):
     x_bits, w, ref = _gemm_case(cr, m, n, k, seed=m + n + k)
