@@ -96,6 +96,13 @@ const char *convrot_status_string(convrot_status_t status);
 /* Library version as 10000 * major + 100 * minor + patch. */
 int convrot_version(void);
 
+/* Identity of this build: 16 hex digits of SHA-256 over the compile flags
+   and the CUDA sources the library was compiled from ("unknown" for a build
+   made without the build script).  Static string, never NULL.  The Python
+   binding refuses a library whose id differs from its sources' hash and
+   rebuilds it; no passage of the source pages corresponds to this call. */
+const char *convrot_build_id(void);
+
 /* Text of the last CUDA error this thread's calls turned into
    CONVROT_ERR_CUDA ("no error" if none).  Static string, never NULL. */
 const char *convrot_last_error_string(void);
@@ -281,15 +288,21 @@ size_t convrot_linear_batch_workspace_bytes(int64_t m, int count, const convrot_
  * convrot_gemm_i8 for callers that cannot allocate device memory: the same
  * product and outputs (xq, sx, w, y_bf16, acc as for convrot_gemm_i8), but
  * with no workspace argument.  Its scratch is an array of 8 MiB built into
- * the library (held on every GPU that loads the library until the process
- * exits).  It is meant for code that must not call cudaMalloc where it runs
- * the layer -- for example a plugin inside an engine that owns all device
- * memory through its own pool -- and cannot be handed a workspace either.
- * (The source pages have no counterpart of this entry point; it is an
- * integration convenience.)
- *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before
- *     any stream capture.
+ * the library.  The array is part of the library's single device module, so
+ * every process that loads libconvrot pays its 8 MiB on each device the
+ * library is used on, until the process exits, whether or not it ever calls
+ * this entry point.  It is meant for code that must not call cudaMalloc
+ * where it runs the layer -- for example a plugin inside an engine that owns
+ * all device memory through its own pool -- and cannot be handed a
+ * workspace either.  (The source pages have no counterpart of this entry
+ * point; it is an integration convenience.)
+ *   - The first call in a CUDA context looks up the array's device address
+ *     (with cudaGetSymbolAddress, with that context's device current) and
+ *     keeps it for that context; a new context (after cudaDeviceReset, for
+ *     instance) looks it up again.  The lookup can load the library's
+ *     module (lazily, under CUDA_MODULE_LOADING=LAZY), which must not
+ *     happen during a stream capture: make the first call on each device
+ *     before any stream capture starts, whatever is being captured.
  *   - Problems whose scratch needs more than 8 MiB are rejected with
  *     CONVROT_ERR_WORKSPACE before anything is launched
  *     (convrot_last_error_string says so).  convrot_gemm_workspace_bytes

@@ -95,6 +95,7 @@ _WP = ctypes.POINTER(convrot_weight_t)
 SIGNATURES = {
     "convrot_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "convrot_version": ([], ctypes.c_int),
+    "convrot_build_id": ([], ctypes.c_char_p),
     "convrot_dynamic_group": ([_I64, _I32], _I32),
     "convrot_quantize_tensor": ([_P, _I64, _P, _P, _P], ctypes.c_int),
     "convrot_conv2d_shape": ([_P, _P, _P], ctypes.c_int),
@@ -130,9 +131,17 @@ _lib = None
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libconvrot.so (raises if it has not been built)."""
+    """Load libconvrot.so.  The in-tree library is first rebuilt if it is
+    missing or its build id differs from the hash of the sources beside it;
+    after loading, its id must equal that hash (ImportError otherwise:
+    there is no fallback path)."""
     global _lib
     if _lib is None:
+        from . import build as _build
+        expected = None
+        if os.path.abspath(path) == os.path.abspath(LIB_PATH):
+            _build.build()
+            expected = _build.source_hash()
         if not os.path.exists(path):
             raise ImportError("libconvrot.so is not built (run rotated_int8_quantized_b200/build.py); "
                               "there is no fallback path")
@@ -141,8 +150,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.argtypes = args
             fn.restype = res
+        if expected is not None and lib.convrot_build_id().decode() != expected:
+            raise ImportError("libconvrot.so (build %s) was not built from the sources beside it (%s)"
+                              % (lib.convrot_build_id().decode(), expected))
         _lib = lib
     return _lib
+
+
+def build_id() -> str:
+    """The loaded library's build id (hash of the sources it was built from)."""
+    return load_library().convrot_build_id().decode()
 
 
 def _check(status: int, where: str) -> None:

@@ -11,6 +11,12 @@
 #include "gemm_i8.h"
 #include "rotate_quant.h"
 
+// Hash of the sources and flags this library was compiled from (set by the
+// build script; a build without it says so).
+#ifndef CONVROT_BUILD_ID
+#define CONVROT_BUILD_ID "unknown"
+#endif
+
 namespace {
 
 constexpr int64_t kGroup = 256;         // the pages' group; also the largest
@@ -124,6 +130,8 @@ const char *convrot_status_string(convrot_status_t s) {
 }
 
 int convrot_version(void) { return 100; }
+
+const char *convrot_build_id(void) { return CONVROT_BUILD_ID; }
 
 int32_t convrot_dynamic_group(int64_t k, int32_t max_group) {
     if (k < 1 || max_group < 1) return 0;

@@ -11,13 +11,16 @@
 // inputs and outputs.
 //
 // The array holds kStaticScratchBytes (8 MiB) on every GPU that loads the
-// library, until the process exits.  Problems whose scratch would not fit
-// are rejected with CONVROT_ERR_WORKSPACE before anything is launched.
-// Every call on a device uses the same array, so calls whose GPU work
-// overlaps (different streams, or host threads racing) corrupt each other.
+// library's module, until the process exits -- also in processes that
+// never call this entry point, since the array is part of the library's one
+// module.  Problems whose scratch would not fit are rejected with
+// CONVROT_ERR_WORKSPACE before anything is launched.  Every call on a
+// device uses the same array, so calls whose GPU work overlaps (different
+// streams, or host threads racing) corrupt each other.
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace {
@@ -28,26 +31,80 @@ constexpr size_t kStaticScratchBytes = 8u << 20;
 // the address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void *g_scratch_addr[kMaxDevices] = {};
+// The array's address belongs to the module loaded in one CUDA context: a
+// cudaDeviceReset (or any teardown of the primary context) unloads the
+// module, and the next context may place the array elsewhere.  So the
+// cached address is keyed on the current context's unique id, not on the
+// device index, and is looked up again whenever the id changes.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Device address of the array on the current device, looked up once per
-// device (with that device current) and cached.
-convrot_status_t static_scratch_address(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        cudaGetLastError();
-        return CONVROT_ERR_CUDA;
-    }
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
+struct ScratchEntry {
+    unsigned long long ctx_id;   // 0: empty
+    void *addr;
+};
+constexpr int kScratchEntries = 64;
+std::mutex g_scratch_mutex;
+ScratchEntry g_scratch_cache[kScratchEntries] = {};
+
+// Unique id of the current context, 0 if none is current or the driver
+// entry points are unavailable.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
         void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess || !p) return from_cuda(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
-        g_scratch_addr[dev] = p;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+        cudaGetLastError();
+        looked_up = true;
     }
-    *out = g_scratch_addr[dev];
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of the array in the current context.  The first call in
+// a context looks it up with cudaGetSymbolAddress (which may load the
+// library's module into that context); later calls in the same context
+// reuse it.  Without a context id (no driver entry points) every call looks
+// it up.
+convrot_status_t static_scratch_address(void **out) {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    unsigned long long id = current_context_id();
+    if (id != 0) {
+        for (int i = 0; i < kScratchEntries; ++i) {
+            if (g_scratch_cache[i].ctx_id == id) {
+                *out = g_scratch_cache[i].addr;
+                return CONVROT_OK;
+            }
+        }
+    }
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p) return from_cuda(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+    // the lookup makes the context current if none was: take its id now
+    if (id == 0) id = current_context_id();
+    if (id != 0) {
+        int slot = (int)(id % kScratchEntries);     // table full: overwrite one entry
+        for (int i = 0; i < kScratchEntries; ++i) {
+            if (g_scratch_cache[i].ctx_id == 0) {
+                slot = i;
+                break;
+            }
+        }
+        g_scratch_cache[slot] = {id, p};
+    }
+    *out = p;
     return CONVROT_OK;
 }
 

@@ -1,9 +1,12 @@
 """convrot_gemm_i8_noalloc: the GEMM entry point for callers that cannot pass
 a device workspace (for example a plugin whose host engine owns all device
 memory and forbids outside allocations).  It keeps its scratch in an array
-built into the library.  Checked against convrot_gemm_i8 (which uses a
-caller workspace) through the C ABI, on two calls in a row, so a second call
-sees the array the first one left behind.
+built into the library.  Checked through the C ABI, on two calls in a row (so
+the second call sees the array the first one left behind), against the
+oracle and against convrot_gemm_i8 (which uses a caller workspace): the same
+plan and kernel, so the INT32 accumulators and the BF16 outputs must be
+bit-identical.  The shapes take the stream-K paths, where the scratch is
+actually used.
 
 This file is named to be collected last, so that a run stopping at the
 first failure has already run every other test.
@@ -14,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -49,7 +53,10 @@ def test_noalloc_matches_workspace_entry_point(cr, m, n, k):
     dev = "cuda"
     seed = 7 * m + n + k
     x = synth.draw_torch(synth.stream_key(seed, 0), m, k, device=dev)
-    w = cr.quantize_weight(synth.draw_torch(synth.stream_key(seed, 1), n, k, synth.W_SIGMA, device=dev))
+    w_bits = synth.draw_np(synth.stream_key(seed, 1), n, k, synth.W_SIGMA)
+    w = cr.quantize_weight(torch.from_numpy(w_bits.view(np.int16)).view(torch.bfloat16).to(dev))
+    wq_ref, sw_ref = oracle.rotate_quantize(w_bits)
+    ref = oracle.linear_int8(synth.draw_np(synth.stream_key(seed, 0), m, k), wq_ref, sw_ref)
     xq = torch.empty((m, k), dtype=torch.int8, device=dev)
     sx = torch.empty((m,), dtype=torch.float32, device=dev)
     cr.convrot_quantize_act(x, xq, sx)
@@ -63,6 +70,9 @@ def test_noalloc_matches_workspace_entry_point(cr, m, n, k):
         cr.convrot_device_status()
         assert _rel_err(y, y_ref) <= TOL, "call %d" % call
         assert torch.equal(acc, acc_ref), "call %d" % call
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16)), "call %d" % call
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"]), "call %d" % call
+        assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), ref["y"]), "call %d" % call
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cr):
