@@ -41,8 +41,8 @@ METRIC = "ConvRot INT8 linear TOPS & weight-stream GB/s on 1 B200, % of INT8/HBM
 UNIT = "GB/s"
 WORKLOAD = "qwen3vl32b_layer_7linears_decode_m12"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-INT8_OVER_BF16 = 2.0     # nominal dense ratio (4.5 / 2.25 PFLOP/s)
-CPU_SAMPLE_ROWS_DIV = 64  # oracle sample: the first N/64 weight rows of every linear
+INT8_OVER_BF16 = 2.0     # nominal dense ratio (4.5 / 2.25 PFLOP/s), a note beside the measured INT8 peak
+CPU_SAMPLE_ROWS_DIV = 64  # reference arm: each step one linear with its first N/64 weight rows
 
 
 # --------------------------------------------------------------------------- helpers
@@ -131,15 +131,21 @@ class ClockSampler:
     def mark(self, t0, t1):
         self.windows.append((t0, t1))
 
-    def stop(self):
+    def stop(self, windows=None):
+        """Stop sampling; the summary over the marked windows (or the given
+        ones)."""
         if self.proc is None:
             return None
-        time.sleep(0.1)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
+        if self.proc.poll() is None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return self.summary(self.windows if windows is None else windows)
+
+    def summary(self, windows):
         sm, smax, reasons, n_all = [], None, set(), 0
         for t, line in self.rows:
             parts = [p.strip() for p in line.split(",")]
@@ -148,7 +154,7 @@ class ClockSampler:
             if self.pci and not parts[2].lower().endswith(self.pci):
                 continue
             n_all += 1
-            if not any(a - 0.05 <= t <= b + 0.05 for a, b in self.windows):
+            if not any(a - 0.05 <= t <= b + 0.05 for a, b in windows):
                 continue
             try:
                 sm.append(float(parts[3]))
@@ -161,6 +167,33 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
                 "reasons": sorted(reasons), "samples": len(sm), "samples_all": n_all}
+
+
+def measure_int8_peak(device, n: int = 8192, reps: int = 10):
+    """The dense INT8 tensor peak as a library reaches it on this GPU: a
+    large torch._int_mm (cuBLASLt INT8 x INT8 -> INT32, A row-major, B
+    column-major) of n x n x n, 2 n^3 ops, best of `reps` CUDA-event-timed
+    launches after warm-up (run, not read)."""
+    gen = torch.Generator(device=device).manual_seed(8)
+    a = torch.randint(-127, 128, (n, n), generator=gen, device=device, dtype=torch.int32).to(torch.int8)
+    b = torch.randint(-127, 128, (n, n), generator=gen, device=device, dtype=torch.int32).to(torch.int8)
+    bt = b.t()
+    for _ in range(3):
+        torch._int_mm(a, bt)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(a, bt)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    ops = 2.0 * n ** 3
+    del a, b, bt
+    torch.cuda.empty_cache()
+    return {"tops": ops / min(times) / 1e12, "median_tops": ops / statistics.median(times) / 1e12,
+            "shape": [n, n, n], "how": "torch._int_mm (cuBLASLt INT8 -> INT32), best of %d, CUDA events" % reps}
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -289,23 +322,34 @@ def gemm_kernel_times(cr, layer, lins, xs, reps, stream, device):
     return out
 
 
-def prologue_kernel_times(cr, lins, xs, reps, stream, device):
+def prologue_kernel_times(cr, lins, xs, reps, stream, device, l2_bytes=126 << 20):
     """Per-launch time of the activation prologue (rotation + row
-    quantisation) per linear, CUDA events on the launching stream."""
+    quantisation) per linear, CUDA events on the launching stream.  The
+    launches cycle through enough distinct inputs and outputs (copies of the
+    linear's activations) that together they exceed twice the L2, so every
+    launch reads its input from HBM."""
     out = []
     for lin, x in zip(lins, xs):
-        xq = torch.empty((lin.m, lin.k), dtype=torch.int8, device=device)
-        sx = torch.empty((lin.m,), dtype=torch.float32, device=device)
+        per = 3 * lin.m * lin.k
+        copies = max(1, min(8, -(-2 * l2_bytes // per)))
+        srcs = [x] + [x.clone() for _ in range(copies - 1)]
+        xqs = [torch.empty((lin.m, lin.k), dtype=torch.int8, device=device) for _ in range(copies)]
+        sxs = [torch.empty((lin.m,), dtype=torch.float32, device=device) for _ in range(copies)]
         torch.cuda.synchronize()
-        cr.convrot_quantize_act(x, xq, sx, stream=stream)
+        for i in range(copies):
+            cr.convrot_quantize_act(srcs[i], xqs[i], sxs[i], stream=stream)
+        n = max(reps, 2 * copies)
         keep_busy(stream, 200.0)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(reps):
-            cr.convrot_quantize_act(x, xq, sx, stream=stream)
+        for r in range(n):
+            i = r % copies
+            cr.convrot_quantize_act(srcs[i], xqs[i], sxs[i], stream=stream)
         e1.record(stream)
         torch.cuda.synchronize()
-        out.append((lin, e0.elapsed_time(e1) / reps / 1e3))
+        out.append((lin, e0.elapsed_time(e1) / n / 1e3, copies))
+        del srcs, xqs, sxs
+    torch.cuda.empty_cache()
     return out
 
 
@@ -330,35 +374,149 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def cpu_baseline(lins, seconds: float = 10.0):
-    """The oracle, as it stands (single-threaded C), on a bounded sample:
-    every linear of the step with its first N/64 weight rows and all M
-    token rows; whole passes repeated for >= `seconds`."""
-    import oracle
-    prepared = []
-    for lin in lins:
-        ns = max(1, math.ceil(lin.n / CPU_SAMPLE_ROWS_DIV))
-        wq, sw = oracle.rotate_quantize(lin.w_rows_np(np.arange(ns)))
-        prepared.append((lin, ns, lin.x_np(), wq, sw))
-    passes, t0 = 0, time.perf_counter()
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def _time_calls(fn, min_seconds):
+    n, t0 = 0, time.perf_counter()
     while True:
-        for lin, ns, x, wq, sw in prepared:
-            oracle.linear_int8(x, wq, sw)
-        passes += 1
+        fn()
+        n += 1
         el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    nbytes = passes * sum(linear_bytes(lin.m, ns, lin.k) for lin, ns, *_ in prepared)
-    return {"value": nbytes / el / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "%d passes over the 7 linears at M=%d with the first N/%d weight rows each "
-                      "(%.2f MB INT8 weights per pass), %.1f s" % (
-                          passes, lins[0].m, CPU_SAMPLE_ROWS_DIV,
-                          sum(ns * lin.k for lin, ns, *_ in prepared) / 1e6, el)}
+        if el >= min_seconds:
+            return el / n, n
 
 
-def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
+def cpu_baseline(lins, single_seconds: float = 8.0, all_seconds: float = 4.0):
+    """The oracle, as it stands (plain C), on the host cores: the decode
+    layer (the seven linears at M = 12) in full against full-size weights,
+    single-threaded and built with OpenMP over all cores; the tiny layer in
+    full; the q matrix of the prefill layer (M = 4096), all cores in full
+    when that fits in about 15 s, else a stated sample.  The weight codes of
+    the timing runs are uniform random INT8 from numpy: the oracle's
+    per-call work (activation rotation and quantisation, INT64 GEMM,
+    dequantisation) does not depend on their values, and the offline weight
+    conversion is not part of a step."""
+    import oracle
+    cores = host_cores()
+    os.environ["OMP_NUM_THREADS"] = str(cores)
+    rng = np.random.default_rng(0)
+    prep = [(lin.x_np(), rng.integers(-127, 128, (lin.n, lin.k), dtype=np.int8),
+             np.full(lin.n, 1e-4, np.float32)) for lin in lins]
+    bytes_step = sum(linear_bytes(lin.m, lin.n, lin.k) for lin in lins)
+
+    def decode_step():
+        for x, wq, sw in prep:
+            oracle.linear_int8(x, wq, sw)
+    out = {"unit": UNIT, "kind": "oracle", "cores": cores}
+    oracle.set_parallel(False)
+    t1, n1 = _time_calls(decode_step, single_seconds)
+    oracle.set_parallel(True)
+    decode_step()
+    ta, na = _time_calls(decode_step, all_seconds)
+    out["value"] = bytes_step / ta / 1e9
+    out["single_thread"] = {"value": bytes_step / t1 / 1e9, "ms_per_step": t1 * 1e3, "steps": n1, "cores": 1}
+    out["all_cores"] = {"value": bytes_step / ta / 1e9, "ms_per_step": ta * 1e3, "steps": na, "cores": cores}
+    # tiny layer in full (weights converted by the oracle itself)
+    tl = synth.tiny()[0]
+    twq, tsw = oracle.rotate_quantize(tl.w_np())
+    tx = tl.x_np()
+    oracle.set_parallel(False)
+    tt, _ = _time_calls(lambda: oracle.linear_int8(tx, twq, tsw), 1.0)
+    out["tiny_m4_k512_n256"] = {"us_per_call_single_thread": tt * 1e6,
+                                "gb_s_single_thread": linear_bytes(tl.m, tl.n, tl.k) / tt / 1e9}
+    # one matrix of the prefill layer: q (K = 5120, N = 8192) at M = 4096
+    q = synth.qwen_layer(4096)[0]
+    qwq = rng.integers(-127, 128, (q.n, q.k), dtype=np.int8)
+    qsw = np.full(q.n, 1e-4, np.float32)
+    macs_per_row = q.n * q.k
+    rate_all = sum(12 * lin.n * lin.k for lin in lins) / ta       # MAC/s seen on the decode layer
+    rows_all = q.m if q.m * macs_per_row / rate_all <= 15.0 else max(64, int(15.0 * rate_all / macs_per_row))
+    oracle.set_parallel(True)
+    xa = q.x_rows_np(np.arange(rows_all))
+    t0 = time.perf_counter()
+    oracle.linear_int8(xa, qwq, qsw)
+    ta_q = (time.perf_counter() - t0) * q.m / rows_all
+    oracle.set_parallel(False)
+    rows_1 = 64
+    x1 = q.x_rows_np(np.arange(rows_1))
+    t0 = time.perf_counter()
+    oracle.linear_int8(x1, qwq, qsw)
+    t1_q = (time.perf_counter() - t0) * q.m / rows_1
+    ops = 2 * q.m * q.n * q.k
+    out["prefill_q_m4096"] = {
+        "all_cores": {"tops": ops / ta_q / 1e12, "s": ta_q, "rows_timed": rows_all,
+                      "extrapolated": rows_all < q.m},
+        "single_thread": {"tops": ops / t1_q / 1e12, "s": t1_q, "rows_timed": rows_1, "extrapolated": True}}
+    out["sample"] = ("decode layer (7 linears, M=12, full-size weights with random INT8 codes) in full: "
+                     "%d single-threaded steps, %d all-core steps; tiny layer in full; prefill q at M=4096: "
+                     "%d token rows on all cores, 64 single-threaded, scaled to 4096 rows"
+                     % (n1, na, rows_all))
+    del prep, qwq
+    return out
+
+
+def method_error_report():
+    """What the rotation buys, computed by the oracle in FP64 on the host:
+    for the tiny layer (in full), the decode layer (all 12 tokens, 256
+    sampled output channels per linear) and the MiniMax qkv projection (64
+    sampled tokens x 256 output channels): the relative Frobenius error
+    against the unquantised FP64 product X W^T of (a) ConvRot INT8 (rotated,
+    the layer built here; the BF16 output and its FP64 dequantised product)
+    and (b) plain row-wise INT8 of the same X and W without rotation; and
+    the activations' per-group max/RMS ratio before and after rotation."""
+    import oracle
+    oracle.set_parallel(True)
+
+    def one(x_bits, w_bits):
+        x = oracle.bf16_bits_to_f64(x_bits)
+        w = oracle.bf16_bits_to_f64(w_bits)
+        ref = oracle.matmul_nt_f64(x, w)
+        nrm = float(np.linalg.norm(ref))
+        wq, sw = oracle.rotate_quantize(w_bits)
+        r = oracle.linear_int8(x_bits, wq, sw)
+        ydq = oracle.matmul_nt_f64(r["xq"].astype(np.float64) * r["sx"][:, None].astype(np.float64),
+                                   wq.astype(np.float64) * sw[:, None].astype(np.float64))
+        y = oracle.bf16_bits_to_f64(r["y"])
+        xq0, sx0, _ = oracle.quantize_rows(x.astype(np.float32))
+        wq0, sw0, _ = oracle.quantize_rows(w.astype(np.float32))
+        yu = oracle.matmul_nt_f64(xq0.astype(np.float64) * sx0[:, None].astype(np.float64),
+                                  wq0.astype(np.float64) * sw0[:, None].astype(np.float64))
+        yr, _ = oracle.rotate_rows(x_bits)
+        g0 = x.reshape(x.shape[0], -1, 256)
+        g1 = yr.astype(np.float64).reshape(x.shape[0], -1, 256)
+        ratio0 = np.max(np.abs(g0), axis=2) / np.maximum(np.sqrt(np.mean(g0 ** 2, axis=2)), 1e-300)
+        ratio1 = np.max(np.abs(g1), axis=2) / np.maximum(np.sqrt(np.mean(g1 ** 2, axis=2)), 1e-300)
+        return {"rel_err_convrot_int8_bf16_out": float(np.linalg.norm(y - ref) / nrm),
+                "rel_err_convrot_int8_dq64": float(np.linalg.norm(ydq - ref) / nrm),
+                "rel_err_plain_int8_dq64": float(np.linalg.norm(yu - ref) / nrm),
+                "group_max_over_rms_x": {"before_mean": float(ratio0.mean()), "before_max": float(ratio0.max()),
+                                         "after_mean": float(ratio1.mean()), "after_max": float(ratio1.max())}}
+    rep = {}
+    t = synth.tiny()[0]
+    rep["tiny"] = one(t.x_np(), t.w_np())
+    rng = np.random.default_rng(5)
+    dec = {}
+    for lin in synth.qwen_layer(12):
+        rows = np.sort(rng.choice(lin.n, 256, replace=False))
+        dec[lin.name] = one(lin.x_np(), lin.w_rows_np(rows))
+    rep["qwen_decode_m12"] = dec
+    mm = synth.minimax_qkv(8192)[0]
+    rep["minimax_qkv"] = one(mm.x_rows_np(np.sort(rng.choice(mm.m, 64, replace=False))),
+                             mm.w_rows_np(np.sort(rng.choice(mm.n, 256, replace=False))))
+    rep["sample"] = ("tiny in full; decode: all 12 tokens x 256 random output channels per linear; "
+                     "MiniMax qkv: 64 random tokens x 256 random output channels")
+    oracle.set_parallel(False)
+    return rep
+
+
+def prefill_secondary(cr, layer, device, stream, peaks, steps=20, warmup=3):
     """The same seven linears at M = 4096 (same weights): TOPS vs the dense
-    INT8 peak (the bf16 peak measured on this machine x the nominal 2x)."""
+    INT8 peak measured on this GPU (a large library INT8 GEMM)."""
     lins = synth.qwen_layer(4096)
     xs = [lin.x_torch(device) for lin in lins]
     ys = [torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device) for lin in lins]
@@ -371,11 +529,11 @@ def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
     keep_busy(stream)
     t = time_region(fn, steps, stream) / steps
     ops = sum(2 * lin.m * lin.n * lin.k for lin in lins)
-    g = gemm_kernel_times(cr, layer, lins, xs, 3, stream, device)
+    g = gemm_kernel_times(cr, layer, lins, xs, 10, stream, device)
     gops = sum(2 * lin.m * lin.n * lin.k for lin, _ in g)
     gt = sum(tt for _, tt in g)
-    peak = peaks["bf16_tflops"] * INT8_OVER_BF16
-    pro = prologue_kernel_times(cr, lins, xs, 5, stream, device)
+    peak = peaks["int8_tops"]
+    pro = prologue_kernel_times(cr, lins, xs, 10, stream, device)
     del batch
     # as the model feeds the layer: q, k, v read one input and gate, up
     # another, so their rotation and quantisation run once per input
@@ -399,13 +557,18 @@ def prefill_secondary(cr, layer, device, stream, peaks, steps=5, warmup=2):
                               "ms_per_step": t_shared * 1e3},
             "gemm_tops": gops / gt / 1e12,
             "roofline": {"bound": "tensor", "achieved": gops / gt / 1e12, "peak": peak, "unit": "TOP/s",
-                         "frac": gops / gt / 1e12 / peak,
-                         "peak_note": "measured bf16 burst x 2 (nominal int8/bf16 ratio)"},
+                         "frac": gops / gt / 1e12 / peak, "peak_source": peaks["int8_source"],
+                         "frac_of_bf16_x2": gops / gt / 1e12 / (peaks["bf16_tflops"] * INT8_OVER_BF16)},
             "per_linear_gemm_tops": {lin.name: 2 * lin.m * lin.n * lin.k / tt / 1e12 for lin, tt in g},
             "prologue": {"bytes": "2MK read + MK + 4M written",
-                         "per_linear_us": {lin.name: tt * 1e6 for lin, tt in pro},
-                         "per_linear_gbs": {lin.name: (3 * lin.m * lin.k + 4 * lin.m) / tt / 1e9 for lin, tt in pro},
-                         "layer_us": sum(tt for _, tt in pro) * 1e6}}
+                         "timing": "launches cycle through distinct copies of the input (> 2x L2 together)",
+                         "per_linear_us": {lin.name: tt * 1e6 for lin, tt, _ in pro},
+                         "per_linear_gbs": {lin.name: (3 * lin.m * lin.k + 4 * lin.m) / tt / 1e9
+                                            for lin, tt, _ in pro},
+                         "per_linear_frac_of_hbm": {lin.name: (3 * lin.m * lin.k + 4 * lin.m) / tt / 1e9
+                                                    / peaks["hbm_gbs"] for lin, tt, _ in pro},
+                         "copies": {lin.name: c for lin, _, c in pro},
+                         "layer_us": sum(tt for _, tt, _ in pro) * 1e6}}
 
 
 def shared_input_secondary(cr, layer, lins, device, stream, peaks, steps=2000, warmup=20):
@@ -474,7 +637,7 @@ def conv_secondary(cr, device, stream, peaks, steps=10, warmup=3):
     """VAE-decoder-shaped 3x3 convolutions (int8_convrot): NHWC BF16 in and
     out, im2col rows gathered by the prologue, INT8 GEMM; TOPS (2MNK)."""
     out = {}
-    peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    peak = peaks["int8_tops"]
     for (h, c) in ((128, 512), (256, 256)):
         seed = 77 + c
         x = synth.Linear("conv_x", h * h, c, 1, seed, None).x_torch(device).view(1, h, h, c)
@@ -507,12 +670,12 @@ def ctypes_byref(obj):
     return ctypes.byref(obj)
 
 
-def minimax_secondary(cr, device, stream, peaks, steps=5, warmup=2):
+def minimax_secondary(cr, device, stream, peaks, steps=10, warmup=3):
     """MiniMax-H3-shaped qkv projection (K = 5376, N = 16128) at M = 8192 and
     32768 video tokens through the single-linear entry point: INT8 TOPS."""
     out = {"workload": "minimax_h3_qkv_k5376_n16128", "metric": "INT8 TOPS (2MNK)"}
     w = None
-    peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    peak = peaks["int8_tops"]
     for m in (8192, 32768):
         lin = synth.minimax_qkv(m)[0]
         if w is None:
@@ -529,7 +692,7 @@ def minimax_secondary(cr, device, stream, peaks, steps=5, warmup=2):
         torch.cuda.synchronize()
         keep_busy(stream)
         t = time_region(fn, steps, stream) / steps
-        g = gemm_kernel_times(cr, _OneWeight(w), [lin], [x], 3, stream, device)[0][1]
+        g = gemm_kernel_times(cr, _OneWeight(w), [lin], [x], 10, stream, device)[0][1]
         ops = 2 * m * lin.n * lin.k
         out["m%d" % m] = {"linear_tops": ops / t / 1e12, "ms": t * 1e3, "gemm_tops": ops / g / 1e12,
                           "gemm_frac": ops / g / 1e12 / peak, "gemm_ms": g * 1e3}
@@ -639,6 +802,19 @@ def run_ours(args):
     cr.load_library()
     peaks, peak_kind = load_peaks()
 
+    try:
+        pr = torch.cuda.get_device_properties(device)
+        pci = "%02x:%02x.0" % (int(pr.pci_bus_id), int(pr.pci_device_id))
+    except Exception:
+        pci = None
+    clocks = ClockSampler(pci)
+    clocks.start()
+    w0 = time.time()
+    int8_peak = measure_int8_peak(device)
+    int8_window = (w0, time.time())
+    peaks["int8_tops"] = int8_peak["tops"]
+    peaks["int8_source"] = "measured"
+
     lins = synth.qwen_layer(12)
     layer = Layer(cr, lins, device)
     xs, ys, wss = make_io(cr, layer, lins, device)
@@ -661,14 +837,6 @@ def run_ours(args):
             step()
     torch.cuda.synchronize()
     cr.convrot_device_status(stream)
-
-    try:
-        pr = torch.cuda.get_device_properties(device)
-        pci = "%02x:%02x.0" % (int(pr.pci_bus_id), int(pr.pci_device_id))
-    except Exception:
-        pci = None
-    clocks = ClockSampler(pci)
-    clocks.start()
 
     barrier(world)
     torch.cuda.synchronize()
@@ -785,6 +953,8 @@ def run_ours(args):
     e2e_value, e2e_t = job_throughput(bytes_step, e2e_steps, e2e_t, world)
     serial_value, serial_t = job_throughput(bytes_step, e2e_steps, serial_t, world)
     clk = clocks.stop()
+    if clk is not None:
+        int8_peak["clocks"] = clocks.summary([int8_window])
     h2d = sum(2 * lin.m * lin.k for lin in lins)
     d2h = sum(2 * lin.m * lin.n for lin in lins)
     e2e = {"value": e2e_value, "unit": UNIT,
@@ -811,8 +981,10 @@ def run_ours(args):
         cr.convrot_device_status(stream)
 
     cpu = None
+    method_error = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(lins)
+        method_error = method_error_report()
 
     if rank == 0:
         line = {
@@ -832,7 +1004,8 @@ def run_ours(args):
             "per_linear_entry_point": {"ms_per_step": per_linear_t * 1e3,
                                        "value": bytes_step / per_linear_t / 1e9,
                                        "launches_per_step": 2 * len(lins)},
-            "secondary": secondary, "more": others or None, "kernel_sources": kernel_source_hash(),
+            "secondary": secondary, "more": others or None, "method_error": method_error,
+            "int8_peak": int8_peak, "library_build_id": cr.build_id(), "kernel_sources": kernel_source_hash(),
             "gemm_sources": kernel_source_hash(GEMM_SOURCES),
         }
         print(json.dumps(line), flush=True)

@@ -45,26 +45,38 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "convrot_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+_LIB_OMP = os.path.join(_HERE, "liboracle_omp.so")
 _CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c99", "-Wall",
            "-shared", "-fPIC"]
 
-_lib = None
+_libs = {}
+_parallel = False
 
 
-def build(force: bool = False) -> str:
-    """Compile ``convrot_oracle.c`` into ``liboracle.so`` next to it."""
-    if force or not os.path.exists(_LIB) or (
-            os.path.getmtime(_LIB) < os.path.getmtime(_SRC)):
-        tmp = _LIB + ".tmp.%d" % os.getpid()
-        subprocess.check_call(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile ``convrot_oracle.c`` into ``liboracle.so`` next to it (with
+    ``openmp``: ``liboracle_omp.so``, the same source built with -fopenmp,
+    rows split over threads, for the timed all-cores CPU baseline)."""
+    lib = _LIB_OMP if openmp else _LIB
+    if force or not os.path.exists(lib) or (
+            os.path.getmtime(lib) < os.path.getmtime(_SRC)):
+        tmp = lib + ".tmp.%d" % os.getpid()
+        extra = ["-fopenmp"] if openmp else []
+        subprocess.check_call(["gcc", *_CFLAGS, *extra, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, lib)
+    return lib
+
+
+def set_parallel(on: bool) -> None:
+    """Route the calls below to the OpenMP build (all host cores, or
+    OMP_NUM_THREADS) or back to the single-threaded one."""
+    global _parallel
+    _parallel = bool(on)
 
 
 def _load():
-    global _lib
-    if _lib is None:
-        lib = ctypes.CDLL(build())
+    if _parallel not in _libs:
+        lib = ctypes.CDLL(build(openmp=_parallel))
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         lib.oracle_sylvester_hadamard.argtypes = [ctypes.c_int, P]
@@ -104,8 +116,8 @@ def _load():
         lib.oracle_matmul_nt_f64.restype = None
         lib.oracle_float_to_bf16.argtypes = [ctypes.c_float]
         lib.oracle_float_to_bf16.restype = ctypes.c_uint16
-        _lib = lib
-    return _lib
+        _libs[_parallel] = lib
+    return _libs[_parallel]
 
 
 def _ptr(a: np.ndarray):

@@ -41,7 +41,10 @@
  *
  * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC -lm
  * (IEEE single and double arithmetic with round-to-nearest-even, no
- * contraction into fused multiply-adds).
+ * contraction into fused multiply-adds).  The same file built with
+ * -fopenmp splits independent rows (and output elements) over threads for
+ * the timed all-cores CPU baseline; every value is computed by the same
+ * operations in the same order either way.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -193,12 +196,25 @@ int oracle_rotate_rows(const uint16_t *a, int64_t rows, int64_t k, int group,
 {
     if (!is_power_of_two(group) || k % group != 0) return -1;
     int32_t *H = (int32_t *)malloc(sizeof(int32_t) * group * group);
-    double *x = (double *)malloc(sizeof(double) * group);
-    if (!H || !x) { free(H); free(x); return -1; }
+    if (!H) return -1;
     oracle_sylvester_hadamard(group, H);
     double root = sqrt((double)group);
     int64_t bad = 0;
+    int nomem = 0;
+    /* The rows are independent: an OpenMP build (the timed all-cores CPU
+       baseline) splits them over threads; the arithmetic of a row is the
+       same in either build. */
+#ifdef _OPENMP
+#pragma omp parallel reduction(+:bad, nomem)
+#endif
+    {
+    double *x = (double *)malloc(sizeof(double) * group);
+    if (!x) ++nomem;
+#ifdef _OPENMP
+#pragma omp for schedule(static)
+#endif
     for (int64_t r = 0; r < rows; ++r) {
+        if (!x) continue;
         for (int64_t g0 = 0; g0 < k; g0 += group) {
             int emin = 1000, emax = -1000;
             for (int i = 0; i < group; ++i) {
@@ -219,10 +235,11 @@ int oracle_rotate_rows(const uint16_t *a, int64_t rows, int64_t k, int group,
             }
         }
     }
+    free(x);
+    }
     if (inexact) *inexact = bad;
     free(H);
-    free(x);
-    return 0;
+    return nomem ? -1 : 0;
 }
 
 /*
@@ -264,6 +281,9 @@ int64_t oracle_quantize_rows(const float *y, int64_t rows, int64_t k,
                              int8_t *q, float *s)
 {
     int64_t ties = 0;
+#ifdef _OPENMP
+#pragma omp parallel for reduction(+:ties) schedule(static)
+#endif
     for (int64_t r = 0; r < rows; ++r) {
         float a = 0.0f;
         for (int64_t c = 0; c < k; ++c) {
@@ -349,6 +369,9 @@ int64_t oracle_embed_lookup(const int32_t *tokens, int64_t t, const int8_t *q, f
 int64_t oracle_quantize_rows4(const float *y, int64_t rows, int64_t k, int8_t *q, float *s)
 {
     int64_t ties = 0;
+#ifdef _OPENMP
+#pragma omp parallel for reduction(+:ties) schedule(static)
+#endif
     for (int64_t r = 0; r < rows; ++r) {
         float a = 0.0f;
         for (int64_t c = 0; c < k; ++c) {
@@ -482,6 +505,9 @@ int64_t oracle_gemm_i32(const int8_t *xq, const int8_t *wq, int64_t m,
                         int64_t n, int64_t k, int32_t *acc)
 {
     int64_t overflow = 0;
+#ifdef _OPENMP
+#pragma omp parallel for collapse(2) reduction(+:overflow) schedule(static)
+#endif
     for (int64_t i = 0; i < m; ++i)
         for (int64_t j = 0; j < n; ++j) {
             int64_t sum = 0;
@@ -501,6 +527,9 @@ int64_t oracle_gemm_i32(const int8_t *xq, const int8_t *wq, int64_t m,
 void oracle_dequant_bf16(const int32_t *acc, const float *sx, const float *sw,
                          int64_t m, int64_t n, uint16_t *y)
 {
+#ifdef _OPENMP
+#pragma omp parallel for collapse(2) schedule(static)
+#endif
     for (int64_t i = 0; i < m; ++i)
         for (int64_t j = 0; j < n; ++j) {
             float v = (float)acc[i * n + j];
@@ -520,6 +549,9 @@ void oracle_dequant_bf16(const int32_t *acc, const float *sx, const float *sw,
 void oracle_dequant_bf16_bias(const int32_t *acc, const float *sx, const float *sw,
                               const uint16_t *bias, int64_t m, int64_t n, uint16_t *y)
 {
+#ifdef _OPENMP
+#pragma omp parallel for collapse(2) schedule(static)
+#endif
     for (int64_t i = 0; i < m; ++i)
         for (int64_t j = 0; j < n; ++j) {
             float v = (float)acc[i * n + j];

@@ -722,3 +722,115 @@ def test_conv2d_int8_bit_exact(cr, n, h, w, c, o, k, stride, pad, dil):
     assert yb.shape == ref["y"].shape
     assert rel_err(yb, ref["y"]) <= TOL
     assert np.array_equal(yb, ref["y"])
+
+
+# ---------------------------------------------------------------- benchmarked configurations at full size
+def _sampled_batch_check(cr, lins, rows_w, rows_x, dev="cuda"):
+    """The layer's linears in one LinearBatch call (the bench's entry point),
+    whole-size weights quantised on the GPU; the oracle recomputes the
+    sampled weight rows and token rows of every linear from the counter-based
+    generator and checks weight codes and scales and the BF16 outputs bit for
+    bit."""
+    weights, xs, ys = [], [], []
+    for lin in lins:
+        w_bf = lin.w_torch(dev)
+        weights.append(cr.quantize_weight(w_bf))
+        del w_bf
+        xs.append(lin.x_torch(dev))
+        ys.append(torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=dev))
+    batch = cr.LinearBatch(xs, weights, ys)
+    batch()
+    batch()                      # the batched workspace is left reusable
+    cr.convrot_device_status()
+    for j, (lin, w, y) in enumerate(zip(lins, weights, ys)):
+        rw = np.asarray(rows_w[j])
+        rx = np.asarray(rows_x)
+        wq_ref, sw_ref = oracle.rotate_quantize(lin.w_rows_np(rw))
+        rwt = torch.as_tensor(rw, device=dev)
+        assert np.array_equal(w.q[rwt].cpu().numpy(), wq_ref), lin.name
+        assert np.array_equal(w.scale[rwt].cpu().numpy(), sw_ref), lin.name
+        ref = oracle.linear_int8(lin.x_rows_np(rx), wq_ref, sw_ref)
+        yb = to_bits(y[torch.as_tensor(rx, device=dev)][:, rwt])
+        assert rel_err(yb, ref["y"]) <= TOL, lin.name
+        assert np.array_equal(yb, ref["y"]), lin.name
+    del batch, weights, xs, ys
+    torch.cuda.empty_cache()
+
+
+def _edge_rows(n, rng, count, tile=256):
+    # first and last rows, both sides of the first tile boundary, random others
+    picks = [0, n - 1, min(tile - 1, n - 1), min(tile, n - 1)]
+    return np.unique(np.concatenate([picks, rng.integers(0, n, count)]))
+
+
+def test_stack_layer_m512_batch_sampled(cr):
+    # one layer of the 50-layer stack at M = 512 exactly as the bench runs it:
+    # seven Qwen-shaped weights in one batched GEMM launch (activations = A,
+    # four 128-row tiles replicated over CTA groups, stream-K over the K
+    # blocks of the 256-row weight tiles of all seven weights)
+    lins = synth.qwen_stack(512, layers=1)
+    plan = cr.gemm_plan(512, [l.n for l in lins], [l.k for l in lins])
+    assert plan.swap == 0 and plan.rep == 4 and plan.njobs == 7
+    rng = np.random.default_rng(512)
+    rows_w = [_edge_rows(lin.n, rng, 12) for lin in lins]
+    rows_x = np.unique(np.concatenate([[0, 127, 128, 255, 256, 383, 384, 511], rng.integers(0, 512, 8)]))
+    _sampled_batch_check(cr, lins, rows_w, rows_x)
+
+
+def test_qwen_prefill_layer_batch_sampled(cr):
+    # the prefill layer as the bench runs it: all seven linears at M = 4096
+    # through LinearBatch (one GEMM launch per linear, whole 128 x 256 tiles
+    # in full waves; gate and up have 3200 tiles = 21 waves + a 92-tile tail)
+    lins = synth.qwen_layer(4096)
+    rng = np.random.default_rng(4096)
+    rows_w = [_edge_rows(lin.n, rng, 10) for lin in lins]
+    rows_x = np.unique(np.concatenate([[0, 127, 128, 2047, 2048, 4095], rng.integers(0, 4096, 8)]))
+    _sampled_batch_check(cr, lins, rows_w, rows_x)
+
+
+def _conv_rows_oracle(x_rows_fn, h, w, c, pixels):
+    """im2col rows (3x3, stride 1, pad 1) of the sampled output pixels, each
+    from its 3 x 3 input window (zeros outside the image) through the
+    oracle's own im2col."""
+    out = []
+    for (oy, ox) in pixels:
+        win = np.zeros((1, 3, 3, c), dtype=np.uint16)
+        for dy in range(3):
+            for dx in range(3):
+                iy, ix = oy - 1 + dy, ox - 1 + dx
+                if 0 <= iy < h and 0 <= ix < w:
+                    win[0, dy, dx] = x_rows_fn([iy * w + ix])[0]
+        out.append(oracle.im2col_nhwc(win, 3, 3, 1, 0, 1)[0])
+    return np.stack(out)
+
+
+@pytest.mark.parametrize("h,c", [(128, 512), (256, 256)])
+def test_vae_conv_bench_shapes_sampled(cr, h, c):
+    # the two VAE-decoder-shaped 3x3 convolutions the bench times, drawn as
+    # the bench draws them, through the same entry point and tile plan
+    seed = 77 + c
+    xl = synth.Linear("conv_x", h * h, c, 1, seed, None)
+    wl = synth.Linear("conv_w", 1, 9 * c, c, seed, None)
+    x = xl.x_torch("cuda").view(1, h, h, c)
+    w_oihw = wl.w_torch("cuda").view(c, c, 3, 3)
+    plan = cr.conv2d_gather_plan(tuple(x.shape), 3, 3, 1, 1, 1)
+    assert plan.tiled == 1
+    wq = cr.quantize_conv_weight(w_oihw)
+    y = cr.conv2d_int8(x, wq, 3, 3, 1, 1, 1)
+    y2 = cr.conv2d_int8(x, wq, 3, 3, 1, 1, 1)
+    cr.convrot_device_status()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    rng = np.random.default_rng(h + c)
+    chans = np.unique(np.concatenate([[0, c - 1], rng.integers(0, c, 10)]))
+    w_rows = oracle.conv_weight_rows(wl.w_rows_np(chans).reshape(len(chans), c, 3, 3))
+    wq_ref, sw_ref = oracle.rotate_quantize(w_rows)
+    ct = torch.as_tensor(chans, device="cuda")
+    assert np.array_equal(wq.q[ct].cpu().numpy(), wq_ref)
+    assert np.array_equal(wq.scale[ct].cpu().numpy(), sw_ref)
+    pix = [(0, 0), (0, h - 1), (h - 1, 0), (h - 1, h - 1), (1, 1), (h // 2, 0)]
+    pix += [tuple(p) for p in rng.integers(0, h, (10, 2))]
+    rows = _conv_rows_oracle(xl.x_rows_np, h, h, c, pix)
+    ref = oracle.linear_int8(rows, wq_ref, sw_ref)
+    got = np.stack([to_bits(y[0, oy, ox][ct]) for (oy, ox) in pix])
+    assert rel_err(got, ref["y"]) <= TOL
+    assert np.array_equal(got, ref["y"])

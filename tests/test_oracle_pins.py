@@ -564,3 +564,42 @@ def test_matmul_f64_matches_numpy():
     a = rng.standard_normal((4, 37))
     b = rng.standard_normal((6, 37))
     assert np.allclose(oracle.matmul_nt_f64(a, b), a @ b.T, rtol=1e-13, atol=1e-13)
+
+
+def test_openmp_build_equals_single_threaded_build():
+    # the all-cores CPU baseline runs the same C source built with -fopenmp
+    # (rows split over threads); every output must equal the single-threaded
+    # oracle's bit for bit, inexact-group counts and ties included
+    import os
+    import synth
+    lin = synth.qwen_layer(37)[1]
+    x = lin.x_np()
+    w_bits = lin.w_rows_np(np.arange(300))
+    y_in = np.random.default_rng(11).standard_normal((40, 768)).astype(np.float32)
+    y_in[3, :] = np.float32(2.5)                        # s = 1: a row of exact ties
+    y_in[3, 0] = np.float32(127.0)
+    tiny = np.zeros((3, 512), np.uint16)
+    tiny[0, 0] = 0x3F80                                 # 1.0 and 2^-60 in one group: inexact
+    tiny[0, 1] = synth.f32_to_bf16_bits(np.array([2.0 ** -60], np.float32))[0]
+    results = []
+    old = os.environ.get("OMP_NUM_THREADS")
+    os.environ["OMP_NUM_THREADS"] = "4"
+    try:
+        for par in (False, True):
+            oracle.set_parallel(par)
+            wq, sw = oracle.rotate_quantize(w_bits)
+            ref = oracle.linear_int8(x, wq, sw)
+            y, bad = oracle.rotate_rows(tiny)
+            q, s, ties = oracle.quantize_rows(y_in)
+            results.append([wq, sw, ref["y"], ref["acc"], ref["xq"], y, q, s, bad, ties])
+    finally:
+        oracle.set_parallel(False)
+        if old is None:
+            del os.environ["OMP_NUM_THREADS"]
+        else:
+            os.environ["OMP_NUM_THREADS"] = old
+    a, b = results
+    for u, v in zip(a[:8], b[:8]):
+        assert np.array_equal(u, v)
+    assert a[8] == b[8] == 1
+    assert a[9] == b[9] > 0
