@@ -22,7 +22,14 @@
  *   y_j  = fp32( (sum_i a_i * H[i][j]) / 16 )   per 256-group, H Sylvester,
  *          the sum exact (FP64; exact while the nonzero magnitudes inside a
  *          group span at most 37 binades -- finite BF16 inputs outside that
- *          range give unspecified low bits).  Groups G of 16 .. 128 (the
+ *          range give unspecified low bits).  Every rotating kernel records
+ *          CONVROT_WARN_INEXACT_DOMAIN for convrot_device_status() when a row
+ *          holds a nonzero input |a| < 2^(e(amax) - 33), amax the row's
+ *          largest |y| and e() the frexp exponent: every group spanning more
+ *          than 37 binades meets this (its largest input is at most 16 amax),
+ *          so rows without the warning are inside the exact domain; a row
+ *          whose groups differ greatly in scale can raise it although each
+ *          group is exact.  Groups G of 16 .. 128 (the
  *          sizes --dynamic-convrot falls back to, see convrot_dynamic_group):
  *          the same with H_G and sqrt(G); for G = 32 and 128 the exact sum
  *          is divided by fp64(sqrt(G)) in FP64 and that quotient rounded to
@@ -67,7 +74,8 @@ typedef enum {
     CONVROT_ERR_UNSUPPORTED_ARCH = 4,  /* current device is not compute capability 10.0 */
     CONVROT_ERR_WORKSPACE = 5,         /* workspace missing or smaller than required */
     CONVROT_ERR_CUDA = 6,              /* a CUDA runtime/driver call failed */
-    CONVROT_ERR_DEVICE_TIMEOUT = 7     /* a bounded in-kernel wait ran out */
+    CONVROT_ERR_DEVICE_TIMEOUT = 7,    /* a bounded in-kernel wait ran out */
+    CONVROT_WARN_INEXACT_DOMAIN = 8    /* an input row may lie outside the exact-rotation domain (see below) */
 } convrot_status_t;
 
 /*
@@ -483,7 +491,11 @@ convrot_status_t convrot_embed_lookup(const int32_t *tokens, int64_t t, const in
  * the current device.  Returns CONVROT_OK, CONVROT_ERR_DEVICE_TIMEOUT if a
  * bounded wait ran out in some kernel since the last call (the workspace
  * must then be re-initialised), CONVROT_ERR_INVALID_ARG if a lookup met a
- * token outside its table, or CONVROT_ERR_CUDA.
+ * token outside its table, CONVROT_WARN_INEXACT_DOMAIN if a rotation met an
+ * input row that may lie outside the exact-sum domain (the results were
+ * written; their low bits may differ from the exact-sum definition), or
+ * CONVROT_ERR_CUDA.  A timeout overrides an earlier warning; the first
+ * other status recorded is kept until this call clears it.
  */
 convrot_status_t convrot_device_status(void *stream);
 

@@ -29,6 +29,7 @@ _STATUS = {
     0: "CONVROT_OK", 1: "CONVROT_ERR_INVALID_ARG", 2: "CONVROT_ERR_ALIGNMENT",
     3: "CONVROT_ERR_UNSUPPORTED_SHAPE", 4: "CONVROT_ERR_UNSUPPORTED_ARCH",
     5: "CONVROT_ERR_WORKSPACE", 6: "CONVROT_ERR_CUDA", 7: "CONVROT_ERR_DEVICE_TIMEOUT",
+    8: "CONVROT_WARN_INEXACT_DOMAIN",
 }
 
 

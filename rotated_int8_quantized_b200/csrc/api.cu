@@ -125,6 +125,7 @@ const char *convrot_status_string(convrot_status_t s) {
         case CONVROT_ERR_WORKSPACE: return "CONVROT_ERR_WORKSPACE";
         case CONVROT_ERR_CUDA: return "CONVROT_ERR_CUDA";
         case CONVROT_ERR_DEVICE_TIMEOUT: return "CONVROT_ERR_DEVICE_TIMEOUT";
+        case CONVROT_WARN_INEXACT_DOMAIN: return "CONVROT_WARN_INEXACT_DOMAIN";
     }
     return "CONVROT_ERR_UNKNOWN";
 }

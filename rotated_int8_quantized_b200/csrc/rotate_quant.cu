@@ -310,6 +310,72 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// max(|a|, |b|, |c|) in one instruction (sm_100).
+__device__ __forceinline__ float max3abs(float a, float b, float c) {
+    float d;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t min_s16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Per 16-bit half of a word of two BF16 values: 0x7FFF + |x| for x != 0,
+// and 0x7FFF for a zero, so that a signed 16-bit minimum ignores zeros and
+// otherwise orders by magnitude (no carry crosses the halves: each half sum
+// is at most 0xFFFE).
+__device__ __forceinline__ uint32_t nonzero_mag_key(uint32_t w) {
+    return (w & 0x7FFF7FFFu) + 0x7FFF7FFFu;
+}
+// The smallest nonzero BF16 magnitude (bits) a key minimum stands for, or
+// 0x7FFF + 1 when every value was zero.
+__device__ __forceinline__ int key_min_magnitude(uint32_t k) {
+    const int lo = (int)(int16_t)(k & 0xFFFFu), hi = (int)(int16_t)(k >> 16);
+    const int m = lo < hi ? lo : hi;
+    return m == 0x7FFF ? 0x8000 : m + 0x8001;
+}
+
+// Exactness threshold of a row (BF16 magnitude bits): the FP64 sums of a
+// group are exact while its nonzero inputs span at most 37 binades
+// (frexp exponents e_max - e_min <= 37).  The group's largest input is at
+// most max_j |S_j| = sqrt(G) max_j |y_j| <= 16 amax (Parseval), so
+// e_max <= e(16 amax) <= e(amax) + 4; a row whose nonzero inputs are all at
+// least 2^(e(amax) - 33) is inside the domain (one binade of slack).
+// Returns the bits of 2^(e(amax) - 33) (0: no BF16 value is below it, or
+// amax == 0); a nonzero input with smaller magnitude bits MAY be outside
+// the domain.
+__device__ __forceinline__ int exactness_threshold_bits(float amax) {
+    if (!(amax > 0.f) || !isfinite(amax)) return 0;
+    int e;
+    frexpf(amax, &e);
+    const int p = e - 33;
+    if (p >= -126) return (p + 127) << 7;
+    if (p >= -133) return 1 << (p + 133);
+    return 0;
+}
+
+// Record a possible exactness-domain violation (keeps an earlier status).
+__device__ __forceinline__ void report_inexact_domain() {
+    atomicCAS(&g_device_status, 0, 8 /* CONVROT_WARN_INEXACT_DOMAIN */);
+}
+
 // Layout of the rotated pixels (MODE 5 / 6, rotate_pixels_kernel): FP32
 // [pixels, c], and inside each 16-value chunk ci of a pixel, float4 part j
 // stored at position
@@ -432,6 +498,7 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
 
     double *xb = xch + cta_slot * kXchStride;
     float amax = 0.f;
+    uint32_t mkey = 0x7FFF7FFFu;       // smallest nonzero input magnitude (exactness domain)
 #pragma unroll
     for (int gi = 0; gi < GPS; ++gi) {
         const int g = g0 + slot + gi * slots;
@@ -440,7 +507,10 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
             const uint32_t w[8] = {raw[gi][0].x, raw[gi][0].y, raw[gi][0].z, raw[gi][0].w,
                                    raw[gi][1].x, raw[gi][1].y, raw[gi][1].z, raw[gi][1].w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
+            for (int i = 0; i < 8; ++i) {
+                mkey = min_s16x2(mkey, nonzero_mag_key(w[i]));
+                bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
+            }
             if (DYN)
                 fwht16_regs_upto(v, J.group < 16 ? J.group : 16);
             else
@@ -517,6 +587,12 @@ __global__ void __launch_bounds__(kMaxSlots * 16, (GPS == 1 && !HALF) ? 2 : 1)
         cluster_arrive();   // this CTA no longer reads its peers; matched by the wait before exit
     }
     const RowScale rs = MODE == 2 ? make_row_scale_levels(rmax, 7.0f) : make_row_scale(rmax);
+    {
+        const unsigned all = __activemask();
+        if (__any_sync(all, key_min_magnitude(mkey) < exactness_threshold_bits(rmax)) &&
+            (threadIdx.x & 31) == (unsigned)(__ffs(all) - 1))
+            report_inexact_domain();
+    }
 
     // quantise 16 consecutive outputs per thread, one 16-byte store
     int8_t *qrow = J.q + (size_t)row * k + (size_t)g0 * 256;
@@ -691,8 +767,12 @@ __global__ void __launch_bounds__(kPixThreads) rotate_pixels_kernel(const __nv_b
         }
         double v[16];
         const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+        uint32_t mkey = 0x7FFF7FFFu;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
+        for (int i = 0; i < 8; ++i) {
+            mkey = min_s16x2(mkey, nonzero_mag_key(w[i]));
+            bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
+        }
         fwht16_regs(v);                                  // index bits 0-3
 #pragma unroll
         for (int i = 0; i < 16; ++i) xb[17 * t + i] = v[i];
@@ -713,6 +793,9 @@ __global__ void __launch_bounds__(kPixThreads) rotate_pixels_kernel(const __nv_b
 #pragma unroll
         for (int o = 8 * CH; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(pix_mask, amax, o));
         if (t == 0 && chunk == 0) pmax[p] = amax;
+        if (__any_sync(pix_mask, key_min_magnitude(mkey) < exactness_threshold_bits(amax)) &&
+            (threadIdx.x & (CH == 1 ? 15 : 31)) == 0)
+            report_inexact_domain();
         r0 = n0;
         r1 = n1;
     }
@@ -745,31 +828,63 @@ static cudaError_t launch_rotate_pixels(const void *x, int64_t pixels, int c, fl
 
 // ---------------------------------------------------------------------------
 // Many long rows with groups of 256 (activations at prefill, weights
-// offline): persistent CTAs of S slots (one per group, in whole warps, or 32
-// when a slot takes several groups) walk the rows, the same arithmetic as
-// rotate_quant_rows_slots MODE 0 without its per-row bookkeeping (no job
-// table, parts or row packing), and each row's loads are issued while the
-// previous row is reduced and quantised.  Slot s takes groups s, s + S, ...
+// offline): persistent CTAs of S slots walk the rows (slot s takes groups
+// s, s + S, ...; GPS groups per slot), each row's loads issued while the
+// previous row is reduced and quantised.  Same values as
+// rotate_quant_rows_slots MODE 0, with a leaner instruction and shared-
+// memory budget (the kernel is issue- and shared-memory-bound, not HBM-bound):
+//   * BF16 -> FP32 by a shift or mask, scaled by 1/16 there (exact: every
+//     BF16 value times 2^-4 is an FP32 number), so the FP64 result only needs
+//     one conversion to FP32 and no multiply;
+//   * the 16 x 16 transpose between the two 16-point halves of the transform
+//     writes 16-byte rows (8 x 128-bit stores, rows padded to 18 doubles) and
+//     reads 8-byte columns;
+//   * the row maximum is reduced by 3-input max instructions, then once per
+//     CTA: warp 0 alone derives s, 1/s and the exactness threshold and hands
+//     them out through shared memory (two barriers per row);
+//   * REG (rows of at most 2 x 32 groups): a thread's 16 (32) rotated values
+//     stay in registers until the row maximum is known; it quantises them
+//     itself -- they are outputs 16 i + t of the group -- and a byte
+//     transpose through the slot's transpose buffer turns them into one
+//     16-byte store of 16 consecutive codes (no FP32 staging of the row);
+//     otherwise the row is staged in shared memory as FP32 and quantised by
+//     consecutive 16-value chunks;
+//   * the quantiser tests the rounding with a fused multiply-add:
+//     e = fl(y * (1/s) + 1.5 * 2^23) carries rne(y * (1/s)) in its low byte and
+//     d = fl(y * (1/s) - rne) is the distance to that integer; |d| < 0.49997
+//     proves that fl(y / s) rounds to the same integer (|y (1/s) - y / s|
+//     <= 127 * 2^-24, |fl(y / s) - y / s| <= 127 * 2^-24, so fl(y / s) is
+//     within 0.49997 + 1.6e-5 < 0.5 of it), else the IEEE division decides;
+//     three FP32-pair instructions per two values and one 3-input max.
+// Every row also reports, conservatively, whether it may lie outside the
+// domain where the FP64 sums are exact (see exactness_threshold_bits).
 // ---------------------------------------------------------------------------
 constexpr int kLeanThreads = 512;
 constexpr int kLeanMinGroups = 16;      // below this most slots would idle
 constexpr int kLeanMaxGps = 4;
+constexpr int kLeanXchStride = 18;      // doubles per transpose row: 16 + 2 (16-byte-aligned rows)
+constexpr int kLeanXch = 16 * kLeanXchStride;
+constexpr int kLeanRegMaxGps = 2;       // rows of more groups per slot stage the row in shared memory
 
-template <int GPS, bool DYNS>
-__global__ void __launch_bounds__(kLeanThreads, GPS == 1 ? 2 : 1)
+template <int GPS, bool REG>
+__global__ void __launch_bounds__(kLeanThreads, 1)
     rotate_quant_rows_lean(const __nv_bfloat16 *a, int64_t rows, int k, int8_t *q, float *s) {
     extern __shared__ __align__(16) uint8_t lsm[];
     __shared__ float red[kLeanThreads / 32];
+    __shared__ float rinfo[4];          // s, 1/s, exactness threshold bits, fast flag
     pdl_wait();
     pdl_launch_dependents();
     const int tid = threadIdx.x, slot = tid >> 4, t = tid & 15, lane = tid & 31, warp = tid >> 5;
-    // DYNS: as many slots as the launch has; otherwise 32, a constant for the compiler
-    const int S = DYNS ? (int)blockDim.x >> 4 : kLeanThreads / 16;
-    const int nthreads = S * 16, nwarps = nthreads >> 5;
+    const int S = (int)blockDim.x >> 4;     // even: whole warps
+    const int nwarps = (int)blockDim.x >> 5;
     const unsigned half_mask = 0xFFFFu << (16 * (slot & 1));
     const int groups = k >> 8, chunks = k >> 4;
-    double *xb = reinterpret_cast<double *>(lsm) + slot * kXchFull;
-    float *ybuf = reinterpret_cast<float *>(lsm + (size_t)S * kXchFull * 8);
+    double *xb = reinterpret_cast<double *>(lsm) + slot * kLeanXch;
+    // the slot's byte-transpose buffer (inside its transpose buffer; odd
+    // slots 64 bytes in, so the two slots of a warp use different banks)
+    uint8_t *xbytes = reinterpret_cast<uint8_t *>(xb) + (slot & 1) * 64;
+    float *ybuf = reinterpret_cast<float *>(lsm + (size_t)S * kLeanXch * 8);   // !REG: the row in FP32
+    const uint64_t sixteenth = pack_f32x2(0.0625f, 0.0625f);
     uint4 raw[GPS][2];
     auto load = [&](int64_t r) {
 #pragma unroll
@@ -782,34 +897,51 @@ __global__ void __launch_bounds__(kLeanThreads, GPS == 1 ? 2 : 1)
             }
         }
     };
+    float yv[REG ? GPS : 1][16];
     int64_t row = blockIdx.x;
     if (row < rows) load(row);
     for (; row < rows; row += gridDim.x) {
         float amax = 0.f;
+        uint32_t mkey = 0x7FFF7FFFu;
 #pragma unroll
         for (int gi = 0; gi < GPS; ++gi) {
             const int g = slot + S * gi;
             if (g < groups) {
-                double v[16];
                 const uint32_t w[8] = {raw[gi][0].x, raw[gi][0].y, raw[gi][0].z, raw[gi][0].w,
                                        raw[gi][1].x, raw[gi][1].y, raw[gi][1].z, raw[gi][1].w};
+                double v[16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) bf16x2_to_f64(w[i], v[2 * i], v[2 * i + 1]);
+                for (int i = 0; i < 8; ++i) {
+                    mkey = min_s16x2(mkey, nonzero_mag_key(w[i]));
+                    float lo, hi;
+                    unpack_f32x2(mul_f32x2(pack_f32x2(__uint_as_float(w[i] << 16),
+                                                      __uint_as_float(w[i] & 0xFFFF0000u)), sixteenth),
+                                 lo, hi);
+                    v[2 * i] = (double)lo;
+                    v[2 * i + 1] = (double)hi;
+                }
                 fwht16_regs(v);                              // index bits 0-3
+                double2 *row_t = reinterpret_cast<double2 *>(xb + kLeanXchStride * t);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) xb[17 * t + i] = v[i];
+                for (int i = 0; i < 8; ++i) row_t[i] = make_double2(v[2 * i], v[2 * i + 1]);
                 __syncwarp(half_mask);
                 double x[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) x[i] = xb[t + 17 * i];
+                for (int i = 0; i < 16; ++i) x[i] = xb[kLeanXchStride * i + t];
                 __syncwarp(half_mask);
                 fwht16_regs(x);                              // index bits 4-7: x[i] is output 16 i + t
-                float *yg = ybuf + (size_t)g * kYGroupStride + (t & 3);
+                float y[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float y = __double2float_rn(x[i] * 0.0625);     // / sqrt(256), exact
-                    yg[16 * i + 4 * ((t >> 2) ^ ((i >> 1) & 3))] = y;
-                    amax = fmaxf(amax, fabsf(y));
+                for (int i = 0; i < 16; ++i) y[i] = __double2float_rn(x[i]);
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) amax = max3abs(y[i], y[i + 1], amax);
+                if (REG) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) yv[REG ? gi : 0][i] = y[i];
+                } else {
+                    float *yg = ybuf + (size_t)g * kYGroupStride + (t & 3);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) yg[16 * i + 4 * ((t >> 2) ^ ((i >> 1) & 3))] = y[i];
                 }
             }
         }
@@ -819,52 +951,132 @@ __global__ void __launch_bounds__(kLeanThreads, GPS == 1 ? 2 : 1)
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         if (lane == 0) red[warp] = amax;
         __syncthreads();
-        float rmax = red[0];
-        for (int w = 1; w < nwarps; ++w) rmax = fmaxf(rmax, red[w]);
-        const RowScale rs = make_row_scale(rmax);
-        int8_t *qrow = q + row * k;
-        for (int c0 = 0; c0 < chunks; c0 += nthreads) {
-            const int c = c0 + tid;
-            const unsigned mask = __ballot_sync(0xffffffffu, c < chunks);
-            if (c < chunks) {
-                const int ci = c & 15;
-                const float4 *src = reinterpret_cast<const float4 *>(ybuf + (size_t)(c >> 4) * kYGroupStride + ci * 16);
-                float y[16];
+        if (warp == 0) {
+            float m = lane < nwarps ? red[lane] : 0.f;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 f = src[i ^ ((ci >> 1) & 3)];
-                    y[4 * i] = f.x;
-                    y[4 * i + 1] = f.y;
-                    y[4 * i + 2] = f.z;
-                    y[4 * i + 3] = f.w;
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) {
+                const RowScale rs0 = make_row_scale(m);
+                rinfo[0] = rs0.s;
+                rinfo[1] = rs0.r;
+                rinfo[2] = __int_as_float(exactness_threshold_bits(m));
+                rinfo[3] = __int_as_float((rs0.fast ? 1 : 0) | (rs0.zero ? 2 : 0));
+            }
+        }
+        __syncthreads();
+        RowScale rs;
+        rs.s = rinfo[0];
+        rs.r = rinfo[1];
+        const int tbits = __float_as_int(rinfo[2]);
+        const int flags = __float_as_int(rinfo[3]);
+        rs.fast = (flags & 1) != 0;
+        rs.zero = (flags & 2) != 0;
+        if (__any_sync(0xffffffffu, key_min_magnitude(mkey) < tbits) && lane == 0) report_inexact_domain();
+        int8_t *qrow = q + row * k;
+        if (REG) {
+            const uint64_t r2 = pack_f32x2(rs.r, rs.r), m2 = pack_f32x2(kRoundMagic, kRoundMagic);
+#pragma unroll
+            for (int gi = 0; gi < GPS; ++gi) {
+                const int g = slot + S * gi;
+                const bool on = g < groups;
+                const unsigned mask = __ballot_sync(0xffffffffu, on);
+                if (on) {
+                    const float(&y)[16] = yv[REG ? gi : 0];
+                    uint32_t e[16];
+                    float dmax = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint64_t y2 = pack_f32x2(y[2 * i], y[2 * i + 1]);
+                        const uint64_t e2 = fma_f32x2(y2, r2, m2);          // rne(y r) in the low byte
+                        const uint64_t d2 = fma_f32x2(y2, r2, sub_f32x2(m2, e2));   // y r - rne(y r)
+                        float d0, d1, e0, e1;
+                        unpack_f32x2(d2, d0, d1);
+                        unpack_f32x2(e2, e0, e1);
+                        e[2 * i] = __float_as_uint(e0);
+                        e[2 * i + 1] = __float_as_uint(e1);
+                        dmax = max3abs(d0, d1, dmax);
+                    }
+                    const bool slow = !(dmax < 0.49997f) || !rs.fast;   // NaN too; zero rows (codes set below)
+                    if (__any_sync(mask, slow) && slow) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float ei = __fmaf_rn(y[i], rs.r, kRoundMagic);
+                            const float di = __fmaf_rn(y[i], rs.r, __fsub_rn(kRoundMagic, ei));
+                            if (!rs.fast || !(fabsf(di) < 0.49997f)) {
+                                const int c =
+                                    __float_as_int(__fadd_rn(__fdiv_rn(y[i], rs.s), kRoundMagic)) - kRoundMagicBits;
+                                e[i] = (uint32_t)min(max(c, -127), 127);
+                            }
+                        }
+                    }
+                    if (rs.zero) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) e[i] = 0u;
+                    }
+                    // codes of outputs 16 i + t -> bytes 16 i + t of the slot's buffer;
+                    // then this thread stores outputs 16 t .. 16 t + 15
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) xbytes[16 * i + t] = (uint8_t)e[i];
+                    __syncwarp(mask & half_mask);
+                    const uint4 pk = *reinterpret_cast<const uint4 *>(xbytes + 16 * t);
+                    __syncwarp(mask & half_mask);
+                    *reinterpret_cast<uint4 *>(qrow + g * 256 + 16 * t) = pk;
                 }
-                *reinterpret_cast<uint4 *>(qrow + c * 16) = quant16x2(y, rs, mask);
+            }
+        } else {
+            for (int c0 = 0; c0 < chunks; c0 += (int)blockDim.x) {
+                const int c = c0 + tid;
+                const unsigned mask = __ballot_sync(0xffffffffu, c < chunks);
+                if (c < chunks) {
+                    const int ci = c & 15;
+                    const float4 *src =
+                        reinterpret_cast<const float4 *>(ybuf + (size_t)(c >> 4) * kYGroupStride + ci * 16);
+                    float y[16];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float4 f = src[i ^ ((ci >> 1) & 3)];
+                        y[4 * i] = f.x;
+                        y[4 * i + 1] = f.y;
+                        y[4 * i + 2] = f.z;
+                        y[4 * i + 3] = f.w;
+                    }
+                    *reinterpret_cast<uint4 *>(qrow + c * 16) = quant16x2(y, rs, mask);
+                }
             }
         }
         if (tid == 0) s[row] = rs.s;
-        __syncthreads();                     // ybuf and red are written again by the next row
+        if (!REG) __syncthreads();           // ybuf is written again by the next row
     }
 }
 
-template <int GPS, bool DYNS>
-static cudaError_t launch_lean(const RQProblem &pr, int64_t rows, int sms, cudaStream_t stream, bool pdl) {
+// Shape of a lean launch for `groups` groups per row: GPS groups per slot,
+// an even number of slots (whole warps), at most 32 (512 threads).  Rows of
+// up to 64 groups keep their rotated values in registers (GPS <= 2); longer
+// rows stage them in shared memory.
+static void lean_shape(int groups, int *gps, int *slots, bool *reg) {
+    const int g = (groups + 31) / 32;
+    const int sl = (groups + g - 1) / g;
+    *gps = g;
+    *slots = (sl + 1) & ~1;
+    *reg = g <= kLeanRegMaxGps;
+}
+
+template <int GPS, bool REG>
+static cudaError_t launch_lean(const RQProblem &pr, int64_t rows, int sms, int slots, cudaStream_t stream, bool pdl) {
     const int groups = (int)(pr.k >> 8);
-    // one group per slot: as many slots as groups (whole warps); several:
-    // all 32 slots (more warps per SM measured faster for the longest rows)
-    const int slots = DYNS ? (groups + 1) & ~1 : kLeanThreads / 16;
-    const size_t smem = (size_t)slots * kXchFull * 8 + (size_t)groups * kYGroupStride * 4;
+    const size_t smem = (size_t)slots * kLeanXch * 8 + (REG ? 0 : (size_t)groups * kYGroupStride * 4);
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(rotate_quant_rows_lean<GPS, DYNS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(rotate_quant_rows_lean<GPS, REG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSlotsSmemMax);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev] = true;
     }
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_rows_lean<GPS, DYNS>, slots * 16, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_rows_lean<GPS, REG>, slots * 16, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t cap = (int64_t)sms * per_sm;
@@ -878,7 +1090,7 @@ static cudaError_t launch_lean(const RQProblem &pr, int64_t rows, int sms, cudaS
     cfg.stream = stream;
     cfg.attrs = pdl ? attr : nullptr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_lean<GPS, DYNS>, static_cast<const __nv_bfloat16 *>(pr.a), rows,
+    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_lean<GPS, REG>, static_cast<const __nv_bfloat16 *>(pr.a), rows,
                               (int)pr.k, pr.q, pr.s);
 }
 
@@ -909,15 +1121,17 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
     if (conv_mode == 0 && !int4 && njobs == 1 && probs[0].group == 256 && (probs[0].k & 255) == 0 &&
         rows >= 2 * (int64_t)num_sms) {
         const int groups = (int)(probs[0].k >> 8);
-        const int gps = (groups + 31) / 32;
+        int gps, slots;
+        bool reg;
+        lean_shape(groups, &gps, &slots, &reg);
         if (groups >= kLeanMinGroups && gps <= kLeanMaxGps) {
+            if (reg) {
+                return gps == 1 ? launch_lean<1, true>(probs[0], rows, num_sms, slots, stream, pdl)
+                                : launch_lean<2, true>(probs[0], rows, num_sms, slots, stream, pdl);
+            }
             switch (gps) {
-                case 1:
-                    return groups >= 31 ? launch_lean<1, false>(probs[0], rows, num_sms, stream, pdl)
-                                        : launch_lean<1, true>(probs[0], rows, num_sms, stream, pdl);
-                case 2: return launch_lean<2, false>(probs[0], rows, num_sms, stream, pdl);
-                case 3: return launch_lean<3, false>(probs[0], rows, num_sms, stream, pdl);
-                default: return launch_lean<4, false>(probs[0], rows, num_sms, stream, pdl);
+                case 3: return launch_lean<3, false>(probs[0], rows, num_sms, slots, stream, pdl);
+                default: return launch_lean<4, false>(probs[0], rows, num_sms, slots, stream, pdl);
             }
         }
     }

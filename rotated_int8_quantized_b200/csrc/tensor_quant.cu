@@ -101,7 +101,9 @@ __global__ void __launch_bounds__(kTqThreads) embed_lookup_kernel(const int32_t 
                 pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
             }
         } else if (c == 0) {
-            atomicExch(&g_device_status, 1 /* CONVROT_ERR_INVALID_ARG */);
+            // an error replaces a recorded warning, never a recorded error
+            if (atomicCAS(&g_device_status, 0, 1 /* CONVROT_ERR_INVALID_ARG */) == 8)
+                atomicCAS(&g_device_status, 8, 1);
         }
         uint4 *dst = reinterpret_cast<uint4 *>(out + i * dim) + 2 * c;
         dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);

@@ -834,3 +834,67 @@ def test_vae_conv_bench_shapes_sampled(cr, h, c):
     got = np.stack([to_bits(y[0, oy, ox][ct]) for (oy, ox) in pix])
     assert rel_err(got, ref["y"]) <= TOL
     assert np.array_equal(got, ref["y"])
+
+
+# ---------------------------------------------------------------- exactness domain of the rotation
+def _plant_wide_group(x_bits, row, group):
+    # 1.0 and 2^-60 in one group: its nonzero magnitudes span 61 binades
+    x = x_bits.copy()
+    x[row, 256 * group] = 0x3F80
+    x[row, 256 * group + 1] = synth.f32_to_bf16_bits(np.array([2.0 ** -60], np.float32))[0]
+    return x
+
+
+def _status_after(cr, fn):
+    fn()
+    try:
+        cr.convrot_device_status()
+    except cr.ConvrotError as e:
+        return e.status
+    return 0
+
+
+@pytest.mark.parametrize("m,k", [(300, 4096), (3, 512), (400, 25600), (5, 25600), (310, 12288)])
+def test_inexact_domain_is_reported(cr, m, k):
+    # the lean prefill kernel (register and staged rows), the row kernel
+    # (few rows, clusters), through the activation and the weight entry points
+    x_bits = synth.draw_np(synth.stream_key(m + k, 0), m, k, 1.0)
+    assert oracle.rotate_rows(x_bits)[1] == 0
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+    assert _status_after(cr, lambda: cr.convrot_quantize_act(from_bits(x_bits), xq, sx)) == 0
+    planted = _plant_wide_group(x_bits, m // 2, (k // 256) // 2)
+    assert oracle.rotate_rows(planted)[1] == 1
+    assert _status_after(cr, lambda: cr.convrot_quantize_act(from_bits(planted), xq, sx)) == 8
+    assert _status_after(cr, lambda: cr.quantize_weight(from_bits(planted))) == 8
+    assert _status_after(cr, lambda: cr.quantize_weight(from_bits(x_bits))) == 0
+
+
+def test_inexact_domain_warning_is_conservative(cr):
+    # every group exact on its own (one group of ~1, one of ~2^-40), but the
+    # row's scale cannot tell them apart: the warning is raised although the
+    # oracle finds no inexact group, and the codes are still bit-exact
+    m, k = 300, 4096
+    x = synth.bf16_bits_to_f32(synth.draw_np(synth.stream_key(9, 0), m, k, 1.0))
+    x[7, 256:512] *= np.float32(2.0 ** -40)
+    bits = synth.f32_to_bf16_bits(x)
+    assert oracle.rotate_rows(bits)[1] == 0
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+    assert _status_after(cr, lambda: cr.convrot_quantize_act(from_bits(bits), xq, sx)) == 8
+    q_ref, s_ref = oracle.rotate_quantize(bits)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def test_inexact_domain_reported_by_convolution_pixels(cr):
+    # 3x3 convolution: every input pixel is rotated once; a pixel holding a
+    # 61-binade group raises the warning
+    n, h, w, c, o = 1, 20, 20, 256, 64
+    x_bits = synth.draw_np(synth.stream_key(21, 0), n * h * w, c, 1.0)
+    w_bits = synth.draw_np(synth.stream_key(21, 1), o, c * 9, synth.W_SIGMA).reshape(o, c, 3, 3)
+    wq = cr.quantize_conv_weight(from_bits(w_bits))
+    xd = from_bits(x_bits.reshape(n, h, w, c))
+    assert _status_after(cr, lambda: cr.conv2d_int8(xd, wq, 3, 3, 1, 1, 1)) == 0
+    planted = _plant_wide_group(x_bits, 123, 0).reshape(n, h, w, c)
+    assert _status_after(cr, lambda: cr.conv2d_int8(from_bits(planted), wq, 3, 3, 1, 1, 1)) == 8
