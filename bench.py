@@ -625,12 +625,27 @@ def w4a8_secondary(cr, lins, device, stream, peaks, steps=2000, warmup=20):
         t = time_region(g.replay, steps, stream) / steps
     m = lins[0].m
     nbytes = sum(lin.n * lin.k // 2 + 4 * lin.n + 2 * m * lin.k + 2 * m * lin.k + 4 * m + 2 * m * lin.n for lin in lins)
-    del g, batch, ws4
+    del g, batch
+    # the same INT4 weights at prefill size (M = 4096): tensor-bound
+    pl = synth.qwen_layer(4096)
+    pxs = [lin.x_torch(device) for lin in pl]
+    pys = [torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device) for lin in pl]
+    pbatch = cr.LinearBatchW4(pxs, ws4, pys)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        pbatch(stream)
+    torch.cuda.synchronize()
+    keep_busy(stream)
+    tp = time_region(lambda: pbatch(stream), 10, stream) / 10
+    pops = sum(2 * lin.m * lin.n * lin.k for lin in pl)
+    del pbatch, pxs, pys, ws4
     torch.cuda.empty_cache()
     return {"workload": "qwen3vl32b_layer_7linears_decode_m12_w4a8", "int4_weight_bytes": sum(l.n * l.k // 2 for l in lins),
             "gb_s": nbytes / t / 1e9, "us_per_step": t * 1e6,
             "frac_of_measured_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"],
-            "weight_stream_gb_s_int8_equivalent": sum(l.n * l.k for l in lins) / t / 1e9}
+            "weight_stream_gb_s_int8_equivalent": sum(l.n * l.k for l in lins) / t / 1e9,
+            "prefill_m4096": {"layer_tops": pops / tp / 1e12, "ms_per_step": tp * 1e3,
+                              "frac_of_int8_peak": pops / tp / 1e12 / peaks["int8_tops"]}}
 
 
 def conv_secondary(cr, device, stream, peaks, steps=10, warmup=3):

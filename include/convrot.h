@@ -169,7 +169,7 @@ size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * points (convrot_gemm_i8 / convrot_linear_int8) for m x k against n x k;
  * count in 2..8 (m <= 512): one batched launch of `count` products with the
  * same m (convrot_gemm_i8_batch / convrot_linear_int8_batch), w4 = 1 for
- * INT4 weights (m <= 256).  A CTA c of the `grid` takes, in order: whole
+ * INT4 weights.  A CTA c of the `grid` takes, in order: whole
  * tiles wave * grid + c for wave < full_waves while below full_tiles; piece
  * c of the split tail when c < split_pieces (tile full_tiles + c / split_ways,
  * K blocks [s * kbpt / ways, (s + 1) * kbpt / ways) with s = c % ways); then
@@ -367,12 +367,13 @@ typedef struct {
 } convrot_linear4_job_t;
 
 /*
- * count (<= 8) W4A8 linears with the same token count m in two launches:
- * the activation prologue (INT8 codes, shared by jobs with the same input),
- * then one weight-streaming GEMM whose K blocks of all weights are dealt out
- * to every SM, the packed tiles unpacked to INT8 by four dedicated warps per
- * CTA.  1 <= m <= 256 (larger m: CONVROT_ERR_UNSUPPORTED_SHAPE; there the
- * layer is tensor-bound and the INT4 format saves no time).  Results:
+ * count (<= 8) W4A8 linears with the same token count m: the activation
+ * prologue (INT8 codes, shared by jobs with the same input), then the INT8
+ * tensor-core GEMM with the packed weight tiles unpacked to INT8 in shared
+ * memory by eight dedicated warps per CTA.  m <= 512: one GEMM launch for all
+ * jobs (for m <= 256 weight-streaming, the K blocks of all weights dealt out
+ * to every SM); larger m (prefill, video tokens): one GEMM launch per job,
+ * whole 128 x 256 tiles with the weight as the 256-row operand.  Results:
  * y = bf16(((float)acc * sx[m]) * sw[n] [+ bias[n]]) with acc the exact INT32
  * product of the INT8 activation codes and the INT4 weight codes.
  * Workspace: convrot_linear_w4a8_workspace_bytes, zero-filled before first

@@ -26,7 +26,6 @@ constexpr int64_t kMaxK = 133120;
 constexpr int64_t kMaxRows = 0x7FFFFFFF;
 constexpr int kDefaultSms = 148;
 constexpr int kMaxBatch = convrot::kMaxJobs;
-constexpr int64_t kMaxW4Rows = 256;     // INT4 weights: the swapped (weight-streaming) orientation only
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -195,10 +194,10 @@ convrot_status_t convrot_gemm_plan(int64_t m, int32_t count, const int64_t *n, c
     if (!out || !n || !k || count < 1 || count > kMaxBatch || m < 1 || sms < 1) return CONVROT_ERR_INVALID_ARG;
     for (int j = 0; j < count; ++j)
         if (n[j] < 1 || k[j] < 1) return CONVROT_ERR_INVALID_ARG;
-    if ((count > 1 && m > convrot::kMaxSwapM) || (w4 && m > 256)) return CONVROT_ERR_UNSUPPORTED_SHAPE;
+    if (count > 1 && m > convrot::kMaxSwapM) return CONVROT_ERR_UNSUPPORTED_SHAPE;
     convrot::GemmPlan p;
-    if (count == 1 && !w4)
-        convrot::plan_gemm(m, n[0], k[0], sms, &p);
+    if (count == 1)
+        convrot::plan_gemm(m, n[0], k[0], sms, &p, w4 != 0);
     else
         convrot::plan_gemm_batch(m, count, n, k, sms, &p, w4 != 0);
     *out = convrot_gemm_plan_t{};
@@ -311,8 +310,7 @@ convrot_status_t collect_jobs(int64_t m, int count, const convrot_linear_job_t *
 }
 
 convrot_status_t collect_jobs4(int64_t m, int count, const convrot_linear4_job_t *jobs, LinJob *out) {
-    if (!jobs || count < 1 || count > kMaxBatch) return CONVROT_ERR_INVALID_ARG;
-    if (m < 1 || m > kMaxW4Rows) return m < 1 ? CONVROT_ERR_INVALID_ARG : CONVROT_ERR_UNSUPPORTED_SHAPE;
+    if (!jobs || count < 1 || count > kMaxBatch || m < 1) return CONVROT_ERR_INVALID_ARG;
     for (int j = 0; j < count; ++j) {
         const convrot_linear4_job_t &J = jobs[j];
         convrot_status_t s = check_weight4(J.w);
@@ -332,7 +330,7 @@ struct LinearLayout {
 };
 
 void linear_layout(int64_t m, int count, const LinJob *jobs, bool w4, int sms, LinearLayout *L) {
-    L->batched_gemm = w4 || (m <= convrot::kMaxSwapM);
+    L->batched_gemm = m <= convrot::kMaxSwapM;
     size_t g = 0;
     if (L->batched_gemm) {
         int64_t n[kMaxBatch], k[kMaxBatch];
@@ -345,7 +343,7 @@ void linear_layout(int64_t m, int count, const LinJob *jobs, bool w4, int sms, L
     } else {
         for (int j = 0; j < count; ++j) {
             convrot::GemmPlan p;
-            convrot::plan_gemm(m, jobs[j].n, jobs[j].k, sms, &p);
+            convrot::plan_gemm(m, jobs[j].n, jobs[j].k, sms, &p, w4);
             g = p.ws_bytes > g ? p.ws_bytes : g;
         }
     }
@@ -393,7 +391,7 @@ convrot_status_t run_linear(int64_t m, int count, const LinJob *jobs, bool w4, v
     if (L.batched_gemm) return from_cuda(convrot::launch_gemm_i8(L.batch, gp, base, st, true, true));
     for (int j = 0; j < count; ++j) {
         convrot::GemmPlan p;
-        convrot::plan_gemm(m, jobs[j].n, jobs[j].k, dev.num_sms, &p);
+        convrot::plan_gemm(m, jobs[j].n, jobs[j].k, dev.num_sms, &p, w4);
         // the first product may prefetch weights under the prologue; later
         // ones follow another GEMM that could still be reading the scratch
         e = convrot::launch_gemm_i8(p, &gp[j], base, st, true, j == 0);

@@ -49,7 +49,7 @@ constexpr int kTileA = 128;            // UMMA M
 constexpr int kBlockK = 128;           // bytes of K per stage (one 128-byte swizzle row)
 constexpr int kUmmaK = 32;             // K per tcgen05.mma kind::i8
 constexpr int kATileBytes = kTileA * kBlockK;
-constexpr uint32_t kPackedTileBytes = kTileA * kBlockK / 2;   // 128 rows x 64 bytes of INT4 codes
+constexpr uint32_t kPackedRowBytes = kBlockK / 2;   // INT4 codes of one 128-byte K block of a weight row
 constexpr int kL2PrefetchBlocks = 16;  // weight K blocks pulled into L2 ahead of the grid-dependency wait
 constexpr int kMaxSplitWays = 6;       // K ranges per split tail tile (large M)
 constexpr long long kGroupABytes = 48ll << 20;   // INT8 A operand above this is taken in tile groups
@@ -305,8 +305,9 @@ __device__ __forceinline__ uint32_t sext_nibbles(uint32_t v) {
     return (v & 0x08080808u) * 30u + v;
 }
 
-// W4: the weight (A operand, swapped orientation) arrives as packed INT4
-// codes; warps 6-9 unpack each 128 x 64-byte tile into the 128 x 128-byte
+// W4: the weight arrives as packed INT4 codes (wrows x 64 bytes per K
+// block: the A tile of 128 rows in the swapped orientation, the B tile of bn
+// rows otherwise); warps 6-13 unpack it into the wrows x 128-byte
 // 128B-swizzled INT8 tile the MMA reads.
 template <bool W4>
 __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
@@ -322,8 +323,10 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
     const uint32_t a_off = 0;
     const uint32_t b_off = (uint32_t)S * kATileBytes;
     // W4: a staging slot per stage where the packed weight tile lands
+    const int wrows = a.swap ? kTileA : a.bn;           // rows of the weight tile
+    const uint32_t packed_bytes = (uint32_t)wrows * kPackedRowBytes;
     const uint32_t p_off = b_off + (uint32_t)S * b_bytes;
-    const uint32_t bar_off = p_off + (W4 ? (uint32_t)S * kPackedTileBytes : 0u);
+    const uint32_t bar_off = p_off + (W4 ? (uint32_t)S * packed_bytes : 0u);
     // barriers: full[S], empty[S], tfull[2], tempty[2], drain, red[2], W4: pfull[S]
     const uint32_t full_bar = base + bar_off;
     const uint32_t empty_bar = full_bar + 8u * S;
@@ -386,7 +389,8 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
         if (lane == 0) {
             // W4: the packed weight tile lands in the stage's staging slot
             // (unpacked into its operand slot by the unpacking warps)
-            const uint32_t tx = (W4 ? kPackedTileBytes : (uint32_t)kATileBytes) + b_bytes;
+            const uint32_t tx = W4 ? packed_bytes + (a.swap ? b_bytes : (uint32_t)kATileBytes)
+                                   : (uint32_t)kATileBytes + b_bytes;
             const int RS = S;
             const uint32_t free_bar = empty_bar;
             int stage = 0;
@@ -419,7 +423,7 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
                     const uint32_t sa = base + a_off + (uint32_t)stage * kATileBytes;
                     const uint32_t sb = base + b_off + (uint32_t)stage * b_bytes;
                     const int kx = kb * kBlockK;
-                    const uint32_t sp = base + p_off + (uint32_t)stage * kPackedTileBytes;   // W4 staging
+                    const uint32_t sp = base + p_off + (uint32_t)stage * packed_bytes;   // W4 staging
                     const uint32_t sW = W4 ? sp : (a.swap ? sa : sb);
                     const uint32_t sX = a.swap ? sb : sa;
                     tma_load_2d(sW, tmW, lb, W4 ? kx / 2 : kx, rowW);
@@ -543,9 +547,10 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
         // ------------------------------------------------ INT4 unpacking (kW4Warps warps)
         // All unpacking warps walk every K block in ring order (so no wait
         // runs ahead of a phase) and each unpacks its share of the stage:
-        // 128 rows x 8 chunks of 16 codes, 8 B of nibbles -> 16 B of INT8 at
-        // the chunk's swizzled position (chunk c of row r sits at
-        // 16 * (c ^ (r & 7)) in the row's 128 bytes); then full[stage].
+        // wrows rows x 8 chunks of 16 codes, 8 B of nibbles -> 16 B of INT8
+        // at the chunk's swizzled position (chunk c of row r sits at
+        // 16 * (c ^ (r & 7)) in the row's 128 bytes) in the weight operand's
+        // slot (A when swapped, else B); then full[stage].
         const int ct = (int)threadIdx.x - kThreads;
         constexpr int kCT = 32 * kW4Warps;
         int stage = 0;
@@ -560,11 +565,11 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
                     ok = false;
                     break;
                 }
-                const uint8_t *src = smem + p_off + (uint32_t)stage * kPackedTileBytes;
-                uint8_t *dst = smem + a_off + (uint32_t)stage * kATileBytes;
-#pragma unroll
-                for (int i = 0; i < 1024 / kCT; ++i) {
-                    const int item = ct + kCT * i;
+                const uint8_t *src = smem + p_off + (uint32_t)stage * packed_bytes;
+                uint8_t *dst = a.swap ? smem + a_off + (uint32_t)stage * kATileBytes
+                                      : smem + b_off + (uint32_t)stage * b_bytes;
+#pragma unroll 4
+                for (int item = ct; item < wrows * 8; item += kCT) {
                     const int r = item >> 3, c = item & 7;
                     const uint2 w = *reinterpret_cast<const uint2 *>(src + r * 64 + c * 8);
                     uint4 o;
@@ -689,7 +694,8 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
                 } else {
                     const int others = ways - 1;
                     // column rounds, double-buffered in the operand ring
-                    const uint32_t ring = (uint32_t)S * ((uint32_t)kATileBytes + b_bytes);
+                    // (W4: the packed staging slots follow the operand slots and are idle too)
+                    const uint32_t ring = (uint32_t)S * ((uint32_t)kATileBytes + b_bytes + (W4 ? packed_bytes : 0u));
                     int cols = (int)(ring / (2u * (uint32_t)others * kTileA * 4u)) / 32 * 32;
                     if (cols > a.bn) cols = a.bn;
                     const int rounds = (a.bn + cols - 1) / cols;
@@ -849,7 +855,8 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
 
 static void plan_common(GemmPlan *p) {
     // W4: every stage also holds the packed weight tile it is unpacked from
-    const int stage_bytes = kATileBytes + p->bn * kBlockK + (p->w4 ? (int)kPackedTileBytes : 0);
+    const int wrows = p->swap ? kTileA : p->bn;
+    const int stage_bytes = kATileBytes + p->bn * kBlockK + (p->w4 ? wrows * (int)kPackedRowBytes : 0);
     int stages = (200 * 1024) / stage_bytes;
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) stages = 2;
@@ -868,14 +875,15 @@ static void plan_common(GemmPlan *p) {
     p->ws_bytes = cnt + (size_t)p->slots * per_slot * p->bn * kTileA * 4;
 }
 
-void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
+void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p, bool w4) {
     if (m > 256 && m <= kMaxSwapM) {
         // a few hundred rows: too few 128 x 256 tiles for 148 SMs; stream-K
         // over all of them, as in a batched launch
-        plan_gemm_batch(m, 1, &n, &k, num_sms, p);
+        plan_gemm_batch(m, 1, &n, &k, num_sms, p, w4);
         return;
     }
     *p = GemmPlan{};
+    p->w4 = w4 ? 1 : 0;
     p->njobs = 1;
     p->swap = (m <= 256) ? 1 : 0;
     // an A operand streamed once from HBM against a single B tile (a
@@ -942,7 +950,7 @@ void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p) {
 void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p,
                      bool w4) {
     *p = GemmPlan{};
-    p->w4 = w4 ? 1 : 0;         // INT4 weights: the swapped orientation only (m <= 256)
+    p->w4 = w4 ? 1 : 0;         // INT4 weights, unpacked into whichever operand holds them
     p->njobs = njobs;
     // m <= 256: the weights are the 128-row A operand and the activations
     // one B tile of roundup16(m) rows.  256 < m <= 512: activations are A
@@ -1049,14 +1057,15 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
         const GemmProblem &q = probs[j];
         const int8_t *A = p.swap ? q.wq : q.xq;
         const int8_t *B = p.swap ? q.xq : q.wq;
-        if (p.w4) {
-            // packed INT4 weight [n, k/2] bytes, plain (unswizzled) 64-byte boxes
-            if (!p.swap || !make_tmap_plain(&maps.a[j], A, p.rows_a[j], q.k / 2, kTileA, (int)kPackedTileBytes / kTileA))
-                return cudaErrorInvalidValue;
-        } else if (!make_tmap(&maps.a[j], A, p.rows_a[j], q.k, kTileA)) {
+        // the weight's map: packed INT4 [n, k/2] bytes in plain (unswizzled)
+        // 64-byte boxes, or INT8 [n, k] in 128-byte swizzled boxes
+        const bool a_w4 = p.w4 && p.swap, b_w4 = p.w4 && !p.swap;
+        if (a_w4 ? !make_tmap_plain(&maps.a[j], A, p.rows_a[j], q.k / 2, kTileA, (int)kPackedRowBytes)
+                 : !make_tmap(&maps.a[j], A, p.rows_a[j], q.k, kTileA))
             return cudaErrorInvalidValue;
-        }
-        if (!make_tmap(&maps.b[j], B, p.rows_b[j], q.k, p.bn)) return cudaErrorInvalidValue;
+        if (b_w4 ? !make_tmap_plain(&maps.b[j], B, p.rows_b[j], q.k / 2, p.bn, (int)kPackedRowBytes)
+                 : !make_tmap(&maps.b[j], B, p.rows_b[j], q.k, p.bn))
+            return cudaErrorInvalidValue;
         GemmJob &J = a.job[j];
         J.m = (int)q.m;
         J.n = (int)q.n;

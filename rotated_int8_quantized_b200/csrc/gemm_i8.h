@@ -84,12 +84,13 @@ struct GemmPlan {
 };
 
 // Single product: whole tiles dealt round-robin in full waves, the last
-// partial wave split along K (stream-K).
-void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p);
+// partial wave split along K (stream-K).  w4: INT4 weights (packed two
+// codes per byte), unpacked in shared memory.
+void plan_gemm(int64_t m, int64_t n, int64_t k, int num_sms, GemmPlan *p, bool w4 = false);
 // Several products with the same m <= kMaxSwapM in one launch: every K
 // block of every (weight tile, activation tile) pair dealt out evenly by
 // stream-K.
-// w4: INT4 weights (packed two codes per byte; m <= 256 only).
+// w4: INT4 weights (packed two codes per byte).
 void plan_gemm_batch(int64_t m, int njobs, const int64_t *n, const int64_t *k, int num_sms, GemmPlan *p,
                      bool w4 = false);
 

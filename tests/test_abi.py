@@ -176,9 +176,12 @@ def test_weight4_validation(lib):
     assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10001), P(0x20000), 8, 512, 256) == 2
     job = (cr.convrot_linear4_job_t * 1)()
     job[0].x_bf16, job[0].w, job[0].y_bf16 = P(0x100000), ctypes.pointer(h), P(0x200000)
-    assert lib.convrot_linear_w4a8(257, 1, job, P(0x300000), 1 << 30, P(0)) == 3     # m > 256
     assert lib.convrot_linear_w4a8(0, 1, job, P(0x300000), 1 << 30, P(0)) == 1
     assert lib.convrot_linear_w4a8_workspace_bytes(12, 1, job) > 0
+    # any token count: prefill sizes take per-job GEMM launches
+    assert lib.convrot_linear_w4a8_workspace_bytes(300, 1, job) > 0
+    job[0].y_bf16 = P(0x10000000)        # clear of the 4 MB input at m = 4096
+    assert lib.convrot_linear_w4a8_workspace_bytes(4096, 1, job) > 0
 
 
 def test_conv2d_shape_and_validation(lib):

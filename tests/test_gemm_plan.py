@@ -105,6 +105,14 @@ def test_int4_batch_and_other_gpu_sizes():
     import rotated_int8_quantized_b200 as cr
     p = cr.gemm_plan(12, QWEN_N, QWEN_K, w4=True, sms=SMS)
     check(p, 12, QWEN_N, QWEN_K)
+    # INT4 weights at any m: the batched stream-K plan up to 512 rows, whole
+    # tiles (weights the 256-row B operand) for single products beyond
+    for m in (300, 512):
+        check(cr.gemm_plan(m, QWEN_N, QWEN_K, w4=True, sms=SMS), m, QWEN_N, QWEN_K)
+    for (m, n, k) in ((4096, 8192, 5120), (4096, 5120, 25600), (700, 1000, 1536)):
+        p = cr.gemm_plan(m, [n], [k], w4=True, sms=SMS)
+        assert p.swap == 0 and p.bn == 256 and p.stages >= 3
+        check(p, m, [n], [k])
     for sms in (1, 7, 64, 132):
         for (m, n, k) in ((12, 5120, 8192), (4096, 8192, 5120), (400, 5120, 5120)):
             check(cr.gemm_plan(m, [n], [k], sms=sms), m, [n], [k])
@@ -114,8 +122,6 @@ def test_plan_rejections():
     import rotated_int8_quantized_b200 as cr
     with pytest.raises(cr.ConvrotError):
         cr.gemm_plan(600, [1024, 1024], [512, 512])      # batches are for m <= 512
-    with pytest.raises(cr.ConvrotError):
-        cr.gemm_plan(300, [1024], [512], w4=True)        # INT4 weights: m <= 256
     with pytest.raises(cr.ConvrotError):
         cr.gemm_plan(12, [1024], [512], sms=0)
 
@@ -132,11 +138,11 @@ def test_random_shapes_cover_every_block_once():
             m = int(rng.choice([1, 5, 12, 100, 256, 257, 300, 511, 512, 513, 1000, 3000, 9000]))
             n = int(rng.integers(1, 40)) * 16 * int(rng.choice([1, 4, 16]))
             k = int(rng.integers(1, 64)) * 16 * int(rng.choice([1, 2, 8]))
-            check(cr.gemm_plan(m, [n], [k], sms=sms), m, [n], [k])
+            check(cr.gemm_plan(m, [n], [k], w4=bool(rng.random() < 0.3), sms=sms), m, [n], [k])
         else:
             m = int(rng.choice([1, 7, 12, 64, 200, 256, 300, 512]))
             count = int(rng.integers(2, 9))
             ns = [int(rng.integers(1, 50)) * 64 for _ in range(count)]
             ks = [int(rng.integers(1, 40)) * 128 for _ in range(count)]
-            w4 = bool(m <= 256 and rng.random() < 0.3)
+            w4 = bool(rng.random() < 0.3)
             check(cr.gemm_plan(m, ns, ks, w4=w4, sms=sms), m, ns, ks)

@@ -627,6 +627,14 @@ W4_CASES = [
     (4, [(640, 384)]),
     (100, [(1536, 640), (512, 1000)]),
     (256, [(1024, 512)]),
+    # activations = A, the INT4 weight unpacked into the 256-row B operand:
+    # replicated stream-K (m <= 512), whole tiles with a split tail, ragged
+    # tiles both ways, a K not a multiple of 128 (dynamic group)
+    (300, [(1024, 512), (768, 384)]),
+    (512, [(2560, 640), (2560, 1000)]),
+    (700, [(1536, 640), (512, 1000)]),
+    (1200, [(5120, 1000), (640, 384)]),
+    (9500, [(1024, 500)]),
 ]
 
 
@@ -898,3 +906,33 @@ def test_inexact_domain_reported_by_convolution_pixels(cr):
     assert _status_after(cr, lambda: cr.conv2d_int8(xd, wq, 3, 3, 1, 1, 1)) == 0
     planted = _plant_wide_group(x_bits, 123, 0).reshape(n, h, w, c)
     assert _status_after(cr, lambda: cr.conv2d_int8(from_bits(planted), wq, 3, 3, 1, 1, 1)) == 8
+
+
+def test_w4a8_qwen_prefill_layer_sampled(cr):
+    # INT4 weights at prefill size: every linear of the layer at M = 4096
+    # through LinearBatchW4 (one whole-tile GEMM launch per linear)
+    lins = synth.qwen_layer(4096)
+    xs, ws4, ys = [], [], []
+    for lin in lins:
+        w_bf = lin.w_torch("cuda")
+        ws4.append(cr.quantize_weight4(w_bf))
+        del w_bf
+        xs.append(lin.x_torch("cuda"))
+        ys.append(torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device="cuda"))
+    batch = cr.LinearBatchW4(xs, ws4, ys)
+    batch()
+    batch()
+    cr.convrot_device_status()
+    rng = np.random.default_rng(4094)
+    rows_x = np.unique(np.concatenate([[0, 127, 128, 4095], rng.integers(0, 4096, 8)]))
+    for lin, w4, y in zip(lins, ws4, ys):
+        rows = _edge_rows(lin.n, rng, 8)
+        packed_ref, s_ref = oracle.rotate_quantize4(lin.w_rows_np(rows))
+        rw = torch.as_tensor(rows, device="cuda")
+        assert np.array_equal(w4.q[rw].cpu().numpy(), packed_ref), lin.name
+        ref = oracle.linear_w4a8(lin.x_rows_np(rows_x), packed_ref, s_ref)
+        yb = to_bits(y[torch.as_tensor(rows_x, device="cuda")][:, rw])
+        assert rel_err(yb, ref["y"]) <= TOL, lin.name
+        assert np.array_equal(yb, ref["y"]), lin.name
+    del batch, ws4, xs, ys
+    torch.cuda.empty_cache()
