@@ -866,12 +866,39 @@ constexpr int kLeanXchStride = 18;      // doubles per transpose row: 16 + 2 (16
 constexpr int kLeanXch = 16 * kLeanXchStride;
 constexpr int kLeanRegMaxGps = 2;       // rows of more groups per slot stage the row in shared memory
 
+// Warp maximum of non-negative floats in one instruction (their bit
+// patterns order like unsigned integers).
+__device__ __forceinline__ uint32_t warp_max_bits(uint32_t v) {
+    uint32_t r;
+    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+    return r;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// The row quantiser of the lean kernel.  s = fl(amax / 127) is the IEEE
+// quotient (stored, and the divisor of the rare exact path); the rounding
+// test multiplies by r = fl(127 * rcp.approx(amax)) instead of fl(1 / s), which
+// needs no division on the row's critical path: rcp.approx is within 1 ulp
+// (2^-23 relative) of 1/amax, so r is within 2^-23 + 2^-24 + 2^-24 (the
+// product's and s's roundings) of 1/s, |y r - y/s| <= 127 * 2^-22 = 3.03e-5,
+// and with |fl(y/s) - y/s| <= 7.6e-6 a distance |y r - rne(y r)| below
+// 0.49995 still proves that fl(y/s) rounds to rne(y r).  Rows with a subnormal
+// s (amax < 127 * 2^-126) or amax >= 2^125 (a subnormal 1/amax) take the
+// division for every element.
+constexpr float kLeanNear = 0.49995f;
+
+#ifndef CONVROT_LEAN_BOUNDS
+#define CONVROT_LEAN_BOUNDS kLeanThreads, 1
+#endif
 template <int GPS, bool REG>
-__global__ void __launch_bounds__(kLeanThreads, 1)
+__global__ void __launch_bounds__(CONVROT_LEAN_BOUNDS)
     rotate_quant_rows_lean(const __nv_bfloat16 *a, int64_t rows, int k, int8_t *q, float *s) {
     extern __shared__ __align__(16) uint8_t lsm[];
-    __shared__ float red[kLeanThreads / 32];
-    __shared__ float rinfo[4];          // s, 1/s, exactness threshold bits, fast flag
+    __shared__ uint32_t red[2][kLeanThreads / 32];    // per-warp maxima (bits), by row parity
     pdl_wait();
     pdl_launch_dependents();
     const int tid = threadIdx.x, slot = tid >> 4, t = tid & 15, lane = tid & 31, warp = tid >> 5;
@@ -899,8 +926,9 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
     };
     float yv[REG ? GPS : 1][16];
     int64_t row = blockIdx.x;
+    int par = 0;
     if (row < rows) load(row);
-    for (; row < rows; row += gridDim.x) {
+    for (; row < rows; row += gridDim.x, par ^= 1) {
         float amax = 0.f;
         uint32_t mkey = 0x7FFF7FFFu;
 #pragma unroll
@@ -947,34 +975,23 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
         }
         const int64_t nrow = row + gridDim.x;
         if (nrow < rows) load(nrow);         // in flight during this row's reduction and quantisation
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        if (lane == 0) red[warp] = amax;
-        __syncthreads();
-        if (warp == 0) {
-            float m = lane < nwarps ? red[lane] : 0.f;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) {
-                const RowScale rs0 = make_row_scale(m);
-                rinfo[0] = rs0.s;
-                rinfo[1] = rs0.r;
-                rinfo[2] = __int_as_float(exactness_threshold_bits(m));
-                rinfo[3] = __int_as_float((rs0.fast ? 1 : 0) | (rs0.zero ? 2 : 0));
-            }
+        {
+            const uint32_t wm = warp_max_bits(__float_as_uint(amax));
+            if (lane == 0) red[par][warp] = wm;
         }
+        // one barrier per row: afterwards every warp reads the per-warp maxima
+        // of this row (red[par] is written again two rows later, after the
+        // next row's barrier, by when every warp has read it)
         __syncthreads();
-        RowScale rs;
-        rs.s = rinfo[0];
-        rs.r = rinfo[1];
-        const int tbits = __float_as_int(rinfo[2]);
-        const int flags = __float_as_int(rinfo[3]);
-        rs.fast = (flags & 1) != 0;
-        rs.zero = (flags & 2) != 0;
+        const float rmax = __uint_as_float(warp_max_bits(lane < nwarps ? red[par][lane] : 0u));
+        const bool zero = rmax == 0.f;
+        const bool fast = rmax >= 127.0f * 1.17549435e-38f && rmax < 4.2535295865117308e37f;   // 2^125
+        const float rr = __fmul_rn(127.0f, rcp_approx(rmax));
+        const int tbits = exactness_threshold_bits(rmax);
         if (__any_sync(0xffffffffu, key_min_magnitude(mkey) < tbits) && lane == 0) report_inexact_domain();
         int8_t *qrow = q + row * k;
         if (REG) {
-            const uint64_t r2 = pack_f32x2(rs.r, rs.r), m2 = pack_f32x2(kRoundMagic, kRoundMagic);
+            const uint64_t r2 = pack_f32x2(rr, rr), m2 = pack_f32x2(kRoundMagic, kRoundMagic);
 #pragma unroll
             for (int gi = 0; gi < GPS; ++gi) {
                 const int g = slot + S * gi;
@@ -996,20 +1013,21 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
                         e[2 * i + 1] = __float_as_uint(e1);
                         dmax = max3abs(d0, d1, dmax);
                     }
-                    const bool slow = !(dmax < 0.49997f) || !rs.fast;   // NaN too; zero rows (codes set below)
+                    const bool slow = !(dmax < kLeanNear) || !fast;   // NaN too; zero rows (codes set below)
                     if (__any_sync(mask, slow) && slow) {
+                        const float sd = __fdiv_rn(rmax, 127.0f);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const float ei = __fmaf_rn(y[i], rs.r, kRoundMagic);
-                            const float di = __fmaf_rn(y[i], rs.r, __fsub_rn(kRoundMagic, ei));
-                            if (!rs.fast || !(fabsf(di) < 0.49997f)) {
+                            const float ei = __fmaf_rn(y[i], rr, kRoundMagic);
+                            const float di = __fmaf_rn(y[i], rr, __fsub_rn(kRoundMagic, ei));
+                            if (!fast || !(fabsf(di) < kLeanNear)) {
                                 const int c =
-                                    __float_as_int(__fadd_rn(__fdiv_rn(y[i], rs.s), kRoundMagic)) - kRoundMagicBits;
+                                    __float_as_int(__fadd_rn(__fdiv_rn(y[i], sd), kRoundMagic)) - kRoundMagicBits;
                                 e[i] = (uint32_t)min(max(c, -127), 127);
                             }
                         }
                     }
-                    if (rs.zero) {
+                    if (zero) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) e[i] = 0u;
                     }
@@ -1024,6 +1042,7 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
                 }
             }
         } else {
+            const RowScale rs = make_row_scale(rmax);
             for (int c0 = 0; c0 < chunks; c0 += (int)blockDim.x) {
                 const int c = c0 + tid;
                 const unsigned mask = __ballot_sync(0xffffffffu, c < chunks);
@@ -1044,7 +1063,7 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
                 }
             }
         }
-        if (tid == 0) s[row] = rs.s;
+        if (tid == 0) s[row] = __fdiv_rn(rmax, 127.0f);
         if (!REG) __syncthreads();           // ybuf is written again by the next row
     }
 }
