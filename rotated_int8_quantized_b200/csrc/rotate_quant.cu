@@ -891,11 +891,11 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // division for every element.
 constexpr float kLeanNear = 0.49995f;
 
-#ifndef CONVROT_LEAN_BOUNDS
-#define CONVROT_LEAN_BOUNDS kLeanThreads, 1
-#endif
+// One group per slot: capped at 64 registers (16 bytes of spill), so that
+// two 512-thread or three 320-thread CTAs share an SM; the variants with
+// more groups per slot keep their registers.
 template <int GPS, bool REG>
-__global__ void __launch_bounds__(CONVROT_LEAN_BOUNDS)
+__global__ void __launch_bounds__(kLeanThreads, (GPS == 1 && REG) ? 2 : 1)
     rotate_quant_rows_lean(const __nv_bfloat16 *a, int64_t rows, int k, int8_t *q, float *s) {
     extern __shared__ __align__(16) uint8_t lsm[];
     __shared__ uint32_t red[2][kLeanThreads / 32];    // per-warp maxima (bits), by row parity
