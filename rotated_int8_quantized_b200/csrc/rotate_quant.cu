@@ -362,10 +362,12 @@ __device__ __forceinline__ int key_min_magnitude(uint32_t k) {
 // amax == 0); a nonzero input with smaller magnitude bits MAY be outside
 // the domain.
 __device__ __forceinline__ int exactness_threshold_bits(float amax) {
-    if (!(amax > 0.f) || !isfinite(amax)) return 0;
-    int e;
-    frexpf(amax, &e);
-    const int p = e - 33;
+    // e(amax) from the FP32 exponent field (e = field - 126 for a normal
+    // amax); a subnormal, zero or non-finite amax has no threshold that a
+    // BF16 input could fall below except in the subnormal range: 0 there
+    const int field = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
+    const int p = field - 159;                      // e(amax) - 33
+    if (field == 0 || field == 0xFF) return 0;
     if (p >= -126) return (p + 127) << 7;
     if (p >= -133) return 1 << (p + 133);
     return 0;
@@ -891,12 +893,19 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // division for every element.
 constexpr float kLeanNear = 0.49995f;
 
-// One group per slot: capped at 64 registers (16 bytes of spill), so that
-// two 512-thread or three 320-thread CTAs share an SM; the variants with
-// more groups per slot keep their registers.
-template <int GPS, bool REG>
-__global__ void __launch_bounds__(kLeanThreads, (GPS == 1 && REG) ? 2 : 1)
-    rotate_quant_rows_lean(const __nv_bfloat16 *a, int64_t rows, int k, int8_t *q, float *s) {
+// RCAP: register cap per thread (0: the 512-thread bound's 128), chosen per
+// launch so that two or three CTAs of the row's width share an SM.
+// The matrices of a lean launch: up to kMaxJobs with the same row count
+// and row length; the launch walks all their rows as one sequence.
+struct LeanJobs {
+    const __nv_bfloat16 *a[kMaxJobs];
+    int8_t *q[kMaxJobs];
+    float *s[kMaxJobs];
+};
+
+template <int GPS, bool REG, int RCAP>
+__global__ void __launch_bounds__(kLeanThreads, 1) __maxnreg__(RCAP ? RCAP : 128)
+    rotate_quant_rows_lean(const __grid_constant__ LeanJobs jobs, int njobs, int64_t rows, int k) {
     extern __shared__ __align__(16) uint8_t lsm[];
     __shared__ uint32_t red[2][kLeanThreads / 32];    // per-warp maxima (bits), by row parity
     pdl_wait();
@@ -912,23 +921,28 @@ __global__ void __launch_bounds__(kLeanThreads, (GPS == 1 && REG) ? 2 : 1)
     uint8_t *xbytes = reinterpret_cast<uint8_t *>(xb) + (slot & 1) * 64;
     float *ybuf = reinterpret_cast<float *>(lsm + (size_t)S * kLeanXch * 8);   // !REG: the row in FP32
     const uint64_t sixteenth = pack_f32x2(0.0625f, 0.0625f);
+    const int64_t total = rows * njobs;
     uint4 raw[GPS][2];
-    auto load = [&](int64_t r) {
+    auto load = [&](int64_t gr) {
+        const int jb = (int)(gr / rows);
+        const __nv_bfloat16 *arow = jobs.a[jb] + (gr - (int64_t)jb * rows) * k;
 #pragma unroll
         for (int gi = 0; gi < GPS; ++gi) {
             const int g = slot + S * gi;
             if (g < groups) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(a + r * k + g * 256 + t * 16);
+                const uint4 *src = reinterpret_cast<const uint4 *>(arow + g * 256 + t * 16);
                 raw[gi][0] = __ldg(src);
                 raw[gi][1] = __ldg(src + 1);
             }
         }
     };
     float yv[REG ? GPS : 1][16];
-    int64_t row = blockIdx.x;
+    int64_t grow = blockIdx.x;
     int par = 0;
-    if (row < rows) load(row);
-    for (; row < rows; row += gridDim.x, par ^= 1) {
+    if (grow < total) load(grow);
+    for (; grow < total; grow += gridDim.x, par ^= 1) {
+        const int jb = (int)(grow / rows);
+        const int64_t row = grow - (int64_t)jb * rows;
         float amax = 0.f;
         uint32_t mkey = 0x7FFF7FFFu;
 #pragma unroll
@@ -973,8 +987,8 @@ __global__ void __launch_bounds__(kLeanThreads, (GPS == 1 && REG) ? 2 : 1)
                 }
             }
         }
-        const int64_t nrow = row + gridDim.x;
-        if (nrow < rows) load(nrow);         // in flight during this row's reduction and quantisation
+        const int64_t nrow = grow + gridDim.x;
+        if (nrow < total) load(nrow);        // in flight during this row's reduction and quantisation
         {
             const uint32_t wm = warp_max_bits(__float_as_uint(amax));
             if (lane == 0) red[par][warp] = wm;
@@ -987,9 +1001,8 @@ __global__ void __launch_bounds__(kLeanThreads, (GPS == 1 && REG) ? 2 : 1)
         const bool zero = rmax == 0.f;
         const bool fast = rmax >= 127.0f * 1.17549435e-38f && rmax < 4.2535295865117308e37f;   // 2^125
         const float rr = __fmul_rn(127.0f, rcp_approx(rmax));
-        const int tbits = exactness_threshold_bits(rmax);
-        if (__any_sync(0xffffffffu, key_min_magnitude(mkey) < tbits) && lane == 0) report_inexact_domain();
-        int8_t *qrow = q + row * k;
+        if (key_min_magnitude(mkey) < exactness_threshold_bits(rmax)) report_inexact_domain();
+        int8_t *qrow = jobs.q[jb] + row * k;
         if (REG) {
             const uint64_t r2 = pack_f32x2(rr, rr), m2 = pack_f32x2(kRoundMagic, kRoundMagic);
 #pragma unroll
@@ -1063,7 +1076,7 @@ __global__ void __launch_bounds__(kLeanThreads, (GPS == 1 && REG) ? 2 : 1)
                 }
             }
         }
-        if (tid == 0) s[row] = __fdiv_rn(rmax, 127.0f);
+        if (tid == 0) jobs.s[jb][row] = __fdiv_rn(rmax, 127.0f);
         if (!REG) __syncthreads();           // ybuf is written again by the next row
     }
 }
@@ -1073,15 +1086,20 @@ __global__ void __launch_bounds__(kLeanThreads, (GPS == 1 && REG) ? 2 : 1)
 // up to 64 groups keep their rotated values in registers (GPS <= 2); longer
 // rows stage them in shared memory.
 static void lean_shape(int groups, int *gps, int *slots, bool *reg) {
-    const int g = (groups + 31) / 32;
+    // two groups per slot up to 64 groups when they pair up evenly
+    // (measured: K = 4096, 5120 and 8192 at M = 4096 a few per cent faster
+    // than one group per slot; K = 5376's 21 groups were not)
+    const int g = (groups <= 64 && groups % 4 == 0) ? 2 : (groups + 31) / 32;
     const int sl = (groups + g - 1) / g;
     *gps = g;
     *slots = (sl + 1) & ~1;
     *reg = g <= kLeanRegMaxGps;
 }
 
-template <int GPS, bool REG>
-static cudaError_t launch_lean(const RQProblem &pr, int64_t rows, int sms, int slots, cudaStream_t stream, bool pdl) {
+template <int GPS, bool REG, int RCAP>
+static cudaError_t launch_lean(int njobs, const RQProblem *probs, int64_t rows, int sms, int slots, cudaStream_t stream,
+                               bool pdl) {
+    const RQProblem &pr = probs[0];
     const int groups = (int)(pr.k >> 8);
     const size_t smem = (size_t)slots * kLeanXch * 8 + (REG ? 0 : (size_t)groups * kYGroupStride * 4);
     static bool configured[64] = {};
@@ -1089,28 +1107,66 @@ static cudaError_t launch_lean(const RQProblem &pr, int64_t rows, int sms, int s
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(rotate_quant_rows_lean<GPS, REG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(rotate_quant_rows_lean<GPS, REG, RCAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSlotsSmemMax);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev] = true;
     }
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_rows_lean<GPS, REG>, slots * 16, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_rows_lean<GPS, REG, RCAP>, slots * 16, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t cap = (int64_t)sms * per_sm;
+    const int64_t total = rows * njobs;
+    LeanJobs jobs;
+    memset(&jobs, 0, sizeof(jobs));
+    for (int j = 0; j < njobs; ++j) {
+        jobs.a[j] = static_cast<const __nv_bfloat16 *>(probs[j].a);
+        jobs.q[j] = probs[j].q;
+        jobs.s[j] = probs[j].s;
+    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3((unsigned)(rows < cap ? rows : cap));
+    cfg.gridDim = dim3((unsigned)(total < cap ? total : cap));
     cfg.blockDim = dim3(slots * 16);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cfg.attrs = pdl ? attr : nullptr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_lean<GPS, REG>, static_cast<const __nv_bfloat16 *>(pr.a), rows,
-                              (int)pr.k, pr.q, pr.s);
+    return cudaLaunchKernelEx(&cfg, rotate_quant_rows_lean<GPS, REG, RCAP>, jobs, njobs, rows, (int)pr.k);
+}
+
+// The lean kernel takes INT8 codes of groups of 256 over rows of 16 to 128
+// groups, when there are at least two rows per SM in the launch.
+static bool lean_applies(const RQProblem &pr, int64_t total_rows, int num_sms) {
+    if (pr.int4 || pr.group != 256 || (pr.k & 255) != 0 || total_rows < 2 * (int64_t)num_sms) return false;
+    const int groups = (int)(pr.k >> 8);
+    int gps, slots;
+    bool reg;
+    lean_shape(groups, &gps, &slots, &reg);
+    return groups >= kLeanMinGroups && gps <= kLeanMaxGps;
+}
+
+// One lean launch over `nj` matrices of the same row length and row count.
+static cudaError_t launch_lean_any(int nj, const RQProblem *probs, int64_t rows, int num_sms, cudaStream_t stream,
+                                   bool pdl) {
+    int gps, slots;
+    bool reg;
+    lean_shape((int)(probs[0].k >> 8), &gps, &slots, &reg);
+    if (reg && gps == 1) {
+        // one group per slot: a register cap that lets three (up to 336
+        // threads) or two CTAs share an SM
+        const int threads = slots * 16;
+        if (threads <= 256) return launch_lean<1, true, 80>(nj, probs, rows, num_sms, slots, stream, pdl);
+        if (threads <= 336) return launch_lean<1, true, 64>(nj, probs, rows, num_sms, slots, stream, pdl);
+        if (threads <= 384) return launch_lean<1, true, 80>(nj, probs, rows, num_sms, slots, stream, pdl);
+        return launch_lean<1, true, 64>(nj, probs, rows, num_sms, slots, stream, pdl);
+    }
+    if (reg) return launch_lean<2, true, 0>(nj, probs, rows, num_sms, slots, stream, pdl);
+    if (gps == 3) return launch_lean<3, false, 0>(nj, probs, rows, num_sms, slots, stream, pdl);
+    return launch_lean<4, false, 0>(nj, probs, rows, num_sms, slots, stream, pdl);
 }
 
 cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs, cudaStream_t stream, bool pdl,
@@ -1120,11 +1176,29 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     const bool few_rows = rows * njobs < num_sms;
     if (!few_rows && njobs > 1) {
-        // rows fill the GPU: one launch per matrix, each with the CTA shape of
-        // its own row length (a shared shape would size every CTA for the
-        // longest rows)
+        // rows fill the GPU: one launch per row length (matrices of the same
+        // row length walked together by the lean kernel, which then has
+        // fewer tails), each with the CTA shape of its own row length (a
+        // shared shape would size every CTA for the longest rows)
+        bool done[kMaxJobs] = {};
         for (int jj = 0; jj < njobs; ++jj) {
-            cudaError_t e = launch_rotate_quant(1, rows, probs + jj, stream, pdl, conv);
+            if (done[jj]) continue;
+            RQProblem same[kMaxJobs];
+            int ns = 0;
+            for (int j2 = jj; j2 < njobs; ++j2) {
+                if (!done[j2] && probs[j2].k == probs[jj].k && probs[j2].group == probs[jj].group &&
+                    probs[j2].int4 == probs[jj].int4) {
+                    same[ns++] = probs[j2];
+                    done[j2] = true;
+                }
+            }
+            cudaError_t e = cudaSuccess;
+            if (!conv && lean_applies(same[0], rows * ns, num_sms)) {
+                e = launch_lean_any(ns, same, rows, num_sms, stream, pdl);
+            } else {
+                for (int j2 = 0; j2 < ns && e == cudaSuccess; ++j2)
+                    e = launch_rotate_quant(1, rows, same + j2, stream, pdl, conv);
+            }
             if (e != cudaSuccess) return e;
         }
         return cudaSuccess;
@@ -1137,23 +1211,8 @@ cudaError_t launch_rotate_quant(int njobs, int64_t rows, const RQProblem *probs,
     if (conv_mode == 5 && njobs == 1 && probs[0].group == 256 && (probs[0].k == 256 || probs[0].k == 512))
         return launch_rotate_pixels(probs[0].a, rows, (int)probs[0].k, reinterpret_cast<float *>(probs[0].q),
                                     probs[0].s, stream, pdl);
-    if (conv_mode == 0 && !int4 && njobs == 1 && probs[0].group == 256 && (probs[0].k & 255) == 0 &&
-        rows >= 2 * (int64_t)num_sms) {
-        const int groups = (int)(probs[0].k >> 8);
-        int gps, slots;
-        bool reg;
-        lean_shape(groups, &gps, &slots, &reg);
-        if (groups >= kLeanMinGroups && gps <= kLeanMaxGps) {
-            if (reg) {
-                return gps == 1 ? launch_lean<1, true>(probs[0], rows, num_sms, slots, stream, pdl)
-                                : launch_lean<2, true>(probs[0], rows, num_sms, slots, stream, pdl);
-            }
-            switch (gps) {
-                case 3: return launch_lean<3, false>(probs[0], rows, num_sms, slots, stream, pdl);
-                default: return launch_lean<4, false>(probs[0], rows, num_sms, slots, stream, pdl);
-            }
-        }
-    }
+    if (conv_mode == 0 && njobs == 1 && lean_applies(probs[0], rows, num_sms))
+        return launch_lean_any(1, probs, rows, num_sms, stream, pdl);
     const bool half = few_rows && !int4 && conv_mode == 0;
     const int parts = rq_parts(njobs, rows, probs, num_sms, half);
     cudaLaunchConfig_t cfg = {};

@@ -362,6 +362,9 @@ BATCH_CASES = [
     (300, [(768, 512), (512, 1000)]),
     (512, [(5120, 1024), (2560, 640), (512, 384)]),
     (600, [(768, 512), (512, 1000)]),
+    # several inputs of the same row length rotated by one persistent launch
+    (400, [(4096, 640), (4096, 384), (5120, 512), (4096, 256)]),
+    (700, [(4096, 256), (4096, 384)]),
 ]
 
 
