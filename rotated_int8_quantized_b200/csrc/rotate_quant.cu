@@ -921,11 +921,20 @@ __global__ void __launch_bounds__(kLeanThreads, 1) __maxnreg__(RCAP ? RCAP : 128
     uint8_t *xbytes = reinterpret_cast<uint8_t *>(xb) + (slot & 1) * 64;
     float *ybuf = reinterpret_cast<float *>(lsm + (size_t)S * kLeanXch * 8);   // !REG: the row in FP32
     const uint64_t sixteenth = pack_f32x2(0.0625f, 0.0625f);
-    const int64_t total = rows * njobs;
+    // rows are walked as one sequence over the jobs; (job, row) of the
+    // current and of the prefetched row advance by gridDim.x without a
+    // division (one job's rows subtracted per boundary crossed)
+    const int64_t stride = gridDim.x;
     uint4 raw[GPS][2];
-    auto load = [&](int64_t gr) {
-        const int jb = (int)(gr / rows);
-        const __nv_bfloat16 *arow = jobs.a[jb] + (gr - (int64_t)jb * rows) * k;
+    auto advance = [&](int &jb, int64_t &r) {
+        r += stride;
+        while (r >= rows && jb < njobs) {
+            r -= rows;
+            ++jb;
+        }
+    };
+    auto load = [&](int jb, int64_t r) {
+        const __nv_bfloat16 *arow = jobs.a[jb] + r * k;
 #pragma unroll
         for (int gi = 0; gi < GPS; ++gi) {
             const int g = slot + S * gi;
@@ -937,12 +946,17 @@ __global__ void __launch_bounds__(kLeanThreads, 1) __maxnreg__(RCAP ? RCAP : 128
         }
     };
     float yv[REG ? GPS : 1][16];
-    int64_t grow = blockIdx.x;
+    int jb = 0, njb = 0;
+    int64_t row = blockIdx.x, nrow = blockIdx.x;
+    while (row >= rows && jb < njobs) {           // a grid larger than one job's rows
+        row -= rows;
+        ++jb;
+    }
+    njb = jb;
+    nrow = row;
+    if (jb < njobs) load(jb, row);
     int par = 0;
-    if (grow < total) load(grow);
-    for (; grow < total; grow += gridDim.x, par ^= 1) {
-        const int jb = (int)(grow / rows);
-        const int64_t row = grow - (int64_t)jb * rows;
+    for (; jb < njobs; par ^= 1) {
         float amax = 0.f;
         uint32_t mkey = 0x7FFF7FFFu;
 #pragma unroll
@@ -987,8 +1001,8 @@ __global__ void __launch_bounds__(kLeanThreads, 1) __maxnreg__(RCAP ? RCAP : 128
                 }
             }
         }
-        const int64_t nrow = grow + gridDim.x;
-        if (nrow < total) load(nrow);        // in flight during this row's reduction and quantisation
+        advance(njb, nrow);
+        if (njb < njobs) load(njb, nrow);     // in flight during this row's reduction and quantisation
         {
             const uint32_t wm = warp_max_bits(__float_as_uint(amax));
             if (lane == 0) red[par][warp] = wm;
@@ -1078,6 +1092,8 @@ __global__ void __launch_bounds__(kLeanThreads, 1) __maxnreg__(RCAP ? RCAP : 128
         }
         if (tid == 0) jobs.s[jb][row] = __fdiv_rn(rmax, 127.0f);
         if (!REG) __syncthreads();           // ybuf is written again by the next row
+        jb = njb;
+        row = nrow;
     }
 }
 
