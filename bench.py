@@ -789,8 +789,30 @@ def run_profile(args):
         cr.convrot_device_status()
         print("profile run ok: conv, %d steps" % args.steps)
         return
-    m = {"decode": 12, "prefill": 4096}[args.profile]
-    lins = synth.qwen_layer(m)
+    if args.profile == "w4a8":
+        # the decode layer with INT4 weights (seven weight conversions, then
+        # the W4A8 steps)
+        lins = synth.qwen_layer(12)
+        ws4 = []
+        for lin in lins:
+            w_bf = lin.w_torch(device)
+            ws4.append(cr.quantize_weight4(w_bf))
+            del w_bf
+        xs = [lin.x_torch(device) for lin in lins]
+        ys = [torch.empty((lin.m, lin.n), dtype=torch.bfloat16, device=device) for lin in lins]
+        batch = cr.LinearBatchW4(xs, ws4, ys)
+        torch.cuda.synchronize()
+        for _ in range(args.steps):
+            batch()
+        torch.cuda.synchronize()
+        cr.convrot_device_status()
+        print("profile run ok: w4a8, %d steps" % args.steps)
+        return
+    if args.profile == "m512":
+        # one layer of the 50-layer stack at M = 512
+        lins = synth.qwen_stack(512, layers=1)
+    else:
+        lins = synth.qwen_layer({"decode": 12, "prefill": 4096}[args.profile])
     layer = Layer(cr, lins, device)
     xs, ys, wss = make_io(cr, layer, lins, device)
     stream = torch.cuda.current_stream()
@@ -1078,7 +1100,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-minimax", action="store_true", help="skip the MiniMax qkv TOPS measurement")
     ap.add_argument("--no-stack", action="store_true", help="skip the 50-layer stack measurement")
-    ap.add_argument("--profile", choices=["decode", "prefill", "conv"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill", "conv", "w4a8", "m512"], default=None,
                     help="run a few eager steps of one workload for ncu (no timing)")
     args = ap.parse_args()
     if args.profile:
