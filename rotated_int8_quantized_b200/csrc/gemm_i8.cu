@@ -309,8 +309,10 @@ __device__ __forceinline__ uint32_t sext_nibbles(uint32_t v) {
 // block: the A tile of 128 rows in the swapped orientation, the B tile of bn
 // rows otherwise); warps 6-13 unpack it into the wrows x 128-byte
 // 128B-swizzled INT8 tile the MMA reads.
-template <bool W4>
-__global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
+// WO: where INT4 weights go -- 0: INT8 weights (no unpacking), 1: the A
+// operand (weight-streaming, a 128-row tile), 2: the B operand (bn rows).
+template <int WO>
+__global__ void __launch_bounds__(WO ? kThreadsW4 : kThreads, 1)
     gemm_i8_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled operand tiles
@@ -323,7 +325,8 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
     const uint32_t a_off = 0;
     const uint32_t b_off = (uint32_t)S * kATileBytes;
     // W4: a staging slot per stage where the packed weight tile lands
-    const int wrows = a.swap ? kTileA : a.bn;           // rows of the weight tile
+    constexpr bool W4 = WO != 0;
+    const int wrows = WO == 1 ? kTileA : a.bn;          // rows of the weight tile
     const uint32_t packed_bytes = (uint32_t)wrows * kPackedRowBytes;
     const uint32_t p_off = b_off + (uint32_t)S * b_bytes;
     const uint32_t bar_off = p_off + (W4 ? (uint32_t)S * packed_bytes : 0u);
@@ -389,7 +392,7 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
         if (lane == 0) {
             // W4: the packed weight tile lands in the stage's staging slot
             // (unpacked into its operand slot by the unpacking warps)
-            const uint32_t tx = W4 ? packed_bytes + (a.swap ? b_bytes : (uint32_t)kATileBytes)
+            const uint32_t tx = W4 ? packed_bytes + (WO == 1 ? b_bytes : (uint32_t)kATileBytes)
                                    : (uint32_t)kATileBytes + b_bytes;
             const int RS = S;
             const uint32_t free_bar = empty_bar;
@@ -566,10 +569,9 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
                     break;
                 }
                 const uint8_t *src = smem + p_off + (uint32_t)stage * packed_bytes;
-                uint8_t *dst = a.swap ? smem + a_off + (uint32_t)stage * kATileBytes
-                                      : smem + b_off + (uint32_t)stage * b_bytes;
-#pragma unroll 4
-                for (int item = ct; item < wrows * 8; item += kCT) {
+                uint8_t *dst = WO == 1 ? smem + a_off + (uint32_t)stage * kATileBytes
+                                       : smem + b_off + (uint32_t)stage * b_bytes;
+                auto unpack = [&](int item) {
                     const int r = item >> 3, c = item & 7;
                     const uint2 w = *reinterpret_cast<const uint2 *>(src + r * 64 + c * 8);
                     uint4 o;
@@ -578,6 +580,14 @@ __global__ void __launch_bounds__(W4 ? kThreadsW4 : kThreads, 1)
                     o.z = sext_nibbles((w.x >> 4) & 0x0F0F0F0Fu);     // codes 8-11
                     o.w = sext_nibbles((w.y >> 4) & 0x0F0F0F0Fu);     // codes 12-15
                     *reinterpret_cast<uint4 *>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = o;
+                };
+                if (WO == 1) {
+                    // weight-streaming: a 128-row tile, a fixed trip count (fully unrolled)
+#pragma unroll
+                    for (int i = 0; i < kTileA * 8 / kCT; ++i) unpack(ct + kCT * i);
+                } else {
+#pragma unroll 4
+                    for (int item = ct; item < wrows * 8; item += kCT) unpack(item);
                 }
                 fence_proxy_async_shared();      // the tensor core reads these stores
                 __syncwarp();
@@ -1088,9 +1098,11 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(gemm_i8_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        e = cudaFuncSetAttribute(gemm_i8_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(gemm_i8_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        e = cudaFuncSetAttribute(gemm_i8_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(gemm_i8_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev] = true;
     }
@@ -1105,8 +1117,8 @@ cudaError_t launch_gemm_i8(const GemmPlan &p, const GemmProblem *probs, void *ws
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if (p.w4) return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel<true>, maps, a);
-    return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel<false>, maps, a);
+    if (p.w4) return cudaLaunchKernelEx(&cfg, p.swap ? gemm_i8_tc_kernel<1> : gemm_i8_tc_kernel<2>, maps, a);
+    return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel<0>, maps, a);
 }
 
 }  // namespace convrot
