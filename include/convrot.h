@@ -372,8 +372,11 @@ typedef struct {
  * tensor-core GEMM with the packed weight tiles unpacked to INT8 in shared
  * memory by eight dedicated warps per CTA.  m <= 512: one GEMM launch for all
  * jobs (for m <= 256 weight-streaming, the K blocks of all weights dealt out
- * to every SM); larger m (prefill, video tokens): one GEMM launch per job,
- * whole 128 x 256 tiles with the weight as the 256-row operand.  Results:
+ * to every SM).  Larger m (prefill, video tokens), where the layer is
+ * tensor-bound: per job, the weight is first unpacked to INT8 into the
+ * workspace (one pass over it) and then multiplied by the INT8 GEMM (whole
+ * 128 x 256 tiles); the workspace then also holds one unpacked weight (the
+ * largest n * k of the jobs, in bytes).  Results:
  * y = bf16(((float)acc * sx[m]) * sw[n] [+ bias[n]]) with acc the exact INT32
  * product of the INT8 activation codes and the INT4 weight codes.
  * Workspace: convrot_linear_w4a8_workspace_bytes, zero-filled before first

@@ -322,10 +322,12 @@ convrot_status_t collect_jobs4(int64_t m, int count, const convrot_linear4_job_t
 }
 
 // Workspace layout of the layer entry points: [GEMM scratch][xq_0][sx_0][xq_1][sx_1]...
+// and, for INT4 weights with per-job GEMMs, [one weight unpacked to INT8].
 struct LinearLayout {
     bool batched_gemm;
     convrot::GemmPlan batch;       // when batched_gemm
     size_t gemm_bytes;
+    size_t unpack_off, unpack_bytes;
     size_t total;
 };
 
@@ -343,14 +345,27 @@ void linear_layout(int64_t m, int count, const LinJob *jobs, bool w4, int sms, L
     } else {
         for (int j = 0; j < count; ++j) {
             convrot::GemmPlan p;
-            convrot::plan_gemm(m, jobs[j].n, jobs[j].k, sms, &p, w4);
+            convrot::plan_gemm(m, jobs[j].n, jobs[j].k, sms, &p);    // INT4 weights: unpacked first (below)
             g = p.ws_bytes > g ? p.ws_bytes : g;
         }
     }
     L->gemm_bytes = round256(g);
     size_t t = L->gemm_bytes;
     for (int j = 0; j < count; ++j) t += round256((size_t)m * (size_t)jobs[j].k) + round256((size_t)m * 4);
-    L->total = t;
+    // INT4 weights beyond the batched sizes: each weight is unpacked to INT8
+    // once per call (one HBM pass) and multiplied by the INT8 GEMM, instead
+    // of every CTA unpacking every weight tile it reads (shared-memory-bound)
+    L->unpack_off = t;
+    L->unpack_bytes = 0;
+    if (w4 && !L->batched_gemm) {
+        size_t mx = 0;
+        for (int j = 0; j < count; ++j) {
+            const size_t b = (size_t)jobs[j].n * (size_t)jobs[j].k;
+            mx = b > mx ? b : mx;
+        }
+        L->unpack_bytes = round256(mx);
+    }
+    L->total = t + L->unpack_bytes;
 }
 
 convrot_status_t run_linear(int64_t m, int count, const LinJob *jobs, bool w4, void *ws, size_t ws_bytes,
@@ -391,10 +406,24 @@ convrot_status_t run_linear(int64_t m, int count, const LinJob *jobs, bool w4, v
     if (L.batched_gemm) return from_cuda(convrot::launch_gemm_i8(L.batch, gp, base, st, true, true));
     for (int j = 0; j < count; ++j) {
         convrot::GemmPlan p;
-        convrot::plan_gemm(m, jobs[j].n, jobs[j].k, dev.num_sms, &p, w4);
-        // the first product may prefetch weights under the prologue; later
-        // ones follow another GEMM that could still be reading the scratch
-        e = convrot::launch_gemm_i8(p, &gp[j], base, st, true, j == 0);
+        if (w4) {
+            // the unpacked weight is written by the launch just before the
+            // GEMM (which waits for it: no weight prefetch ahead of the wait);
+            // the unpack itself waits for the previous GEMM, which read the
+            // same buffer
+            int8_t *wq8 = reinterpret_cast<int8_t *>(base + L.unpack_off);
+            e = convrot::launch_unpack_int4(reinterpret_cast<const uint8_t *>(jobs[j].wq), jobs[j].n, jobs[j].k, wq8,
+                                            st, true);
+            if (e != cudaSuccess) return from_cuda(e);
+            gp[j].wq = wq8;
+            convrot::plan_gemm(m, jobs[j].n, jobs[j].k, dev.num_sms, &p);
+            e = convrot::launch_gemm_i8(p, &gp[j], base, st, true, false);
+        } else {
+            convrot::plan_gemm(m, jobs[j].n, jobs[j].k, dev.num_sms, &p);
+            // the first product may prefetch weights under the prologue; later
+            // ones follow another GEMM that could still be reading the scratch
+            e = convrot::launch_gemm_i8(p, &gp[j], base, st, true, j == 0);
+        }
         if (e != cudaSuccess) return from_cuda(e);
     }
     return CONVROT_OK;

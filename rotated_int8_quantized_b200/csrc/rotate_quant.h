@@ -46,6 +46,8 @@ cudaError_t launch_conv_gather_quant(const float *yrot, const float *pmax, const
 
 // ------------------------------------------------------------------ tensor-wise INT8 (embedding table)
 cudaError_t launch_quantize_tensor(const void *a, int64_t count, int8_t *q, float *scale, cudaStream_t stream);
+// Packed INT4 weight [n, k/2] -> INT8 codes [n, k] (natural order).
+cudaError_t launch_unpack_int4(const uint8_t *packed, int64_t n, int64_t k, int8_t *out, cudaStream_t stream, bool pdl);
 cudaError_t launch_embed_lookup(const int32_t *tokens, int64_t t, const int8_t *q, const float *scale,
                                 int64_t vocab, int64_t dim, void *out, cudaStream_t stream);
 

@@ -111,6 +111,12 @@ __global__ void __launch_bounds__(kTqThreads) embed_lookup_kernel(const int32_t 
     }
 }
 
+// Sign-extend the low nibble of each byte of v (bytes 0..15) to int8: bit 3
+// of a byte times 30 is 0xF0, which lands in its empty high nibble.
+__device__ __forceinline__ uint32_t sext_nibbles4(uint32_t v) {
+    return (v & 0x08080808u) * 30u + v;
+}
+
 static int tq_grid(int64_t work) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -130,6 +136,47 @@ cudaError_t launch_quantize_tensor(const void *a, int64_t count, int8_t *q, floa
                                                        reinterpret_cast<uint4 *>(q));
     tensor_scale_kernel<<<1, 1, 0, stream>>>(scale);
     return cudaGetLastError();
+}
+
+// INT4 weight codes (this library's packing: within each 16-code chunk, byte
+// j holds code j in its low nibble and code 8 + j in its high nibble) to
+// INT8 codes in their natural order, two chunks (16 packed bytes -> 32 code
+// bytes) per thread and step.  HBM-bound; used before an INT8 GEMM at
+// prefill sizes, where unpacking every weight tile inside each CTA that
+// reads it would cost far more shared-memory bandwidth than one pass here.
+__global__ void __launch_bounds__(kTqThreads) unpack_int4_kernel(const uint4 *packed, int64_t pairs, uint4 *out) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < pairs; i += stride) {
+        const uint4 w = __ldg(packed + i);
+        const uint32_t h[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint32_t lo = h[2 * c], hi = h[2 * c + 1];     // the chunk's 8 packed bytes
+            uint4 o;
+            o.x = sext_nibbles4(lo & 0x0F0F0F0Fu);               // codes 0-3
+            o.y = sext_nibbles4(hi & 0x0F0F0F0Fu);               // codes 4-7
+            o.z = sext_nibbles4((lo >> 4) & 0x0F0F0F0Fu);        // codes 8-11
+            o.w = sext_nibbles4((hi >> 4) & 0x0F0F0F0Fu);        // codes 12-15
+            out[2 * i + c] = o;
+        }
+    }
+}
+
+cudaError_t launch_unpack_int4(const uint8_t *packed, int64_t n, int64_t k, int8_t *out, cudaStream_t stream, bool pdl) {
+    const int64_t pairs = n * k / 32;          // k % 32 == 0 for INT4 weights
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)tq_grid(pairs));
+    cfg.blockDim = dim3(kTqThreads);
+    cfg.stream = stream;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, unpack_int4_kernel, reinterpret_cast<const uint4 *>(packed), pairs,
+                              reinterpret_cast<uint4 *>(out));
 }
 
 cudaError_t launch_embed_lookup(const int32_t *tokens, int64_t t, const int8_t *q, const float *scale,
