@@ -750,6 +750,7 @@ def stack_secondary(cr, device, stream, peaks, layers=50, steps=5, warmup=2):
         with torch.cuda.stream(stream):
             one_pass()
         torch.cuda.synchronize()
+        launches_per_layer = count_launches(lambda: batches[0](stream), stream)
         g = capture(one_pass, stream)
         with torch.cuda.stream(stream):
             for _ in range(warmup):
@@ -761,7 +762,7 @@ def stack_secondary(cr, device, stream, peaks, layers=50, steps=5, warmup=2):
         ops = sum(2 * lin.m * lin.n * lin.k for lin in lins)
         out["m%d" % m] = {"gb_s": nbytes / t / 1e9, "ms_per_pass": t * 1e3, "tops": ops / t / 1e12,
                           "frac_of_measured_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"],
-                          "launches_per_pass": 2 * layers if m <= 512 else None}
+                          "launches_per_pass": launches_per_layer * layers if launches_per_layer > 0 else None}
         del g, batches, xs, ys
         torch.cuda.empty_cache()
     del ws

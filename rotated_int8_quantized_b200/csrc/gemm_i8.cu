@@ -195,9 +195,14 @@ __device__ __forceinline__ float dq_row(int32_t acc, float sxm, const float *sws
     return bias ? __fadd_rn(f, sws[kBiasStage + e]) : f;
 }
 
-__device__ __forceinline__ void emit_row16(const GemmJob &J, int m, int j0, const int32_t (&v)[16], float sxm,
-                                           const float *sws) {
+// sh: the accumulators are 2^sh times the products' sums (INT4 weights are
+// unpacked as 16 x code); the exact sum is v >> sh.
+__device__ __forceinline__ void emit_row16(const GemmJob &J, int m, int j0, const int32_t (&v_in)[16], float sxm,
+                                           const float *sws, int sh) {
     if (m >= J.m) return;
+    int32_t v[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = v_in[e] >> sh;
     const bool full = (j0 + 16 <= J.n) && ((J.n & 7) == 0);
     if (J.acc) {
         int32_t *dst = J.acc + (size_t)m * J.n + j0;
@@ -235,9 +240,12 @@ __device__ __forceinline__ void emit_row16(const GemmJob &J, int m, int j0, cons
 // buffer) so that each output row leaves as 16-byte segments instead of
 // 2-byte scatters.  Called by all 128 epilogue threads (it holds a barrier).
 __device__ __forceinline__ void emit_swap16(const GemmJob &J, int a0, int row, int tid, int j0,
-                                            const int32_t (&v)[16], float srow, float brow, const float *scol,
-                                            __nv_bfloat16 *stg) {
+                                            const int32_t (&v_in)[16], float srow, float brow, const float *scol,
+                                            __nv_bfloat16 *stg, int sh) {
     const int n = a0 + row;
+    int32_t v[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = v_in[e] >> sh;
     if (J.acc && n < J.n) {
 #pragma unroll
         for (int e = 0; e < 16; ++e)
@@ -274,15 +282,15 @@ __device__ __forceinline__ void emit_swap16(const GemmJob &J, int a0, int row, i
 // sw[n] for large M, sw[n] and sx[m] for the swapped (weights = A)
 // orientation.  Both compute bf16(((float)acc * sx[m]) * sw[n]).  Called by
 // all 128 epilogue threads; `chunk` counts the calls (it picks the transpose
-// buffer of the swapped orientation).
+// buffer of the swapped orientation).  sh: see emit_row16.
 __device__ __forceinline__ void emit16s(const GemmJob &J, int swap, int a0, int row, int tid, int j0,
                                         const int32_t (&v)[16], float srow, float brow, const float *scol,
-                                        __nv_bfloat16 *y_stage, int &chunk) {
+                                        __nv_bfloat16 *y_stage, int &chunk, int sh) {
     if (!swap) {
-        emit_row16(J, a0 + row, j0, v, srow, scol);
+        emit_row16(J, a0 + row, j0, v, srow, scol, sh);
         return;
     }
-    emit_swap16(J, a0, row, tid, j0, v, srow, brow, scol, y_stage + (chunk & 1) * 16 * kTileA);
+    emit_swap16(J, a0, row, tid, j0, v, srow, brow, scol, y_stage + (chunk & 1) * 16 * kTileA, sh);
     ++chunk;
 }
 
@@ -297,12 +305,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, int32_t (&v0)[16], int
         v0[e] = (int32_t)r0[e];
         v1[e] = (int32_t)r1[e];
     }
-}
-
-// Sign-extend the low nibble of each byte of v (bytes 0..15) to int8: the
-// bit 3 of a byte times 30 is 0xF0, which lands in its empty high nibble.
-__device__ __forceinline__ uint32_t sext_nibbles(uint32_t v) {
-    return (v & 0x08080808u) * 30u + v;
 }
 
 // W4: the weight arrives as packed INT4 codes (wrows x 64 bytes per K
@@ -326,6 +328,9 @@ __global__ void __launch_bounds__(WO ? kThreadsW4 : kThreads, 1)
     const uint32_t b_off = (uint32_t)S * kATileBytes;
     // W4: a staging slot per stage where the packed weight tile lands
     constexpr bool W4 = WO != 0;
+    // W4: the unpacked weight bytes are 16 x code, so the accumulators are
+    // 16 x the sums (exact: |16 * 7 * 127 * k| < 2^31 for every accepted k)
+    constexpr int kAccShift = W4 ? 4 : 0;
     const int wrows = WO == 1 ? kTileA : a.bn;          // rows of the weight tile
     const uint32_t packed_bytes = (uint32_t)wrows * kPackedRowBytes;
     const uint32_t p_off = b_off + (uint32_t)S * b_bytes;
@@ -574,11 +579,14 @@ __global__ void __launch_bounds__(WO ? kThreadsW4 : kThreads, 1)
                 auto unpack = [&](int item) {
                     const int r = item >> 3, c = item & 7;
                     const uint2 w = *reinterpret_cast<const uint2 *>(src + r * 64 + c * 8);
+                    // a two's-complement nibble in the high half of a byte,
+                    // low half zero, is the int8 value 16 x code: no sign
+                    // extension (the epilogue divides the exact sums by 16)
                     uint4 o;
-                    o.x = sext_nibbles(w.x & 0x0F0F0F0Fu);            // codes 0-3 of the chunk
-                    o.y = sext_nibbles(w.y & 0x0F0F0F0Fu);            // codes 4-7
-                    o.z = sext_nibbles((w.x >> 4) & 0x0F0F0F0Fu);     // codes 8-11
-                    o.w = sext_nibbles((w.y >> 4) & 0x0F0F0F0Fu);     // codes 12-15
+                    o.x = (w.x << 4) & 0xF0F0F0F0u;     // codes 0-3 of the chunk
+                    o.y = (w.y << 4) & 0xF0F0F0F0u;     // codes 4-7
+                    o.z = w.x & 0xF0F0F0F0u;            // codes 8-11
+                    o.w = w.y & 0xF0F0F0F0u;            // codes 12-15
                     *reinterpret_cast<uint4 *>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = o;
                 };
                 if (WO == 1) {
@@ -646,8 +654,8 @@ __global__ void __launch_bounds__(WO ? kThreadsW4 : kThreads, 1)
                     __syncwarp();
                     tmem_ld32(tbase + (uint32_t)c, v0, v1);
                     const int j0 = tb * a.bn + c;
-                    emit_row16(J, i, j0, v0, srow, scol + c);
-                    emit_row16(J, i, j0 + 16, v1, srow, scol + c + 16);
+                    emit_row16(J, i, j0, v0, srow, scol + c, kAccShift);
+                    emit_row16(J, i, j0 + 16, v1, srow, scol + c + 16, kAccShift);
                 }
             } else if (sg.split < 0) {
                 for (int c = 0; c < a.bn / 16; ++c) {
@@ -660,7 +668,7 @@ __global__ void __launch_bounds__(WO ? kThreadsW4 : kThreads, 1)
                     for (int e = 0; e < 16; ++e) v[e] = (int32_t)r[e];
                     if (whole) {
                         emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + c * 16, v, srow, brow, scol + c * 16,
-                                y_stage, ychunk);
+                                y_stage, ychunk, kAccShift);
                     } else {
                         int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
 #pragma unroll
@@ -771,8 +779,8 @@ __global__ void __launch_bounds__(WO ? kThreadsW4 : kThreads, 1)
                                 }
                             }
                             const int j0 = tb * a.bn + col0 + cc;
-                            emit_row16(J, i, j0, v0, srow, scol + col0 + cc);
-                            emit_row16(J, i, j0 + 16, v1, srow, scol + col0 + cc + 16);
+                            emit_row16(J, i, j0, v0, srow, scol + col0 + cc, kAccShift);
+                            emit_row16(J, i, j0 + 16, v1, srow, scol + col0 + cc + 16, kAccShift);
                         }
                         named_bar_sync(1, 128);     // buffer (r & 1) is read by everyone
                         if (r + 2 < rounds && ew == 0 && lane == 0) {
@@ -833,7 +841,7 @@ __global__ void __launch_bounds__(WO ? kThreadsW4 : kThreads, 1)
 #pragma unroll
                         for (int h = 0; h < 4; ++h)
                             emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + (c + h) * 16, v[h], srow, brow,
-                                    scol + (c + h) * 16, y_stage, ychunk);
+                                    scol + (c + h) * 16, y_stage, ychunk, kAccShift);
                     }
                     for (; c < chunks; ++c) {
                         int32_t *p = a.partial + ((size_t)sg.slot * a.bn + c * 16) * kTileA + row;
@@ -843,7 +851,7 @@ __global__ void __launch_bounds__(WO ? kThreadsW4 : kThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 16; ++e) __stcg(p + (size_t)e * kTileA, 0);
                         emit16s(J, a.swap, ta * kTileA, row, tid, tb * a.bn + c * 16, v, srow, brow, scol + c * 16,
-                                y_stage, ychunk);
+                                y_stage, ychunk, kAccShift);
                     }
                     if (ew == 0 && lane == 0) a.counters[sg.slot] = 0;
                 }
