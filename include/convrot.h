@@ -22,7 +22,8 @@
  *   y_j  = fp32( (sum_i a_i * H[i][j]) / 16 )   per 256-group, H Sylvester,
  *          the sum exact (FP64; exact while the nonzero magnitudes inside a
  *          group span at most 37 binades -- finite BF16 inputs outside that
- *          range give unspecified low bits).  Every rotating kernel records
+ *          range give unspecified low bits; non-finite inputs give
+ *          unspecified codes).  Every rotating kernel records
  *          CONVROT_WARN_INEXACT_DOMAIN for convrot_device_status() when a row
  *          holds a nonzero input |a| < 2^(e(amax) - 33), amax the row's
  *          largest |y| and e() the frexp exponent: every group spanning more

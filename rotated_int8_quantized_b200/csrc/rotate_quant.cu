@@ -121,8 +121,41 @@ __device__ __forceinline__ uint4 quant16(const float (&y)[16], const RowScale &r
 
 
 // The same codes with the FP32 pair instructions of sm_100 (two values per
-// multiply or add): identical arithmetic, each operation still rounded to
-// nearest even per value, half the instructions on the FP32 pipe.
+// instruction) and fused multiply-adds: e = fl(y r + 1.5 * 2^23) rounds the
+// exact product y r to the nearest integer (ties to even; the sum's ulp is
+// 1), and d = fl(y r - (e - 1.5 * 2^23)) is the exact residual rounded once
+// (|d| <= 0.5, error <= 2^-25).  With |y r - y/s| <= |y/s| 2^-24 and
+// |fl(y/s) - y/s| <= |y/s| 2^-24, |y/s| <= 127 (1 + 2^-23), a residual
+// below 0.49997 puts fl(y/s) within 0.49999 of the same integer, so e's low
+// byte is rne(fl(y/s)) there; elsewhere the division decides, as in
+// quant16.  The largest |d| of the 16 values comes from 3-input maxima of
+// magnitudes.  Inputs are finite (non-finite values give unspecified codes).
+// max(|a|, |b|, |c|) in one instruction (sm_100).
+__device__ __forceinline__ float max3abs(float a, float b, float c) {
+    float d;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t min_s16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 __device__ __forceinline__ uint64_t pack_f32x2(float a, float b) {
     uint64_t d;
     asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(a), "f"(b));
@@ -134,30 +167,27 @@ __device__ __forceinline__ void unpack_f32x2(uint64_t d, float &a, float &b) {
 
 __device__ __forceinline__ uint4 quant16x2(const float (&y)[16], const RowScale &rs, unsigned mask) {
     uint32_t b[16];
-    bool nr[4] = {false, false, false, false};     // four short "near" chains instead of one of 16
+    float dmax = 0.f;
     const uint64_t r2 = pack_f32x2(rs.r, rs.r), m2 = pack_f32x2(kRoundMagic, kRoundMagic);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        uint64_t t2, big2, rnd2, d2;
-        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(pack_f32x2(y[2 * i], y[2 * i + 1])), "l"(r2));
-        asm("add.rn.f32x2 %0, %1, %2;" : "=l"(big2) : "l"(t2), "l"(m2));
-        asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rnd2) : "l"(big2), "l"(m2));
-        asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d2) : "l"(t2), "l"(rnd2));
-        float d0, d1, b0, b1;
+        const uint64_t y2 = pack_f32x2(y[2 * i], y[2 * i + 1]);
+        const uint64_t e2 = fma_f32x2(y2, r2, m2);                   // rne(y r) in the low byte
+        const uint64_t d2 = fma_f32x2(y2, r2, sub_f32x2(m2, e2));    // y r - rne(y r), rounded once
+        float d0, d1, e0, e1;
         unpack_f32x2(d2, d0, d1);
-        unpack_f32x2(big2, b0, b1);
-        b[2 * i] = __float_as_uint(b0);                               // low byte: rne(t)
-        b[2 * i + 1] = __float_as_uint(b1);
-        nr[i & 3] |= !(fabsf(d0) < 0.49997f);                         // NaN too
-        nr[i & 3] |= !(fabsf(d1) < 0.49997f);
+        unpack_f32x2(e2, e0, e1);
+        b[2 * i] = __float_as_uint(e0);
+        b[2 * i + 1] = __float_as_uint(e1);
+        dmax = max3abs(d0, d1, dmax);
     }
-    const bool slow = (nr[0] || nr[1]) || (nr[2] || nr[3]) || !rs.fast;   // zero rows too (codes set below)
+    const bool slow = !(dmax < 0.49997f) || !rs.fast;   // zero rows too (codes set below)
     if (__any_sync(mask, slow) && slow) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            const float t = __fmul_rn(y[e], rs.r);
-            const float f = __fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic);
-            if (!rs.fast || !(fabsf(__fsub_rn(t, f)) < 0.49997f)) {
+            const float ei = __fmaf_rn(y[e], rs.r, kRoundMagic);
+            const float di = __fmaf_rn(y[e], rs.r, __fsub_rn(kRoundMagic, ei));
+            if (!rs.fast || !(fabsf(di) < 0.49997f)) {
                 const int c = __float_as_int(__fadd_rn(__fdiv_rn(y[e], rs.s), kRoundMagic)) - kRoundMagicBits;
                 b[e] = (uint32_t)min(max(c, -127), 127);
             }
@@ -310,32 +340,6 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// max(|a|, |b|, |c|) in one instruction (sm_100).
-__device__ __forceinline__ float max3abs(float a, float b, float c) {
-    float d;
-    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-__device__ __forceinline__ uint32_t min_s16x2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("min.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 
 // Per 16-bit half of a word of two BF16 values: 0x7FFF + |x| for x != 0,
 // and 0x7FFF for a zero, so that a signed 16-bit minimum ignores zeros and
@@ -1040,7 +1044,7 @@ __global__ void __launch_bounds__(kLeanThreads, 1) __maxnreg__(RCAP ? RCAP : 128
                         e[2 * i + 1] = __float_as_uint(e1);
                         dmax = max3abs(d0, d1, dmax);
                     }
-                    const bool slow = !(dmax < kLeanNear) || !fast;   // NaN too; zero rows (codes set below)
+                    const bool slow = !(dmax < kLeanNear) || !fast;   // zero rows too (codes set below)
                     if (__any_sync(mask, slow) && slow) {
                         const float sd = __fdiv_rn(rmax, 127.0f);
 #pragma unroll
