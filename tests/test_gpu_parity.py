@@ -668,6 +668,37 @@ def test_w4a8_linear_bit_exact(cr, m, shapes):
         assert np.array_equal(yb, ref["y"])
 
 
+@pytest.mark.parametrize("m", [12, 300, 1200])
+def test_w4a8_largest_sums_at_max_k(cr, m):
+    """The largest products the W4A8 path can accumulate, at the largest K
+    the API accepts: one unit spike per 256-group rotates to a constant
+    group (the first Hadamard row is all ones), so every activation code is
+    127 and every weight code +7 or -7, and each output sums K products of
+    +-889.  The GEMM's tensor cores see the unpacked weights as 16 x code,
+    so their INT32 sums reach 16 * 889 * 133120 = 1.89e9 (< 2^31) before the
+    epilogue divides by 16.  Decode (weights as A), 256 < M <= 512 (weights
+    as B) and larger M (the weight unpacked to INT8 first) are covered; all
+    rows of x are equal, so the oracle runs on one."""
+    k, n = 133120, 256
+    x_bits = np.zeros((1, k), dtype=np.uint16)
+    x_bits[0, ::256] = 0x3F80                        # 1.0 at the start of every group
+    w_bits = np.zeros((n, k), dtype=np.uint16)
+    w_bits[: n // 2, ::256] = 0x3F80                 # rows of +7 codes
+    w_bits[n // 2:, ::256] = 0xBF80                  # rows of -7 codes
+    packed_ref, s_ref = oracle.rotate_quantize4(w_bits)
+    assert np.array_equal(oracle.unpack_int4(packed_ref[:1]), np.full((1, k), 7, dtype=np.int8))
+    ref = oracle.linear_w4a8(x_bits, packed_ref, s_ref)
+    assert int(ref["acc"][0, 0]) == 889 * k and int(ref["acc"][0, n - 1]) == -889 * k
+    w4 = cr.quantize_weight4(from_bits(w_bits))
+    assert np.array_equal(w4.q.cpu().numpy(), packed_ref)
+    x = from_bits(x_bits).expand(m, k).contiguous()
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    cr.LinearBatchW4([x], [w4], [y])()
+    cr.convrot_device_status()
+    yb = to_bits(y)
+    assert np.array_equal(yb, np.broadcast_to(ref["y"], (m, n)))
+
+
 def test_w4a8_qwen_decode_layer_sampled(cr):
     lins = synth.qwen_layer(12)
     xs, ws4, ys = [], [], []
