@@ -170,7 +170,9 @@ size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * points (convrot_gemm_i8 / convrot_linear_int8) for m x k against n x k;
  * count in 2..8 (m <= 512): one batched launch of `count` products with the
  * same m (convrot_gemm_i8_batch / convrot_linear_int8_batch), w4 = 1 for
- * INT4 weights.  A CTA c of the `grid` takes, in order: whole
+ * INT4 weights unpacked inside the GEMM (what convrot_linear_w4a8 launches
+ * for m <= 512; for larger m it unpacks the weights to INT8 first and runs
+ * the INT8 plan, w4 = 0).  A CTA c of the `grid` takes, in order: whole
  * tiles wave * grid + c for wave < full_waves while below full_tiles; piece
  * c of the split tail when c < split_pieces (tile full_tiles + c / split_ways,
  * K blocks [s * kbpt / ways, (s + 1) * kbpt / ways) with s = c % ways); then
@@ -180,8 +182,7 @@ size_t convrot_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * job j is (A tile, B tile) with tiles_a[j] x tiles_b[j] tiles; 128-byte K
  * blocks, kbpt[j] per tile.  swap = 1: the weights are the 128-row A operand.
  * Errors: CONVROT_ERR_INVALID_ARG (null pointers, count out of range, sizes
- * < 1, sms < 1), CONVROT_ERR_UNSUPPORTED_SHAPE (a batch with m > 512, INT4
- * with m > 256).
+ * < 1, sms < 1), CONVROT_ERR_UNSUPPORTED_SHAPE (a batch with m > 512).
  */
 typedef struct {
     int32_t njobs, swap, bn, grid;
