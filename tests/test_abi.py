@@ -174,6 +174,14 @@ def test_weight4_validation(lib):
     assert h.k == 512 and h.group == 256
     assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10000), P(0x20000), 8, 48, 16) == 3   # k % 32
     assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10001), P(0x20000), 8, 512, 256) == 2
+    # the GEMM accumulates INT4 weights as 16 x code, exact while
+    # 16 * 7 * 127 * k < 2^31: the largest accepted k keeps that, the next one
+    # is refused when the handle is made
+    kmax = 133120
+    assert 16 * 7 * 127 * kmax < 2 ** 31
+    assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10000), P(0x20000), 8, kmax, 256) == 0
+    assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10000), P(0x20000), 8, kmax + 256, 256) == 3
+    assert lib.convrot_weight4_init(ctypes.byref(h), P(0x10000), P(0x20000), 8, 512, 256) == 0
     job = (cr.convrot_linear4_job_t * 1)()
     job[0].x_bf16, job[0].w, job[0].y_bf16 = P(0x100000), ctypes.pointer(h), P(0x200000)
     assert lib.convrot_linear_w4a8(0, 1, job, P(0x300000), 1 << 30, P(0)) == 1
